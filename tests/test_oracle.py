@@ -1,0 +1,385 @@
+"""Pins for the fp64 oracle, checked against things other than itself.
+
+Each pin cites the passage it follows.  The attention oracle is pinned by:
+torch's fp64 scaled_dot_product_attention with an explicit boolean mask built
+from tril/triu diagonals (a library routine); pure-Python brute force on tiny
+inputs that normalises without a max shift; closed forms (Q = 0, a single
+key, causal row 0, empty band); invariants (key permutation, key shift,
+linearity in V); and special-case reductions (GQA, varlen, window, decode).
+The quantiser is pinned by exact half-way rounding against numpy.rint, by its
+invariants, and by the compression ratio printed on the fkl page.
+``test_mutants_are_caught`` plants plausible mistakes in a copy of the C
+oracle and checks that the pins reject every one of them.
+"""
+import math
+import os
+import shutil
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from flashattention_attention_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------
+# helpers (test side)
+
+def band_mask(s_q, s_k, causal, window):
+    """Boolean [s_q, s_k] visibility mask from tril/triu diagonals.
+    Bottom-right alignment: query i sits at key position i + s_k - s_q."""
+    m = torch.ones(s_q, s_k, dtype=torch.bool)
+    off = s_k - s_q
+    if causal:
+        m = torch.tril(m, diagonal=off)
+    if window > 0:
+        m = m & torch.triu(torch.ones(s_q, s_k, dtype=torch.bool), diagonal=off - window + 1)
+    return m
+
+
+def sdpa_reference(q, k, v, hq, hkv, causal, window, scale):
+    """torch fp64 SDPA over dense [B*h, s, d] inputs, GQA via repeat_interleave."""
+    B = q.shape[0] // hq
+    s_q, s_k, d = q.shape[1], k.shape[1], q.shape[2]
+    qt = torch.as_tensor(q, dtype=torch.float64).reshape(B, hq, s_q, d)
+    kt = torch.as_tensor(k, dtype=torch.float64).reshape(B, hkv, s_k, d)
+    vt = torch.as_tensor(v, dtype=torch.float64).reshape(B, hkv, s_k, d)
+    kt = kt.repeat_interleave(hq // hkv, dim=1)
+    vt = vt.repeat_interleave(hq // hkv, dim=1)
+    mask = band_mask(s_q, s_k, causal, window)
+    out = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale)
+    return out.reshape(B * hq, s_q, d).numpy(), mask.numpy()
+
+
+def rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+# ----------------------------------------------------------------------------
+# pins, written as plain functions so the mutation test can rerun them
+
+SDPA_CASES = [
+    # B, hq, hkv, s_q, s_k, d, causal, window
+    (1, 1, 1, 7, 7, 8, False, 0),
+    (2, 4, 2, 9, 9, 16, True, 0),
+    (1, 8, 2, 5, 13, 8, True, 0),       # s_q < s_k: bottom-right causal
+    (2, 2, 1, 11, 11, 4, True, 3),      # causal + window
+    (1, 3, 3, 6, 10, 8, False, 4),      # window without causal (left bound only)
+    (1, 4, 1, 16, 16, 32, True, 16),    # window == s: same as causal
+    (1, 2, 2, 12, 5, 8, True, 0),       # s_q > s_k: leading rows empty (excluded here)
+]
+
+
+def pin_sdpa():
+    """fkl_python PR #6, Summary: softmax(q k^T) v, causal flag, (batch*heads,
+    seq, head_dim) layout; GQA per SKaiNET-transformers PR #419, Summary."""
+    rng = np.random.default_rng(1)
+    for (B, hq, hkv, s_q, s_k, d, causal, window) in SDPA_CASES:
+        q, k, v = rand(rng, B * hq, s_q, d), rand(rng, B * hkv, s_k, d), rand(rng, B * hkv, s_k, d)
+        scale = 0.37 + 0.1 * d ** -0.5
+        got = oracle.attention(q, k, v, hq=hq, hkv=hkv, causal=causal, window=window, scale=scale)
+        ref, mask = sdpa_reference(q, k, v, hq, hkv, causal, window, scale)
+        rows = mask.any(axis=1)
+        assert rows.any()
+        np.testing.assert_allclose(got[:, rows], ref[:, rows], rtol=0, atol=1e-12)
+
+
+def brute_force(q, k, v, hq, hkv, causal, window, scale):
+    """Pure-Python loops; weights exp(x_j) / sum exp(x_l) with no max shift."""
+    B = len(q) // hq
+    G = hq // hkv
+    out = []
+    for b in range(B):
+        for h in range(hq):
+            qq = q[b * hq + h]
+            kk = k[b * hkv + h // G]
+            vv = v[b * hkv + h // G]
+            s_q, s_k, d = len(qq), len(kk), len(qq[0])
+            rows = []
+            for i in range(s_q):
+                vis = []
+                for j in range(s_k):
+                    p = i + s_k - s_q
+                    ok = (not causal or j <= p) and (window <= 0 or j > p - window)
+                    if ok:
+                        vis.append(j)
+                if vis:
+                    e = {j: math.exp(scale * sum(qq[i][c] * kk[j][c] for c in range(d))) for j in vis}
+                    z = sum(e.values())
+                    rows.append([sum(e[j] * vv[j][c] for j in vis) / z for c in range(d)])
+                else:
+                    rows.append([sum(vv[j][c] for j in range(s_k)) / s_k if s_k else 0.0
+                                 for c in range(d)])
+            out.append(rows)
+    return np.array(out)
+
+
+def pin_brute_force():
+    rng = np.random.default_rng(2)
+    for (B, hq, hkv, s_q, s_k, d, causal, window) in [(1, 2, 1, 3, 4, 3, True, 0),
+                                                       (2, 2, 2, 4, 4, 2, False, 0),
+                                                       (1, 4, 2, 4, 3, 4, True, 2),
+                                                       (1, 1, 1, 4, 2, 3, True, 0)]:
+        q, k, v = rand(rng, B * hq, s_q, d), rand(rng, B * hkv, s_k, d), rand(rng, B * hkv, s_k, d)
+        got = oracle.attention(q, k, v, hq=hq, hkv=hkv, causal=causal, window=window, scale=0.7)
+        ref = brute_force(q.tolist(), k.tolist(), v.tolist(), hq, hkv, causal, window, 0.7)
+        np.testing.assert_allclose(got, ref, rtol=0, atol=1e-13)
+
+
+def pin_zero_query():
+    """Q = 0 makes every visible score equal: the output is the mean of V over
+    the band (closed form)."""
+    rng = np.random.default_rng(3)
+    s_q, s_k, d, W = 9, 12, 8, 4
+    v = rand(rng, 1, s_k, d)
+    k = rand(rng, 1, s_k, d)
+    q = np.zeros((1, s_q, d))
+    got = oracle.attention(q, k, v, hq=1, hkv=1, causal=True, window=W)
+    mask = band_mask(s_q, s_k, True, W).numpy()
+    for i in range(s_q):
+        np.testing.assert_allclose(got[0, i], v[0, mask[i]].mean(axis=0), rtol=0, atol=1e-14)
+
+
+def pin_single_key_and_row0():
+    """One key: o = v_0 exactly.  Causal row 0 of a square problem: o = v_0."""
+    rng = np.random.default_rng(4)
+    q, k, v = rand(rng, 3, 5, 16), rand(rng, 3, 1, 16), rand(rng, 3, 1, 16)
+    got = oracle.attention(q, k, v, hq=3, hkv=3, causal=False)
+    assert np.array_equal(got, np.broadcast_to(v, got.shape))
+    q, k, v = rand(rng, 2, 6, 16), rand(rng, 2, 6, 16), rand(rng, 2, 6, 16)
+    got = oracle.attention(q, k, v, hq=2, hkv=2, causal=True)
+    assert np.array_equal(got[:, 0], v[:, 0])
+
+
+def pin_empty_band():
+    """SKaiNET-transformers PR #419, Summary: an empty sliding-window band
+    reproduces the uniform softmax, i.e. the mean of all V rows.  Here s_q > s_k
+    under causal masking leaves the first s_q - s_k rows with no visible key."""
+    rng = np.random.default_rng(5)
+    s_q, s_k, d = 10, 4, 8
+    q, k, v = rand(rng, 2, s_q, d), rand(rng, 2, s_k, d), rand(rng, 2, s_k, d)
+    got = oracle.attention(q, k, v, hq=2, hkv=2, causal=True)
+    for h in range(2):
+        for i in range(s_q - s_k):
+            np.testing.assert_allclose(got[h, i], v[h].mean(axis=0), rtol=0, atol=1e-15)
+    # decode against an empty cache gives zeros
+    out = oracle.decode(rand(rng, 2, 1, d), np.zeros((1, 8, d)), np.ones((1, 8, d)), [0],
+                        hq=2, hkv=1)
+    assert not out.any()
+
+
+def pin_invariants():
+    """Non-causal attention is invariant under a joint permutation of the
+    (k, v) rows; adding one vector to every key shifts each row's scores by a
+    constant and leaves the output unchanged; the output is linear in V."""
+    rng = np.random.default_rng(6)
+    q, k, v = rand(rng, 2, 7, 8), rand(rng, 2, 11, 8), rand(rng, 2, 11, 8)
+    base = oracle.attention(q, k, v, hq=2, hkv=2)
+    perm = rng.permutation(11)
+    np.testing.assert_allclose(oracle.attention(q, k[:, perm], v[:, perm], hq=2, hkv=2), base,
+                               rtol=0, atol=1e-13)
+    shifted = oracle.attention(q, k + rand(rng, 1, 1, 8), v, hq=2, hkv=2)
+    np.testing.assert_allclose(shifted, base, rtol=0, atol=1e-12)
+    v2 = rand(rng, 2, 11, 8)
+    lin = oracle.attention(q, k, 2.0 * v - 3.0 * v2, hq=2, hkv=2, causal=True, window=5)
+    ref = (2.0 * oracle.attention(q, k, v, hq=2, hkv=2, causal=True, window=5)
+           - 3.0 * oracle.attention(q, k, v2, hq=2, hkv=2, causal=True, window=5))
+    np.testing.assert_allclose(lin, ref, rtol=0, atol=1e-12)
+
+
+def pin_reductions():
+    """GQA == MHA with KV heads repeated; varlen == per-sequence dense calls;
+    a window >= s_k == plain causal; decode == the last row of a prefill."""
+    rng = np.random.default_rng(7)
+    hq, hkv, s, d = 8, 2, 10, 8
+    q, k, v = rand(rng, hq, s, d), rand(rng, hkv, s, d), rand(rng, hkv, s, d)
+    gqa = oracle.attention(q, k, v, hq=hq, hkv=hkv, causal=True)
+    mha = oracle.attention(q, np.repeat(k, hq // hkv, axis=0), np.repeat(v, hq // hkv, axis=0),
+                           hq=hq, hkv=hq, causal=True)
+    assert np.array_equal(gqa, mha)
+
+    lengths = [5, 1, 9, 3]
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    tot = cu[-1]
+    qv, kv, vv = rand(rng, hq, tot, d), rand(rng, hkv, tot, d), rand(rng, hkv, tot, d)
+    var = oracle.attention(qv, kv, vv, hq=hq, hkv=hkv, causal=True, window=3, cu_seqlens_q=cu)
+    for b in range(len(lengths)):
+        sl = slice(cu[b], cu[b + 1])
+        dense = oracle.attention(qv[:, sl], kv[:, sl], vv[:, sl], hq=hq, hkv=hkv, causal=True,
+                                 window=3)
+        assert np.array_equal(var[:, sl], dense)
+
+    wide = oracle.attention(q, k, v, hq=hq, hkv=hkv, causal=True, window=s)
+    assert np.array_equal(wide, gqa)
+
+    L = [10, 6]
+    cap = 12
+    kc, vc = np.zeros((2 * hkv, cap, d)), np.zeros((2 * hkv, cap, d))
+    qd = rand(rng, 2 * hq, 1, d)
+    for b in range(2):
+        kc[b * hkv:(b + 1) * hkv, :L[b]] = rand(rng, hkv, L[b], d)
+        vc[b * hkv:(b + 1) * hkv, :L[b]] = rand(rng, hkv, L[b], d)
+    dec = oracle.decode(qd, kc, vc, L, hq=hq, hkv=hkv)
+    for b in range(2):
+        qp = np.concatenate([rand(rng, hq, L[b] - 1, d), qd[b * hq:(b + 1) * hq]], axis=1)
+        pre = oracle.attention(qp, kc[b * hkv:(b + 1) * hkv, :L[b]], vc[b * hkv:(b + 1) * hkv, :L[b]],
+                               hq=hq, hkv=hkv, causal=True)
+        np.testing.assert_allclose(dec[b * hq:(b + 1) * hq, 0], pre[:, -1], rtol=0, atol=1e-15)
+
+
+def pin_epilogue():
+    """fkl_python PR #6, Summary: epilogue=[Mul(2.0), Add(0.5)] runs on the
+    attention output, in order (Mul first, then Add)."""
+    rng = np.random.default_rng(8)
+    q, k, v = rand(rng, 2, 6, 8), rand(rng, 2, 6, 8), rand(rng, 2, 6, 8)
+    o = oracle.attention(q, k, v, hq=2, hkv=2, causal=True)
+    ma = oracle.attention(q, k, v, hq=2, hkv=2, causal=True, epilogue=[("mul", 2.0), ("add", 0.5)])
+    am = oracle.attention(q, k, v, hq=2, hkv=2, causal=True, epilogue=[("add", 0.5), ("mul", 2.0)])
+    np.testing.assert_allclose(ma, 2.0 * o + 0.5, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(am, 2.0 * (o + 0.5), rtol=0, atol=1e-15)
+
+
+def pin_row_selection():
+    """Computing a subset of rows gives those rows of the full result."""
+    rng = np.random.default_rng(9)
+    q, k, v = rand(rng, 4, 9, 8), rand(rng, 2, 9, 8), rand(rng, 2, 9, 8)
+    full = oracle.attention(q, k, v, hq=2, hkv=1, causal=True, window=4)
+    sel = [(0, 1, 3), (1, 0, 8), (1, 1, 0)]
+    part = oracle.attention(q, k, v, hq=2, hkv=1, causal=True, window=4, rows=sel)
+    for (b, h, i) in sel:
+        assert np.array_equal(part[b * 2 + h, i], full[b * 2 + h, i])
+
+
+def pin_quantiser_rounding():
+    """fkl_python PR #6, Summary: per-token int8 with one fp32 scale.  A row
+    whose max |x| is 127 has scale exactly 1, so its codes are x rounded half
+    to even, which numpy.rint computes."""
+    halves = np.array([0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.5, 126.5, -126.5, 0.49999997, 2.5000002],
+                      dtype=np.float32)
+    row = np.concatenate([halves, np.array([127.0, -3.25, 64.75], dtype=np.float32)])
+    codes, scales = oracle.compress_kv(row[None, :])
+    assert scales[0] == np.float32(1.0)
+    assert np.array_equal(codes[0].astype(np.int64), np.rint(row).astype(np.int64))
+
+
+def pin_quantiser_invariants():
+    """|c| <= 127; each row's max-|x| element maps to +-127; |x - c s| <= s/2
+    (to rounding); an all-zero row has scale 0 and zero codes."""
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((64, 128)).astype(np.float32) * rng.uniform(1e-3, 1e3, (64, 1)).astype(np.float32)
+    x[5] = 0.0
+    codes, scales = oracle.compress_kv(x)
+    assert np.abs(codes.astype(np.int32)).max() <= 127
+    assert scales[5] == 0 and not codes[5].any()
+    for r in range(64):
+        if r == 5:
+            continue
+        a = np.argmax(np.abs(x[r]))
+        assert abs(int(codes[r, a])) == 127 and np.sign(codes[r, a]) == np.sign(x[r, a])
+        err = np.abs(x[r].astype(np.float64) - codes[r].astype(np.float64) * float(scales[r]))
+        assert err.max() <= 0.5 * float(scales[r]) * (1 + 1e-5)
+        np.testing.assert_allclose(float(scales[r]), np.abs(x[r]).max() / 127.0, rtol=1e-7)
+
+
+def pin_compression_ratio():
+    """fkl_python PR #6, Verification: 'KV compression ratio 3.76x (>3.5x)'.
+    Measured from the oracle's output buffers at head_dim 64 against fp32."""
+    with open(os.path.join(GOLDEN, "compression_ratio.txt")) as f:
+        fields = dict(line.split("=", 1) for line in f.read().split("\n")
+                      if "=" in line and not line.startswith("#"))
+    d = int(fields["head_dim"])
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((1000, d)).astype(np.float32)
+    codes, scales = oracle.compress_kv(x)
+    ratio = x.nbytes / (codes.nbytes + scales.nbytes)
+    assert f"{ratio:.2f}" == fields["ratio"].strip()
+    assert ratio > float(fields["gate"])
+    assert abs(ratio - d / (d / 4 + 1)) < 1e-12
+
+
+def pin_int8_end_to_end():
+    """fkl_python PR #6, Summary and Verification: attention over the int8
+    cache stays within ~1e-3-order error of the unquantised result (the page
+    measured 3.9e-3).  A loose bound: the error is nonzero and below 2e-2."""
+    rng = np.random.default_rng(12)
+    q, k, v = rand(rng, 4, 64, 64), rand(rng, 4, 64, 64), rand(rng, 4, 64, 64)
+    exact = oracle.attention(q, k, v, hq=4, hkv=4, causal=True)
+    kq = oracle.dequantize(*oracle.compress_kv(k.astype(np.float32)))
+    vq = oracle.dequantize(*oracle.compress_kv(v.astype(np.float32)))
+    approx = oracle.attention(q, kq, vq, hq=4, hkv=4, causal=True)
+    err = np.abs(approx - exact).max()
+    assert 1e-5 < err < 2e-2
+
+
+ALL_PINS = [pin_sdpa, pin_brute_force, pin_zero_query, pin_single_key_and_row0, pin_empty_band,
+            pin_invariants, pin_reductions, pin_epilogue, pin_row_selection,
+            pin_quantiser_rounding, pin_quantiser_invariants, pin_compression_ratio,
+            pin_int8_end_to_end]
+
+
+@pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
+def test_pin(pin):
+    pin()
+
+
+# ----------------------------------------------------------------------------
+# mutation test: plausible mistakes planted in a copy of the C oracle
+
+MUTANTS = {
+    "dropped_scale": ("score[j] = scale * dot;", "score[j] = dot;"),
+    "causal_top_left": ("int64_t p = i + s_k - s_q;", "int64_t p = i;"),
+    "causal_strict": ("if (causal && j > p) return 0;", "if (causal && j >= p) return 0;"),
+    "window_off_by_one": ("if (window > 0 && j <= p - window) return 0;",
+                          "if (window > 0 && j < p - window) return 0;"),
+    "gqa_modulo": ("int64_t g = h / group;", "int64_t g = h % hkv;"),
+    "empty_band_zero": ("for (c = 0; c < d; ++c) out_row[c] /= (double)s_k;",
+                        "for (c = 0; c < d; ++c) out_row[c] = 0.0;"),
+    "no_max_shift_sign": ("score[j] = exp(score[j] - m);", "score[j] = exp(m - score[j]);"),
+    "transposed_kv": ("out_row[c] += w * v_rows[j * kv_row_stride + c];",
+                      "out_row[c] += w * k_rows[j * kv_row_stride + c];"),
+    "epilogue_reversed": ("for (int e = 0; e < n_epi; ++e) {", "for (int e = n_epi - 1; e >= 0; --e) {"),
+    "quant_truncate": ("float t = nearbyintf(xr[c] / s);", "float t = truncf(xr[c] / s);"),
+    "quant_scale_128": ("float s = amax / 127.0f;", "float s = amax / 128.0f;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutants_are_caught(name, monkeypatch):
+    old, new = MUTANTS[name]
+    src = open(oracle._SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not unique"
+    tmp = tempfile.mkdtemp()
+    try:
+        path = os.path.join(tmp, "mutant.c")
+        with open(path, "w") as f:
+            f.write(src.replace(old, new))
+        lib = os.path.join(tmp, "libmutant.so")
+        subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
+                               "-std=c99", "-shared", "-fPIC", "-o", lib, path, "-lm"])
+        monkeypatch.setattr(oracle, "_LIB", lib)
+        monkeypatch.setattr(oracle, "_SRC", path)
+        monkeypatch.setattr(oracle, "_lib", None)
+        caught = []
+        for pin in ALL_PINS:
+            try:
+                pin()
+            except AssertionError:
+                caught.append(pin.__name__)
+        assert caught, f"mutant {name} passed every pin"
+    finally:
+        monkeypatch.setattr(oracle, "_lib", None)
+        shutil.rmtree(tmp)
+
+
+def test_workload_lengths():
+    """The seeded lengths of the benchmarked workloads are reproducible."""
+    w = inputs.varlen_lengths(0, 8, 33, 8192)
+    assert w == [6974, 5230, 4203, 2234, 2544, 367, 646, 167]
+    lens = np.random.default_rng(0).integers(1024, 32769, 16)
+    assert int(lens.sum()) == 272568
