@@ -1,0 +1,290 @@
+// fa_api.cu -- the C ABI of libfa.so (declared in include/fa.h): argument
+// checks, dispatch to the kernels, the per-device status word, TMA
+// descriptor encoding, and the watchdog self-test kernel.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <mutex>
+#include <set>
+
+#include "internal.h"
+
+namespace fa {
+namespace {
+
+std::mutex g_mu;
+constexpr int kMaxDevices = 64;
+unsigned int* g_status[kMaxDevices] = {};
+long long g_budget = 0;
+std::set<const void*>* g_variants = nullptr;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+long long watchdog_budget() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_budget == 0) {
+    const char* e = std::getenv("FA_WATCHDOG_CYCLES");
+    long long v = e ? std::atoll(e) : 0;
+    g_budget = v > 0 ? v : 4000000000LL;  // about 2 s at the boost clock
+  }
+  return g_budget;
+}
+
+fa_status status_word(unsigned int** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_status[dev] == nullptr) {
+    unsigned int* p = nullptr;
+    if (cudaMalloc(&p, 16) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMemset(p, 0, 16) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+      cudaFree(p);
+      return FA_ERR_CUDA;
+    }
+    g_status[dev] = p;
+  }
+  *out = g_status[dev];
+  return FA_OK;
+}
+
+fa_status make_ctx(fa_stream_t s, LaunchCtx* ctx) {
+  ctx->stream = reinterpret_cast<cudaStream_t>(s);
+  ctx->wd.budget = watchdog_budget();
+  return status_word(&ctx->wd.word);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool epilogue_ok(const fa_epi_op* ops, int n) {
+  if (n < 0 || n > FA_MAX_EPILOGUE) return false;
+  for (int i = 0; i < n; ++i) {
+    if (ops[i].op != FA_EPI_MUL && ops[i].op != FA_EPI_ADD) return false;
+  }
+  return true;
+}
+
+__global__ void watchdog_selftest_kernel(Watchdog wd) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);  // expects one arrival that never comes
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_parity(&bar, 0, wd, &abort_flag);
+  __syncthreads();
+}
+
+}  // namespace
+
+Epilogue make_epilogue(const fa_epi_op* ops, int n) {
+  Epilogue e;
+  e.n = n;
+  for (int i = 0; i < 8; ++i) {
+    e.op[i] = i < n ? ops[i].op : 0;
+    e.val[i] = i < n ? ops[i].value : 0.f;
+  }
+  return e;
+}
+
+void note_variant(const void* kernel_fn) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_variants == nullptr) g_variants = new std::set<const void*>();
+  g_variants->insert(kernel_fn);
+}
+
+fa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                            const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                            CUtensorMapSwizzle swizzle) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return FA_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  cuuint64_t d[5];
+  cuuint64_t s[4];
+  cuuint32_t b[5], e[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    e[i] = 1;
+    if (i + 1 < rank) s[i] = strides_bytes[i];
+  }
+  CUresult r = g_encode(map, dtype, rank, const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported combination";
+    case FA_ERR_CUDA: return "CUDA call failed";
+    case FA_ERR_TIMEOUT: return "bounded device wait timed out";
+    case FA_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+fa_status fa_compress_kv(const void* x, fa_dtype x_dtype, int64_t rows, int32_t d, int8_t* codes, float* scales,
+                         fa_stream_t stream) {
+  if (rows < 0 || d < 16 || d > 1024 || d % 16 != 0) return FA_ERR_INVALID;
+  if (x_dtype != FA_BF16 && x_dtype != FA_F32) return FA_ERR_INVALID;
+  if (rows == 0) return FA_OK;
+  if (x == nullptr || codes == nullptr || scales == nullptr) return FA_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return FA_ERR_INVALID;
+  LaunchCtx ctx;
+  fa_status st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  return launch_compress(x, x_dtype, rows, d, codes, scales, ctx);
+}
+
+fa_status fa_attention_fwd(const fa_fwd_params* p, fa_stream_t stream) {
+  if (p == nullptr) return FA_ERR_INVALID;
+  if (p->batch < 0 || p->hq <= 0 || p->hkv <= 0 || p->hq % p->hkv != 0) return FA_ERR_INVALID;
+  if (!epilogue_ok(p->epilogue, p->n_epilogue)) return FA_ERR_INVALID;
+  if (!std::isfinite(p->softmax_scale)) return FA_ERR_INVALID;
+  const bool varlen = p->cu_seqlens_q != nullptr;
+  if (varlen) {
+    if (p->total_q < 0 || p->total_k < 0 || p->max_seqlen_q < 0 || p->max_seqlen_k < 0) return FA_ERR_INVALID;
+  } else {
+    if (p->seqlen_q < 0 || p->seqlen_k < 0) return FA_ERR_INVALID;
+    if (p->cu_seqlens_k != nullptr) return FA_ERR_INVALID;
+  }
+  if (p->q_dtype == FA_F32) {
+    if (p->kv_dtype != FA_F32) return FA_ERR_INVALID;
+    if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
+    if (p->head_dim > 256) return FA_ERR_UNSUPPORTED;
+  } else if (p->q_dtype == FA_BF16) {
+    if (p->kv_dtype != FA_BF16 && p->kv_dtype != FA_I8) return FA_ERR_INVALID;
+    if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
+    if (p->kv_dtype == FA_I8 && (p->k_scales == nullptr || p->v_scales == nullptr)) return FA_ERR_INVALID;
+    if (p->kv_dtype == FA_I8 && (!aligned16(p->k_scales) || !aligned16(p->v_scales))) return FA_ERR_INVALID;
+    if (p->head_dim != 64 && p->head_dim != 128) return FA_ERR_UNSUPPORTED;
+  } else {
+    return FA_ERR_INVALID;
+  }
+  const bool empty = p->batch == 0 || (varlen ? p->total_q == 0 : p->seqlen_q == 0);
+  if (empty) return FA_OK;
+  if (p->q == nullptr || p->k == nullptr || p->v == nullptr || p->out == nullptr) return FA_ERR_INVALID;
+  if (!aligned16(p->q) || !aligned16(p->k) || !aligned16(p->v) || !aligned16(p->out)) return FA_ERR_INVALID;
+  LaunchCtx ctx;
+  fa_status st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  st = (p->q_dtype == FA_F32) ? launch_attn_f32(*p, ctx) : launch_prefill_tc(*p, ctx);
+  if (st != FA_OK) return st;
+  return launch_empty_rows(*p, ctx);
+}
+
+size_t fa_decode_workspace_size(int32_t batch, int32_t hq, int32_t capacity, int32_t head_dim) {
+  if (batch <= 0 || hq <= 0 || capacity <= 0 || head_dim <= 0) return 0;
+  const size_t n_split_max = (static_cast<size_t>(capacity) + 255) / 256;
+  const size_t recs = static_cast<size_t>(batch) * hq * n_split_max;
+  const size_t o_bytes = recs * head_dim * sizeof(float);
+  return o_bytes + recs * 2 * sizeof(float);
+}
+
+fa_status fa_attention_decode(const fa_decode_params* p, fa_stream_t stream) {
+  if (p == nullptr) return FA_ERR_INVALID;
+  if (p->batch < 0 || p->hq <= 0 || p->hkv <= 0 || p->hq % p->hkv != 0) return FA_ERR_INVALID;
+  if (p->capacity <= 0 || p->capacity % 32 != 0) return FA_ERR_INVALID;
+  if (p->max_seqlen < 0 || p->max_seqlen > p->capacity) return FA_ERR_INVALID;
+  if (p->split_keys < 0 || p->split_keys % 256 != 0) return FA_ERR_INVALID;
+  if (!epilogue_ok(p->epilogue, p->n_epilogue)) return FA_ERR_INVALID;
+  if (!std::isfinite(p->softmax_scale)) return FA_ERR_INVALID;
+  if (p->kv_dtype != FA_I8 && p->kv_dtype != FA_BF16) return FA_ERR_INVALID;
+  if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
+  if (p->head_dim != 64 && p->head_dim != 128) return FA_ERR_UNSUPPORTED;
+  if (p->hq / p->hkv > 8) return FA_ERR_UNSUPPORTED;
+  if (p->batch == 0) return FA_OK;
+  if (p->q == nullptr || p->k_cache == nullptr || p->v_cache == nullptr || p->out == nullptr ||
+      p->cache_seqlens == nullptr)
+    return FA_ERR_INVALID;
+  if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->out))
+    return FA_ERR_INVALID;
+  if (p->kv_dtype == FA_I8) {
+    if (p->k_scales == nullptr || p->v_scales == nullptr) return FA_ERR_INVALID;
+    if (!aligned16(p->k_scales) || !aligned16(p->v_scales)) return FA_ERR_INVALID;
+  }
+  const size_t need = fa_decode_workspace_size(p->batch, p->hq, p->capacity, p->head_dim);
+  if (p->workspace == nullptr || p->workspace_bytes < need || !aligned16(p->workspace)) return FA_ERR_WORKSPACE;
+
+  const int max_len = p->max_seqlen > 0 ? p->max_seqlen : p->capacity;
+  int split = p->split_keys;
+  if (split == 0) {
+    // Aim for about four CTAs per SM slot over the (sequence, kv-head) pairs.
+    const long long pairs = static_cast<long long>(p->batch) * p->hkv;
+    const long long want_units = 148LL * 2 * 4;
+    long long per = (static_cast<long long>(max_len) * pairs + want_units - 1) / want_units;
+    per = ((per + 255) / 256) * 256;
+    if (per < 256) per = 256;
+    if (per > 4096) per = 4096;
+    split = static_cast<int>(per);
+  }
+  const int n_splits = (max_len + split - 1) / split;
+  LaunchCtx ctx;
+  fa_status st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  if (n_splits == 0) {
+    // every cache is empty: the merge alone writes the epilogue of zeros
+    return launch_decode(*p, split, 1, ctx);
+  }
+  return launch_decode(*p, split, n_splits, ctx);
+}
+
+fa_status fa_check_device_error(fa_stream_t stream) {
+  unsigned int* word = nullptr;
+  fa_status st = status_word(&word);
+  if (st != FA_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  unsigned int host = 0;
+  if (cudaMemcpy(&host, word, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+  if (host != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if (host & kStatusTimeout) return FA_ERR_TIMEOUT;
+  return FA_OK;
+}
+
+fa_status fa_selftest_watchdog(uint64_t budget_cycles, fa_stream_t stream) {
+  LaunchCtx ctx;
+  fa_status st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  unsigned long long b = budget_cycles;
+  if (b < 1000ULL) b = 1000ULL;
+  if (b > 1000000000ULL) b = 1000000000ULL;
+  return launch_watchdog_selftest(b, ctx);
+}
+
+int32_t fa_kernel_variants_used(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return g_variants ? static_cast<int32_t>(g_variants->size()) : 0;
+}
+
+}  // extern "C"
+
+namespace fa {
+fa_status launch_watchdog_selftest(unsigned long long budget, const LaunchCtx& ctx) {
+  Watchdog wd = ctx.wd;
+  wd.budget = static_cast<long long>(budget);
+  note_variant(reinterpret_cast<const void*>(watchdog_selftest_kernel));
+  watchdog_selftest_kernel<<<1, 32, 0, ctx.stream>>>(wd);
+  return cuda_status(cudaGetLastError());
+}
+}  // namespace fa

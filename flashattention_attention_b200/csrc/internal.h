@@ -1,0 +1,37 @@
+// internal.h -- launchers shared between the C-ABI host layer (fa_api.cu) and
+// the kernel files.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "device.cuh"
+#include "fa.h"
+
+namespace fa {
+
+struct LaunchCtx {
+  cudaStream_t stream;
+  Watchdog wd;
+};
+
+Epilogue make_epilogue(const fa_epi_op* ops, int n);
+
+// Records that a kernel instantiation was launched (distinct-variant count).
+void note_variant(const void* kernel_fn);
+
+fa_status launch_compress(const void* x, int x_dtype, int64_t rows, int d, int8_t* codes, float* scales,
+                          const LaunchCtx& ctx);
+fa_status launch_attn_f32(const fa_fwd_params& p, const LaunchCtx& ctx);
+fa_status launch_empty_rows(const fa_fwd_params& p, const LaunchCtx& ctx);
+fa_status launch_prefill_tc(const fa_fwd_params& p, const LaunchCtx& ctx);
+fa_status launch_decode(const fa_decode_params& p, int split_keys, int n_splits, const LaunchCtx& ctx);
+fa_status launch_watchdog_selftest(unsigned long long budget, const LaunchCtx& ctx);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+fa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                            const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                            CUtensorMapSwizzle swizzle);
+
+inline fa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+}  // namespace fa

@@ -1,0 +1,232 @@
+"""Thin ctypes binding of libfa.so (include/fa.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI.  torch supplies device memory and the current
+stream.  Importing this module loads ``lib/libfa.so`` and raises ImportError
+when it is missing -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libfa.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libfa.so not built ({_LIB_PATH}); run __graft_entry__.build() "
+                      "or python flashattention_attention_b200/build.py")
+lib = ctypes.CDLL(_LIB_PATH)
+
+# --- fa.h mirrors -------------------------------------------------------------
+FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+FA_F32, FA_BF16, FA_I8 = 0, 1, 2
+FA_EPI_MUL, FA_EPI_ADD = 1, 2
+FA_MAX_EPILOGUE = 8
+
+
+class EpiOp(ctypes.Structure):
+    _fields_ = [("op", ctypes.c_int32), ("value", ctypes.c_float)]
+
+
+class FwdParams(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("out", ctypes.c_void_p), ("k_scales", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
+                ("q_dtype", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
+                ("batch", ctypes.c_int32), ("hq", ctypes.c_int32), ("hkv", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("seqlen_q", ctypes.c_int32), ("seqlen_k", ctypes.c_int32),
+                ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
+                ("total_q", ctypes.c_int32), ("total_k", ctypes.c_int32),
+                ("max_seqlen_q", ctypes.c_int32), ("max_seqlen_k", ctypes.c_int32),
+                ("causal", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float), ("n_epilogue", ctypes.c_int32),
+                ("epilogue", EpiOp * FA_MAX_EPILOGUE)]
+
+
+class DecodeParams(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("k_scales", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
+                ("cache_seqlens", ctypes.c_void_p), ("out", ctypes.c_void_p),
+                ("kv_dtype", ctypes.c_int32), ("batch", ctypes.c_int32), ("hq", ctypes.c_int32),
+                ("hkv", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("capacity", ctypes.c_int32),
+                ("max_seqlen", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float), ("split_keys", ctypes.c_int32),
+                ("n_epilogue", ctypes.c_int32), ("epilogue", EpiOp * FA_MAX_EPILOGUE),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
+lib.fa_compress_kv.restype = ctypes.c_int
+lib.fa_compress_kv.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int32,
+                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+lib.fa_attention_fwd.restype = ctypes.c_int
+lib.fa_attention_fwd.argtypes = [ctypes.POINTER(FwdParams), ctypes.c_void_p]
+lib.fa_decode_workspace_size.restype = ctypes.c_size_t
+lib.fa_decode_workspace_size.argtypes = [ctypes.c_int32] * 4
+lib.fa_attention_decode.restype = ctypes.c_int
+lib.fa_attention_decode.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_void_p]
+lib.fa_status_string.restype = ctypes.c_char_p
+lib.fa_status_string.argtypes = [ctypes.c_int]
+lib.fa_check_device_error.restype = ctypes.c_int
+lib.fa_check_device_error.argtypes = [ctypes.c_void_p]
+lib.fa_selftest_watchdog.restype = ctypes.c_int
+lib.fa_selftest_watchdog.argtypes = [ctypes.c_uint64, ctypes.c_void_p]
+lib.fa_kernel_variants_used.restype = ctypes.c_int32
+lib.fa_kernel_variants_used.argtypes = []
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {lib.fa_status_string(status).decode()} (status {status})")
+        self.status = status
+
+
+def _check(status: int, what: str):
+    if status != FA_OK:
+        raise FAError(status, what)
+
+
+_DT = {torch.float32: FA_F32, torch.bfloat16: FA_BF16, torch.int8: FA_I8}
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _fill_epilogue(arr, epilogue: Sequence[Tuple[str, float]]) -> int:
+    if len(epilogue) > FA_MAX_EPILOGUE:
+        raise ValueError(f"at most {FA_MAX_EPILOGUE} epilogue ops")
+    for i, (op, val) in enumerate(epilogue):
+        name = op.lower() if isinstance(op, str) else op
+        arr[i].op = {"mul": FA_EPI_MUL, "add": FA_EPI_ADD}.get(name, name)
+        arr[i].value = float(val)
+    return len(epilogue)
+
+
+def _contig_cuda(t: torch.Tensor, name: str):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+# --- API ----------------------------------------------------------------------
+
+def compress_kv(x: torch.Tensor, codes: Optional[torch.Tensor] = None,
+                scales: Optional[torch.Tensor] = None, stream=None):
+    """Per-row int8 codes + fp32 scales of x [..., d] (bf16 or fp32)."""
+    _contig_cuda(x, "x")
+    d = x.shape[-1]
+    rows = x.numel() // d if d else 0
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _check(lib.fa_compress_kv(_ptr(x), _DT[x.dtype], rows, d, _ptr(codes), _ptr(scales), _stream(stream)),
+           "fa_compress_kv")
+    return codes, scales
+
+
+def fwd_params(q, k, v, out, *, hq, hkv, causal=False, window=0, scale=None, epilogue=(),
+               k_scales=None, v_scales=None, cu_seqlens_q=None, cu_seqlens_k=None,
+               max_seqlen_q=None, max_seqlen_k=None) -> FwdParams:
+    p = FwdParams()
+    p.q, p.k, p.v, p.out = q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr()
+    p.k_scales = None if k_scales is None else k_scales.data_ptr()
+    p.v_scales = None if v_scales is None else v_scales.data_ptr()
+    p.q_dtype, p.kv_dtype = _DT[q.dtype], _DT[k.dtype]
+    p.hq, p.hkv, p.head_dim = hq, hkv, q.shape[-1]
+    if cu_seqlens_q is None:
+        p.batch = q.shape[0] // hq
+        p.seqlen_q, p.seqlen_k = q.shape[1], k.shape[1]
+    else:
+        p.batch = cu_seqlens_q.numel() - 1
+        p.cu_seqlens_q = cu_seqlens_q.data_ptr()
+        p.cu_seqlens_k = None if cu_seqlens_k is None else cu_seqlens_k.data_ptr()
+        p.total_q, p.total_k = q.shape[1], k.shape[1]
+        p.max_seqlen_q = int(max_seqlen_q)
+        p.max_seqlen_k = int(max_seqlen_k if max_seqlen_k is not None else max_seqlen_q)
+    p.causal, p.window = int(bool(causal)), int(window)
+    p.softmax_scale = float(scale if scale is not None else 1.0 / math.sqrt(q.shape[-1]))
+    p.n_epilogue = _fill_epilogue(p.epilogue, epilogue)
+    return p
+
+
+def attention_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, hq: int, hkv: int,
+                  causal: bool = False, window: int = 0, scale: Optional[float] = None,
+                  epilogue: Sequence[Tuple[str, float]] = (), k_scales=None, v_scales=None,
+                  cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None, max_seqlen_k=None,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Fused attention forward; layouts and semantics as fa_attention_fwd in fa.h."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _contig_cuda(t, name)
+    if out is None:
+        out = torch.empty_like(q)
+    p = fwd_params(q, k, v, out, hq=hq, hkv=hkv, causal=causal, window=window, scale=scale,
+                   epilogue=epilogue, k_scales=k_scales, v_scales=v_scales, cu_seqlens_q=cu_seqlens_q,
+                   cu_seqlens_k=cu_seqlens_k, max_seqlen_q=max_seqlen_q, max_seqlen_k=max_seqlen_k)
+    _check(lib.fa_attention_fwd(ctypes.byref(p), _stream(stream)), "fa_attention_fwd")
+    return out
+
+
+def decode_workspace_size(batch: int, hq: int, capacity: int, head_dim: int) -> int:
+    return int(lib.fa_decode_workspace_size(batch, hq, capacity, head_dim))
+
+
+def decode_params(q, k_cache, v_cache, cache_seqlens, out, workspace, *, hq, hkv, k_scales=None,
+                  v_scales=None, window=0, scale=None, epilogue=(), max_seqlen=0,
+                  split_keys=0) -> DecodeParams:
+    p = DecodeParams()
+    p.q, p.k_cache, p.v_cache = q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr()
+    p.k_scales = None if k_scales is None else k_scales.data_ptr()
+    p.v_scales = None if v_scales is None else v_scales.data_ptr()
+    p.cache_seqlens, p.out = cache_seqlens.data_ptr(), out.data_ptr()
+    p.kv_dtype = _DT[k_cache.dtype]
+    p.batch = cache_seqlens.numel()
+    p.hq, p.hkv, p.head_dim, p.capacity = hq, hkv, q.shape[-1], k_cache.shape[1]
+    p.max_seqlen, p.window = int(max_seqlen), int(window)
+    p.softmax_scale = float(scale if scale is not None else 1.0 / math.sqrt(q.shape[-1]))
+    p.split_keys = int(split_keys)
+    p.n_epilogue = _fill_epilogue(p.epilogue, epilogue)
+    p.workspace = workspace.data_ptr()
+    p.workspace_bytes = workspace.numel() * workspace.element_size()
+    return p
+
+
+def attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                     cache_seqlens: torch.Tensor, *, hq: int, hkv: int, k_scales=None, v_scales=None,
+                     window: int = 0, scale: Optional[float] = None,
+                     epilogue: Sequence[Tuple[str, float]] = (), max_seqlen: int = 0,
+                     split_keys: int = 0, workspace: Optional[torch.Tensor] = None,
+                     out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """s_q = 1 decode; q [B*hq, d] (or [B*hq, 1, d]) bf16, caches [B*hkv, cap, d]."""
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                    ("cache_seqlens", cache_seqlens)):
+        _contig_cuda(t, name)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        nbytes = decode_workspace_size(cache_seqlens.numel(), hq, k_cache.shape[1], q.shape[-1])
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    p = decode_params(q, k_cache, v_cache, cache_seqlens, out, workspace, hq=hq, hkv=hkv,
+                      k_scales=k_scales, v_scales=v_scales, window=window, scale=scale,
+                      epilogue=epilogue, max_seqlen=max_seqlen, split_keys=split_keys)
+    _check(lib.fa_attention_decode(ctypes.byref(p), _stream(stream)), "fa_attention_decode")
+    return out
+
+
+def check_device_error(stream=None) -> int:
+    """Synchronise and return (then clear) the device status: FA_OK or FA_ERR_TIMEOUT."""
+    return int(lib.fa_check_device_error(_stream(stream)))
+
+
+def selftest_watchdog(budget_cycles: int, stream=None) -> int:
+    return int(lib.fa_selftest_watchdog(budget_cycles, _stream(stream)))
+
+
+def kernel_variants_used() -> int:
+    return int(lib.fa_kernel_variants_used())

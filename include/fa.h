@@ -1,0 +1,214 @@
+/*
+ * fa.h -- C ABI of the B200 fused attention library (libfa.so).
+ *
+ * The operations follow fkl_python PR #6 ("fkl.flash_attention: FA-2 forward
+ * with fused epilogue + compressed int8 KV cache"), Summary:
+ *   - flash_attention(q, k, v, causal, epilogue=[ops])  -> fa_attention_fwd
+ *   - compress_kv(k): per-token int8 + one fp32 scale   -> fa_compress_kv
+ *   - the decode step s_q = 1 over the int8 cache        -> fa_attention_decode
+ * and the C style of Foundry attention/README.md, API (fa_* calls over raw
+ * buffers).
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never frees them and keeps none of them after the call returns.
+ *   - Every pointer must be 16-byte aligned and every row contiguous.
+ *   - Work is enqueued asynchronously on the given stream (0 = legacy default
+ *     stream).  Argument checks run on the host before any launch; a call that
+ *     returns an error has enqueued nothing.
+ *   - The library allocates only one small device status word per device, on
+ *     first use, plus cached TMA descriptors.  It never prints and never
+ *     throws across the ABI.
+ *   - Bounded device waits: every spin on an mbarrier or flag in a kernel has
+ *     a cycle budget; on expiry the kernel records FA_ERR_TIMEOUT in the
+ *     status word and returns.  fa_check_device_error() reports it.
+ */
+#ifndef FA_H
+#define FA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *fa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID = 1,     /* bad argument: null pointer, shape, alignment, ... */
+    FA_ERR_UNSUPPORTED = 2, /* well-formed, but no kernel for this combination */
+    FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (launch, descriptor) */
+    FA_ERR_TIMEOUT = 4,     /* a bounded device wait gave up (see fa_check_device_error) */
+    FA_ERR_WORKSPACE = 5    /* decode workspace missing or too small */
+} fa_status;
+
+typedef enum {
+    FA_F32 = 0,  /* IEEE fp32 */
+    FA_BF16 = 1, /* bfloat16 */
+    FA_I8 = 2    /* int8 codes, with one fp32 scale per row (token, kv-head) */
+} fa_dtype;
+
+/* Epilogue ops (fkl_python PR #6, Summary: "epilogue=[ops]: any fkl compute
+ * ops run in-register on the attention output inside the same kernel";
+ * example [Mul(2.0), Add(0.5)]).  They are applied to the normalised fp32
+ * output in list order, each rounded to fp32 (no fused multiply-add), before
+ * the cast to the output dtype.  Values are plain kernel arguments, so
+ * changing them -- or the list's shape -- never compiles anything. */
+typedef enum { FA_EPI_MUL = 1, FA_EPI_ADD = 2 } fa_epi_kind;
+#define FA_MAX_EPILOGUE 8
+typedef struct {
+    int32_t op;  /* fa_epi_kind */
+    float value;
+} fa_epi_op;
+
+/*
+ * fa_compress_kv -- per-row int8 quantisation (fkl_python PR #6, Summary,
+ * "compress_kv(): GPU-side per-token int8 quantization (one fp32
+ * scale/token)").
+ *   x       [rows, d] FA_BF16 or FA_F32, row-major.  A row is one (token,
+ *           kv-head) vector; K and V are compressed by separate calls.
+ *   codes   [rows, d] int8 out;  scales [rows] fp32 out.
+ * For each row: amax = max|x| (in fp32), s = amax / 127 (IEEE fp32 division),
+ * c = clamp(round_half_even(x / s), -127, 127); an all-zero row gets s = 0
+ * and zero codes.  Non-finite inputs give unspecified codes.
+ * Requirements: rows >= 0 (0 enqueues nothing), 1 <= d <= 1024 with d % 16 == 0,
+ * pointers 16-byte aligned.
+ */
+FA_API fa_status fa_compress_kv(const void *x, fa_dtype x_dtype, int64_t rows, int32_t d,
+                         int8_t *codes, float *scales, fa_stream_t stream);
+
+/*
+ * Forward attention parameters (fkl_python PR #6, Summary: layout
+ * (batch*heads, seq, head_dim), fp32 accumulation, head_dim multiple of 32).
+ *
+ * out = softmax(scale * q k^T + mask) v, then the epilogue chain.
+ *
+ * Dense layout (cu_seqlens_q == NULL):
+ *     q, out [batch*hq, seqlen_q, d];  k, v [batch*hkv, seqlen_k, d].
+ * Varlen layout (cu_seqlens_q != NULL; device int32 [batch+1], ascending,
+ * cu[0] = 0; cu_seqlens_k NULL means the same as cu_seqlens_q):
+ *     q, out [hq, total_q, d];  k, v [hkv, total_k, d]; sequence b owns rows
+ *     cu[b] .. cu[b+1]-1 of every head plane.  total_q/total_k are the head
+ *     plane heights and max_seqlen_q/k host-side upper bounds of the
+ *     per-sequence lengths (used to size the grid; they must hold).
+ * GQA: query head h reads KV head h / (hq / hkv); hq % hkv == 0.
+ * Masks (per sequence with s_q queries and s_k keys; query i sits at key
+ * position p = i + s_k - s_q, bottom-right aligned):
+ *     causal != 0 keeps keys j <= p;  window > 0 keeps keys j > p - window;
+ *     window <= 0 means no window.
+ * A row with no visible key gets uniform weights over all s_k keys of its
+ * sequence (the mean of V; zeros when s_k = 0) -- SKaiNET-transformers
+ * PR #419, Summary, "empty sliding-window bands reproduce the engine's
+ * uniform softmax".
+ * dtypes: q_dtype FA_F32 (then kv_dtype FA_F32, CUDA-core fp32 path) or
+ * FA_BF16 (then kv_dtype FA_BF16, or FA_I8 with k_scales/v_scales
+ * [batch*hkv, seqlen_k] dense or [hkv, total_k] varlen, one fp32 scale per
+ * (token, kv-head) as fa_compress_kv writes them).  out has q's dtype.
+ * head_dim: F32 path any multiple of 32 up to 256; BF16/I8 paths 64 or 128.
+ */
+typedef struct {
+    const void *q;
+    const void *k;
+    const void *v;
+    void *out;
+    const float *k_scales; /* FA_I8 only, else NULL */
+    const float *v_scales; /* FA_I8 only, else NULL */
+    int32_t q_dtype;       /* fa_dtype */
+    int32_t kv_dtype;      /* fa_dtype */
+    int32_t batch, hq, hkv, head_dim;
+    int32_t seqlen_q, seqlen_k;          /* dense layout */
+    const int32_t *cu_seqlens_q;         /* varlen layout (device) */
+    const int32_t *cu_seqlens_k;
+    int32_t total_q, total_k;            /* varlen head-plane heights */
+    int32_t max_seqlen_q, max_seqlen_k;  /* varlen host-side bounds */
+    int32_t causal;
+    int32_t window;
+    float softmax_scale;                 /* e.g. 1/sqrt(head_dim) */
+    int32_t n_epilogue;                  /* 0 .. FA_MAX_EPILOGUE */
+    fa_epi_op epilogue[FA_MAX_EPILOGUE];
+} fa_fwd_params;
+
+FA_API fa_status fa_attention_fwd(const fa_fwd_params *p, fa_stream_t stream);
+
+/*
+ * Single-query decode against a KV cache (fkl_python PR #6, Verification,
+ * "FA decode step s_q=1 vs s_k=256 int8"; Summary: the compressed cache is
+ * dequantised in-register and never inflated in global memory).
+ *   q        [batch*hq, d] bf16 (one query per sequence and head)
+ *   k_cache, v_cache [batch*hkv, capacity, d], kv_dtype FA_I8 (with k_scales,
+ *            v_scales [batch*hkv, capacity] fp32) or FA_BF16
+ *   cache_seqlens  device int32 [batch]: sequence b attends to keys
+ *            0 .. L_b-1 (the current token already appended), 0 <= L_b <= capacity
+ *   out      [batch*hq, d] bf16
+ * The query sits at position L_b - 1, so every cached key is visible; a
+ * window W > 0 keeps the last W.  L_b = 0 gives the epilogue applied to zeros.
+ * Work is split along the keys; per-split (m, l, O) partials go to the
+ * caller's workspace (>= fa_decode_workspace_size bytes, 16-byte aligned,
+ * contents need no initialisation) and a merge kernel combines them.
+ * max_seqlen: host-side upper bound of the L_b (0 means capacity);
+ * split_keys: keys per split (a multiple of 256), chosen by the library
+ * when 0.  capacity must be a multiple of 32; cache entries at or past L_b
+ * may hold any bytes (they never reach the result).
+ * Supported: head_dim 128 (FA_I8 and FA_BF16) or 64; hq / hkv <= 8.
+ */
+typedef struct {
+    const void *q;
+    const void *k_cache;
+    const void *v_cache;
+    const float *k_scales;
+    const float *v_scales;
+    const int32_t *cache_seqlens;
+    void *out;
+    int32_t kv_dtype; /* fa_dtype: FA_I8 or FA_BF16 */
+    int32_t batch, hq, hkv, head_dim, capacity;
+    int32_t max_seqlen;
+    int32_t window;
+    float softmax_scale;
+    int32_t split_keys; /* keys per split, multiple of 256; 0 = library choice */
+    int32_t n_epilogue;
+    fa_epi_op epilogue[FA_MAX_EPILOGUE];
+    void *workspace;
+    size_t workspace_bytes;
+} fa_decode_params;
+
+/* Bytes of decode workspace for any split choice at these sizes. */
+FA_API size_t fa_decode_workspace_size(int32_t batch, int32_t hq, int32_t capacity, int32_t head_dim);
+
+FA_API fa_status fa_attention_decode(const fa_decode_params *p, fa_stream_t stream);
+
+/* Static text for a status code (never NULL). */
+FA_API const char *fa_status_string(fa_status s);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status
+ * word: FA_ERR_TIMEOUT if a bounded wait in any kernel gave up since the last
+ * check, FA_ERR_CUDA if the synchronisation itself failed, else FA_OK.
+ */
+FA_API fa_status fa_check_device_error(fa_stream_t stream);
+
+/*
+ * Diagnostic: launches one tiny kernel that waits on an mbarrier no thread
+ * ever arrives on, with a budget of `budget_cycles` SM cycles (clamped to
+ * [1e3, 1e9]).  The wait runs out, the kernel records FA_ERR_TIMEOUT and
+ * returns; fa_check_device_error() must then report FA_ERR_TIMEOUT.  Used to
+ * test the watchdog path without faulting or hanging the device.
+ */
+FA_API fa_status fa_selftest_watchdog(uint64_t budget_cycles, fa_stream_t stream);
+
+/* Number of distinct kernel instantiations launched so far by this process
+ * (the epilogue never adds one: values and list length are runtime data). */
+FA_API int32_t fa_kernel_variants_used(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H */

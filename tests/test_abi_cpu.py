@@ -1,0 +1,168 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry
+point include/fa.h declares, and rejects bad arguments on the host before any
+CUDA call (fa.h: "Argument checks run on the host before any launch")."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "fa.h")).read()
+    return re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)
+
+
+def test_header_declares_the_three_calls():
+    names = header_functions()
+    for n in ("fa_compress_kv", "fa_attention_fwd", "fa_attention_decode"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    from flashattention_attention_b200 import fa
+    for name in header_functions():
+        assert hasattr(fa.lib, name), name
+
+
+@pytest.fixture(scope="module")
+def fa():
+    from flashattention_attention_b200 import fa as mod
+    return mod
+
+
+class FakeTensor:
+    """Carries a (never dereferenced) address through the fa.py marshalling."""
+    def __init__(self, addr, shape, dtype):
+        self._a, self.shape, self.dtype = addr, shape, dtype
+
+    def data_ptr(self):
+        return self._a
+
+    def numel(self):
+        n = 1
+        for s in self.shape:
+            n *= s
+        return n
+
+    def element_size(self):
+        return 1
+
+
+def fwd(fa, **kw):
+    import torch
+    base = dict(hq=4, hkv=2, causal=True)
+    q = FakeTensor(0x10000, (4, 64, 128), torch.bfloat16)
+    k = FakeTensor(0x20000, (2, 64, 128), torch.bfloat16)
+    v = FakeTensor(0x30000, (2, 64, 128), torch.bfloat16)
+    o = FakeTensor(0x40000, (4, 64, 128), torch.bfloat16)
+    tensors = dict(q=q, k=k, v=v, out=o)
+    for name in ("q", "k", "v", "out"):
+        if name in kw:
+            tensors[name] = kw.pop(name)
+    base.update(kw)
+    p = fa.fwd_params(tensors["q"], tensors["k"], tensors["v"], tensors["out"], **base)
+    return p
+
+
+def call_fwd(fa, p):
+    return fa.lib.fa_attention_fwd(ctypes.byref(p), None)
+
+
+def test_fwd_rejects_bad_arguments(fa):
+    import torch
+    assert fa.lib.fa_attention_fwd(None, None) == fa.FA_ERR_INVALID
+    p = fwd(fa)
+    p.hq = 3  # hq % hkv != 0
+    assert call_fwd(fa, p) == fa.FA_ERR_INVALID
+    p = fwd(fa)
+    p.head_dim = 48  # not a multiple of 32
+    assert call_fwd(fa, p) == fa.FA_ERR_INVALID
+    p = fwd(fa)
+    p.head_dim = 96  # multiple of 32 but no bf16 tensor-core kernel
+    assert call_fwd(fa, p) == fa.FA_ERR_UNSUPPORTED
+    p = fwd(fa)
+    p.n_epilogue = 9
+    assert call_fwd(fa, p) == fa.FA_ERR_INVALID
+    p = fwd(fa)
+    p.n_epilogue = 1
+    p.epilogue[0].op = 7  # unknown op
+    assert call_fwd(fa, p) == fa.FA_ERR_INVALID
+    p = fwd(fa)
+    p.q = 0x10008  # misaligned
+    assert call_fwd(fa, p) == fa.FA_ERR_INVALID
+    p = fwd(fa)
+    p.out = None
+    assert call_fwd(fa, p) == fa.FA_ERR_INVALID
+    p = fwd(fa, k=FakeTensor(0x20000, (2, 64, 128), torch.int8),
+            v=FakeTensor(0x30000, (2, 64, 128), torch.int8))
+    assert call_fwd(fa, p) == fa.FA_ERR_INVALID  # int8 without scales
+    p = fwd(fa, q=FakeTensor(0x10000, (4, 64, 128), torch.float32))
+    assert call_fwd(fa, p) == fa.FA_ERR_INVALID  # fp32 q with bf16 kv
+    p = fwd(fa)
+    p.softmax_scale = float("nan")
+    assert call_fwd(fa, p) == fa.FA_ERR_INVALID
+
+
+def test_fwd_empty_problem_is_a_noop(fa):
+    p = fwd(fa)
+    p.seqlen_q = 0
+    p.q = p.k = p.v = p.out = None
+    assert call_fwd(fa, p) == fa.FA_OK
+
+
+def test_compress_rejects_bad_arguments(fa):
+    lib = fa.lib
+    assert lib.fa_compress_kv(0x1000, fa.FA_BF16, 4, 15, 0x2000, 0x3000, None) == fa.FA_ERR_INVALID
+    assert lib.fa_compress_kv(0x1000, fa.FA_I8, 4, 64, 0x2000, 0x3000, None) == fa.FA_ERR_INVALID
+    assert lib.fa_compress_kv(0x1008, fa.FA_BF16, 4, 64, 0x2000, 0x3000, None) == fa.FA_ERR_INVALID
+    assert lib.fa_compress_kv(None, fa.FA_BF16, 4, 64, 0x2000, 0x3000, None) == fa.FA_ERR_INVALID
+    assert lib.fa_compress_kv(None, fa.FA_BF16, 0, 64, None, None, None) == fa.FA_OK
+    assert lib.fa_compress_kv(0x1000, fa.FA_BF16, -1, 64, 0x2000, 0x3000, None) == fa.FA_ERR_INVALID
+
+
+def decode_p(fa, **over):
+    import torch
+    q = FakeTensor(0x10000, (16, 128), torch.bfloat16)
+    kc = FakeTensor(0x20000, (4, 1024, 128), torch.int8)
+    vc = FakeTensor(0x30000, (4, 1024, 128), torch.int8)
+    sl = FakeTensor(0x40000, (2,), torch.int32)
+    o = FakeTensor(0x50000, (16, 128), torch.bfloat16)
+    need = fa.decode_workspace_size(2, 16, 1024, 128)
+    ws = FakeTensor(0x100000, (need,), torch.uint8)
+    p = fa.decode_params(q, kc, vc, sl, o, ws, hq=8, hkv=2, k_scales=FakeTensor(0x60000, (4, 1024), None),
+                         v_scales=FakeTensor(0x70000, (4, 1024), None))
+    for k, v in over.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_decode_rejects_bad_arguments(fa):
+    lib = fa.lib
+    call = lambda p: lib.fa_attention_decode(ctypes.byref(p), None)
+    assert lib.fa_attention_decode(None, None) == fa.FA_ERR_INVALID
+    assert call(decode_p(fa, hq=9)) == fa.FA_ERR_INVALID
+    assert call(decode_p(fa, capacity=1000)) == fa.FA_ERR_INVALID       # not a multiple of 32
+    assert call(decode_p(fa, max_seqlen=2048)) == fa.FA_ERR_INVALID     # above capacity
+    assert call(decode_p(fa, split_keys=100)) == fa.FA_ERR_INVALID
+    assert call(decode_p(fa, head_dim=96)) == fa.FA_ERR_UNSUPPORTED
+    assert call(decode_p(fa, hq=32, hkv=2)) == fa.FA_ERR_UNSUPPORTED    # group of 16
+    assert call(decode_p(fa, k_scales=None)) == fa.FA_ERR_INVALID
+    assert call(decode_p(fa, workspace_bytes=16)) == fa.FA_ERR_WORKSPACE
+    assert call(decode_p(fa, workspace=None)) == fa.FA_ERR_WORKSPACE
+    assert call(decode_p(fa, q=0x10004)) == fa.FA_ERR_INVALID
+
+
+def test_workspace_size_formula(fa):
+    # one (d + 2)-float record per (sequence, q-head, 256-key split)
+    assert fa.decode_workspace_size(16, 32, 32768, 128) == 16 * 32 * 128 * (128 + 2) * 4
+    assert fa.decode_workspace_size(1, 1, 1, 64) == 1 * 1 * 1 * 66 * 4
+    assert fa.decode_workspace_size(0, 1, 1, 64) == 0
+
+
+def test_status_strings(fa):
+    for s in range(6):
+        assert fa.lib.fa_status_string(s)
+    assert fa.lib.fa_status_string(99) == b"unknown status"
