@@ -1,10 +1,410 @@
-// prefill_tc.cu -- tensor-core (tcgen05) prefill; under construction.
+// prefill_tc.cu -- fused attention forward on the 5th-generation tensor cores
+// (tcgen05 + TMEM + TMA), bf16 Q/K/V, fp32 accumulation.
+//
+// What it computes: fkl_python PR #6, Summary -- FlashAttention-2 style
+// forward softmax(q k^T * scale + mask) v with fused epilogue ops, layout
+// (batch*heads, seq, head_dim) or varlen; online softmax rescaling (Foundry
+// attention/README.md, References: the FlashAttention paper and the online
+// softmax trick), so the score matrix never leaves the SM.
+//
+// CTA work tile: two 128-row Q tiles = the same 128 query rows of two query
+// heads of one GQA group (SKaiNET-transformers PR #419, Summary: one task per
+// GQA group).  Both tiles see the same mask, so they walk the same key range
+// and every K/V tile brought in by TMA serves both heads.  (An odd group
+// size runs one Q tile per CTA.)  Key tiles outside the causal / window band
+// are never loaded; only boundary tiles get an element mask.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax of Q tile 0 (one thread per row = one TMEM lane)
+//   warps 4-7  softmax of Q tile 1
+//   warp 8     TMA producer: Q once, then a K ring and a V ring
+//   warp 9     MMA issuer (one thread) and TMEM owner
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 after it.
+// P (bf16, two per 32-bit column) overwrites the first 64 columns of its S
+// tile and is the A operand of O += P V straight from TMEM.
+//
+// MMA issue order per key tile j (ping-pong between the two Q tiles):
+//   PV0(j-1), S0(j), PV1(j-1), S1(j)
+// so the tensor core works on one tile while the other tile's softmax runs.
+// Softmax of tile t at step j: wait S_t(j) (its commit also covers PV_t(j-1)),
+// read the row, raise the running max only when it grows by more than 8 (in
+// log2 units; the final O / l uses the same stale max, so the result is
+// exact), rescale O_t in TMEM when it did, write P_t, signal the MMA warp.
+// Every wait is bounded (device.cuh); a timeout aborts all roles cleanly.
 #include "internal.h"
+#include "layout.cuh"
+#include "umma.cuh"
 
 namespace fa {
+namespace {
+
+constexpr int kBM = 128;  // query rows per Q tile
+constexpr int kBN = 128;  // keys per K/V tile
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr uint32_t kChunkBytes = kSwizzleChunkRows * 128;  // [128 rows x 64 bf16]
+
+template <int D>
+struct TcGeom {
+  static constexpr int kStages = (D == 128) ? 2 : 3;
+  static constexpr uint32_t kQBytes = kBM * D * 2;
+  static constexpr uint32_t kKVBytes = kBN * D * 2;
+  static constexpr uint32_t kKOff = 2 * kQBytes;
+  static constexpr uint32_t kVOff = kKOff + kStages * kKVBytes;
+  static constexpr uint32_t kBarOff = kVOff + kStages * kKVBytes;
+  static constexpr uint32_t kSmem = kBarOff + 256 + 1024;
+};
+
+struct PrefillArgs {
+  SeqLayout L;
+  __nv_bfloat16* out;
+  int batch, hq, hkv, group, n_qblocks, two_tiles;
+  float scale_log2;
+  Epilogue epi;
+  Watchdog wd;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const PrefillArgs A) {
+  using G = TcGeom<D>;
+  constexpr int S = G::kStages;
+  extern __shared__ uint8_t tc_smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G::kBarOff);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + S;
+  uint64_t* v_full = k_empty + S;
+  uint64_t* v_empty = v_full + S;
+  uint64_t* s_full = v_empty + S;  // [2]
+  uint64_t* p_full = s_full + 2;   // [2]
+  uint64_t* o_done = p_full + 2;   // [2]
+  uint64_t* drain = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  __shared__ int abort_flag;
+
+  // ---- work tile: longest (highest q-block) first, then sequence, then head pair
+  const int n_pairs = A.two_tiles ? A.hq / 2 : A.hq;
+  const int per_qb = A.batch * n_pairs;
+  const int qb = A.n_qblocks - 1 - static_cast<int>(blockIdx.x) / per_qb;
+  const int rem = static_cast<int>(blockIdx.x) % per_qb;
+  const int b = rem / n_pairs, pair = rem % n_pairs;
+  const int h0 = A.two_tiles ? 2 * pair : pair;
+  const int ntile = A.two_tiles ? 2 : 1;
+  const int g = h0 / A.group;
+  const Seq sq = seq_of(A.L, b, h0, g);
+  const int i0 = qb * kBM;
+  if (i0 >= sq.s_q) return;
+  const int i_last = min(i0 + kBM, sq.s_q) - 1;
+  int lo_first, hi_first, lo_last, hi_last;
+  band_of(A.L, i0, sq.s_q, sq.s_k, lo_first, hi_first);
+  band_of(A.L, i_last, sq.s_q, sq.s_k, lo_last, hi_last);
+  const int k_lo = max(0, lo_first);
+  const int k_hi = min(sq.s_k, hi_last);
+  const int j_lo = k_lo / kBN;
+  const int n_iter = k_hi > k_lo ? (k_hi + kBN - 1) / kBN - j_lo : 0;
+  if (n_iter == 0) return;  // no row of this tile sees a key: the empty-band kernel writes them
+
+  // TMA coordinates: dense planes are (b*h + h), varlen planes are h with the
+  // sequence starting at cu[b] inside the plane.
+  const bool varlen = A.L.cu_q != nullptr;
+  const int q_plane = varlen ? h0 : b * A.hq + h0;
+  const int q_prow = (varlen ? A.L.cu_q[b] : 0) + i0;
+  const int k_plane = varlen ? g : b * A.hkv + g;
+  const int k_prow0 = varlen ? A.L.cu_k[b] : 0;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(q_full, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(s_full + t, 1);
+      mbar_init(p_full + t, kBM);
+      mbar_init(o_done + t, 1);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      mbar_expect_tx(q_full, ntile * G::kQBytes);
+      for (int t = 0; t < ntile; ++t)
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + t * G::kQBytes + c * kChunkBytes, &tm_q, q_full, 64 * c, q_prow, q_plane + t);
+      for (int it = 0; it < n_iter; ++it) {
+        const int s = it % S, u = it / S;
+        const int krow = k_prow0 + (j_lo + it) * kBN;
+        if (u > 0 && !wait_parity(k_empty + s, (u - 1) & 1, A.wd, &abort_flag)) break;
+        mbar_expect_tx(k_full + s, G::kKVBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + G::kKOff + s * G::kKVBytes + c * kChunkBytes, &tm_k, k_full + s, 64 * c, krow,
+                      k_plane);
+        if (u > 0 && !wait_parity(v_empty + s, (u - 1) & 1, A.wd, &abort_flag)) break;
+        mbar_expect_tx(v_full + s, G::kKVBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + G::kVOff + s * G::kKVBytes + c * kChunkBytes, &tm_v, v_full + s, 64 * c, krow,
+                      k_plane);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = umma_idesc_f16(kBM, kBN, 1, 1, false);
+      constexpr uint32_t idesc_o = umma_idesc_f16(kBM, D, 1, 1, true);
+      const uint32_t q_base = smem_u32(smem);
+      auto issue_s = [&](int t, int s) {
+        const uint32_t qa = q_base + t * G::kQBytes;
+        const uint32_t kb = q_base + G::kKOff + s * G::kKVBytes;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k / 4) * kChunkBytes + (k % 4) * 32;
+          mma_ss(tmem + t * kBN, umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
+                 idesc_s, k > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int s, bool accumulate) {
+        const uint32_t vb = q_base + G::kVOff + s * G::kKVBytes;
+#pragma unroll
+        for (int k = 0; k < kBN / 16; ++k) {
+          mma_ts(tmem + 256 + t * D, tmem + t * kBN + k * 8, umma_desc_sw128(vb + k * 2048, kChunkBytes, 1024),
+                 idesc_o, (accumulate || k > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = wait_parity(q_full, 0, A.wd, &abort_flag);
+      for (int it = 0; ok && it < n_iter; ++it) {
+        const int s = it % S;
+        if (!(ok = wait_parity(k_full + s, (it / S) & 1, A.wd, &abort_flag))) break;
+        tc_fence_after();
+        for (int t = 0; t < ntile; ++t) {
+          if (it > 0) {
+            const int vs = (it - 1) % S;
+            if (!(ok = wait_parity(p_full + t, (it - 1) & 1, A.wd, &abort_flag))) break;
+            if (t == 0 && !(ok = wait_parity(v_full + vs, ((it - 1) / S) & 1, A.wd, &abort_flag))) break;
+            tc_fence_after();
+            issue_pv(t, vs, it - 1 > 0);
+            if (t == ntile - 1) mma_commit(v_empty + vs);
+          }
+          issue_s(t, s);
+          mma_commit(s_full + t);
+        }
+        if (ok) mma_commit(k_empty + s);
+      }
+      if (ok) {
+        const int vs = (n_iter - 1) % S;
+        for (int t = 0; t < ntile; ++t) {
+          if (!(ok = wait_parity(p_full + t, (n_iter - 1) & 1, A.wd, &abort_flag))) break;
+          if (t == 0 && !(ok = wait_parity(v_full + vs, ((n_iter - 1) / S) & 1, A.wd, &abort_flag))) break;
+          tc_fence_after();
+          issue_pv(t, vs, n_iter - 1 > 0);
+          mma_commit(o_done + t);
+        }
+      }
+      // every MMA this thread issued has completed before TMEM is released
+      mma_commit(drain);
+      wait_parity(drain, 0, A.wd);
+    }
+  } else if (warp / 4 < ntile) {
+    // ------------------------------------------------------------ softmax
+    const int t = warp / 4, quarter = warp % 4;
+    const int r = quarter * 32 + lane;
+    const int i = i0 + r;
+    int lo, hi;
+    band_of(A.L, i, sq.s_q, sq.s_k, lo, hi);
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_tm = tmem + lane_base + t * kBN;
+    const uint32_t o_tm = tmem + lane_base + 256 + t * D;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int it = 0; it < n_iter; ++it) {
+      ok = __all_sync(0xffffffffu, wait_parity(s_full + t, it & 1, A.wd, &abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t raw[4][32];
+      tmem_ld32(s_tm + 0, raw[0]);
+      tmem_ld32(s_tm + 32, raw[1]);
+      tmem_ld32(s_tm + 64, raw[2]);
+      tmem_ld32(s_tm + 96, raw[3]);
+      tmem_wait_ld();
+      const int kb = (j_lo + it) * kBN;
+      const bool whole = kb >= lo && kb + kBN <= hi;
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float x = __uint_as_float(raw[cc][e]) * A.scale_log2;
+          if (!whole) {
+            const int kj = kb + cc * 32 + e;
+            x = (kj >= lo && kj < hi) ? x : -INFINITY;
+          }
+          raw[cc][e] = __float_as_uint(x);
+          mx[cc] = fmaxf(mx[cc], x);
+        }
+      }
+      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float m_new = fmaxf(m_used, m_tile);
+      const bool need = m_new > m_used + kRescaleThreshold;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2_approx(m_used - m_new);
+        m_used = m_new;
+      }
+      const float mref = m_used == -INFINITY ? 0.f : m_used;
+      l *= alpha;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2_approx(__uint_as_float(raw[cc][2 * e]) - mref);
+          const float p1 = ex2_approx(__uint_as_float(raw[cc][2 * e + 1]) - mref);
+          ls[cc] += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(s_tm + cc * 16, pk);
+      }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      if (it > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int oc = 0; oc < D / 32; ++oc) {
+          uint32_t o[32];
+          tmem_ld32(o_tm + oc * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(o_tm + oc * 32, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full + t);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, wait_parity(o_done + t, 0, A.wd, &abort_flag));
+    if (ok) {
+      tc_fence_after();
+      const bool store = i < sq.s_q && lo < hi;
+      const float inv_l = 1.f / l;
+      __nv_bfloat16* orow = A.out + (sq.q_row0 + static_cast<int64_t>(t) * A.L.q_hstride + i) * D;
+#pragma unroll
+      for (int oc = 0; oc < D / 32; ++oc) {
+        uint32_t o[32];
+        tmem_ld32(o_tm + oc * 32, o);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float y0 = apply_epilogue(__uint_as_float(o[2 * e]) * inv_l, A.epi);
+          const float y1 = apply_epilogue(__uint_as_float(o[2 * e + 1]) * inv_l, A.epi);
+          pk[e] = pack_bf16x2(y0, y1);
+        }
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + oc * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+fa_status launch_bf16(const fa_fwd_params& p, const LaunchCtx& ctx) {
+  using G = TcGeom<D>;
+  const bool varlen = p.cu_seqlens_q != nullptr;
+  const uint64_t q_rows = varlen ? p.total_q : p.seqlen_q;
+  const uint64_t k_rows = varlen ? p.total_k : p.seqlen_k;
+  const uint64_t q_planes = varlen ? p.hq : static_cast<uint64_t>(p.batch) * p.hq;
+  const uint64_t k_planes = varlen ? p.hkv : static_cast<uint64_t>(p.batch) * p.hkv;
+  if (k_rows == 0) return FA_OK;  // no keys anywhere: only the empty-band kernel writes
+  CUtensorMap tq, tk, tv;
+  const uint32_t box[3] = {64, static_cast<uint32_t>(kSwizzleChunkRows), 1};
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(D), q_rows, q_planes};
+    const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, q_rows * D * 2};
+    fa_status st = encode_tensor_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.q, dims, strides, box,
+                                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != FA_OK) return st;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(D), k_rows, k_planes};
+    const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, k_rows * D * 2};
+    fa_status st = encode_tensor_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.k, dims, strides, box,
+                                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != FA_OK) return st;
+    st = encode_tensor_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.v, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != FA_OK) return st;
+  }
+  PrefillArgs A;
+  A.L = SeqLayout::from(p);
+  A.out = static_cast<__nv_bfloat16*>(p.out);
+  A.batch = p.batch;
+  A.hq = p.hq;
+  A.hkv = p.hkv;
+  A.group = p.hq / p.hkv;
+  A.two_tiles = (A.group % 2 == 0) ? 1 : 0;
+  const int max_sq = varlen ? p.max_seqlen_q : p.seqlen_q;
+  A.n_qblocks = (max_sq + kBM - 1) / kBM;
+  A.scale_log2 = p.softmax_scale * kLog2e;
+  A.epi = make_epilogue(p.epilogue, p.n_epilogue);
+  A.wd = ctx.wd;
+  const long long n_pairs = A.two_tiles ? p.hq / 2 : p.hq;
+  const long long grid = static_cast<long long>(A.n_qblocks) * p.batch * n_pairs;
+  if (grid == 0) return FA_OK;
+  if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  auto kern = prefill_bf16_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem) != cudaSuccess)
+    return FA_ERR_CUDA;
+  note_variant(reinterpret_cast<const void*>(kern));
+  kern<<<static_cast<unsigned>(grid), kThreads, G::kSmem, ctx.stream>>>(tq, tk, tv, A);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
 fa_status launch_prefill_tc(const fa_fwd_params& p, const LaunchCtx& ctx) {
-  (void)p;
-  (void)ctx;
+  if (p.kv_dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (p.head_dim == 128) return launch_bf16<128>(p, ctx);
+  if (p.head_dim == 64) return launch_bf16<64>(p, ctx);
   return FA_ERR_UNSUPPORTED;
 }
+
 }  // namespace fa
