@@ -1,0 +1,376 @@
+"""Benchmark of the fused attention hot path on B200.
+
+One step = one causal GQA prefill forward through the C ABI on the workload
+the headline metric is quoted on: B=4, Hq=32, Hkv=8, S_q=S_k=4096, d=128,
+bf16 in/out, fp32 accumulation, scale 1/sqrt(128), seeded N(0,1) inputs.
+FLOPs per step count the 128x128 tiles of a fixed grid that intersect the
+causal band: 4*d*128*128 per tile (0.5669 TFLOP).  The same run also times
+the int8-KV decode (B=16, Hq=32, Hkv=8, d=128, cache lengths U[1024,32768]
+from seed 0; bytes = codes + scales + Q + O) and the KV quantiser on that
+cache's 4,361,088 rows, each against its roofline.
+
+Inputs of every timed launch are larger than L2 (126 MB): prefill reads
+201 MB of Q/K/V, decode 576 MB of cache, the quantiser 1.1 GB; no flush.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun (N > 1) every rank runs its own replica of the workload (the
+path shards by independent (sequence, head) units: no collective), and the
+step time is the max over ranks.  ``--impl reference`` times the fp64 CPU
+oracle on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "prefill attention TFLOP/s and int8-KV decode GB/s, as % of B200 roofline"
+TILE = 128
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def band_tiles(s_q, s_k, causal, window):
+    """128x128 tiles of a fixed grid that intersect the visible band of one
+    (sequence, head), and the exact number of visible (query, key) pairs."""
+    tiles = 0
+    pairs = 0
+    for qb in range((s_q + TILE - 1) // TILE):
+        i0, i1 = qb * TILE, min(s_q, qb * TILE + TILE) - 1
+        lo = max(0, i0 + s_k - s_q - window + 1) if window > 0 else 0
+        hi = min(s_k, i1 + s_k - s_q + 1) if causal else s_k
+        if hi > lo:
+            tiles += (hi + TILE - 1) // TILE - lo // TILE
+    for i in range(s_q):
+        p = i + s_k - s_q
+        lo = max(0, p - window + 1) if window > 0 else 0
+        hi = min(s_k, p + 1) if causal else s_k
+        pairs += max(0, hi - lo)
+    return tiles, pairs
+
+
+def prefill_flops(w):
+    tiles, pairs = band_tiles(w.seqlen_q, w.seqlen_k, w.causal, w.window)
+    per = w.batch * w.hq * 4 * w.d
+    return per * tiles * TILE * TILE, per * pairs
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"fa_bench_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                    rows.append(f)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        busy = [r for r in rows if pw and float(r[3]) > 0.5 * max(pw)] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in busy for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(float(r[1]) for r in busy),
+                "sm_max_mhz": max(float(r[2]) for r in rows), "reasons": reasons,
+                "samples": len(busy), "power_w_max": max(pw) if pw else None}
+
+
+# ---------------------------------------------------------------------------- GPU arm
+def time_launches(fn, steps, warmup, torch, dist=None):
+    """Warm up, then time exactly `steps` calls between barriers and
+    synchronisations with CUDA events on the current stream; max over ranks."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms / steps
+
+
+def gpu_arm(args, rank, world, dist):
+    import torch
+    from flashattention_attention_b200 import fa, inputs
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    w = inputs.gqa_causal_prefill()
+    flops_tiles, flops_exact = prefill_flops(w)
+    q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
+    out = torch.empty_like(q)
+
+    def prefill():
+        fa.attention_fwd(q, k, v, hq=w.hq, hkv=w.hkv, causal=True, out=out)
+
+    if args.only in ("decode", "quant"):
+        return decode_and_quant(args, dev, peaks, world, dist, {})
+    l0 = fa.kernel_launches()
+    with ClockSampler(dev.index or 0) as clocks:
+        ms = time_launches(prefill, args.steps, args.warmup, torch, dist)
+    launches = fa.kernel_launches() - l0 - args.warmup * 1
+    clk = clocks.summary()
+    assert fa.check_device_error() == fa.FA_OK
+    tflops = flops_tiles / (ms * 1e-3) / 1e12
+
+    # e2e: the same call with host buffers: pinned H2D of q/k/v, the kernel,
+    # D2H of the output, every step
+    hq_, hk_, hv_ = w.q.pin_memory(), w.k.pin_memory(), w.v.pin_memory()
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(hq_, non_blocking=True)
+        k.copy_(hk_, non_blocking=True)
+        v.copy_(hv_, non_blocking=True)
+        prefill()
+        ho.copy_(out, non_blocking=True)
+
+    e2e_steps = max(3, args.steps // 10)
+    e2e_ms = time_launches(e2e_step, e2e_steps, 2, torch, dist)
+    h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_))
+    d2h = ho.numel() * ho.element_size()
+    del q, k, v, out, hq_, hk_, hv_, ho
+    torch.cuda.empty_cache()
+
+    result = {
+        "metric": METRIC, "value": round(tflops * world, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1), numpy PCG64 -> fp32 -> bf16)",
+        "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "seq_len": w.seqlen_q,
+                   "head_dim": w.d, "causal": True, "window": 0, "epilogue": [],
+                   "flops_per_step": flops_tiles, "flops_counting": "128x128 tiles intersecting the band",
+                   "flops_exact_pairs": flops_exact, "l2": "inputs larger than L2 (201 MB), no flush",
+                   "parallelism": f"replicas x{world} (no collective)"},
+        "roofline": {"bound": "tensor", "kernel": "prefill_bf16_kernel<128>", "achieved": round(tflops, 2),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(tflops / peaks["bf16_tflops"], 4),
+                     "peak_source": f"{peaks['source']} bf16 burst", "traffic": None,
+                     "frac_of_nominal_2250": round(tflops / 2250.0, 4)},
+        "e2e": {"value": round(flops_tiles / (e2e_ms * 1e-3) / 1e12 * world, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if args.only == "all":
+        decode_and_quant(args, dev, peaks, world, dist, result)
+    if rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, flops_tiles, flops_exact, args.cpu_seconds)
+    return result
+
+
+def decode_and_quant(args, dev, peaks, world, dist, result):
+    """int8-KV decode and the quantiser on the decode workload."""
+    import torch
+    from flashattention_attention_b200 import fa, inputs
+    dw = inputs.int8kv_decode()
+    if args.only in ("all", "quant"):
+        # the quantiser over every valid (token, kv-head) row of K and V, packed
+        rows = torch.cat([t[b * dw.hkv:(b + 1) * dw.hkv, :dw.lengths[b]].reshape(-1, dw.d)
+                          for t in (dw.k, dw.v) for b in range(dw.batch)]).to(dev)
+        codes = torch.empty(rows.shape, dtype=torch.int8, device=dev)
+        scales = torch.empty(rows.shape[0], dtype=torch.float32, device=dev)
+        quant_ms = time_launches(lambda: fa.compress_kv(rows, codes, scales), max(10, args.steps // 4),
+                                 args.warmup, torch, dist)
+        quant_rows = int(rows.shape[0])
+        quant_bytes = quant_rows * (2 * dw.d + dw.d + 4)
+        quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+        result["quantiser"] = {"rows": quant_rows, "value": round(quant_gbs * world, 1), "unit": "GB/s",
+                               "us_per_step": round(quant_ms * 1e3, 2), "bytes_per_step": quant_bytes,
+                               "roofline": {"bound": "hbm", "kernel": "compress_kernel",
+                                            "achieved": round(quant_gbs, 1), "peak": peaks["hbm_gbs"],
+                                            "unit": "GB/s", "frac": round(quant_gbs / peaks["hbm_gbs"], 4),
+                                            "traffic": None}}
+        del rows, codes, scales
+    if args.only in ("all", "decode"):
+        kc, ks = fa.compress_kv(dw.k.to(dev))
+        vc, vs = fa.compress_kv(dw.v.to(dev))
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()  # the bf16 copies are gone: only the int8 cache stays resident
+        lens = torch.tensor(dw.lengths, dtype=torch.int32, device=dev)
+        dq = dw.q.reshape(-1, dw.d).to(dev)
+        dout = torch.empty_like(dq)
+        ws = torch.empty(fa.decode_workspace_size(dw.batch, dw.hq, dw.cache_capacity, dw.d),
+                         dtype=torch.uint8, device=dev)
+        maxlen = max(dw.lengths)
+
+        def decode():
+            fa.attention_decode(dq, kc, vc, lens, hq=dw.hq, hkv=dw.hkv, k_scales=ks, v_scales=vs,
+                                max_seqlen=maxlen, workspace=ws, out=dout)
+
+        dec_ms = time_launches(decode, max(20, args.steps), args.warmup, torch, dist)
+        dec_bytes = sum(dw.lengths) * dw.hkv * 2 * (dw.d + 4) + 2 * dq.numel() * 2
+        dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
+        result["decode"] = {"workload": dw.name, "value": round(dec_gbs * world, 1), "unit": "GB/s",
+                            "us_per_step": round(dec_ms * 1e3, 2), "bytes_per_step": dec_bytes,
+                            "roofline": {"bound": "hbm", "kernel": "decode_i8_kernel<128> + merge",
+                                         "achieved": round(dec_gbs, 1), "peak": peaks["hbm_gbs"],
+                                         "unit": "GB/s", "frac": round(dec_gbs / peaks["hbm_gbs"], 4),
+                                         "frac_of_nominal_8000": round(dec_gbs / 8000.0, 4), "traffic": None}}
+    assert fa.check_device_error() == fa.FA_OK
+    return result
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def _oracle_sample(w, n_rows, seed):
+    """Time the fp64 oracle, as it stands, on n_rows random causal rows of
+    one head plane of the prefill workload (its cost is per row).  Returns
+    (seconds, visible pairs)."""
+    import numpy as np
+
+    import oracle
+    rng = np.random.default_rng(seed)
+    qf = w.q[0:1].double().numpy()
+    kf = w.k[0:1].double().numpy()
+    vf = w.v[0:1].double().numpy()
+    rows = [(0, 0, int(i)) for i in rng.integers(0, w.seqlen_q, n_rows)]
+    t0 = time.perf_counter()
+    oracle.attention(qf, kf, vf, hq=1, hkv=1, causal=True, rows=rows)
+    dt = time.perf_counter() - t0
+    return dt, sum(i + 1 for _, _, i in rows)
+
+
+def _cores():
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return int(os.environ.get("OMP_NUM_THREADS", cores))
+
+
+def cpu_baseline(w, flops_tiles, flops_exact, budget_s):
+    """The oracle on the host cores over a bounded sample (about budget_s
+    seconds of CPU work), scaled to the whole step by the exact pair count."""
+    dt, pairs = _oracle_sample(w, 64, 1)
+    n = int(min(w.seqlen_q * 4, max(64, 64 * budget_s / max(dt, 1e-3))))
+    dt, pairs = _oracle_sample(w, n, 2)
+    full_s = dt * flops_exact / (4 * w.d * pairs)
+    return {"value": flops_tiles / full_s / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"{n} random causal rows of one head plane ({pairs} visible pairs, {dt:.2f} s of fp64 "
+                      f"CPU work), scaled to the whole step by its exact pair count",
+            "seconds_sampled": round(dt, 3)}
+
+
+def reference_arm(args, world):
+    """The oracle timed on host cores on this arm's workload, metric and unit;
+    each step is a bounded sample of 256 rows scaled by the exact pair count."""
+    from flashattention_attention_b200 import inputs
+    w = inputs.gqa_causal_prefill()
+    flops_tiles, flops_exact = prefill_flops(w)
+    vals = []
+    for s in range(args.warmup + args.steps):
+        dt, pairs = _oracle_sample(w, 256, 100 + s)
+        if s >= args.warmup:
+            vals.append(flops_tiles / (dt * flops_exact / (4 * w.d * pairs)) / 1e12)
+    value = statistics.median(vals)
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": flops_tiles / (value * 1e12) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1), numpy PCG64 -> fp32 -> bf16)",
+            "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "seq_len": w.seqlen_q,
+                       "head_dim": w.d, "causal": True, "flops_per_step": flops_tiles},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+                             "sample": "each step: 256 random causal rows of one head plane, fp64, scaled to "
+                                       "the whole step by its exact pair count"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "quant"],
+                    help="time one part only (used for profiler captures)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        # rank 0 alone times the CPU oracle; other ranks exit without work
+        if rank == 0:
+            print(json.dumps(reference_arm(args, world)), flush=True)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        res = gpu_arm(args, rank, world, dist)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

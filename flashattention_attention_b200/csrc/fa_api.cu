@@ -5,6 +5,7 @@
 
 #include <cmath>
 #include <cstdlib>
+#include <atomic>
 #include <mutex>
 #include <set>
 
@@ -18,6 +19,7 @@ constexpr int kMaxDevices = 64;
 unsigned int* g_status[kMaxDevices] = {};
 long long g_budget = 0;
 std::set<const void*>* g_variants = nullptr;
+std::atomic<long long> g_launches{0};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 long long watchdog_budget() {
@@ -90,6 +92,7 @@ Epilogue make_epilogue(const fa_epi_op* ops, int n) {
 }
 
 void note_variant(const void* kernel_fn) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_variants == nullptr) g_variants = new std::set<const void*>();
   g_variants->insert(kernel_fn);
@@ -271,6 +274,8 @@ fa_status fa_selftest_watchdog(uint64_t budget_cycles, fa_stream_t stream) {
   if (b > 1000000000ULL) b = 1000000000ULL;
   return launch_watchdog_selftest(b, ctx);
 }
+
+int64_t fa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int32_t fa_kernel_variants_used(void) {
   std::lock_guard<std::mutex> lk(g_mu);

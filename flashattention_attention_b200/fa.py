@@ -74,6 +74,8 @@ lib.fa_selftest_watchdog.restype = ctypes.c_int
 lib.fa_selftest_watchdog.argtypes = [ctypes.c_uint64, ctypes.c_void_p]
 lib.fa_kernel_variants_used.restype = ctypes.c_int32
 lib.fa_kernel_variants_used.argtypes = []
+lib.fa_kernel_launches.restype = ctypes.c_int64
+lib.fa_kernel_launches.argtypes = []
 
 
 class FAError(RuntimeError):
@@ -230,3 +232,7 @@ def selftest_watchdog(budget_cycles: int, stream=None) -> int:
 
 def kernel_variants_used() -> int:
     return int(lib.fa_kernel_variants_used())
+
+
+def kernel_launches() -> int:
+    return int(lib.fa_kernel_launches())

@@ -207,6 +207,10 @@ FA_API fa_status fa_selftest_watchdog(uint64_t budget_cycles, fa_stream_t stream
  * (the epilogue never adds one: values and list length are runtime data). */
 FA_API int32_t fa_kernel_variants_used(void);
 
+/* Total kernel launches made by this library in this process (all devices);
+ * a diagnostic for counting launches inside a timed region. */
+FA_API int64_t fa_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif
