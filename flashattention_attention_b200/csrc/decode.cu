@@ -460,3 +460,131 @@ fa_status launch_decode(const fa_decode_params& p, int split_keys, int n_splits,
 }
 
 }  // namespace fa
+
+// ----------------------------------------------------------------------------
+// Decode without caller workspace.
+//
+// For callers that cannot allocate device memory at call time -- for example
+// a plug-in inside a serving runtime that owns every device byte through its
+// own pre-planned arena and forbids allocations outside it, or a caller that
+// must not risk the implicit device synchronisation a cudaMalloc can cause --
+// the per-split partials (O, m, l) live in this file-scope device array
+// instead of a caller workspace.  Every device that loads the library holds
+// it until the process exits.  All calls on a device share it and it keeps
+// the last call's contents; nothing in it needs clearing, because the merge
+// only reads records that the same call's split kernel wrote.  Calls whose
+// work overlaps on the GPU (different streams, or different host threads on
+// the same device) race on the array and must be serialised by the caller.
+#include <mutex>
+
+namespace fa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[kNoAllocScratchBytes];
+// Watchdog word of this path (the library's shared status word is allocated
+// lazily, which this path must not do).
+static __device__ unsigned int g_decode_noalloc_status;
+
+// Device addresses of the scratch array and status word for the current
+// device.  The first call on each device looks them up (cudaGetSymbolAddress,
+// with that device current); later calls reuse them.
+fa_status noalloc_scratch(void** scratch, unsigned int** status) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  static void* word[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    void* w = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess || p == nullptr) return FA_ERR_CUDA;
+    if (cudaGetSymbolAddress(&w, g_decode_noalloc_status) != cudaSuccess || w == nullptr) return FA_ERR_CUDA;
+    word[dev] = w;
+    addr[dev] = p;
+  }
+  *scratch = addr[dev];
+  *status = static_cast<unsigned int*>(word[dev]);
+  return FA_OK;
+}
+
+template <int D>
+fa_status launch_decode_i8_noalloc(const fa_decode_params& p, int split_keys, int n_splits, void* scratch,
+                                   const LaunchCtx& ctx) {
+  using G = Geom<D>;
+  const uint64_t rows = static_cast<uint64_t>(p.batch) * p.hkv * p.capacity;
+  CUtensorMap tmk, tmv;
+  const uint64_t dims[2] = {static_cast<uint64_t>(D), rows};
+  const uint64_t strides[1] = {static_cast<uint64_t>(D)};
+  const uint32_t box[2] = {static_cast<uint32_t>(D), static_cast<uint32_t>(kTile)};
+  const CUtensorMapSwizzle sw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  fa_status st = encode_tensor_map(&tmk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p.k_cache, dims, strides, box, sw);
+  if (st != FA_OK) return st;
+  st = encode_tensor_map(&tmv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p.v_cache, dims, strides, box, sw);
+  if (st != FA_OK) return st;
+
+  // partial records are packed with a stride of the launched split count
+  const size_t o_bytes = static_cast<size_t>(p.batch) * p.hq * n_splits * D * sizeof(float);
+  DecodeArgs A;
+  A.q = static_cast<const __nv_bfloat16*>(p.q);
+  A.k_scales = p.k_scales;
+  A.v_scales = p.v_scales;
+  A.seqlens = p.cache_seqlens;
+  A.part_o = static_cast<float*>(scratch);
+  A.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + o_bytes);
+  A.hq = p.hq;
+  A.hkv = p.hkv;
+  A.group = p.hq / p.hkv;
+  A.cap = p.capacity;
+  A.window = p.window;
+  A.split_keys = split_keys;
+  A.n_split_max = n_splits;
+  A.n_split_launched = n_splits;
+  A.scale_log2 = p.softmax_scale * kLog2e;
+  A.wd = ctx.wd;
+
+  auto kern = decode_i8_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem) != cudaSuccess)
+    return FA_ERR_CUDA;
+  // (no note_variant here: its bookkeeping set may allocate host memory)
+  dim3 grid(n_splits, p.hkv, p.batch);
+  kern<<<grid, kWarps * 32, G::kSmem, ctx.stream>>>(tmk, tmv, A);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  auto merge = decode_merge_kernel<D>;
+  merge<<<p.batch * p.hq, 128, 0, ctx.stream>>>(A, static_cast<__nv_bfloat16*>(p.out),
+                                                make_epilogue(p.epilogue, p.n_epilogue));
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+size_t decode_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+fa_status launch_decode_noalloc(const fa_decode_params& p, int split_keys, long long budget, cudaStream_t stream) {
+  if (p.kv_dtype != FA_I8) return FA_ERR_UNSUPPORTED;
+  const int max_len = p.max_seqlen > 0 ? p.max_seqlen : p.capacity;
+  const size_t per_split = static_cast<size_t>(p.batch) * p.hq * (p.head_dim + 2) * sizeof(float);
+  if (per_split > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;  // even one split does not fit
+  const int fit = static_cast<int>(kNoAllocScratchBytes / per_split);
+  int n_splits = max_len > 0 ? (max_len + split_keys - 1) / split_keys : 1;
+  if (n_splits > fit) {
+    if (p.split_keys > 0) return FA_ERR_WORKSPACE;  // the caller's split count does not fit
+    split_keys = ((max_len + fit - 1) / fit + 255) / 256 * 256;
+    n_splits = (max_len + split_keys - 1) / split_keys;
+    if (n_splits > fit) return FA_ERR_WORKSPACE;
+  }
+  if (n_splits < 1) n_splits = 1;
+  void* scratch = nullptr;
+  LaunchCtx ctx;
+  ctx.stream = stream;
+  ctx.wd.budget = budget;
+  fa_status st = noalloc_scratch(&scratch, &ctx.wd.word);
+  if (st != FA_OK) return st;
+  if (p.head_dim == 128) return launch_decode_i8_noalloc<128>(p, split_keys, n_splits, scratch, ctx);
+  if (p.head_dim == 64) return launch_decode_i8_noalloc<64>(p, split_keys, n_splits, scratch, ctx);
+  return FA_ERR_UNSUPPORTED;
+}
+
+}  // namespace fa

@@ -250,6 +250,42 @@ fa_status fa_attention_decode(const fa_decode_params* p, fa_stream_t stream) {
   return launch_decode(*p, split, n_splits, ctx);
 }
 
+fa_status fa_attention_decode_noalloc(const fa_decode_params* p, fa_stream_t stream) {
+  if (p == nullptr) return FA_ERR_INVALID;
+  if (p->batch < 0 || p->hq <= 0 || p->hkv <= 0 || p->hq % p->hkv != 0) return FA_ERR_INVALID;
+  if (p->capacity <= 0 || p->capacity % 32 != 0) return FA_ERR_INVALID;
+  if (p->max_seqlen < 0 || p->max_seqlen > p->capacity) return FA_ERR_INVALID;
+  if (p->split_keys < 0 || p->split_keys % 256 != 0) return FA_ERR_INVALID;
+  if (!epilogue_ok(p->epilogue, p->n_epilogue)) return FA_ERR_INVALID;
+  if (!std::isfinite(p->softmax_scale)) return FA_ERR_INVALID;
+  if (p->kv_dtype != FA_I8 && p->kv_dtype != FA_BF16) return FA_ERR_INVALID;
+  if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
+  if (p->head_dim != 64 && p->head_dim != 128) return FA_ERR_UNSUPPORTED;
+  if (p->hq / p->hkv > 8) return FA_ERR_UNSUPPORTED;
+  if (p->kv_dtype != FA_I8) return FA_ERR_UNSUPPORTED;
+  if (p->batch == 0) return FA_OK;
+  if (p->q == nullptr || p->k_cache == nullptr || p->v_cache == nullptr || p->out == nullptr ||
+      p->cache_seqlens == nullptr || p->k_scales == nullptr || p->v_scales == nullptr)
+    return FA_ERR_INVALID;
+  if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->out) ||
+      !aligned16(p->k_scales) || !aligned16(p->v_scales))
+    return FA_ERR_INVALID;
+  const size_t per_split = static_cast<size_t>(p->batch) * p->hq * (p->head_dim + 2) * sizeof(float);
+  if (per_split > decode_noalloc_scratch_bytes()) return FA_ERR_WORKSPACE;
+  const int max_len = p->max_seqlen > 0 ? p->max_seqlen : p->capacity;
+  int split = p->split_keys;
+  if (split == 0) {
+    const long long pairs = static_cast<long long>(p->batch) * p->hkv;
+    const long long want_units = 148LL * 2 * 4;
+    long long per = (static_cast<long long>(max_len) * pairs + want_units - 1) / want_units;
+    per = ((per + 255) / 256) * 256;
+    if (per < 256) per = 256;
+    if (per > 4096) per = 4096;
+    split = static_cast<int>(per);
+  }
+  return launch_decode_noalloc(*p, split, watchdog_budget(), reinterpret_cast<cudaStream_t>(stream));
+}
+
 fa_status fa_check_device_error(fa_stream_t stream) {
   unsigned int* word = nullptr;
   fa_status st = status_word(&word);

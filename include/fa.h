@@ -184,6 +184,39 @@ FA_API size_t fa_decode_workspace_size(int32_t batch, int32_t hq, int32_t capaci
 
 FA_API fa_status fa_attention_decode(const fa_decode_params *p, fa_stream_t stream);
 
+/*
+ * fa_attention_decode_noalloc -- fa_attention_decode for callers that cannot
+ * allocate device memory when they call.  The paper has no counterpart: this
+ * entry point exists for callers such as a plug-in inside a serving runtime
+ * that owns every device byte through its own pre-planned arena (allocating
+ * outside it is forbidden or breaks its accounting), or code that must not
+ * trigger the implicit device synchronisation a cudaMalloc can cause.
+ *
+ * Same parameters and results as fa_attention_decode, except that
+ * p->workspace and p->workspace_bytes are ignored: the per-split partials go
+ * to a scratch array of FA_DECODE_NOALLOC_SCRATCH_BYTES (8 MiB) built into
+ * the library, which every device that loads the library holds until the
+ * process exits.  The call allocates nothing (no cudaMalloc, no library
+ * allocator).
+ *   - Limit: batch * hq * (head_dim + 2) * 4 bytes per key split must fit in
+ *     the scratch for the number of splits used.  With split_keys == 0 the
+ *     library picks a split large enough to fit; a problem for which even
+ *     one split does not fit (batch * hq * (head_dim + 2) * 4 > 8 MiB), or a
+ *     caller-chosen split_keys that does not fit, returns FA_ERR_WORKSPACE
+ *     and enqueues nothing.  Only the int8 cache (FA_I8) is supported.
+ *   - The first call on each device looks up the scratch array's device
+ *     address (with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the scratch and it keeps the last call's
+ *     contents (nothing in it needs clearing).  Calls that overlap on the GPU
+ *     race on it: serialise them (one stream, or events between streams).
+ *   - A bounded device wait that gives up inside this call is recorded in a
+ *     status word of this entry point's own (the shared one is allocated on
+ *     first use), which fa_check_device_error does not read.
+ */
+#define FA_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+FA_API fa_status fa_attention_decode_noalloc(const fa_decode_params *p, fa_stream_t stream);
+
 /* Static text for a status code (never NULL). */
 FA_API const char *fa_status_string(fa_status s);
 
