@@ -62,7 +62,8 @@ struct PrefillArgs {
   SeqLayout L;
   __nv_bfloat16* out;
   int batch, hq, hkv, group, n_qblocks, two_tiles;
-  float scale_log2;
+  float scale_log2;      // |softmax scale| * log2(e), > 0
+  uint32_t negate_s;     // 1: the MMA negates Q (a negative softmax scale)
   Epilogue epi;
   Watchdog wd;
 };
@@ -179,7 +180,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = umma_idesc_f16(kBM, kBN, 1, 1, false);
+      // a negative softmax scale is folded into the S MMA (negated A operand),
+      // so the softmax only ever sees a positive scale
+      const uint32_t idesc_s = umma_idesc_f16(kBM, kBN, 1, 1, false) | (A.negate_s << 13);
       constexpr uint32_t idesc_o = umma_idesc_f16(kBM, D, 1, 1, true);
       const uint32_t q_base = smem_u32(smem);
       auto issue_s = [&](int t, int s) {
@@ -256,22 +259,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(s_tm + 96, raw[3]);
       tmem_wait_ld();
       const int kb = (j_lo + it) * kBN;
-      const bool whole = kb >= lo && kb + kBN <= hi;
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (!(kb >= lo && kb + kBN <= hi)) {
+        // boundary tile: keys outside this row's band become -inf (raw scores;
+        // the scale is positive, so masking before scaling is the same)
+        const int va = lo - kb, vb = hi - kb;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float x = __uint_as_float(raw[cc][e]) * A.scale_log2;
-          if (!whole) {
-            const int kj = kb + cc * 32 + e;
-            x = (kj >= lo && kj < hi) ? x : -INFINITY;
-          }
-          raw[cc][e] = __float_as_uint(x);
-          mx[cc] = fmaxf(mx[cc], x);
-        }
+        for (int c = 0; c < kBN; ++c)
+          if (c < va || c >= vb) raw[c / 32][c % 32] = 0xff800000u;
       }
-      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      // row max of the raw scores: eight independent chains of 3-input max
+      float g8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t* v = &raw[k / 2][(k % 2) * 16];
+        float g = max3f(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+#pragma unroll
+        for (int e = 3; e < 15; e += 2) g = max3f(g, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+        g8[k] = fmaxf(g, __uint_as_float(v[15]));
+      }
+      const float m_raw = fmaxf(max3f(g8[0], g8[1], g8[2]), max3f(max3f(g8[3], g8[4], g8[5]), g8[6], g8[7]));
+      const float m_tile = m_raw * A.scale_log2;
       const float m_new = fmaxf(m_used, m_tile);
       const bool need = m_new > m_used + kRescaleThreshold;
       float alpha = 1.f;
@@ -279,22 +286,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         alpha = ex2_approx(m_used - m_new);
         m_used = m_new;
       }
-      const float mref = m_used == -INFINITY ? 0.f : m_used;
-      l *= alpha;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+      const float2 sc2 = make_float2(A.scale_log2, A.scale_log2);
+      const float2 nm2 = make_float2(neg_m, neg_m);
+      float2 lacc[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) lacc[k] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2_approx(__uint_as_float(raw[cc][2 * e]) - mref);
-          const float p1 = ex2_approx(__uint_as_float(raw[cc][2 * e + 1]) - mref);
-          ls[cc] += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          // p = 2^(s * scale * log2(e) - m): one packed FMA for two scores
+          const float2 x = fma2(make_float2(__uint_as_float(raw[cc][2 * e]), __uint_as_float(raw[cc][2 * e + 1])),
+                                sc2, nm2);
+          const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          lacc[e % 8] = add2(lacc[e % 8], pp);
+          pk[e] = pack_bf16x2(pp.x, pp.y);
         }
         tmem_st16(s_tm + cc * 16, pk);
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) lacc[k] = add2(lacc[k], lacc[k + 4]);
+      lacc[0] = add2(lacc[0], lacc[2]);
+      lacc[1] = add2(lacc[1], lacc[3]);
+      lacc[0] = add2(lacc[0], lacc[1]);
+      l = l * alpha + (lacc[0].x + lacc[0].y);
       if (it > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
         for (int oc = 0; oc < D / 32; ++oc) {
@@ -321,13 +338,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t o[32];
         tmem_ld32(o_tm + oc * 32, o);
         tmem_wait_ld();
+        float y[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) y[e] = __uint_as_float(o[e]) * inv_l;
+        apply_epilogue_vec(y, A.epi);
         uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float y0 = apply_epilogue(__uint_as_float(o[2 * e]) * inv_l, A.epi);
-          const float y1 = apply_epilogue(__uint_as_float(o[2 * e + 1]) * inv_l, A.epi);
-          pk[e] = pack_bf16x2(y0, y1);
-        }
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
         if (store) {
           uint4* dst = reinterpret_cast<uint4*>(orow + oc * 32);
 #pragma unroll
@@ -383,7 +400,11 @@ fa_status launch_bf16(const fa_fwd_params& p, const LaunchCtx& ctx) {
   A.two_tiles = (A.group % 2 == 0) ? 1 : 0;
   const int max_sq = varlen ? p.max_seqlen_q : p.seqlen_q;
   A.n_qblocks = (max_sq + kBM - 1) / kBM;
-  A.scale_log2 = p.softmax_scale * kLog2e;
+  // the softmax works with a positive scale: a negative one negates Q inside
+  // the S MMA; a zero scale (uniform weights) becomes a vanishing one
+  const float abs_scale = p.softmax_scale < 0.f ? -p.softmax_scale : p.softmax_scale;
+  A.scale_log2 = (abs_scale > 0.f ? abs_scale : 1e-30f) * kLog2e;
+  A.negate_s = p.softmax_scale < 0.f ? 1u : 0u;
   A.epi = make_epilogue(p.epilogue, p.n_epilogue);
   A.wd = ctx.wd;
   const long long n_pairs = A.two_tiles ? p.hq / 2 : p.hq;
