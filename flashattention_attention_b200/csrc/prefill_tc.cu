@@ -31,6 +31,16 @@
 // log2 units; the final O / l uses the same stale max, so the result is
 // exact), rescale O_t in TMEM when it did, write P_t, signal the MMA warp.
 // Every wait is bounded (device.cuh); a timeout aborts all roles cleanly.
+//
+// int8 K/V (fkl_python PR #6, Summary: "dequantizes in-register inside q.k
+// and p.v; the compressed cache is never inflated in global memory"): TMA
+// brings each int8 tile into shared memory (at d = 128 into the upper half of
+// the bf16 slot it becomes), four converter warps rewrite it as exact bf16
+// (|c| <= 127) in the tensor-core layout, and fence it to the async proxy.
+// The per-key K scale multiplies the columns of S after the MMA; the per-key
+// V scale multiplies the columns of P before its bf16 cast (l sums the
+// unscaled p).  That variant runs 16 warps and rebalances registers with
+// setmaxnreg (softmax 200, the rest 56).
 #include "internal.h"
 #include "layout.cuh"
 #include "umma.cuh"
@@ -40,27 +50,43 @@ namespace {
 
 constexpr int kBM = 128;  // query rows per Q tile
 constexpr int kBN = 128;  // keys per K/V tile
-constexpr int kThreads = 320;
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kConvWarp0 = 12;  // int8 variant: warps 12-15 convert K/V tiles
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t kChunkBytes = kSwizzleChunkRows * 128;  // [128 rows x 64 bf16]
 
-template <int D>
+template <int D, bool kI8>
 struct TcGeom {
   static constexpr int kStages = (D == 128) ? 2 : 3;
   static constexpr uint32_t kQBytes = kBM * D * 2;
-  static constexpr uint32_t kKVBytes = kBN * D * 2;
+  static constexpr uint32_t kKVBytes = kBN * D * 2;   // one bf16 K or V tile
+  static constexpr uint32_t kI8Bytes = kBN * D;       // one int8 tile
   static constexpr uint32_t kKOff = 2 * kQBytes;
   static constexpr uint32_t kVOff = kKOff + kStages * kKVBytes;
-  static constexpr uint32_t kBarOff = kVOff + kStages * kKVBytes;
+  // int8 staging: at d = 128 in the upper half of each bf16 slot (a row's
+  // bf16 output overwrites only that row's int8 bytes); at d = 64 separate
+  static constexpr bool kInPlace = (D == 128);
+  static constexpr uint32_t kStageOff = kVOff + kStages * kKVBytes;
+  static constexpr uint32_t kStageBytes = (kI8 && !kInPlace) ? 2 * kStages * kI8Bytes : 0;
+  static constexpr uint32_t kBarOff = kStageOff + kStageBytes;
   static constexpr uint32_t kSmem = kBarOff + 256 + 1024;
+  static constexpr int kThreads = kI8 ? 512 : 320;
+  __host__ __device__ static constexpr uint32_t k_stage(int s) {
+    return kInPlace ? kKOff + s * kKVBytes + kKVBytes / 2 : kStageOff + s * kI8Bytes;
+  }
+  __host__ __device__ static constexpr uint32_t v_stage(int s) {
+    return kInPlace ? kVOff + s * kKVBytes + kKVBytes / 2 : kStageOff + (kStages + s) * kI8Bytes;
+  }
 };
 
 struct PrefillArgs {
   SeqLayout L;
   __nv_bfloat16* out;
+  const float* k_scales;  // int8 variant: one fp32 scale per K / V row
+  const float* v_scales;
+  int64_t k_plane_rows;   // rows per K plane (the scales share K's row numbering)
   int batch, hq, hkv, group, n_qblocks, two_tiles;
   float scale_log2;      // |softmax scale| * log2(e), > 0
   uint32_t negate_s;     // 1: the MMA negates Q (a negative softmax scale)
@@ -73,11 +99,40 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-    prefill_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const PrefillArgs A) {
-  using G = TcGeom<D>;
+// bf16 of the signed bytes 0 and 1 (lo) or 2 and 3 (hi) of w, exact:
+// 0x4300 | (b & 0x7f) is 128 + (b & 0x7f) and 0x4300 | (b & 0x80) is 128 or
+// 256, so their difference is the two's-complement value of b.
+__device__ __forceinline__ uint32_t i8x2_to_bf16x2(uint32_t w, uint32_t sel) {
+  uint32_t t, m, sg, r;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(t) : "r"(w), "r"(sel));
+  asm("lop3.b32 %0, %1, 0x007f007f, 0x43004300, 0xea;" : "=r"(m) : "r"(t));
+  asm("lop3.b32 %0, %1, 0x00800080, 0x43004300, 0xea;" : "=r"(sg) : "r"(t));
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(m), "r"(sg));
+  return r;
+}
+
+// 32 consecutive per-key scales from global memory (read-only path; every
+// lane of a warp reads the same addresses, so each load is one broadcast);
+// entries at or past `valid` read as 0.  Vector loads only from 16-byte
+// aligned addresses (varlen sequences start anywhere).
+__device__ __forceinline__ void load_scales32(const float* p, int valid, float (&v)[32]) {
+  if (valid >= 32 && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(p) + q);
+      v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[e] = e < valid ? __ldg(p + e) : 0.f;
+  }
+}
+
+template <int D, bool kI8>
+__global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const PrefillArgs A) {
+  using G = TcGeom<D, kI8>;
   constexpr int S = G::kStages;
   extern __shared__ uint8_t tc_smem_raw[];
   uint8_t* smem =
@@ -92,7 +147,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_full + 2;   // [2]
   uint64_t* o_done = p_full + 2;   // [2]
   uint64_t* drain = o_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* kraw_full = drain + 1;   // [S] int8 variant: TMA landed the int8 K tile
+  uint64_t* vraw_full = kraw_full + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(vraw_full + S);
   __shared__ int abort_flag;
 
   // ---- work tile: longest (highest q-block) first, then sequence, then head pair
@@ -130,10 +187,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     abort_flag = 0;
     mbar_init(q_full, 1);
     for (int s = 0; s < S; ++s) {
-      mbar_init(k_full + s, 1);
+      // bf16: TMA completes k_full / v_full; int8: the 128 converter threads do
+      mbar_init(k_full + s, kI8 ? 128 : 1);
       mbar_init(k_empty + s, 1);
-      mbar_init(v_full + s, 1);
+      mbar_init(v_full + s, kI8 ? 128 : 1);
       mbar_init(v_empty + s, 1);
+      mbar_init(kraw_full + s, 1);
+      mbar_init(vraw_full + s, 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full + t, 1);
@@ -152,6 +212,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Roles split by warpgroup first: warpgroups 0-1 softmax, 2-3 the rest.
+  // int8 variant registers: 512 threads launched at 128; warpgroups 0-1 take
+  // 200, warpgroups 2-3 give back down to 56: 256*200 + 256*56 = 512*128.
+  if (warp >= 8) {
+  if constexpr (kI8) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -166,15 +231,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = it % S, u = it / S;
         const int krow = k_prow0 + (j_lo + it) * kBN;
         if (u > 0 && !wait_parity(k_empty + s, (u - 1) & 1, A.wd, &abort_flag)) break;
-        mbar_expect_tx(k_full + s, G::kKVBytes);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + G::kKOff + s * G::kKVBytes + c * kChunkBytes, &tm_k, k_full + s, 64 * c, krow,
-                      k_plane);
+        if constexpr (kI8) {
+          mbar_expect_tx(kraw_full + s, G::kI8Bytes);
+          tma_load_3d(smem + G::k_stage(s), &tm_k, kraw_full + s, 0, krow, k_plane);
+        } else {
+          mbar_expect_tx(k_full + s, G::kKVBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem + G::kKOff + s * G::kKVBytes + c * kChunkBytes, &tm_k, k_full + s, 64 * c, krow,
+                        k_plane);
+        }
         if (u > 0 && !wait_parity(v_empty + s, (u - 1) & 1, A.wd, &abort_flag)) break;
-        mbar_expect_tx(v_full + s, G::kKVBytes);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + G::kVOff + s * G::kKVBytes + c * kChunkBytes, &tm_v, v_full + s, 64 * c, krow,
-                      k_plane);
+        if constexpr (kI8) {
+          mbar_expect_tx(vraw_full + s, G::kI8Bytes);
+          tma_load_3d(smem + G::v_stage(s), &tm_v, vraw_full + s, 0, krow, k_plane);
+        } else {
+          mbar_expect_tx(v_full + s, G::kKVBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem + G::kVOff + s * G::kKVBytes + c * kChunkBytes, &tm_v, v_full + s, 64 * c, krow,
+                        k_plane);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
@@ -236,11 +311,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(drain);
       wait_parity(drain, 0, A.wd);
     }
-  } else if (warp / 4 < ntile) {
+  } else if (kI8 && warp >= kConvWarp0) {
+    // ------------------------------------------------------------ int8 -> bf16 converters
+    // thread r rewrites row r of each int8 K and V tile as bf16 in the
+    // 128-byte-swizzled K-major (K) / MN-major (V) operand layout
+    const int r = static_cast<int>(threadIdx.x) - kConvWarp0 * 32;
+    const int64_t scale_row0 = static_cast<int64_t>(k_plane) * A.k_plane_rows + k_prow0;
+    auto convert_row = [&](const uint8_t* src_tile, uint8_t* dst_tile) {
+      constexpr int kChunks8 = D / 16;  // 16-byte int8 chunks per row
+      uint4 w[kChunks8];
+#pragma unroll
+      for (int c = 0; c < kChunks8; ++c) {
+        const int pc = (D == 128) ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
+        w[c] = *reinterpret_cast<const uint4*>(src_tile + r * D + pc * 16);
+      }
+#pragma unroll
+      for (int c = 0; c < kChunks8; ++c) {
+        const int h = c / 4, j0 = 2 * (c % 4);
+        uint8_t* row = dst_tile + h * kChunkBytes + r * 128;
+        const uint4 a = make_uint4(i8x2_to_bf16x2(w[c].x, 0x4140), i8x2_to_bf16x2(w[c].x, 0x4342),
+                                   i8x2_to_bf16x2(w[c].y, 0x4140), i8x2_to_bf16x2(w[c].y, 0x4342));
+        const uint4 bq = make_uint4(i8x2_to_bf16x2(w[c].z, 0x4140), i8x2_to_bf16x2(w[c].z, 0x4342),
+                                    i8x2_to_bf16x2(w[c].w, 0x4140), i8x2_to_bf16x2(w[c].w, 0x4342));
+        *reinterpret_cast<uint4*>(row + ((j0 ^ (r & 7)) * 16)) = a;
+        *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ (r & 7)) * 16)) = bq;
+      }
+    };
+    for (int it = 0; it < n_iter; ++it) {
+      const int s = it % S;
+      const uint32_t ph = (it / S) & 1;
+      const int kb = (j_lo + it) * kBN;
+      if (kb + r < sq.s_k) {  // warm L1 with this tile's scales for the softmax warps
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(A.k_scales + scale_row0 + kb + r));
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(A.v_scales + scale_row0 + kb + r));
+      }
+      if (!__all_sync(0xffffffffu, wait_parity(kraw_full + s, ph, A.wd, &abort_flag))) break;
+      convert_row(smem + G::k_stage(s), smem + G::kKOff + s * G::kKVBytes);
+      fence_proxy_async_smem();
+      mbar_arrive(k_full + s);
+      if (!__all_sync(0xffffffffu, wait_parity(vraw_full + s, ph, A.wd, &abort_flag))) break;
+      convert_row(smem + G::v_stage(s), smem + G::kVOff + s * G::kKVBytes);
+      fence_proxy_async_smem();
+      mbar_arrive(v_full + s);
+    }
+  }
+  } else {
+  if constexpr (kI8) asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+  if (warp / 4 < ntile) {
     // ------------------------------------------------------------ softmax
     const int t = warp / 4, quarter = warp % 4;
     const int r = quarter * 32 + lane;
     const int i = i0 + r;
+    const int64_t scale_row0 = static_cast<int64_t>(k_plane) * A.k_plane_rows + k_prow0;
     int lo, hi;
     band_of(A.L, i, sq.s_q, sq.s_k, lo, hi);
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
@@ -259,9 +381,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(s_tm + 96, raw[3]);
       tmem_wait_ld();
       const int kb = (j_lo + it) * kBN;
+      if constexpr (kI8) {
+        // S columns times the per-key K scale (keys past the sequence get 0
+        // and are masked below)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          float ksv[32];
+          load_scales32(A.k_scales + scale_row0 + kb + cc * 32, sq.s_k - kb - cc * 32, ksv);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float2 x = mul2(make_float2(__uint_as_float(raw[cc][2 * e]), __uint_as_float(raw[cc][2 * e + 1])),
+                                  make_float2(ksv[2 * e], ksv[2 * e + 1]));
+            raw[cc][2 * e] = __float_as_uint(x.x);
+            raw[cc][2 * e + 1] = __float_as_uint(x.y);
+          }
+        }
+      }
       if (!(kb >= lo && kb + kBN <= hi)) {
-        // boundary tile: keys outside this row's band become -inf (raw scores;
-        // the scale is positive, so masking before scaling is the same)
+        // boundary tile: keys outside this row's band become -inf (the
+        // softmax scale is positive, so masking before it is the same)
         const int va = lo - kb, vb = hi - kb;
 #pragma unroll
         for (int c = 0; c < kBN; ++c)
@@ -295,6 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t pk[16];
+        float vsv[32];
+        if constexpr (kI8) load_scales32(A.v_scales + scale_row0 + kb + cc * 32, sq.s_k - kb - cc * 32, vsv);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           // p = 2^(s * scale * log2(e) - m): one packed FMA for two scores
@@ -302,7 +442,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 sc2, nm2);
           const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           lacc[e % 8] = add2(lacc[e % 8], pp);
-          pk[e] = pack_bf16x2(pp.x, pp.y);
+          if constexpr (kI8) {
+            // the V scale multiplies P's columns; l keeps the unscaled p
+            const float2 pv = mul2(pp, make_float2(vsv[2 * e], vsv[2 * e + 1]));
+            pk[e] = pack_bf16x2(pv.x, pv.y);
+          } else {
+            pk[e] = pack_bf16x2(pp.x, pp.y);
+          }
         }
         tmem_st16(s_tm + cc * 16, pk);
       }
@@ -353,6 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
+  }
 
   tc_fence_before();
   __syncthreads();
@@ -362,9 +509,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
-fa_status launch_bf16(const fa_fwd_params& p, const LaunchCtx& ctx) {
-  using G = TcGeom<D>;
+template <int D, bool kI8>
+fa_status launch_tc(const fa_fwd_params& p, const LaunchCtx& ctx) {
+  using G = TcGeom<D, kI8>;
   const bool varlen = p.cu_seqlens_q != nullptr;
   const uint64_t q_rows = varlen ? p.total_q : p.seqlen_q;
   const uint64_t k_rows = varlen ? p.total_k : p.seqlen_k;
@@ -372,15 +519,26 @@ fa_status launch_bf16(const fa_fwd_params& p, const LaunchCtx& ctx) {
   const uint64_t k_planes = varlen ? p.hkv : static_cast<uint64_t>(p.batch) * p.hkv;
   if (k_rows == 0) return FA_OK;  // no keys anywhere: only the empty-band kernel writes
   CUtensorMap tq, tk, tv;
-  const uint32_t box[3] = {64, static_cast<uint32_t>(kSwizzleChunkRows), 1};
   {
+    const uint32_t box[3] = {64, static_cast<uint32_t>(kSwizzleChunkRows), 1};
     const uint64_t dims[3] = {static_cast<uint64_t>(D), q_rows, q_planes};
     const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, q_rows * D * 2};
     fa_status st = encode_tensor_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.q, dims, strides, box,
                                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != FA_OK) return st;
   }
-  {
+  if constexpr (kI8) {
+    // int8 rows of D bytes, one box per tile (128 B or 64 B swizzle)
+    const uint32_t box[3] = {static_cast<uint32_t>(D), static_cast<uint32_t>(kSwizzleChunkRows), 1};
+    const uint64_t dims[3] = {static_cast<uint64_t>(D), k_rows, k_planes};
+    const uint64_t strides[2] = {static_cast<uint64_t>(D), k_rows * D};
+    const CUtensorMapSwizzle sw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    fa_status st = encode_tensor_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, p.k, dims, strides, box, sw);
+    if (st != FA_OK) return st;
+    st = encode_tensor_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, p.v, dims, strides, box, sw);
+    if (st != FA_OK) return st;
+  } else {
+    const uint32_t box[3] = {64, static_cast<uint32_t>(kSwizzleChunkRows), 1};
     const uint64_t dims[3] = {static_cast<uint64_t>(D), k_rows, k_planes};
     const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, k_rows * D * 2};
     fa_status st = encode_tensor_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.k, dims, strides, box,
@@ -393,6 +551,9 @@ fa_status launch_bf16(const fa_fwd_params& p, const LaunchCtx& ctx) {
   PrefillArgs A;
   A.L = SeqLayout::from(p);
   A.out = static_cast<__nv_bfloat16*>(p.out);
+  A.k_scales = p.k_scales;
+  A.v_scales = p.v_scales;
+  A.k_plane_rows = static_cast<int64_t>(k_rows);
   A.batch = p.batch;
   A.hq = p.hq;
   A.hkv = p.hkv;
@@ -411,20 +572,24 @@ fa_status launch_bf16(const fa_fwd_params& p, const LaunchCtx& ctx) {
   const long long grid = static_cast<long long>(A.n_qblocks) * p.batch * n_pairs;
   if (grid == 0) return FA_OK;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-  auto kern = prefill_bf16_kernel<D>;
+  auto kern = prefill_tc_kernel<D, kI8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem) != cudaSuccess)
     return FA_ERR_CUDA;
   note_variant(reinterpret_cast<const void*>(kern));
-  kern<<<static_cast<unsigned>(grid), kThreads, G::kSmem, ctx.stream>>>(tq, tk, tv, A);
+  kern<<<static_cast<unsigned>(grid), G::kThreads, G::kSmem, ctx.stream>>>(tq, tk, tv, A);
   return cuda_status(cudaGetLastError());
 }
 
 }  // namespace
 
 fa_status launch_prefill_tc(const fa_fwd_params& p, const LaunchCtx& ctx) {
-  if (p.kv_dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
-  if (p.head_dim == 128) return launch_bf16<128>(p, ctx);
-  if (p.head_dim == 64) return launch_bf16<64>(p, ctx);
+  if (p.kv_dtype == FA_I8) {
+    if (p.head_dim == 128) return launch_tc<128, true>(p, ctx);
+    if (p.head_dim == 64) return launch_tc<64, true>(p, ctx);
+    return FA_ERR_UNSUPPORTED;
+  }
+  if (p.head_dim == 128) return launch_tc<128, false>(p, ctx);
+  if (p.head_dim == 64) return launch_tc<64, false>(p, ctx);
   return FA_ERR_UNSUPPORTED;
 }
 
