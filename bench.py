@@ -49,7 +49,7 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "prefill_bf16_kernel<128>": ["prefill_tc.cu", "umma.cuh", "device.cuh", "layout.cuh"],
+    "prefill_tc_kernel<128,bf16>": ["prefill_tc.cu", "umma.cuh", "device.cuh", "layout.cuh"],
     "decode_i8_kernel<128>": ["decode.cu", "device.cuh"],
     "compress_kernel": ["quant.cu"],
 }
@@ -192,6 +192,10 @@ def gpu_arm(args, rank, world, dist):
 
     if args.only in ("decode", "quant"):
         return decode_and_quant(args, dev, peaks, world, dist, {})
+    if args.only in ("prefill_int8", "varlen"):
+        res = {}
+        other_prefills(args, dev, peaks, world, dist, res)
+        return res
     l0 = fa.kernel_launches()
     with ClockSampler(dev.index or 0) as clocks:
         ms = time_launches(prefill, args.steps, args.warmup, torch, dist)
@@ -229,11 +233,11 @@ def gpu_arm(args, rank, world, dist):
                    "flops_per_step": flops_tiles, "flops_counting": "128x128 tiles intersecting the band",
                    "flops_exact_pairs": flops_exact, "l2": "inputs larger than L2 (201 MB), no flush",
                    "parallelism": f"replicas x{world} (no collective)"},
-        "roofline": {"bound": "tensor", "kernel": "prefill_bf16_kernel<128>", "achieved": round(tflops, 2),
+        "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel<128,bf16>", "achieved": round(tflops, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(tflops / peaks["bf16_tflops"], 4),
                      "peak_source": f"{peaks['source']} bf16 burst",
-                     "traffic": measured_traffic("prefill_bf16_kernel<128>"),
+                     "traffic": measured_traffic("prefill_tc_kernel<128,bf16>"),
                      "frac_of_nominal_2250": round(tflops / 2250.0, 4)},
         "e2e": {"value": round(flops_tiles / (e2e_ms * 1e-3) / 1e12 * world, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
@@ -241,10 +245,65 @@ def gpu_arm(args, rank, world, dist):
         "clocks": clk,
     }
     if args.only == "all":
+        other_prefills(args, dev, peaks, world, dist, result)
         decode_and_quant(args, dev, peaks, world, dist, result)
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, flops_tiles, flops_exact, args.cpu_seconds)
     return result
+
+
+def varlen_flops(w):
+    tiles = pairs = 0
+    for L in w.lengths:
+        t, pr = band_tiles(L, L, w.causal, w.window)
+        tiles += t
+        pairs += pr
+    per = w.hq * 4 * w.d
+    return per * tiles * TILE * TILE, per * pairs
+
+
+def other_prefills(args, dev, peaks, world, dist, result):
+    """The varlen sliding-window prefill (d=64, epilogue) and the long-context
+    prefill over an int8 KV cache, each timed like the main step."""
+    import torch
+    from flashattention_attention_b200 import fa, inputs
+    steps = max(10, args.steps // 4)
+
+    w = inputs.varlen_window_prefill()
+    cu = inputs.cu_from_lengths(w.lengths).to(dev)
+    q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
+    out = torch.empty_like(q)
+    ms = time_launches(lambda: fa.attention_fwd(q, k, v, hq=w.hq, hkv=w.hkv, causal=True, window=w.window,
+                                                epilogue=w.epilogue, cu_seqlens_q=cu,
+                                                max_seqlen_q=max(w.lengths), out=out),
+                       steps, args.warmup, torch, dist)
+    ft, fe = varlen_flops(w)
+    result["varlen_window_prefill"] = {
+        "workload": w.name, "lengths": w.lengths, "value": round(fe / (ms * 1e-3) / 1e12 * world, 2),
+        "unit": "TFLOP/s", "flops_counting": "exact visible pairs", "flops_per_step": fe,
+        "flops_tile_count": ft, "ms_per_step": round(ms, 4),
+        "frac_of_bf16_peak": round(fe / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
+    del q, k, v, out
+
+    w = inputs.int8kv_long_prefill()
+    kc, ks = fa.compress_kv(w.k.to(dev))
+    vc, vs = fa.compress_kv(w.v.to(dev))
+    q = w.q.to(dev)
+    out = torch.empty_like(q)
+    ms = time_launches(lambda: fa.attention_fwd(q, kc, vc, k_scales=ks, v_scales=vs, hq=w.hq, hkv=w.hkv,
+                                                causal=True, epilogue=w.epilogue, out=out),
+                       steps, args.warmup, torch, dist)
+    ft, fe = prefill_flops(w)
+    tf = ft / (ms * 1e-3) / 1e12
+    result["int8kv_long_prefill"] = {
+        "workload": w.name, "value": round(tf * world, 2), "unit": "TFLOP/s",
+        "flops_counting": "128x128 tiles intersecting the band", "flops_per_step": ft,
+        "flops_exact_pairs": fe, "ms_per_step": round(ms, 4),
+        "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel<128,int8>", "achieved": round(tf, 2),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None}}
+    del q, kc, vc, ks, vs, out
+    torch.cuda.empty_cache()
 
 
 def decode_and_quant(args, dev, peaks, world, dist, result):
@@ -369,7 +428,7 @@ def main():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "quant"],
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "quant", "prefill_int8", "varlen"],
                     help="time one part only (used for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
