@@ -4,11 +4,20 @@
 // global memory; kernbench2 commit ADR-0060: decode splits the keys and
 // reduces the partial softmax states (m, l, O) to one output).
 //
-// Work unit: (split, kv-head g, sequence b).  One CTA of 4 warps owns a
-// split; each warp streams 32-key tiles of K codes, V codes and their fp32
-// scales through its own 3-stage ring (TMA, 128-byte swizzle, bounded
-// mbarrier waits), so a warp never waits on another warp.  All G = hq/hkv
-// query heads of the group are served by every key read.
+// Work decomposition (stream-K): the 32-key tiles of every (sequence, KV
+// head) segment are laid end to end, T tiles in all, and a persistent grid of
+// P warps ("workers", 4 per CTA, 2 CTAs per SM) takes equal contiguous ranges
+// [w*T/P, (w+1)*T/P).  Each worker streams its tiles -- K codes, V codes and
+// their fp32 scales -- through its own 3-stage TMA ring (128-byte swizzle,
+// bounded mbarrier waits), straight across segment boundaries, so the ring
+// never drains and every SM gets the same number of bytes.  When a worker's
+// range leaves a segment it writes its partial softmax state (m, l, O) for
+// the segment's G = hq/hkv query heads to record (segment + worker) and
+// counts itself done on the segment; the last worker to finish a segment
+// merges its records (the segment's workers are W(x) = (x*P + P - 1) / T
+// over its tiles), applies the epilogue and stores bf16.  A one-CTA plan
+// kernel first turns the device-side cache lengths into the per-sequence
+// tile prefix sums, zeroes the counters and writes the rows of empty caches.
 //
 // Per tile (tensor cores through mma.sync m16n8k16, fp16 in, fp32 accumulate):
 //   S^T[32 keys x 8 heads] = K_codes[32 x d] . Q^T    (keys on M, heads on N)
@@ -23,10 +32,8 @@
 // Because d is summed over, each thread owns a contiguous byte slice of every
 // K row; Q's fragments use the same dim order.  The S accumulator fragment
 // becomes the P operand fragment with one 8x8 transpose (movmatrix).
-//
-// The CTA merges its 4 warps' (m, l, O) and writes one partial per
-// (sequence, q-head, split); decode_merge_kernel combines the splits,
-// applies the epilogue and stores bf16.
+#include <mutex>
+
 #include "internal.h"
 
 namespace fa {
@@ -35,24 +42,31 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kTile = 32;    // keys per tile
 constexpr int kStages = 3;
+constexpr int kCtasPerSm = 2;
+constexpr int kMaxWorkers = 4096;
 constexpr float kLog2e = 1.4426950408889634f;
 
-struct DecodeArgs {
-  const __nv_bfloat16* q;  // [B*hq, D]
-  const float* k_scales;   // [B*hkv, cap]
+struct SkArgs {
+  const __nv_bfloat16* q;   // [B*hq, D]
+  const float* k_scales;    // [B*hkv, cap]
   const float* v_scales;
-  const int32_t* seqlens;  // [B]
-  float* part_o;           // [B*hq, n_split_max, D]
-  float* part_ml;          // [B*hq, n_split_max, 2]
-  int hq, hkv, group, cap, window, split_keys, n_split_max, n_split_launched;
+  const int32_t* seqlens;   // [B]
+  const int32_t* prefix;    // [B+1]: tiles (x hkv) before sequence b; prefix[B] = T
+  float* rec_o;             // [B*hkv + P][G][D]
+  float* rec_ml;            // [B*hkv + P][G][2]
+  int32_t* counters;        // [B*hkv]: workers done with each segment (zeroed by the plan)
+  __nv_bfloat16* out;       // [B*hq, D]
+  Epilogue epi;
+  int batch, hq, hkv, group, cap, window;
+  int n_workers;            // P (launched warps)
+  int min_tiles;            // > 0: at least this many tiles per worker
   float scale_log2;
   Watchdog wd;
 };
 
 template <int D>
 struct Geom {
-  static constexpr int kRowBytes = D;  // int8 codes
-  static constexpr int kTileBytes = kTile * D;
+  static constexpr int kTileBytes = kTile * D;  // int8 codes
   static constexpr int kScaleOff = 2 * kTileBytes;
   static constexpr int kStageBytes = ((2 * kTileBytes + 2 * kTile * 4) + 1023) / 1024 * 1024;
   static constexpr int kSwzMask = (D == 128) ? 0x70 : 0x30;  // 128B or 64B swizzle
@@ -91,6 +105,7 @@ __device__ __forceinline__ uint32_t i8x2_to_f16x2_even(uint32_t w) {
 // fp16x2 of the signed bytes 1 and 3 of w (exact).
 __device__ __forceinline__ uint32_t i8x2_to_f16x2_odd(uint32_t w) { return i8x2_to_f16x2_even(w >> 8); }
 
+
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -111,15 +126,115 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 
 // Keys of sequence b handled by the decode: [k_lo, L); tiles start at the
 // 32-aligned t_begin <= k_lo so every tile's scale block is 16-byte aligned.
-__device__ __forceinline__ void key_range(int L, int window, int& k_lo, int& t_begin) {
-  k_lo = window > 0 ? max(0, L - window) : 0;
+__host__ __device__ __forceinline__ void key_range(int L, int window, int& k_lo, int& t_begin) {
+  k_lo = window > 0 ? (L - window > 0 ? L - window : 0) : 0;
   t_begin = (k_lo / kTile) * kTile;
+}
+__device__ __forceinline__ int clamp_len(int L, int cap) { return max(0, min(L, cap)); }
+__device__ __forceinline__ int tiles_of(int L, int window) {
+  int k_lo, t_begin;
+  key_range(L, window, k_lo, t_begin);
+  return L > t_begin ? (L - t_begin + kTile - 1) / kTile : 0;
+}
+
+// The worker whose range [w*T/P, (w+1)*T/P) holds tile x.
+__device__ __forceinline__ int worker_of(long long x, long long T, long long P) {
+  return static_cast<int>((x * P + P - 1) / T);
+}
+__device__ __forceinline__ long long worker_begin(long long w, long long T, long long P) { return (w * T) / P; }
+// Never more workers than tiles, so every worker's range is non-empty and a
+// segment's workers are exactly W(first tile) .. W(last tile).
+__device__ __forceinline__ int effective_workers(const SkArgs& A, long long T) {
+  long long p = min(static_cast<long long>(A.n_workers), max(1LL, T));
+  if (A.min_tiles > 0) p = min(p, max(1LL, T / A.min_tiles));
+  return static_cast<int>(p);
+}
+
+// ---------------------------------------------------------------- plan
+// prefix[b] = sum over earlier sequences of (tiles x hkv); prefix[B] = T.
+template <int D>
+__global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __restrict__ seqlens, int batch,
+                                                           int hq, int hkv, int cap, int window,
+                                                           int32_t* __restrict__ prefix,
+                                                           int32_t* __restrict__ counters,
+                                                           __nv_bfloat16* __restrict__ out, Epilogue epi) {
+  __shared__ int32_t warp_sums[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nthreads = blockDim.x;
+  const int per = (batch + nthreads - 1) / nthreads;
+  const int b0 = min(batch, tid * per), b1 = min(batch, b0 + per);
+  int32_t local = 0;
+  for (int b = b0; b < b1; ++b) local += tiles_of(clamp_len(seqlens[b], cap), window) * hkv;
+  int32_t incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t v = lane < (nthreads >> 5) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t u = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += u;
+    }
+    warp_sums[lane] = v;
+  }
+  __syncthreads();
+  int32_t base = (warp > 0 ? warp_sums[warp - 1] : 0) + incl - local;
+  for (int b = b0; b < b1; ++b) {
+    prefix[b] = base;
+    const int tb = tiles_of(clamp_len(seqlens[b], cap), window);
+    base += tb * hkv;
+    if (tb == 0) {
+      // a sequence with no key to attend: the epilogue of zeros (no worker
+      // sees it); rare, so one thread writes its rows
+      const __nv_bfloat16 zero_row = __float2bfloat16_rn(apply_epilogue(0.f, epi));
+      for (int i = 0; i < hq * D; ++i) out[static_cast<int64_t>(b) * hq * D + i] = zero_row;
+    }
+  }
+  if (tid == nthreads - 1) prefix[batch] = base;
+  for (int i = tid; i < batch * hkv; i += nthreads) counters[i] = 0;
+}
+
+// Position in the global tile sequence: sequence b, KV head g, tile t of Tb.
+struct Cursor {
+  int b, g, t, Tb;
+};
+
+__device__ __forceinline__ int seq_tiles(const SkArgs& A, int b) {
+  return (A.prefix[b + 1] - A.prefix[b]) / A.hkv;
+}
+__device__ __forceinline__ Cursor locate(const SkArgs& A, long long x) {
+  int lo = 0, hi = A.batch - 1;  // largest b with prefix[b] <= x
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (A.prefix[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  Cursor c;
+  c.b = lo;
+  c.Tb = seq_tiles(A, lo);
+  const long long y = x - A.prefix[lo];
+  c.g = static_cast<int>(y / c.Tb);
+  c.t = static_cast<int>(y % c.Tb);
+  return c;
+}
+__device__ __forceinline__ void advance(const SkArgs& A, Cursor& c) {
+  if (++c.t < c.Tb) return;
+  c.t = 0;
+  if (++c.g < A.hkv) return;
+  c.g = 0;
+  do {
+    ++c.b;
+  } while (c.b < A.batch && (c.Tb = seq_tiles(A, c.b)) == 0);
 }
 
 template <int D>
-__global__ void __launch_bounds__(kWarps * 32, 2)
-    decode_i8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                     const DecodeArgs A) {
+__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm)
+    decode_sk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const SkArgs A) {
   using G = Geom<D>;
   constexpr int kSteps = D / 16;      // k-steps of the S MMA
   constexpr int kChunks = D / 64;     // 16-byte chunks per thread per K row
@@ -129,20 +244,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kStages * G::kStageBytes);
   __shared__ int abort_flag;
 
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int L = max(0, min(A.seqlens[b], A.cap));
-  int k_lo, t_begin;
-  key_range(L, A.window, k_lo, t_begin);
-  const int key_begin = t_begin + split * A.split_keys;
-  if (key_begin >= L) return;
-  const int key_end = min(L, key_begin + A.split_keys);
-  const int n_tiles = (key_end - key_begin + kTile - 1) / kTile;
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, qq = lane & 3;
-  const int my_tiles = n_tiles > warp ? (n_tiles - warp + kWarps - 1) / kWarps : 0;
-  const int64_t kv_row0 = (static_cast<int64_t>(b) * A.hkv + g) * A.cap;
-
   if (threadIdx.x == 0) abort_flag = 0;
   if (lane == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[warp * kStages + s], 1);
@@ -150,10 +253,29 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   }
   __syncthreads();
 
+  const long long T = A.prefix[A.batch];
+  const long long P = effective_workers(A, T);
+  const long long w = static_cast<long long>(blockIdx.x) * kWarps + warp;
+  if (T == 0 || w >= P) return;
+  const long long t_first = worker_begin(w, T, P);
+  const int my_tiles = static_cast<int>(worker_begin(w + 1, T, P) - t_first);
+  if (my_tiles <= 0) return;
+
   auto stage_ptr = [&](int s) { return smem + (warp * kStages + s) * G::kStageBytes; };
-  auto issue = [&](int i) {  // tile i of this warp into stage i % kStages
+  auto tile_geom = [&](const Cursor& c, int& key0, int& k_lo, int& L, int64_t& kv_row0) {
+    L = clamp_len(A.seqlens[c.b], A.cap);
+    int t_begin;
+    key_range(L, A.window, k_lo, t_begin);
+    key0 = t_begin + c.t * kTile;
+    kv_row0 = (static_cast<int64_t>(c.b) * A.hkv + c.g) * A.cap;
+  };
+  // issue cursor (lane 0 runs it kStages tiles ahead of the compute cursor)
+  Cursor ic = locate(A, t_first);
+  auto issue = [&](int i) {
     const int s = i % kStages;
-    const int key0 = key_begin + (warp + i * kWarps) * kTile;
+    int key0, k_lo, L;
+    int64_t kv_row0;
+    tile_geom(ic, key0, k_lo, L, kv_row0);
     uint8_t* st = stage_ptr(s);
     uint64_t* bar = &bars[warp * kStages + s];
     mbar_expect_tx(bar, 2 * G::kTileBytes + 2 * kTile * 4);
@@ -161,15 +283,25 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     tma_load_2d(st + G::kTileBytes, &tm_v, bar, 0, static_cast<int>(kv_row0 + key0));
     bulk_load(st + G::kScaleOff, A.k_scales + kv_row0 + key0, kTile * 4, bar);
     bulk_load(st + G::kScaleOff + kTile * 4, A.v_scales + kv_row0 + key0, kTile * 4, bar);
+    advance(A, ic);
   };
   if (lane == 0) {
     for (int i = 0; i < min(kStages, my_tiles); ++i) issue(i);
   }
 
-  // ---- Q fragments: thread (gq, qq) holds head gq, dims [qq*D/4, (qq+1)*D/4)
+  // ---- per-segment state
   uint32_t qb0[kSteps], qb1[kSteps];
-  float qs_own = 0.f;
-  {
+  float qs0 = 0.f, qs1 = 0.f;
+  float o[kMT][4];
+  float m_run[2], l_run[2];
+  auto reset = [&]() {
+#pragma unroll
+    for (int m = 0; m < kMT; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+    m_run[0] = m_run[1] = -INFINITY;
+    l_run[0] = l_run[1] = 0.f;
+  };
+  // Q fragments: thread (gq, qq) holds head gq, dims [qq*D/4, (qq+1)*D/4)
+  auto load_q = [&](int b, int g) {
     float qv[D / 4];
     const bool head_ok = gq < A.group;
     const int hq_idx = b * A.hq + g * A.group + gq;
@@ -178,11 +310,11 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     for (int c = 0; c < D / 32; ++c) {
       uint4 raw = make_uint4(0, 0, 0, 0);
       if (head_ok) raw = *reinterpret_cast<const uint4*>(A.q + static_cast<int64_t>(hq_idx) * D + qq * (D / 4) + 8 * c);
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        qv[8 * c + 2 * e] = __uint_as_float(w[e] << 16);
-        qv[8 * c + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+        qv[8 * c + 2 * e] = __uint_as_float(wv[e] << 16);
+        qv[8 * c + 2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
       }
     }
 #pragma unroll
@@ -192,23 +324,127 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     int ex = 0;
     if (amax > 0.f) frexpf(amax, &ex);
     const int kexp = amax > 0.f ? 15 - ex : 0;  // largest |q| * 2^kexp in [2^14, 2^15)
-    qs_own = ldexpf(A.scale_log2, -kexp);
+    const float qs_own = ldexpf(A.scale_log2, -kexp);
 #pragma unroll
     for (int ks = 0; ks < kSteps; ++ks) {
       qb0[ks] = pack_f16x2(ldexpf(qv[4 * ks + 0], kexp), ldexpf(qv[4 * ks + 2], kexp));
       qb1[ks] = pack_f16x2(ldexpf(qv[4 * ks + 1], kexp), ldexpf(qv[4 * ks + 3], kexp));
     }
-  }
-  // logit multipliers of this thread's two score columns (heads 2qq, 2qq+1)
-  const float qs0 = __shfl_sync(0xffffffffu, qs_own, (2 * qq) * 4);
-  const float qs1 = __shfl_sync(0xffffffffu, qs_own, (2 * qq + 1) * 4);
-
-  float o[kMT][4];
+    // logit multipliers of this thread's two score columns (heads 2qq, 2qq+1)
+    qs0 = __shfl_sync(0xffffffffu, qs_own, (2 * qq) * 4);
+    qs1 = __shfl_sync(0xffffffffu, qs_own, (2 * qq + 1) * 4);
+  };
+  // partial state of segment `seg` -> record (seg + w)
+  auto finalize = [&](int seg) {
+    float l0 = l_run[0], l1 = l_run[1];
 #pragma unroll
-  for (int m = 0; m < kMT; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+    const int64_t rec = static_cast<int64_t>(seg) + w;
+    const int h0 = 2 * qq, h1 = 2 * qq + 1;
+    if (gq == 0) {
+      if (h0 < A.group) {
+        A.rec_ml[(rec * A.group + h0) * 2 + 0] = m_run[0];
+        A.rec_ml[(rec * A.group + h0) * 2 + 1] = l0;
+      }
+      if (h1 < A.group) {
+        A.rec_ml[(rec * A.group + h1) * 2 + 0] = m_run[1];
+        A.rec_ml[(rec * A.group + h1) * 2 + 1] = l1;
+      }
+    }
+#pragma unroll
+    for (int pr = 0; pr < D / 32; ++pr) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int dim0 = 4 * (8 * pr + gq) + 2 * j;
+        const float(&c)[4] = o[2 * pr + j];
+        if (h0 < A.group)
+          *reinterpret_cast<float2*>(A.rec_o + (rec * A.group + h0) * D + dim0) = make_float2(c[0], c[2]);
+        if (h1 < A.group)
+          *reinterpret_cast<float2*>(A.rec_o + (rec * A.group + h1) * D + dim0) = make_float2(c[1], c[3]);
+      }
+    }
+  };
 
+  // The last worker done with a segment merges every record of it.
+  auto segment_workers = [&](int seg, int& w_lo, int& w_hi) {
+    const int b = seg / A.hkv, g = seg % A.hkv;
+    const int Tb = seq_tiles(A, b);
+    const long long a = A.prefix[b] + static_cast<long long>(g) * Tb;
+    w_lo = worker_of(a, T, P);
+    w_hi = worker_of(a + Tb - 1, T, P);
+  };
+  auto finish = [&](int seg) {
+    finalize(seg);
+    __threadfence();  // each lane's record stores are visible device-wide ...
+    __syncwarp();     // ... before lane 0 counts the warp done
+    int prev = 0;
+    if (lane == 0) prev = atomicAdd(&A.counters[seg], 1);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    int w_lo, w_hi;
+    segment_workers(seg, w_lo, w_hi);
+    if (prev != w_hi - w_lo) return;
+    __threadfence();
+    const int b = seg / A.hkv, g = seg % A.hkv;
+    // one pass over the segment's records, all heads at once, online max
+    float M[8], lsum[8], acc[8][D / 32];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      M[h] = -INFINITY;
+      lsum[h] = 0.f;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) acc[h][j] = 0.f;
+    }
+    for (int v = w_lo; v <= w_hi; ++v) {
+      const int64_t r0 = (static_cast<int64_t>(seg) + v) * A.group;
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        if (h >= A.group) break;
+        const float m = __ldcg(&A.rec_ml[(r0 + h) * 2]);
+        const float lv = __ldcg(&A.rec_ml[(r0 + h) * 2 + 1]);
+        float ov[D / 32];
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) ov[j] = __ldcg(&A.rec_o[(r0 + h) * D + lane + 32 * j]);
+        const float mn = fmaxf(M[h], m);
+        const float ref = mn == -INFINITY ? 0.f : mn;
+        const float a_old = ex2_approx(M[h] - ref), a_new = ex2_approx(m - ref);
+        M[h] = mn;
+        lsum[h] = lsum[h] * a_old + lv * a_new;
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) acc[h][j] = acc[h][j] * a_old + ov[j] * a_new;
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      if (h >= A.group) break;
+      const float inv = lsum[h] > 0.f ? 1.f / lsum[h] : 0.f;
+      float y[D / 32];
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) y[j] = acc[h][j] * inv;
+      apply_epilogue_vec(y, A.epi);
+      __nv_bfloat16* orow = A.out + (static_cast<int64_t>(b) * A.hq + g * A.group + h) * D;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) orow[lane + 32 * j] = __float2bfloat16_rn(y[j]);
+    }
+  };
+
+  Cursor cc = locate(A, t_first);
+  int cur_seg = -1;
+  int seg_t_begin = 0, k_lo = 0, key_end = 0;
   for (int i = 0; i < my_tiles; ++i) {
+    const int seg = cc.b * A.hkv + cc.g;
+    if (seg != cur_seg) {
+      if (cur_seg >= 0) finish(cur_seg);
+      reset();
+      load_q(cc.b, cc.g);
+      cur_seg = seg;
+      key_end = clamp_len(A.seqlens[cc.b], A.cap);
+      key_range(key_end, A.window, k_lo, seg_t_begin);
+    }
+    const int key0 = seg_t_begin + cc.t * kTile;
+
     const int s = i % kStages;
     // every lane polls; the decision to continue is warp-uniform because the
     // MMAs and transposes below need the whole warp
@@ -218,7 +454,6 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     const uint32_t vt = kt + G::kTileBytes;
     const float* ksc = reinterpret_cast<const float*>(stage_ptr(s) + G::kScaleOff);
     const float* vsc = ksc + kTile;
-    const int key0 = key_begin + (warp + i * kWarps) * kTile;
 
     // ---- S^T = K . Q^T for the two 16-key halves of the tile
     float sc[2][4];
@@ -266,18 +501,25 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
     }
-    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
-    const float ref0 = mn0 == -INFINITY ? 0.f : mn0, ref1 = mn1 == -INFINITY ? 0.f : mn1;
-    const float al0 = ex2_approx(m_run[0] - ref0), al1 = ex2_approx(m_run[1] - ref1);
-    m_run[0] = mn0;
-    m_run[1] = mn1;
-    l_run[0] *= al0;
-    l_run[1] *= al1;
+    // the running maxima move only when a tile raises them, and the O
+    // rescale runs only when some head of the warp moved
+    const bool up0 = mx0 > m_run[0], up1 = mx1 > m_run[1];
+    if (__any_sync(0xffffffffu, up0 || up1)) {
+      const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+      const float r0 = mn0 == -INFINITY ? 0.f : mn0, r1 = mn1 == -INFINITY ? 0.f : mn1;
+      const float al0 = ex2_approx(m_run[0] - r0), al1 = ex2_approx(m_run[1] - r1);
+      m_run[0] = mn0;
+      m_run[1] = mn1;
+      l_run[0] *= al0;
+      l_run[1] *= al1;
 #pragma unroll
-    for (int m = 0; m < kMT; ++m) {
-      o[m][0] *= al0; o[m][2] *= al0;
-      o[m][1] *= al1; o[m][3] *= al1;
+      for (int m = 0; m < kMT; ++m) {
+        o[m][0] *= al0; o[m][2] *= al0;
+        o[m][1] *= al1; o[m][3] *= al1;
+      }
     }
+    const float ref0 = m_run[0] == -INFINITY ? 0.f : m_run[0];
+    const float ref1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
     uint32_t pb[2][2];  // [mt][b0/b1] P' operand fragments
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
@@ -323,86 +565,39 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       fence_proxy_async_smem();
       issue(i + kStages);
     }
+    advance(A, cc);
   }
-
-  // ---- merge the 4 warps' states; then one partial per (q-head, split)
-  l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], 4);
-  l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], 4);
-  l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], 8);
-  l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], 8);
-  l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], 16);
-  l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], 16);
-  __syncthreads();  // every warp is done with its stages (all issued tiles were waited on)
-  float* red_o = reinterpret_cast<float*>(smem);          // [warp][8 heads][D]
-  float* red_ml = red_o + kWarps * 8 * D;                  // [warp][8 heads][2]
-  if (gq == 0) {
-    red_ml[(warp * 8 + 2 * qq) * 2 + 0] = m_run[0];
-    red_ml[(warp * 8 + 2 * qq) * 2 + 1] = l_run[0];
-    red_ml[(warp * 8 + 2 * qq + 1) * 2 + 0] = m_run[1];
-    red_ml[(warp * 8 + 2 * qq + 1) * 2 + 1] = l_run[1];
-  }
-#pragma unroll
-  for (int pr = 0; pr < D / 32; ++pr) {
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int dim0 = 4 * (8 * pr + gq) + 2 * j;
-      const float(&c)[4] = o[2 * pr + j];
-      red_o[(warp * 8 + 2 * qq) * D + dim0] = c[0];
-      red_o[(warp * 8 + 2 * qq + 1) * D + dim0] = c[1];
-      red_o[(warp * 8 + 2 * qq) * D + dim0 + 1] = c[2];
-      red_o[(warp * 8 + 2 * qq + 1) * D + dim0 + 1] = c[3];
-    }
-  }
-  __syncthreads();
-  const int active_warps = min(kWarps, n_tiles);
-  for (int e = threadIdx.x; e < A.group * D; e += kWarps * 32) {
-    const int h = e / D, dim = e % D;
-    float M = -INFINITY;
-    for (int w = 0; w < active_warps; ++w) M = fmaxf(M, red_ml[(w * 8 + h) * 2]);
-    const float ref = M == -INFINITY ? 0.f : M;
-    float acc = 0.f, lsum = 0.f;
-    for (int w = 0; w < active_warps; ++w) {
-      const float f = ex2_approx(red_ml[(w * 8 + h) * 2] - ref);
-      acc += f * red_o[(w * 8 + h) * D + dim];
-      lsum += f * red_ml[(w * 8 + h) * 2 + 1];
-    }
-    const int64_t rec = (static_cast<int64_t>(b) * A.hq + g * A.group + h) * A.n_split_max + split;
-    A.part_o[rec * D + dim] = acc;
-    if (dim == 0) {
-      A.part_ml[rec * 2 + 0] = M;
-      A.part_ml[rec * 2 + 1] = lsum;
-    }
-  }
+  if (cur_seg >= 0) finish(cur_seg);
 }
 
-// One CTA per (sequence, q-head): log-sum-exp merge of the split partials.
-template <int D>
-__global__ void __launch_bounds__(128)
-    decode_merge_kernel(const DecodeArgs A, __nv_bfloat16* __restrict__ out, Epilogue epi) {
-  const int bh = blockIdx.x;
-  const int b = bh / A.hq;
-  const int L = max(0, min(A.seqlens[b], A.cap));
-  int k_lo, t_begin;
-  key_range(L, A.window, k_lo, t_begin);
-  const int n_split = min(A.n_split_launched, L > t_begin ? (L - t_begin + A.split_keys - 1) / A.split_keys : 0);
-  const int64_t rec0 = static_cast<int64_t>(bh) * A.n_split_max;
-  float M = -INFINITY;
-  for (int s = 0; s < n_split; ++s) M = fmaxf(M, A.part_ml[(rec0 + s) * 2]);
-  const float ref = M == -INFINITY ? 0.f : M;
-  for (int dim = threadIdx.x; dim < D; dim += blockDim.x) {
-    float acc = 0.f, lsum = 0.f;
-    for (int s = 0; s < n_split; ++s) {
-      const float f = ex2_approx(A.part_ml[(rec0 + s) * 2] - ref);
-      acc += f * A.part_o[(rec0 + s) * D + dim];
-      lsum += f * A.part_ml[(rec0 + s) * 2 + 1];
-    }
-    const float y = lsum > 0.f ? acc / lsum : 0.f;
-    out[static_cast<int64_t>(bh) * D + dim] = __float2bfloat16_rn(apply_epilogue(y, epi));
+// SMs of the current device (cached per device).
+int sm_count() {
+  static std::mutex mu;
+  static int counts[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lk(mu);
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    counts[dev] = n;
   }
+  return counts[dev];
 }
 
+// plan (prefix [B+1]) and counters [B*hkv <= B*hq], 256-byte padded
+size_t plan_bytes(int batch, int hq) {
+  return (static_cast<size_t>(batch + 1 + static_cast<size_t>(batch) * hq) * sizeof(int32_t) + 255) / 256 * 256;
+}
+size_t records_bytes(int batch, int hq, int hkv, int d, int n_workers) {
+  const size_t recs = static_cast<size_t>(batch) * hkv + n_workers;
+  return recs * (hq / hkv) * (static_cast<size_t>(d) + 2) * sizeof(float);
+}
+
+// Launch plan + stream-K kernel + merge into `ws` (plan, then records).
 template <int D>
-fa_status launch_decode_i8(const fa_decode_params& p, int split_keys, int n_splits, const LaunchCtx& ctx) {
+fa_status launch_sk(const fa_decode_params& p, int n_workers, int min_tiles, void* ws, bool count_variants,
+                    const LaunchCtx& ctx) {
   using G = Geom<D>;
   const uint64_t rows = static_cast<uint64_t>(p.batch) * p.hkv * p.capacity;
   CUtensorMap tmk, tmv;
@@ -415,47 +610,66 @@ fa_status launch_decode_i8(const fa_decode_params& p, int split_keys, int n_spli
   st = encode_tensor_map(&tmv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p.v_cache, dims, strides, box, sw);
   if (st != FA_OK) return st;
 
-  const int n_split_max = (p.capacity + 255) / 256;
-  const size_t o_bytes = static_cast<size_t>(p.batch) * p.hq * n_split_max * D * sizeof(float);
-  DecodeArgs A;
+  const int group = p.hq / p.hkv;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  SkArgs A;
   A.q = static_cast<const __nv_bfloat16*>(p.q);
   A.k_scales = p.k_scales;
   A.v_scales = p.v_scales;
   A.seqlens = p.cache_seqlens;
-  A.part_o = static_cast<float*>(p.workspace);
-  A.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(p.workspace) + o_bytes);
+  A.prefix = reinterpret_cast<int32_t*>(base);
+  A.counters = reinterpret_cast<int32_t*>(base) + (p.batch + 1);
+  A.out = static_cast<__nv_bfloat16*>(p.out);
+  A.epi = make_epilogue(p.epilogue, p.n_epilogue);
+  const size_t o_recs = static_cast<size_t>(p.batch * p.hkv + n_workers) * group;
+  A.rec_o = reinterpret_cast<float*>(base + plan_bytes(p.batch, p.hq));
+  A.rec_ml = A.rec_o + o_recs * D;
+  A.batch = p.batch;
   A.hq = p.hq;
   A.hkv = p.hkv;
-  A.group = p.hq / p.hkv;
+  A.group = group;
   A.cap = p.capacity;
   A.window = p.window;
-  A.split_keys = split_keys;
-  A.n_split_max = n_split_max;
-  A.n_split_launched = n_splits;
+  A.n_workers = n_workers;
+  A.min_tiles = min_tiles;
   A.scale_log2 = p.softmax_scale * kLog2e;
   A.wd = ctx.wd;
 
-  auto kern = decode_i8_kernel<D>;
+  auto plan = decode_plan_kernel<D>;
+  auto kern = decode_sk_kernel<D>;
+  if (count_variants) {
+    note_variant(reinterpret_cast<const void*>(plan));
+    note_variant(reinterpret_cast<const void*>(kern));
+  }
+  plan<<<1, 1024, 0, ctx.stream>>>(p.cache_seqlens, p.batch, p.hq, p.hkv, p.capacity, p.window,
+                                   reinterpret_cast<int32_t*>(base), A.counters, A.out, A.epi);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem) != cudaSuccess)
     return FA_ERR_CUDA;
-  note_variant(reinterpret_cast<const void*>(kern));
-  dim3 grid(n_splits, p.hkv, p.batch);
-  kern<<<grid, kWarps * 32, G::kSmem, ctx.stream>>>(tmk, tmv, A);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-
-  auto merge = decode_merge_kernel<D>;
-  note_variant(reinterpret_cast<const void*>(merge));
-  merge<<<p.batch * p.hq, 128, 0, ctx.stream>>>(A, static_cast<__nv_bfloat16*>(p.out),
-                                                make_epilogue(p.epilogue, p.n_epilogue));
+  kern<<<n_workers / kWarps, kWarps * 32, G::kSmem, ctx.stream>>>(tmk, tmv, A);
   return cuda_status(cudaGetLastError());
 }
 
+int default_workers() { return min(kMaxWorkers, sm_count() * kCtasPerSm * kWarps); }
+
+int min_tiles_of(int split_keys) { return split_keys > 0 ? split_keys / kTile : 0; }
+
 }  // namespace
 
-fa_status launch_decode(const fa_decode_params& p, int split_keys, int n_splits, const LaunchCtx& ctx) {
+size_t decode_workspace_bytes(int batch, int hq, int head_dim) {
+  // hkv is not known here: bound the group by min(hq, 8) (the kernel's
+  // limit), which covers every (hkv, group) split of hq
+  const size_t g = static_cast<size_t>(hq < 8 ? hq : 8);
+  const size_t workers = static_cast<size_t>(default_workers());
+  return plan_bytes(batch, hq) +
+         (static_cast<size_t>(batch) * hq + workers * g) * (static_cast<size_t>(head_dim) + 2) * sizeof(float);
+}
+
+fa_status launch_decode(const fa_decode_params& p, int split_keys, const LaunchCtx& ctx) {
   if (p.kv_dtype != FA_I8) return FA_ERR_UNSUPPORTED;
-  if (p.head_dim == 128) return launch_decode_i8<128>(p, split_keys, n_splits, ctx);
-  if (p.head_dim == 64) return launch_decode_i8<64>(p, split_keys, n_splits, ctx);
+  const int workers = default_workers();
+  if (p.head_dim == 128) return launch_sk<128>(p, workers, min_tiles_of(split_keys), p.workspace, true, ctx);
+  if (p.head_dim == 64) return launch_sk<64>(p, workers, min_tiles_of(split_keys), p.workspace, true, ctx);
   return FA_ERR_UNSUPPORTED;
 }
 
@@ -468,14 +682,14 @@ fa_status launch_decode(const fa_decode_params& p, int split_keys, int n_splits,
 // a plug-in inside a serving runtime that owns every device byte through its
 // own pre-planned arena and forbids allocations outside it, or a caller that
 // must not risk the implicit device synchronisation a cudaMalloc can cause --
-// the per-split partials (O, m, l) live in this file-scope device array
-// instead of a caller workspace.  Every device that loads the library holds
-// it until the process exits.  All calls on a device share it and it keeps
-// the last call's contents; nothing in it needs clearing, because the merge
-// only reads records that the same call's split kernel wrote.  Calls whose
-// work overlaps on the GPU (different streams, or different host threads on
-// the same device) race on the array and must be serialised by the caller.
-#include <mutex>
+// the plan and the per-worker partials (O, m, l) live in this file-scope
+// device array instead of a caller workspace.  Every device that loads the
+// library holds it until the process exits.  All calls on a device share it
+// and it keeps the last call's contents; nothing in it needs clearing,
+// because each call writes its plan first and the merge only reads records
+// that the same call's workers wrote.  Calls whose work overlaps on the GPU
+// (different streams, or different host threads on the same device) race on
+// the array and must be serialised by the caller.
 
 namespace fa {
 namespace {
@@ -510,80 +724,35 @@ fa_status noalloc_scratch(void** scratch, unsigned int** status) {
   return FA_OK;
 }
 
-template <int D>
-fa_status launch_decode_i8_noalloc(const fa_decode_params& p, int split_keys, int n_splits, void* scratch,
-                                   const LaunchCtx& ctx) {
-  using G = Geom<D>;
-  const uint64_t rows = static_cast<uint64_t>(p.batch) * p.hkv * p.capacity;
-  CUtensorMap tmk, tmv;
-  const uint64_t dims[2] = {static_cast<uint64_t>(D), rows};
-  const uint64_t strides[1] = {static_cast<uint64_t>(D)};
-  const uint32_t box[2] = {static_cast<uint32_t>(D), static_cast<uint32_t>(kTile)};
-  const CUtensorMapSwizzle sw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  fa_status st = encode_tensor_map(&tmk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p.k_cache, dims, strides, box, sw);
-  if (st != FA_OK) return st;
-  st = encode_tensor_map(&tmv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p.v_cache, dims, strides, box, sw);
-  if (st != FA_OK) return st;
-
-  // partial records are packed with a stride of the launched split count
-  const size_t o_bytes = static_cast<size_t>(p.batch) * p.hq * n_splits * D * sizeof(float);
-  DecodeArgs A;
-  A.q = static_cast<const __nv_bfloat16*>(p.q);
-  A.k_scales = p.k_scales;
-  A.v_scales = p.v_scales;
-  A.seqlens = p.cache_seqlens;
-  A.part_o = static_cast<float*>(scratch);
-  A.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + o_bytes);
-  A.hq = p.hq;
-  A.hkv = p.hkv;
-  A.group = p.hq / p.hkv;
-  A.cap = p.capacity;
-  A.window = p.window;
-  A.split_keys = split_keys;
-  A.n_split_max = n_splits;
-  A.n_split_launched = n_splits;
-  A.scale_log2 = p.softmax_scale * kLog2e;
-  A.wd = ctx.wd;
-
-  auto kern = decode_i8_kernel<D>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem) != cudaSuccess)
-    return FA_ERR_CUDA;
-  // (no note_variant here: its bookkeeping set may allocate host memory)
-  dim3 grid(n_splits, p.hkv, p.batch);
-  kern<<<grid, kWarps * 32, G::kSmem, ctx.stream>>>(tmk, tmv, A);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  auto merge = decode_merge_kernel<D>;
-  merge<<<p.batch * p.hq, 128, 0, ctx.stream>>>(A, static_cast<__nv_bfloat16*>(p.out),
-                                                make_epilogue(p.epilogue, p.n_epilogue));
-  return cuda_status(cudaGetLastError());
-}
-
 }  // namespace
 
 size_t decode_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
+// Workers that fit the scratch: plan + (B*hkv + P) * G * (d + 2) floats;
+// 0 when not even one CTA of workers fits.
+int decode_noalloc_workers(int batch, int hq, int hkv, int head_dim) {
+  const size_t fixed = plan_bytes(batch, hq) + records_bytes(batch, hq, hkv, head_dim, 0);
+  if (fixed >= kNoAllocScratchBytes) return 0;
+  const size_t per_worker = static_cast<size_t>(hq / hkv) * (head_dim + 2) * sizeof(float);
+  const size_t fit = (kNoAllocScratchBytes - fixed) / per_worker;
+  int w = static_cast<int>(fit < static_cast<size_t>(kMaxWorkers) ? fit : kMaxWorkers);
+  w = min(w, default_workers());
+  return (w / kWarps) * kWarps;
+}
+
 fa_status launch_decode_noalloc(const fa_decode_params& p, int split_keys, long long budget, cudaStream_t stream) {
   if (p.kv_dtype != FA_I8) return FA_ERR_UNSUPPORTED;
-  const int max_len = p.max_seqlen > 0 ? p.max_seqlen : p.capacity;
-  const size_t per_split = static_cast<size_t>(p.batch) * p.hq * (p.head_dim + 2) * sizeof(float);
-  if (per_split > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;  // even one split does not fit
-  const int fit = static_cast<int>(kNoAllocScratchBytes / per_split);
-  int n_splits = max_len > 0 ? (max_len + split_keys - 1) / split_keys : 1;
-  if (n_splits > fit) {
-    if (p.split_keys > 0) return FA_ERR_WORKSPACE;  // the caller's split count does not fit
-    split_keys = ((max_len + fit - 1) / fit + 255) / 256 * 256;
-    n_splits = (max_len + split_keys - 1) / split_keys;
-    if (n_splits > fit) return FA_ERR_WORKSPACE;
-  }
-  if (n_splits < 1) n_splits = 1;
+  const int workers = decode_noalloc_workers(p.batch, p.hq, p.hkv, p.head_dim);
+  if (workers < kWarps) return FA_ERR_WORKSPACE;
   void* scratch = nullptr;
   LaunchCtx ctx;
   ctx.stream = stream;
   ctx.wd.budget = budget;
   fa_status st = noalloc_scratch(&scratch, &ctx.wd.word);
   if (st != FA_OK) return st;
-  if (p.head_dim == 128) return launch_decode_i8_noalloc<128>(p, split_keys, n_splits, scratch, ctx);
-  if (p.head_dim == 64) return launch_decode_i8_noalloc<64>(p, split_keys, n_splits, scratch, ctx);
+  // (no note_variant here: its bookkeeping set may allocate host memory)
+  if (p.head_dim == 128) return launch_sk<128>(p, workers, min_tiles_of(split_keys), scratch, false, ctx);
+  if (p.head_dim == 64) return launch_sk<64>(p, workers, min_tiles_of(split_keys), scratch, false, ctx);
   return FA_ERR_UNSUPPORTED;
 }
 

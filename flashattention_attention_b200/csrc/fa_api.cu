@@ -196,10 +196,7 @@ fa_status fa_attention_fwd(const fa_fwd_params* p, fa_stream_t stream) {
 
 size_t fa_decode_workspace_size(int32_t batch, int32_t hq, int32_t capacity, int32_t head_dim) {
   if (batch <= 0 || hq <= 0 || capacity <= 0 || head_dim <= 0) return 0;
-  const size_t n_split_max = (static_cast<size_t>(capacity) + 255) / 256;
-  const size_t recs = static_cast<size_t>(batch) * hq * n_split_max;
-  const size_t o_bytes = recs * head_dim * sizeof(float);
-  return o_bytes + recs * 2 * sizeof(float);
+  return decode_workspace_bytes(batch, hq, head_dim);
 }
 
 fa_status fa_attention_decode(const fa_decode_params* p, fa_stream_t stream) {
@@ -226,28 +223,10 @@ fa_status fa_attention_decode(const fa_decode_params* p, fa_stream_t stream) {
   }
   const size_t need = fa_decode_workspace_size(p->batch, p->hq, p->capacity, p->head_dim);
   if (p->workspace == nullptr || p->workspace_bytes < need || !aligned16(p->workspace)) return FA_ERR_WORKSPACE;
-
-  const int max_len = p->max_seqlen > 0 ? p->max_seqlen : p->capacity;
-  int split = p->split_keys;
-  if (split == 0) {
-    // Aim for about four CTAs per SM slot over the (sequence, kv-head) pairs.
-    const long long pairs = static_cast<long long>(p->batch) * p->hkv;
-    const long long want_units = 148LL * 2 * 4;
-    long long per = (static_cast<long long>(max_len) * pairs + want_units - 1) / want_units;
-    per = ((per + 255) / 256) * 256;
-    if (per < 256) per = 256;
-    if (per > 4096) per = 4096;
-    split = static_cast<int>(per);
-  }
-  const int n_splits = (max_len + split - 1) / split;
   LaunchCtx ctx;
   fa_status st = make_ctx(stream, &ctx);
   if (st != FA_OK) return st;
-  if (n_splits == 0) {
-    // every cache is empty: the merge alone writes the epilogue of zeros
-    return launch_decode(*p, split, 1, ctx);
-  }
-  return launch_decode(*p, split, n_splits, ctx);
+  return launch_decode(*p, p->split_keys, ctx);
 }
 
 fa_status fa_attention_decode_noalloc(const fa_decode_params* p, fa_stream_t stream) {
@@ -270,19 +249,8 @@ fa_status fa_attention_decode_noalloc(const fa_decode_params* p, fa_stream_t str
   if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->out) ||
       !aligned16(p->k_scales) || !aligned16(p->v_scales))
     return FA_ERR_INVALID;
-  const size_t per_split = static_cast<size_t>(p->batch) * p->hq * (p->head_dim + 2) * sizeof(float);
-  if (per_split > decode_noalloc_scratch_bytes()) return FA_ERR_WORKSPACE;
-  const int max_len = p->max_seqlen > 0 ? p->max_seqlen : p->capacity;
-  int split = p->split_keys;
-  if (split == 0) {
-    const long long pairs = static_cast<long long>(p->batch) * p->hkv;
-    const long long want_units = 148LL * 2 * 4;
-    long long per = (static_cast<long long>(max_len) * pairs + want_units - 1) / want_units;
-    per = ((per + 255) / 256) * 256;
-    if (per < 256) per = 256;
-    if (per > 4096) per = 4096;
-    split = static_cast<int>(per);
-  }
+  if (decode_noalloc_workers(p->batch, p->hq, p->hkv, p->head_dim) < 4) return FA_ERR_WORKSPACE;
+  const int split = p->split_keys;
   return launch_decode_noalloc(*p, split, watchdog_budget(), reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -150,13 +150,16 @@ FA_API fa_status fa_attention_fwd(const fa_fwd_params *p, fa_stream_t stream);
  *   out      [batch*hq, d] bf16
  * The query sits at position L_b - 1, so every cached key is visible; a
  * window W > 0 keeps the last W.  L_b = 0 gives the epilogue applied to zeros.
- * Work is split along the keys; per-split (m, l, O) partials go to the
- * caller's workspace (>= fa_decode_workspace_size bytes, 16-byte aligned,
- * contents need no initialisation) and a merge kernel combines them.
- * max_seqlen: host-side upper bound of the L_b (0 means capacity);
- * split_keys: keys per split (a multiple of 256), chosen by the library
- * when 0.  capacity must be a multiple of 32; cache entries at or past L_b
- * may hold any bytes (they never reach the result).
+ * Work is split along the keys: the 32-key tiles of all (sequence, KV head)
+ * pairs are divided evenly among a persistent grid of warps, each of which
+ * writes one partial (m, l, O) per pair it touches to the caller's workspace
+ * (>= fa_decode_workspace_size bytes, 16-byte aligned, contents need no
+ * initialisation); a merge kernel combines them.
+ * max_seqlen: host-side upper bound of the L_b (0 means capacity; checked
+ * against capacity only).  split_keys: 0, or a multiple of 256 -- the fewest
+ * keys each warp is given (fewer, longer ranges).  capacity must be a
+ * multiple of 32; cache entries at or past L_b may hold any bytes (they never
+ * reach the result).
  * Supported: head_dim 128 (FA_I8 and FA_BF16) or 64; hq / hkv <= 8.
  */
 typedef struct {
@@ -179,7 +182,8 @@ typedef struct {
     size_t workspace_bytes;
 } fa_decode_params;
 
-/* Bytes of decode workspace for any split choice at these sizes. */
+/* Bytes of decode workspace at these sizes (any hkv dividing hq with
+ * hq / hkv <= 8; the count of SMs of the current device enters it). */
 FA_API size_t fa_decode_workspace_size(int32_t batch, int32_t hq, int32_t capacity, int32_t head_dim);
 
 FA_API fa_status fa_attention_decode(const fa_decode_params *p, fa_stream_t stream);
@@ -198,12 +202,13 @@ FA_API fa_status fa_attention_decode(const fa_decode_params *p, fa_stream_t stre
  * the library, which every device that loads the library holds until the
  * process exits.  The call allocates nothing (no cudaMalloc, no library
  * allocator).
- *   - Limit: batch * hq * (head_dim + 2) * 4 bytes per key split must fit in
- *     the scratch for the number of splits used.  With split_keys == 0 the
- *     library picks a split large enough to fit; a problem for which even
- *     one split does not fit (batch * hq * (head_dim + 2) * 4 > 8 MiB), or a
- *     caller-chosen split_keys that does not fit, returns FA_ERR_WORKSPACE
- *     and enqueues nothing.  Only the int8 cache (FA_I8) is supported.
+ *   - Limit: the scratch holds the per-sequence tile plan ((batch + 1) * 4
+ *     bytes), one partial record per (sequence, KV head) and one per worker
+ *     warp, each hq / hkv * (head_dim + 2) * 4 bytes.  The library uses as
+ *     many workers as fit (up to its usual count); a problem where
+ *     batch * hq * (head_dim + 2) * 4 bytes leave no room for one CTA of 4
+ *     workers returns FA_ERR_WORKSPACE and enqueues nothing.  Only the int8
+ *     cache (FA_I8) is supported.
  *   - The first call on each device looks up the scratch array's device
  *     address (with that device current); make that first call before any
  *     stream capture.

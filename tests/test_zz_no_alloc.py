@@ -74,7 +74,8 @@ def test_noalloc_matches_decode_on_two_calls_in_a_row():
 
 def test_noalloc_rejects_problems_beyond_the_scratch():
     from flashattention_attention_b200 import fa
-    # one split needs batch * hq * (128 + 2) * 4 bytes: 2048 * 8 * 520 > 8 MiB
+    # one record per (sequence, q-head) needs batch * hq * (128 + 2) * 4 bytes:
+    # 2048 * 8 * 520 > 8 MiB leaves no room for the workers' records
     q = torch.empty(16, dtype=torch.bfloat16, device="cuda")
     p = fa.DecodeParams()
     p.q = p.k_cache = p.v_cache = p.out = q.data_ptr()
@@ -82,6 +83,6 @@ def test_noalloc_rejects_problems_beyond_the_scratch():
     p.kv_dtype, p.batch, p.hq, p.hkv, p.head_dim, p.capacity = fa.FA_I8, 2048, 8, 8, 128, 256
     p.softmax_scale = 0.088
     assert fa.lib.fa_attention_decode_noalloc(ctypes.byref(p), None) == fa.FA_ERR_WORKSPACE
-    # a caller-fixed split count that cannot fit is rejected too
-    p.batch, p.hq, p.hkv, p.capacity, p.max_seqlen, p.split_keys = 64, 64, 8, 65536, 65536, 256
+    # the same with grouped heads: 256 sequences x 64 q-heads
+    p.batch, p.hq, p.hkv, p.capacity = 256, 64, 8, 1024
     assert fa.lib.fa_attention_decode_noalloc(ctypes.byref(p), None) == fa.FA_ERR_WORKSPACE
