@@ -59,17 +59,20 @@ constexpr uint32_t kChunkBytes = kSwizzleChunkRows * 128;  // [128 rows x 64 bf1
 
 template <int D, bool kI8>
 struct TcGeom {
-  static constexpr int kStages = (D == 128) ? 2 : 3;
+  // K is consumed one step before V (S(j) precedes PV(j)), so K gets the
+  // deeper ring: a slot refills with the TMA latency hidden behind ~2 steps
+  static constexpr int kKStages = 3;
+  static constexpr int kVStages = (D == 128) ? 2 : 3;
   static constexpr uint32_t kQBytes = kBM * D * 2;
   static constexpr uint32_t kKVBytes = kBN * D * 2;   // one bf16 K or V tile
   static constexpr uint32_t kI8Bytes = kBN * D;       // one int8 tile
   static constexpr uint32_t kKOff = 2 * kQBytes;
-  static constexpr uint32_t kVOff = kKOff + kStages * kKVBytes;
+  static constexpr uint32_t kVOff = kKOff + kKStages * kKVBytes;
   // int8 staging: at d = 128 in the upper half of each bf16 slot (a row's
   // bf16 output overwrites only that row's int8 bytes); at d = 64 separate
   static constexpr bool kInPlace = (D == 128);
-  static constexpr uint32_t kStageOff = kVOff + kStages * kKVBytes;
-  static constexpr uint32_t kStageBytes = (kI8 && !kInPlace) ? 2 * kStages * kI8Bytes : 0;
+  static constexpr uint32_t kStageOff = kVOff + kVStages * kKVBytes;
+  static constexpr uint32_t kStageBytes = (kI8 && !kInPlace) ? (kKStages + kVStages) * kI8Bytes : 0;
   static constexpr uint32_t kBarOff = kStageOff + kStageBytes;
   static constexpr uint32_t kSmem = kBarOff + 256 + 1024;
   static constexpr int kThreads = kI8 ? 512 : 320;
@@ -77,9 +80,12 @@ struct TcGeom {
     return kInPlace ? kKOff + s * kKVBytes + kKVBytes / 2 : kStageOff + s * kI8Bytes;
   }
   __host__ __device__ static constexpr uint32_t v_stage(int s) {
-    return kInPlace ? kVOff + s * kKVBytes + kKVBytes / 2 : kStageOff + (kStages + s) * kI8Bytes;
+    return kInPlace ? kVOff + s * kKVBytes + kKVBytes / 2 : kStageOff + (kKStages + s) * kI8Bytes;
   }
 };
+static_assert(TcGeom<128, false>::kSmem <= 232448, "shared memory budget");
+static_assert(TcGeom<128, true>::kSmem <= 232448, "shared memory budget");
+static_assert(TcGeom<64, true>::kSmem <= 232448, "shared memory budget");
 
 struct PrefillArgs {
   SeqLayout L;
@@ -133,23 +139,23 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const PrefillArgs A) {
   using G = TcGeom<D, kI8>;
-  constexpr int S = G::kStages;
+  constexpr int KS = G::kKStages, VS = G::kVStages;
   extern __shared__ uint8_t tc_smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G::kBarOff);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + S;
-  uint64_t* v_full = k_empty + S;
-  uint64_t* v_empty = v_full + S;
-  uint64_t* s_full = v_empty + S;  // [2]
-  uint64_t* p_full = s_full + 2;   // [2]
-  uint64_t* o_done = p_full + 2;   // [2]
+  uint64_t* k_empty = k_full + KS;
+  uint64_t* v_full = k_empty + KS;
+  uint64_t* v_empty = v_full + VS;
+  uint64_t* s_full = v_empty + VS;  // [2]
+  uint64_t* p_full = s_full + 2;   // [2 tiles][2 halves of the keys]
+  uint64_t* o_done = p_full + 4;   // [2]
   uint64_t* drain = o_done + 2;
-  uint64_t* kraw_full = drain + 1;   // [S] int8 variant: TMA landed the int8 K tile
-  uint64_t* vraw_full = kraw_full + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(vraw_full + S);
+  uint64_t* kraw_full = drain + 1;   // [KS] int8 variant: TMA landed the int8 K tile
+  uint64_t* vraw_full = kraw_full + KS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(vraw_full + VS);
   __shared__ int abort_flag;
 
   // ---- work tile: longest (highest q-block) first, then sequence, then head pair
@@ -186,18 +192,21 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(q_full, 1);
-    for (int s = 0; s < S; ++s) {
-      // bf16: TMA completes k_full / v_full; int8: the 128 converter threads do
+    // bf16: TMA completes k_full / v_full; int8: the 128 converter threads do
+    for (int s = 0; s < KS; ++s) {
       mbar_init(k_full + s, kI8 ? 128 : 1);
       mbar_init(k_empty + s, 1);
+      mbar_init(kraw_full + s, 1);
+    }
+    for (int s = 0; s < VS; ++s) {
       mbar_init(v_full + s, kI8 ? 128 : 1);
       mbar_init(v_empty + s, 1);
-      mbar_init(kraw_full + s, 1);
       mbar_init(vraw_full + s, 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full + t, 1);
-      mbar_init(p_full + t, kBM);
+      mbar_init(p_full + 2 * t, kBM);
+      mbar_init(p_full + 2 * t + 1, kBM);
       mbar_init(o_done + t, 1);
     }
     mbar_init(drain, 1);
@@ -228,7 +237,7 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(smem + t * G::kQBytes + c * kChunkBytes, &tm_q, q_full, 64 * c, q_prow, q_plane + t);
       for (int it = 0; it < n_iter; ++it) {
-        const int s = it % S, u = it / S;
+        int s = it % KS, u = it / KS;
         const int krow = k_prow0 + (j_lo + it) * kBN;
         if (u > 0 && !wait_parity(k_empty + s, (u - 1) & 1, A.wd, &abort_flag)) break;
         if constexpr (kI8) {
@@ -240,6 +249,8 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
             tma_load_3d(smem + G::kKOff + s * G::kKVBytes + c * kChunkBytes, &tm_k, k_full + s, 64 * c, krow,
                         k_plane);
         }
+        s = it % VS;
+        u = it / VS;
         if (u > 0 && !wait_parity(v_empty + s, (u - 1) & 1, A.wd, &abort_flag)) break;
         if constexpr (kI8) {
           mbar_expect_tx(vraw_full + s, G::kI8Bytes);
@@ -260,37 +271,50 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       const uint32_t idesc_s = umma_idesc_f16(kBM, kBN, 1, 1, false) | (A.negate_s << 13);
       constexpr uint32_t idesc_o = umma_idesc_f16(kBM, D, 1, 1, true);
       const uint32_t q_base = smem_u32(smem);
-      auto issue_s = [&](int t, int s) {
-        const uint32_t qa = q_base + t * G::kQBytes;
-        const uint32_t kb = q_base + G::kKOff + s * G::kKVBytes;
+      // operand descriptors are built once; a k-step only moves the start
+      // address (its 14-bit field never carries: every address is < 2^18)
+      const uint64_t dq0 = umma_desc_sw128(q_base, 16, 1024);
+      const uint64_t dk0 = umma_desc_sw128(q_base + G::kKOff, 16, 1024);
+      const uint64_t dv0 = umma_desc_sw128(q_base + G::kVOff, kChunkBytes, 1024);
+      auto issue_s = [&](int t, int st) {
+        const uint64_t dq = dq0 + ((t * G::kQBytes) >> 4);
+        const uint64_t dk = dk0 + ((st * G::kKVBytes) >> 4);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k / 4) * kChunkBytes + (k % 4) * 32;
-          mma_ss(tmem + t * kBN, umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
-                 idesc_s, k > 0 ? 1u : 0u);
+          const uint32_t off = ((k / 4) * kChunkBytes + (k % 4) * 32) >> 4;
+          mma_ss(tmem + t * kBN, dq + off, dk + off, idesc_s, k > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int s, bool accumulate) {
-        const uint32_t vb = q_base + G::kVOff + s * G::kKVBytes;
+      // O_t += P_t V over keys [64 h, 64 h + 64)
+      auto issue_pv_half = [&](int t, int st, int h, bool accumulate) {
+        const uint64_t dv = dv0 + ((st * G::kKVBytes) >> 4);
 #pragma unroll
-        for (int k = 0; k < kBN / 16; ++k) {
-          mma_ts(tmem + 256 + t * D, tmem + t * kBN + k * 8, umma_desc_sw128(vb + k * 2048, kChunkBytes, 1024),
-                 idesc_o, (accumulate || k > 0) ? 1u : 0u);
+        for (int k = 4 * h; k < 4 * h + 4; ++k) {
+          mma_ts(tmem + 256 + t * D, tmem + t * kBN + k * 8, dv + ((k * 2048) >> 4), idesc_o,
+                 (accumulate || k > 0) ? 1u : 0u);
         }
+      };
+      // PV for step `j` of tile t, each half as soon as the softmax wrote it
+      auto issue_pv = [&](int t, int j) -> bool {
+        const int vs = j % VS;
+        if (!wait_parity(p_full + 2 * t, j & 1, A.wd, &abort_flag)) return false;
+        if (t == 0 && !wait_parity(v_full + vs, (j / VS) & 1, A.wd, &abort_flag)) return false;
+        tc_fence_after();
+        issue_pv_half(t, vs, 0, j > 0);
+        if (!wait_parity(p_full + 2 * t + 1, j & 1, A.wd, &abort_flag)) return false;
+        tc_fence_after();
+        issue_pv_half(t, vs, 1, true);
+        return true;
       };
       bool ok = wait_parity(q_full, 0, A.wd, &abort_flag);
       for (int it = 0; ok && it < n_iter; ++it) {
-        const int s = it % S;
-        if (!(ok = wait_parity(k_full + s, (it / S) & 1, A.wd, &abort_flag))) break;
+        const int s = it % KS;
+        if (!(ok = wait_parity(k_full + s, (it / KS) & 1, A.wd, &abort_flag))) break;
         tc_fence_after();
         for (int t = 0; t < ntile; ++t) {
           if (it > 0) {
-            const int vs = (it - 1) % S;
-            if (!(ok = wait_parity(p_full + t, (it - 1) & 1, A.wd, &abort_flag))) break;
-            if (t == 0 && !(ok = wait_parity(v_full + vs, ((it - 1) / S) & 1, A.wd, &abort_flag))) break;
-            tc_fence_after();
-            issue_pv(t, vs, it - 1 > 0);
-            if (t == ntile - 1) mma_commit(v_empty + vs);
+            if (!(ok = issue_pv(t, it - 1))) break;
+            if (t == ntile - 1) mma_commit(v_empty + (it - 1) % VS);
           }
           issue_s(t, s);
           mma_commit(s_full + t);
@@ -298,12 +322,8 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
         if (ok) mma_commit(k_empty + s);
       }
       if (ok) {
-        const int vs = (n_iter - 1) % S;
         for (int t = 0; t < ntile; ++t) {
-          if (!(ok = wait_parity(p_full + t, (n_iter - 1) & 1, A.wd, &abort_flag))) break;
-          if (t == 0 && !(ok = wait_parity(v_full + vs, ((n_iter - 1) / S) & 1, A.wd, &abort_flag))) break;
-          tc_fence_after();
-          issue_pv(t, vs, n_iter - 1 > 0);
+          if (!(ok = issue_pv(t, n_iter - 1))) break;
           mma_commit(o_done + t);
         }
       }
@@ -338,8 +358,8 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       }
     };
     for (int it = 0; it < n_iter; ++it) {
-      const int s = it % S;
-      const uint32_t ph = (it / S) & 1;
+      const int s = it % KS, sv = it % VS;
+      const uint32_t ph = (it / KS) & 1, phv = (it / VS) & 1;
       const int kb = (j_lo + it) * kBN;
       if (kb + r < sq.s_k) {  // warm L1 with this tile's scales for the softmax warps
         asm volatile("prefetch.global.L1 [%0];" ::"l"(A.k_scales + scale_row0 + kb + r));
@@ -349,10 +369,10 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       convert_row(smem + G::k_stage(s), smem + G::kKOff + s * G::kKVBytes);
       fence_proxy_async_smem();
       mbar_arrive(k_full + s);
-      if (!__all_sync(0xffffffffu, wait_parity(vraw_full + s, ph, A.wd, &abort_flag))) break;
-      convert_row(smem + G::v_stage(s), smem + G::kVOff + s * G::kKVBytes);
+      if (!__all_sync(0xffffffffu, wait_parity(vraw_full + sv, phv, A.wd, &abort_flag))) break;
+      convert_row(smem + G::v_stage(sv), smem + G::kVOff + sv * G::kKVBytes);
       fence_proxy_async_smem();
-      mbar_arrive(v_full + s);
+      mbar_arrive(v_full + sv);
     }
   }
   } else {
@@ -440,6 +460,9 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
           // p = 2^(s * scale * log2(e) - m): one packed FMA for two scores
           const float2 x = fma2(make_float2(__uint_as_float(raw[cc][2 * e]), __uint_as_float(raw[cc][2 * e + 1])),
                                 sc2, nm2);
+          // odd 32-column chunks use the FMA-pipe exp2, so each half of P
+          // (the unit the MMA warp waits for) splits its exponentials evenly
+          // between the MUFU and FMA pipes
           const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           lacc[e % 8] = add2(lacc[e % 8], pp);
           if constexpr (kI8) {
@@ -451,6 +474,26 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
           }
         }
         tmem_st16(s_tm + cc * 16, pk);
+        if (cc == 1 && it > 0 && __any_sync(0xffffffffu, need)) {
+          // O_t is idle here (PV_t of the previous step has completed, this
+          // step's starts only after the signal below): rescale it if some
+          // row's max moved (rare; the first half's scores are dead by now)
+#pragma unroll
+          for (int oc = 0; oc < D / 32; ++oc) {
+            uint32_t o[32];
+            tmem_ld32(o_tm + oc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(o_tm + oc * 32, o);
+          }
+        }
+        if (cc % 2 == 1) {
+          // keys [64 h, 64 h + 64) of P are in TMEM: let the PV MMA start on them
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(p_full + 2 * t + cc / 2);
+        }
       }
 #pragma unroll
       for (int k = 0; k < 4; ++k) lacc[k] = add2(lacc[k], lacc[k + 4]);
@@ -458,20 +501,6 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       lacc[1] = add2(lacc[1], lacc[3]);
       lacc[0] = add2(lacc[0], lacc[1]);
       l = l * alpha + (lacc[0].x + lacc[0].y);
-      if (it > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
-        for (int oc = 0; oc < D / 32; ++oc) {
-          uint32_t o[32];
-          tmem_ld32(o_tm + oc * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(o_tm + oc * 32, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full + t);
     }
     if (ok) ok = __all_sync(0xffffffffu, wait_parity(o_done + t, 0, A.wd, &abort_flag));
     if (ok) {
