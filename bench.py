@@ -50,7 +50,7 @@ def load_peaks():
 
 KERNEL_SOURCES = {
     "prefill_tc_kernel<128,bf16>": ["prefill_tc.cu", "umma.cuh", "device.cuh", "layout.cuh"],
-    "decode_i8_kernel<128>": ["decode.cu", "device.cuh"],
+    "decode_sk_kernel<128>": ["decode.cu", "device.cuh"],
     "compress_kernel": ["quant.cu"],
 }
 
@@ -265,10 +265,17 @@ def varlen_flops(w):
 def other_prefills(args, dev, peaks, world, dist, result):
     """The varlen sliding-window prefill (d=64, epilogue) and the long-context
     prefill over an int8 KV cache, each timed like the main step."""
-    import torch
-    from flashattention_attention_b200 import fa, inputs
     steps = max(10, args.steps // 4)
 
+    if args.only != "prefill_int8":
+        varlen_prefill(args, dev, peaks, world, dist, result, steps)
+    if args.only != "varlen":
+        int8_long_prefill(args, dev, peaks, world, dist, result, steps)
+
+
+def varlen_prefill(args, dev, peaks, world, dist, result, steps):
+    import torch
+    from flashattention_attention_b200 import fa, inputs
     w = inputs.varlen_window_prefill()
     cu = inputs.cu_from_lengths(w.lengths).to(dev)
     q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
@@ -285,6 +292,10 @@ def other_prefills(args, dev, peaks, world, dist, result):
         "frac_of_bf16_peak": round(fe / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
     del q, k, v, out
 
+
+def int8_long_prefill(args, dev, peaks, world, dist, result, steps):
+    import torch
+    from flashattention_attention_b200 import fa, inputs
     w = inputs.int8kv_long_prefill()
     kc, ks = fa.compress_kv(w.k.to(dev))
     vc, vs = fa.compress_kv(w.v.to(dev))
@@ -350,11 +361,11 @@ def decode_and_quant(args, dev, peaks, world, dist, result):
         dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
         result["decode"] = {"workload": dw.name, "value": round(dec_gbs * world, 1), "unit": "GB/s",
                             "us_per_step": round(dec_ms * 1e3, 2), "bytes_per_step": dec_bytes,
-                            "roofline": {"bound": "hbm", "kernel": "decode_i8_kernel<128> + merge",
+                            "roofline": {"bound": "hbm", "kernel": "decode_sk_kernel<128> (merge fused) + decode_plan_kernel",
                                          "achieved": round(dec_gbs, 1), "peak": peaks["hbm_gbs"],
                                          "unit": "GB/s", "frac": round(dec_gbs / peaks["hbm_gbs"], 4),
                                          "frac_of_nominal_8000": round(dec_gbs / 8000.0, 4),
-                                         "traffic": measured_traffic("decode_i8_kernel<128>")}}
+                                         "traffic": measured_traffic("decode_sk_kernel<128>")}}
     assert fa.check_device_error() == fa.FA_OK
     return result
 

@@ -35,12 +35,12 @@
 // int8 K/V (fkl_python PR #6, Summary: "dequantizes in-register inside q.k
 // and p.v; the compressed cache is never inflated in global memory"): TMA
 // brings each int8 tile into shared memory (at d = 128 into the upper half of
-// the bf16 slot it becomes), four converter warps rewrite it as exact bf16
-// (|c| <= 127) in the tensor-core layout, and fence it to the async proxy.
-// The per-key K scale multiplies the columns of S after the MMA; the per-key
-// V scale multiplies the columns of P before its bf16 cast (l sums the
-// unscaled p).  That variant runs 16 warps and rebalances registers with
-// setmaxnreg (softmax 200, the rest 56).
+// the bf16 slot it becomes); four converter warps, one thread per key row,
+// dequantise it as c * s in fp32 (exact: |c| <= 127 times an fp32 scale),
+// round once to bf16, the tensor-core operand type, write it in the operand
+// layout and fence it to the async proxy.  The softmax is then the bf16 one.
+// That variant runs 16 warps and rebalances registers with setmaxnreg
+// (softmax 200, the rest 56).
 #include "internal.h"
 #include "layout.cuh"
 #include "umma.cuh"
@@ -105,33 +105,23 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// bf16 of the signed bytes 0 and 1 (lo) or 2 and 3 (hi) of w, exact:
-// 0x4300 | (b & 0x7f) is 128 + (b & 0x7f) and 0x4300 | (b & 0x80) is 128 or
-// 256, so their difference is the two's-complement value of b.
-__device__ __forceinline__ uint32_t i8x2_to_bf16x2(uint32_t w, uint32_t sel) {
-  uint32_t t, m, sg, r;
-  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(t) : "r"(w), "r"(sel));
-  asm("lop3.b32 %0, %1, 0x007f007f, 0x43004300, 0xea;" : "=r"(m) : "r"(t));
-  asm("lop3.b32 %0, %1, 0x00800080, 0x43004300, 0xea;" : "=r"(sg) : "r"(t));
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(m), "r"(sg));
-  return r;
-}
-
-// 32 consecutive per-key scales from global memory (read-only path; every
-// lane of a warp reads the same addresses, so each load is one broadcast);
-// entries at or past `valid` read as 0.  Vector loads only from 16-byte
-// aligned addresses (varlen sequences start anywhere).
-__device__ __forceinline__ void load_scales32(const float* p, int valid, float (&v)[32]) {
-  if (valid >= 32 && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float4 x = __ldg(reinterpret_cast<const float4*>(p) + q);
-      v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 32; ++e) v[e] = e < valid ? __ldg(p + e) : 0.f;
-  }
+// Four signed bytes of w times the row scale, each product rounded once to
+// bf16 (two bf16x2 words).  Each byte b, flipped to b ^ 0x80 = c + 128, is
+// placed in the low mantissa byte of 2^23, so the float is 2^23 + 128 + c and
+// one exact subtraction leaves c; c * s is then exact in fp32 (8 x 24 bits
+// fit), and the bf16 cast is the only rounding.
+__device__ __forceinline__ uint2 dequant4_bf16(uint32_t w, float2 s2) {
+  const uint32_t x = w ^ 0x80808080u;
+  uint32_t f[4];
+  asm("prmt.b32 %0, %1, 0x4b000000, 0x7540;" : "=r"(f[0]) : "r"(x));
+  asm("prmt.b32 %0, %1, 0x4b000000, 0x7541;" : "=r"(f[1]) : "r"(x));
+  asm("prmt.b32 %0, %1, 0x4b000000, 0x7542;" : "=r"(f[2]) : "r"(x));
+  asm("prmt.b32 %0, %1, 0x4b000000, 0x7543;" : "=r"(f[3]) : "r"(x));
+  const float2 bias = make_float2(-8388736.f, -8388736.f);  // -(2^23 + 128)
+  const float2 c01 = add2(make_float2(__uint_as_float(f[0]), __uint_as_float(f[1])), bias);
+  const float2 c23 = add2(make_float2(__uint_as_float(f[2]), __uint_as_float(f[3])), bias);
+  const float2 y01 = mul2(c01, s2), y23 = mul2(c23, s2);
+  return make_uint2(pack_bf16x2(y01.x, y01.y), pack_bf16x2(y23.x, y23.y));
 }
 
 template <int D, bool kI8>
@@ -337,40 +327,37 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
     // 128-byte-swizzled K-major (K) / MN-major (V) operand layout
     const int r = static_cast<int>(threadIdx.x) - kConvWarp0 * 32;
     const int64_t scale_row0 = static_cast<int64_t>(k_plane) * A.k_plane_rows + k_prow0;
-    auto convert_row = [&](const uint8_t* src_tile, uint8_t* dst_tile) {
-      constexpr int kChunks8 = D / 16;  // 16-byte int8 chunks per row
-      uint4 w[kChunks8];
+    auto convert_row = [&](const uint8_t* src_tile, uint8_t* dst_tile, float sc) {
+      const float2 s2 = make_float2(sc, sc);
 #pragma unroll
-      for (int c = 0; c < kChunks8; ++c) {
+      for (int c = 0; c < D / 16; ++c) {  // 16-byte int8 chunks of the row
         const int pc = (D == 128) ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
-        w[c] = *reinterpret_cast<const uint4*>(src_tile + r * D + pc * 16);
-      }
-#pragma unroll
-      for (int c = 0; c < kChunks8; ++c) {
+        const uint4 w = *reinterpret_cast<const uint4*>(src_tile + r * D + pc * 16);
         const int h = c / 4, j0 = 2 * (c % 4);
         uint8_t* row = dst_tile + h * kChunkBytes + r * 128;
-        const uint4 a = make_uint4(i8x2_to_bf16x2(w[c].x, 0x4140), i8x2_to_bf16x2(w[c].x, 0x4342),
-                                   i8x2_to_bf16x2(w[c].y, 0x4140), i8x2_to_bf16x2(w[c].y, 0x4342));
-        const uint4 bq = make_uint4(i8x2_to_bf16x2(w[c].z, 0x4140), i8x2_to_bf16x2(w[c].z, 0x4342),
-                                    i8x2_to_bf16x2(w[c].w, 0x4140), i8x2_to_bf16x2(w[c].w, 0x4342));
-        *reinterpret_cast<uint4*>(row + ((j0 ^ (r & 7)) * 16)) = a;
-        *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ (r & 7)) * 16)) = bq;
+        const uint2 y0 = dequant4_bf16(w.x, s2), y1 = dequant4_bf16(w.y, s2);
+        const uint2 y2 = dequant4_bf16(w.z, s2), y3 = dequant4_bf16(w.w, s2);
+        *reinterpret_cast<uint4*>(row + ((j0 ^ (r & 7)) * 16)) = make_uint4(y0.x, y0.y, y1.x, y1.y);
+        *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ (r & 7)) * 16)) = make_uint4(y2.x, y2.y, y3.x, y3.y);
       }
     };
     for (int it = 0; it < n_iter; ++it) {
       const int s = it % KS, sv = it % VS;
       const uint32_t ph = (it / KS) & 1, phv = (it / VS) & 1;
-      const int kb = (j_lo + it) * kBN;
-      if (kb + r < sq.s_k) {  // warm L1 with this tile's scales for the softmax warps
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(A.k_scales + scale_row0 + kb + r));
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(A.v_scales + scale_row0 + kb + r));
+      // this thread's key row: its two scales, loaded ahead of the waits (0
+      // past the sequence end, so those rows become zeros; the softmax masks them)
+      const int key = (j_lo + it) * kBN + r;
+      float ksc = 0.f, vsc = 0.f;
+      if (key < sq.s_k) {
+        ksc = __ldg(A.k_scales + scale_row0 + key);
+        vsc = __ldg(A.v_scales + scale_row0 + key);
       }
       if (!__all_sync(0xffffffffu, wait_parity(kraw_full + s, ph, A.wd, &abort_flag))) break;
-      convert_row(smem + G::k_stage(s), smem + G::kKOff + s * G::kKVBytes);
+      convert_row(smem + G::k_stage(s), smem + G::kKOff + s * G::kKVBytes, ksc);
       fence_proxy_async_smem();
       mbar_arrive(k_full + s);
       if (!__all_sync(0xffffffffu, wait_parity(vraw_full + sv, phv, A.wd, &abort_flag))) break;
-      convert_row(smem + G::v_stage(sv), smem + G::kVOff + sv * G::kKVBytes);
+      convert_row(smem + G::v_stage(sv), smem + G::kVOff + sv * G::kKVBytes, vsc);
       fence_proxy_async_smem();
       mbar_arrive(v_full + sv);
     }
@@ -382,7 +369,6 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
     const int t = warp / 4, quarter = warp % 4;
     const int r = quarter * 32 + lane;
     const int i = i0 + r;
-    const int64_t scale_row0 = static_cast<int64_t>(k_plane) * A.k_plane_rows + k_prow0;
     int lo, hi;
     band_of(A.L, i, sq.s_q, sq.s_k, lo, hi);
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
@@ -401,22 +387,6 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       tmem_ld32(s_tm + 96, raw[3]);
       tmem_wait_ld();
       const int kb = (j_lo + it) * kBN;
-      if constexpr (kI8) {
-        // S columns times the per-key K scale (keys past the sequence get 0
-        // and are masked below)
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float ksv[32];
-          load_scales32(A.k_scales + scale_row0 + kb + cc * 32, sq.s_k - kb - cc * 32, ksv);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float2 x = mul2(make_float2(__uint_as_float(raw[cc][2 * e]), __uint_as_float(raw[cc][2 * e + 1])),
-                                  make_float2(ksv[2 * e], ksv[2 * e + 1]));
-            raw[cc][2 * e] = __float_as_uint(x.x);
-            raw[cc][2 * e + 1] = __float_as_uint(x.y);
-          }
-        }
-      }
       if (!(kb >= lo && kb + kBN <= hi)) {
         // boundary tile: keys outside this row's band become -inf (the
         // softmax scale is positive, so masking before it is the same)
@@ -453,25 +423,14 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t pk[16];
-        float vsv[32];
-        if constexpr (kI8) load_scales32(A.v_scales + scale_row0 + kb + cc * 32, sq.s_k - kb - cc * 32, vsv);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           // p = 2^(s * scale * log2(e) - m): one packed FMA for two scores
           const float2 x = fma2(make_float2(__uint_as_float(raw[cc][2 * e]), __uint_as_float(raw[cc][2 * e + 1])),
                                 sc2, nm2);
-          // odd 32-column chunks use the FMA-pipe exp2, so each half of P
-          // (the unit the MMA warp waits for) splits its exponentials evenly
-          // between the MUFU and FMA pipes
           const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           lacc[e % 8] = add2(lacc[e % 8], pp);
-          if constexpr (kI8) {
-            // the V scale multiplies P's columns; l keeps the unscaled p
-            const float2 pv = mul2(pp, make_float2(vsv[2 * e], vsv[2 * e + 1]));
-            pk[e] = pack_bf16x2(pv.x, pv.y);
-          } else {
-            pk[e] = pack_bf16x2(pp.x, pp.y);
-          }
+          pk[e] = pack_bf16x2(pp.x, pp.y);
         }
         tmem_st16(s_tm + cc * 16, pk);
         if (cc == 1 && it > 0 && __any_sync(0xffffffffu, need)) {
