@@ -366,6 +366,24 @@ def decode_and_quant(args, dev, peaks, world, dist, result):
                                          "unit": "GB/s", "frac": round(dec_gbs / peaks["hbm_gbs"], 4),
                                          "frac_of_nominal_8000": round(dec_gbs / 8000.0, 4),
                                          "traffic": measured_traffic("decode_sk_kernel<128>")}}
+        del kc, vc, ks, vs
+        torch.cuda.empty_cache()
+        # the same decode over an uncompressed bf16 cache (2 * 2d bytes per key and KV head)
+        kb, vb = dw.k.to(dev), dw.v.to(dev)
+
+        def decode_bf16():
+            fa.attention_decode(dq, kb, vb, lens, hq=dw.hq, hkv=dw.hkv, max_seqlen=maxlen, workspace=ws, out=dout)
+
+        bf_ms = time_launches(decode_bf16, max(20, args.steps), args.warmup, torch, dist)
+        bf_bytes = sum(dw.lengths) * dw.hkv * 2 * (2 * dw.d) + 2 * dq.numel() * 2
+        bf_gbs = bf_bytes / (bf_ms * 1e-3) / 1e9
+        result["decode_bf16"] = {"workload": dw.name.replace("int8kv", "bf16kv"), "value": round(bf_gbs * world, 1),
+                                 "unit": "GB/s", "us_per_step": round(bf_ms * 1e3, 2), "bytes_per_step": bf_bytes,
+                                 "roofline": {"bound": "hbm", "kernel": "decode_sk_kernel<128,bf16> + decode_plan_kernel",
+                                              "achieved": round(bf_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                              "frac": round(bf_gbs / peaks["hbm_gbs"], 4), "traffic": None}}
+        del kb, vb
+        torch.cuda.empty_cache()
     assert fa.check_device_error() == fa.FA_OK
     return result
 

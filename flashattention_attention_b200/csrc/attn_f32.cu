@@ -8,6 +8,10 @@
 // of 4 dims, so the K/V tiles in shared memory are read without bank
 // conflicts.  Keys stream in tiles of 32 through an online softmax (running
 // max m and sum l in fp32, exp2 with log2(e) folded into the scale).
+// With an int8 KV cache (fkl_python PR #6, Verification, "FA int8-KV exact
+// vs dequantized oracle") each K/V element enters the shared tile as c * s
+// computed in fp32, which is exact (|c| <= 127 times an fp32 scale), so the
+// kernel sees the dequantised cache itself.
 //
 // empty_rows_kernel: rows whose band is empty (causal with s_q > s_k leaves
 // rows i < s_q - s_k without keys) get uniform weights over all s_k keys,
@@ -24,9 +28,24 @@ constexpr int kRowsPerCta = 32;
 constexpr int kKeysPerTile = 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D>
+// Four consecutive K or V elements of row `row` as fp32: plain fp32, or int8
+// codes times the row's scale.
+template <bool kI8>
+__device__ __forceinline__ float4 load_kv4(const void* base, const float* scales, int64_t row, int d, int col) {
+  if constexpr (kI8) {
+    const char4 c = *reinterpret_cast<const char4*>(static_cast<const int8_t*>(base) + row * d + col);
+    const float s = scales[row];
+    return make_float4(static_cast<float>(c.x) * s, static_cast<float>(c.y) * s, static_cast<float>(c.z) * s,
+                       static_cast<float>(c.w) * s);
+  } else {
+    return *reinterpret_cast<const float4*>(static_cast<const float*>(base) + row * d + col);
+  }
+}
+
+template <int D, bool kI8>
 __global__ void __launch_bounds__(128)
-    attn_f32_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
+    attn_f32_kernel(const float* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
+                    const float* __restrict__ k_scales, const float* __restrict__ v_scales,
                     float* __restrict__ out, SeqLayout L, int hq, int hkv, float scale_log2, Epilogue epi) {
   constexpr int kPer = D / 4;        // dims per thread
   constexpr int kVec = kPer / 4;     // float4 groups per thread
@@ -71,8 +90,8 @@ __global__ void __launch_bounds__(128)
       const int jj = e / (D / 4), c4 = e % (D / 4);
       float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
       if (j0 + jj < sq.s_k) {
-        kv = *reinterpret_cast<const float4*>(k + (sq.k_row0 + j0 + jj) * D + 4 * c4);
-        vv = *reinterpret_cast<const float4*>(v + (sq.k_row0 + j0 + jj) * D + 4 * c4);
+        kv = load_kv4<kI8>(k, k_scales, sq.k_row0 + j0 + jj, D, 4 * c4);
+        vv = load_kv4<kI8>(v, v_scales, sq.k_row0 + j0 + jj, D, 4 * c4);
       }
       *reinterpret_cast<float4*>(&ks[jj][4 * c4]) = kv;
       *reinterpret_cast<float4*>(&vs[jj][4 * c4]) = vv;
@@ -168,14 +187,14 @@ fa_status launch_f32_d(const fa_fwd_params& p, const LaunchCtx& ctx) {
   const int max_sq = p.cu_seqlens_q ? p.max_seqlen_q : p.seqlen_q;
   dim3 grid((max_sq + kRowsPerCta - 1) / kRowsPerCta, p.hq, p.batch);
   if (grid.x == 0) return FA_OK;
-  auto kern = attn_f32_kernel<D>;
+  auto kern = p.kv_dtype == FA_I8 ? attn_f32_kernel<D, true> : attn_f32_kernel<D, false>;
   constexpr int kSmem = 2 * kKeysPerTile * D * sizeof(float);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
     return FA_ERR_CUDA;
   note_variant(reinterpret_cast<const void*>(kern));
-  kern<<<grid, 128, kSmem, ctx.stream>>>(static_cast<const float*>(p.q), static_cast<const float*>(p.k),
-                                     static_cast<const float*>(p.v), static_cast<float*>(p.out), L, p.hq,
-                                     p.hkv, p.softmax_scale * kLog2e, make_epilogue(p.epilogue, p.n_epilogue));
+  kern<<<grid, 128, kSmem, ctx.stream>>>(static_cast<const float*>(p.q), p.k, p.v, p.k_scales, p.v_scales,
+                                     static_cast<float*>(p.out), L, p.hq, p.hkv, p.softmax_scale * kLog2e,
+                                     make_epilogue(p.epilogue, p.n_epilogue));
   return cuda_status(cudaGetLastError());
 }
 
@@ -205,7 +224,12 @@ fa_status launch_empty_rows(const fa_fwd_params& p, const LaunchCtx& ctx) {
   const SeqLayout L = SeqLayout::from(p);
   const Epilogue epi = make_epilogue(p.epilogue, p.n_epilogue);
   dim3 grid(p.hq, p.batch);
-  if (p.q_dtype == FA_F32) {
+  if (p.q_dtype == FA_F32 && p.kv_dtype == FA_I8) {
+    auto kern = empty_rows_kernel<int8_t, float>;
+    note_variant(reinterpret_cast<const void*>(kern));
+    kern<<<grid, 128, 0, ctx.stream>>>(static_cast<const int8_t*>(p.v), p.v_scales, static_cast<float*>(p.out),
+                                       L, p.hq, p.hkv, p.head_dim, epi);
+  } else if (p.q_dtype == FA_F32) {
     auto kern = empty_rows_kernel<float, float>;
     note_variant(reinterpret_cast<const void*>(kern));
     kern<<<grid, 128, 0, ctx.stream>>>(static_cast<const float*>(p.v), nullptr, static_cast<float*>(p.out),

@@ -32,6 +32,14 @@
 // Because d is summed over, each thread owns a contiguous byte slice of every
 // K row; Q's fragments use the same dim order.  The S accumulator fragment
 // becomes the P operand fragment with one 8x8 transpose (movmatrix).
+//
+// bf16 cache (the same stream-K schedule and merge): tiles arrive as 64-dim
+// chunks of 128-byte rows (128-byte swizzle); K fragments come from ldmatrix,
+// V^T fragments from ldmatrix.trans, Q enters the bf16 MMA as it is and P is
+// rounded to bf16.  A stage is twice as large, so d = 128 runs one CTA per
+// SM.  Cache rows outside [k_lo, L) may hold any bytes (NaN included): their
+// scores are masked, and in a tile that holds such rows the V rows are zeroed
+// in shared memory before P V, so 0 * NaN never reaches O.
 #include <mutex>
 
 #include "internal.h"
@@ -42,7 +50,7 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kTile = 32;    // keys per tile
 constexpr int kStages = 3;
-constexpr int kCtasPerSm = 2;
+constexpr int kCtasPerSm = 2;  // int8 (and bf16 at d = 64); bf16 at d = 128 fits one
 constexpr int kMaxWorkers = 4096;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -64,20 +72,32 @@ struct SkArgs {
   Watchdog wd;
 };
 
-template <int D>
+template <int D, bool kBF>
 struct Geom {
-  static constexpr int kTileBytes = kTile * D;  // int8 codes
+  static constexpr int kTileBytes = kTile * D * (kBF ? 2 : 1);  // int8 codes or bf16
+  static constexpr int kScaleBytes = kBF ? 0 : 2 * kTile * 4;    // K and V scales (int8)
   static constexpr int kScaleOff = 2 * kTileBytes;
-  static constexpr int kStageBytes = ((2 * kTileBytes + 2 * kTile * 4) + 1023) / 1024 * 1024;
-  static constexpr int kSwzMask = (D == 128) ? 0x70 : 0x30;  // 128B or 64B swizzle
+  static constexpr int kStageBytes = ((2 * kTileBytes + kScaleBytes) + 1023) / 1024 * 1024;
+  // int8: 128B (d = 128) or 64B (d = 64) swizzle of whole rows; bf16: 128B
+  // swizzle of 64-dim chunks [32 rows x 128 B]
+  static constexpr int kSwzMask = (kBF || D == 128) ? 0x70 : 0x30;
+  static constexpr int kChunkBytes = kTile * 128;
+  static constexpr int kCtas = (kBF && D == 128) ? 1 : kCtasPerSm;
   static constexpr int kSmem = kWarps * kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
 };
+static_assert(Geom<128, true>::kSmem <= 232448, "shared memory budget");
+static_assert(2 * Geom<128, false>::kSmem <= 232448 && 2 * Geom<64, true>::kSmem <= 232448, "two CTAs per SM");
 
 // TMA swizzle of a byte offset inside a tile whose base is aligned to the
 // swizzle period: bits [4,7) (128B) or [4,6) (64B) ^= bits [7,10) / [7,9).
-template <int D>
+template <int D, bool kBF>
 __device__ __forceinline__ uint32_t swz(uint32_t lin) {
-  return lin ^ ((lin >> 3) & Geom<D>::kSwzMask);
+  return lin ^ ((lin >> 3) & Geom<D, kBF>::kSwzMask);
+}
+// Shared address of element (key r, dim c) of a bf16 tile at `tile`.
+template <int D>
+__device__ __forceinline__ uint32_t bf_addr(uint32_t tile, int r, int c) {
+  return tile + (c / 64) * Geom<D, true>::kChunkBytes + swz<D, true>(r * 128 + (c % 64) * 2);
 }
 
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
@@ -105,6 +125,16 @@ __device__ __forceinline__ uint32_t i8x2_to_f16x2_even(uint32_t w) {
 // fp16x2 of the signed bytes 1 and 3 of w (exact).
 __device__ __forceinline__ uint32_t i8x2_to_f16x2_odd(uint32_t w) { return i8x2_to_f16x2_even(w >> 8); }
 
+// Four 8x8 b16 matrices; lane l gives the row address of matrix l / 8, row l % 8.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -113,6 +143,17 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma16816_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 __device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
   uint32_t y;
@@ -199,13 +240,21 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   for (int i = tid; i < batch * hkv; i += nthreads) counters[i] = 0;
 }
 
-// Position in the global tile sequence: sequence b, KV head g, tile t of Tb.
+// Position in the global tile sequence: sequence b, KV head g, tile t of Tb,
+// with the segment's first tile key and cache row kept for the loads.
 struct Cursor {
   int b, g, t, Tb;
+  int t_begin;      // key of the segment's first tile
+  int64_t kv_row0;  // cache row of key 0 of (b, g)
 };
 
 __device__ __forceinline__ int seq_tiles(const SkArgs& A, int b) {
   return (A.prefix[b + 1] - A.prefix[b]) / A.hkv;
+}
+__device__ __forceinline__ void set_segment(const SkArgs& A, Cursor& c) {
+  int k_lo;
+  key_range(clamp_len(A.seqlens[c.b], A.cap), A.window, k_lo, c.t_begin);
+  c.kv_row0 = (static_cast<int64_t>(c.b) * A.hkv + c.g) * A.cap;
 }
 __device__ __forceinline__ Cursor locate(const SkArgs& A, long long x) {
   int lo = 0, hi = A.batch - 1;  // largest b with prefix[b] <= x
@@ -219,23 +268,28 @@ __device__ __forceinline__ Cursor locate(const SkArgs& A, long long x) {
   const long long y = x - A.prefix[lo];
   c.g = static_cast<int>(y / c.Tb);
   c.t = static_cast<int>(y % c.Tb);
+  set_segment(A, c);
   return c;
 }
 __device__ __forceinline__ void advance(const SkArgs& A, Cursor& c) {
   if (++c.t < c.Tb) return;
   c.t = 0;
-  if (++c.g < A.hkv) return;
+  if (++c.g < A.hkv) {
+    c.kv_row0 += A.cap;
+    return;
+  }
   c.g = 0;
   do {
     ++c.b;
   } while (c.b < A.batch && (c.Tb = seq_tiles(A, c.b)) == 0);
+  if (c.b < A.batch) set_segment(A, c);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm)
+template <int D, bool kBF>
+__global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
     decode_sk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const SkArgs A) {
-  using G = Geom<D>;
+  using G = Geom<D, kBF>;
   constexpr int kSteps = D / 16;      // k-steps of the S MMA
   constexpr int kChunks = D / 64;     // 16-byte chunks per thread per K row
   constexpr int kMT = D / 16;         // O^T m-tiles (dims)
@@ -262,27 +316,27 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm)
   if (my_tiles <= 0) return;
 
   auto stage_ptr = [&](int s) { return smem + (warp * kStages + s) * G::kStageBytes; };
-  auto tile_geom = [&](const Cursor& c, int& key0, int& k_lo, int& L, int64_t& kv_row0) {
-    L = clamp_len(A.seqlens[c.b], A.cap);
-    int t_begin;
-    key_range(L, A.window, k_lo, t_begin);
-    key0 = t_begin + c.t * kTile;
-    kv_row0 = (static_cast<int64_t>(c.b) * A.hkv + c.g) * A.cap;
-  };
   // issue cursor (lane 0 runs it kStages tiles ahead of the compute cursor)
   Cursor ic = locate(A, t_first);
   auto issue = [&](int i) {
     const int s = i % kStages;
-    int key0, k_lo, L;
-    int64_t kv_row0;
-    tile_geom(ic, key0, k_lo, L, kv_row0);
+    const int key0 = ic.t_begin + ic.t * kTile;
+    const int64_t kv_row0 = ic.kv_row0;
     uint8_t* st = stage_ptr(s);
     uint64_t* bar = &bars[warp * kStages + s];
-    mbar_expect_tx(bar, 2 * G::kTileBytes + 2 * kTile * 4);
-    tma_load_2d(st, &tm_k, bar, 0, static_cast<int>(kv_row0 + key0));
-    tma_load_2d(st + G::kTileBytes, &tm_v, bar, 0, static_cast<int>(kv_row0 + key0));
-    bulk_load(st + G::kScaleOff, A.k_scales + kv_row0 + key0, kTile * 4, bar);
-    bulk_load(st + G::kScaleOff + kTile * 4, A.v_scales + kv_row0 + key0, kTile * 4, bar);
+    mbar_expect_tx(bar, 2 * G::kTileBytes + G::kScaleBytes);
+    if constexpr (kBF) {
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_2d(st + c * G::kChunkBytes, &tm_k, bar, 64 * c, static_cast<int>(kv_row0 + key0));
+        tma_load_2d(st + G::kTileBytes + c * G::kChunkBytes, &tm_v, bar, 64 * c, static_cast<int>(kv_row0 + key0));
+      }
+    } else {
+      tma_load_2d(st, &tm_k, bar, 0, static_cast<int>(kv_row0 + key0));
+      tma_load_2d(st + G::kTileBytes, &tm_v, bar, 0, static_cast<int>(kv_row0 + key0));
+      bulk_load(st + G::kScaleOff, A.k_scales + kv_row0 + key0, kTile * 4, bar);
+      bulk_load(st + G::kScaleOff + kTile * 4, A.v_scales + kv_row0 + key0, kTile * 4, bar);
+    }
     advance(A, ic);
   };
   if (lane == 0) {
@@ -302,9 +356,20 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm)
   };
   // Q fragments: thread (gq, qq) holds head gq, dims [qq*D/4, (qq+1)*D/4)
   auto load_q = [&](int b, int g) {
-    float qv[D / 4];
     const bool head_ok = gq < A.group;
     const int hq_idx = b * A.hq + g * A.group + gq;
+    if constexpr (kBF) {
+      // B fragments of head gq: dims 16 ks + 2 qq (+1) and 16 ks + 8 + 2 qq (+1)
+      const uint32_t* qw = reinterpret_cast<const uint32_t*>(A.q + static_cast<int64_t>(hq_idx) * D);
+#pragma unroll
+      for (int ks = 0; ks < kSteps; ++ks) {
+        qb0[ks] = head_ok ? qw[8 * ks + qq] : 0u;
+        qb1[ks] = head_ok ? qw[8 * ks + 4 + qq] : 0u;
+      }
+      qs0 = qs1 = A.scale_log2;
+      return;
+    }
+    float qv[D / 4];
     float amax = 0.f;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
@@ -354,16 +419,32 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm)
         A.rec_ml[(rec * A.group + h1) * 2 + 1] = l1;
       }
     }
+    if constexpr (kBF) {
+      // m-tile mi holds dims 16 mi + gq (c0, c1) and 16 mi + gq + 8 (c2, c3)
 #pragma unroll
-    for (int pr = 0; pr < D / 32; ++pr) {
+      for (int mi = 0; mi < kMT; ++mi) {
+        const int dim = 16 * mi + gq;
+        if (h0 < A.group) {
+          A.rec_o[(rec * A.group + h0) * D + dim] = o[mi][0];
+          A.rec_o[(rec * A.group + h0) * D + dim + 8] = o[mi][2];
+        }
+        if (h1 < A.group) {
+          A.rec_o[(rec * A.group + h1) * D + dim] = o[mi][1];
+          A.rec_o[(rec * A.group + h1) * D + dim + 8] = o[mi][3];
+        }
+      }
+    } else {
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int dim0 = 4 * (8 * pr + gq) + 2 * j;
-        const float(&c)[4] = o[2 * pr + j];
-        if (h0 < A.group)
-          *reinterpret_cast<float2*>(A.rec_o + (rec * A.group + h0) * D + dim0) = make_float2(c[0], c[2]);
-        if (h1 < A.group)
-          *reinterpret_cast<float2*>(A.rec_o + (rec * A.group + h1) * D + dim0) = make_float2(c[1], c[3]);
+      for (int pr = 0; pr < D / 32; ++pr) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int dim0 = 4 * (8 * pr + gq) + 2 * j;
+          const float(&c)[4] = o[2 * pr + j];
+          if (h0 < A.group)
+            *reinterpret_cast<float2*>(A.rec_o + (rec * A.group + h0) * D + dim0) = make_float2(c[0], c[2]);
+          if (h1 < A.group)
+            *reinterpret_cast<float2*>(A.rec_o + (rec * A.group + h1) * D + dim0) = make_float2(c[1], c[3]);
+        }
       }
     }
   };
@@ -388,45 +469,47 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm)
     if (prev != w_hi - w_lo) return;
     __threadfence();
     const int b = seg / A.hkv, g = seg % A.hkv;
-    // one pass over the segment's records, all heads at once, online max
-    float M[8], lsum[8], acc[8][D / 32];
+    // one pass over the segment's records with an online max; lane l owns
+    // head l / 4 and a quarter of its dims (contiguous, read as float4), and
+    // the unrolled record loop keeps several records' loads in flight
+    constexpr int kPer = D / 4;
+    const int hl = lane >> 2, part = lane & 3;
+    if (hl < A.group) {
+      float M = -INFINITY, lsum = 0.f, acc[kPer];
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
-      M[h] = -INFINITY;
-      lsum[h] = 0.f;
+      for (int j = 0; j < kPer; ++j) acc[j] = 0.f;
+#pragma unroll 2
+      for (int v = w_lo; v <= w_hi; ++v) {
+        const int64_t r = (static_cast<int64_t>(seg) + v) * A.group + hl;
+        const float m = __ldcg(&A.rec_ml[r * 2]);
+        const float lv = __ldcg(&A.rec_ml[r * 2 + 1]);
+        const float4* src = reinterpret_cast<const float4*>(A.rec_o + r * D + part * kPer);
+        float4 ov[kPer / 4];
 #pragma unroll
-      for (int j = 0; j < D / 32; ++j) acc[h][j] = 0.f;
-    }
-    for (int v = w_lo; v <= w_hi; ++v) {
-      const int64_t r0 = (static_cast<int64_t>(seg) + v) * A.group;
-#pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        if (h >= A.group) break;
-        const float m = __ldcg(&A.rec_ml[(r0 + h) * 2]);
-        const float lv = __ldcg(&A.rec_ml[(r0 + h) * 2 + 1]);
-        float ov[D / 32];
-#pragma unroll
-        for (int j = 0; j < D / 32; ++j) ov[j] = __ldcg(&A.rec_o[(r0 + h) * D + lane + 32 * j]);
-        const float mn = fmaxf(M[h], m);
+        for (int q = 0; q < kPer / 4; ++q) ov[q] = __ldcg(src + q);
+        const float mn = fmaxf(M, m);
         const float ref = mn == -INFINITY ? 0.f : mn;
-        const float a_old = ex2_approx(M[h] - ref), a_new = ex2_approx(m - ref);
-        M[h] = mn;
-        lsum[h] = lsum[h] * a_old + lv * a_new;
+        const float a_old = ex2_approx(M - ref), a_new = ex2_approx(m - ref);
+        M = mn;
+        lsum = lsum * a_old + lv * a_new;
 #pragma unroll
-        for (int j = 0; j < D / 32; ++j) acc[h][j] = acc[h][j] * a_old + ov[j] * a_new;
+        for (int q = 0; q < kPer / 4; ++q) {
+          acc[4 * q + 0] = acc[4 * q + 0] * a_old + ov[q].x * a_new;
+          acc[4 * q + 1] = acc[4 * q + 1] * a_old + ov[q].y * a_new;
+          acc[4 * q + 2] = acc[4 * q + 2] * a_old + ov[q].z * a_new;
+          acc[4 * q + 3] = acc[4 * q + 3] * a_old + ov[q].w * a_new;
+        }
       }
-    }
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
-      if (h >= A.group) break;
-      const float inv = lsum[h] > 0.f ? 1.f / lsum[h] : 0.f;
-      float y[D / 32];
+      for (int j = 0; j < kPer; ++j) acc[j] *= inv;
+      apply_epilogue_vec(acc, A.epi);
+      uint4* dst = reinterpret_cast<uint4*>(A.out + (static_cast<int64_t>(b) * A.hq + g * A.group + hl) * D +
+                                            part * kPer);
 #pragma unroll
-      for (int j = 0; j < D / 32; ++j) y[j] = acc[h][j] * inv;
-      apply_epilogue_vec(y, A.epi);
-      __nv_bfloat16* orow = A.out + (static_cast<int64_t>(b) * A.hq + g * A.group + h) * D;
-#pragma unroll
-      for (int j = 0; j < D / 32; ++j) orow[lane + 32 * j] = __float2bfloat16_rn(y[j]);
+      for (int q = 0; q < kPer / 8; ++q)
+        dst[q] = make_uint4(pack_bf16x2(acc[8 * q + 0], acc[8 * q + 1]), pack_bf16x2(acc[8 * q + 2], acc[8 * q + 3]),
+                            pack_bf16x2(acc[8 * q + 4], acc[8 * q + 5]), pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]));
     }
   };
 
@@ -457,6 +540,20 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm)
 
     // ---- S^T = K . Q^T for the two 16-key halves of the tile
     float sc[2][4];
+    if constexpr (kBF) {
+      // matrix i of lane l: keys 16 mt + 8 (i % 2) + l % 8, dims 16 ks + 8 (i / 2)
+      const int mi = lane >> 3, mr = lane & 7;
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < kSteps; ++ks) {
+          uint32_t a[4];
+          ldsm_x4(bf_addr<D>(kt, 16 * mt + 8 * (mi % 2) + mr, 16 * ks + 8 * (mi / 2)), a);
+          mma16816_bf16(sc[mt], a, qb0[ks], qb1[ks]);
+        }
+      }
+    } else
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
       sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
@@ -465,8 +562,8 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm)
 #pragma unroll
       for (int c = 0; c < kChunks; ++c) {
         const uint32_t off = (qq * kChunks + c) * 16;
-        ka[c] = lds128(kt + swz<D>(r0 * D + off));
-        kb[c] = lds128(kt + swz<D>(r1 * D + off));
+        ka[c] = lds128(kt + swz<D, false>(r0 * D + off));
+        kb[c] = lds128(kt + swz<D, false>(r1 * D + off));
       }
 #pragma unroll
       for (int ks = 0; ks < kSteps; ++ks) {
@@ -489,7 +586,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm)
         const int kl = 16 * mt + gq + 8 * hf;
         const int key = key0 + kl;
         const bool ok = key >= k_lo && key < key_end;
-        const float kscale = ksc[kl];
+        const float kscale = kBF ? 1.f : ksc[kl];
         x[mt][2 * hf + 0] = ok ? sc[mt][2 * hf + 0] * kscale * qs0 : -INFINITY;
         x[mt][2 * hf + 1] = ok ? sc[mt][2 * hf + 1] * kscale * qs1 : -INFINITY;
         mx0 = fmaxf(mx0, x[mt][2 * hf + 0]);
@@ -533,24 +630,52 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm)
         const float p1 = ex2_approx(x[mt][2 * hf + 1] - ref1);
         l_run[0] += p0;
         l_run[1] += p1;
-        const float vscale = ok ? vsc[kl] : 0.f;
-        packed[hf] = pack_f16x2(ok ? p0 * vscale : 0.f, ok ? p1 * vscale : 0.f);
+        if constexpr (kBF) {
+          packed[hf] = pack_bf16x2(ok ? p0 : 0.f, ok ? p1 : 0.f);
+        } else {
+          const float vscale = ok ? vsc[kl] : 0.f;
+          packed[hf] = pack_f16x2(ok ? p0 * vscale : 0.f, ok ? p1 * vscale : 0.f);
+        }
       }
       pb[mt][0] = transpose8x8(packed[0]);  // (head gq; keys 2qq, 2qq+1)
       pb[mt][1] = transpose8x8(packed[1]);  // (head gq; keys 8+2qq, 8+2qq+1)
     }
 
     // ---- O^T += V^T . P'
+    if constexpr (kBF) {
+      if (key0 < k_lo || key0 + kTile > key_end) {
+        // rows outside the band may hold NaN or Inf: zero them (P is 0 there)
+        const int key = key0 + lane;
+        if (key < k_lo || key >= key_end) {
+#pragma unroll
+          for (int c = 0; c < D; c += 8)
+            asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(bf_addr<D>(vt, lane, c)), "r"(0u) : "memory");
+          fence_proxy_async_smem();  // ordered before the TMA that refills this stage
+        }
+        __syncwarp();
+      }
+      // matrix i of lane l: keys 16 mt + 8 (i / 2) + l % 8, dims 16 mi + 8 (i % 2)
+      const int mi4 = lane >> 3, mr = lane & 7;
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+        for (int mi = 0; mi < kMT; ++mi) {
+          uint32_t a[4];
+          ldsm_x4_trans(bf_addr<D>(vt, 16 * mt + 8 * (mi4 / 2) + mr, 16 * mi + 8 * (mi4 % 2)), a);
+          mma16816_bf16(o[mi], a, pb[mt][0], pb[mt][1]);
+        }
+      }
+    } else
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
       const int kk0 = 16 * mt + 2 * qq;
 #pragma unroll
       for (int pr = 0; pr < D / 32; ++pr) {
         const uint32_t xw = (8 * pr + gq) * 4;  // byte offset of this thread's word
-        const uint32_t w0 = lds32(vt + swz<D>((kk0 + 0) * D + xw));
-        const uint32_t w1 = lds32(vt + swz<D>((kk0 + 1) * D + xw));
-        const uint32_t w2 = lds32(vt + swz<D>((kk0 + 8) * D + xw));
-        const uint32_t w3 = lds32(vt + swz<D>((kk0 + 9) * D + xw));
+        const uint32_t w0 = lds32(vt + swz<D, false>((kk0 + 0) * D + xw));
+        const uint32_t w1 = lds32(vt + swz<D, false>((kk0 + 1) * D + xw));
+        const uint32_t w2 = lds32(vt + swz<D, false>((kk0 + 8) * D + xw));
+        const uint32_t w3 = lds32(vt + swz<D, false>((kk0 + 9) * D + xw));
         const uint32_t t01l = prmt(w0, w1, 0x5410), t01h = prmt(w0, w1, 0x7632);
         const uint32_t t23l = prmt(w2, w3, 0x5410), t23h = prmt(w2, w3, 0x7632);
         mma16816(o[2 * pr], i8x2_to_f16x2_even(t01l), i8x2_to_f16x2_odd(t01l), i8x2_to_f16x2_even(t23l),
@@ -595,19 +720,21 @@ size_t records_bytes(int batch, int hq, int hkv, int d, int n_workers) {
 }
 
 // Launch plan + stream-K kernel + merge into `ws` (plan, then records).
-template <int D>
+template <int D, bool kBF>
 fa_status launch_sk(const fa_decode_params& p, int n_workers, int min_tiles, void* ws, bool count_variants,
                     const LaunchCtx& ctx) {
-  using G = Geom<D>;
+  using G = Geom<D, kBF>;
   const uint64_t rows = static_cast<uint64_t>(p.batch) * p.hkv * p.capacity;
   CUtensorMap tmk, tmv;
   const uint64_t dims[2] = {static_cast<uint64_t>(D), rows};
-  const uint64_t strides[1] = {static_cast<uint64_t>(D)};
-  const uint32_t box[2] = {static_cast<uint32_t>(D), static_cast<uint32_t>(kTile)};
-  const CUtensorMapSwizzle sw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  fa_status st = encode_tensor_map(&tmk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p.k_cache, dims, strides, box, sw);
+  const uint64_t strides[1] = {static_cast<uint64_t>(D) * (kBF ? 2 : 1)};
+  // int8: one box of whole rows; bf16: boxes of 64 dims (128 bytes) per row
+  const uint32_t box[2] = {static_cast<uint32_t>(kBF ? 64 : D), static_cast<uint32_t>(kTile)};
+  const CUtensorMapSwizzle sw = (kBF || D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUtensorMapDataType dt = kBF ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  fa_status st = encode_tensor_map(&tmk, dt, 2, p.k_cache, dims, strides, box, sw);
   if (st != FA_OK) return st;
-  st = encode_tensor_map(&tmv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p.v_cache, dims, strides, box, sw);
+  st = encode_tensor_map(&tmv, dt, 2, p.v_cache, dims, strides, box, sw);
   if (st != FA_OK) return st;
 
   const int group = p.hq / p.hkv;
@@ -636,7 +763,7 @@ fa_status launch_sk(const fa_decode_params& p, int n_workers, int min_tiles, voi
   A.wd = ctx.wd;
 
   auto plan = decode_plan_kernel<D>;
-  auto kern = decode_sk_kernel<D>;
+  auto kern = decode_sk_kernel<D, kBF>;
   if (count_variants) {
     note_variant(reinterpret_cast<const void*>(plan));
     note_variant(reinterpret_cast<const void*>(kern));
@@ -650,7 +777,11 @@ fa_status launch_sk(const fa_decode_params& p, int n_workers, int min_tiles, voi
   return cuda_status(cudaGetLastError());
 }
 
+// the most workers any variant runs (int8 and bf16 at d = 64: two CTAs per
+// SM); the workspace is sized for this many
 int default_workers() { return min(kMaxWorkers, sm_count() * kCtasPerSm * kWarps); }
+template <int D, bool kBF>
+int variant_workers() { return min(kMaxWorkers, sm_count() * Geom<D, kBF>::kCtas * kWarps); }
 
 int min_tiles_of(int split_keys) { return split_keys > 0 ? split_keys / kTile : 0; }
 
@@ -666,10 +797,14 @@ size_t decode_workspace_bytes(int batch, int hq, int head_dim) {
 }
 
 fa_status launch_decode(const fa_decode_params& p, int split_keys, const LaunchCtx& ctx) {
-  if (p.kv_dtype != FA_I8) return FA_ERR_UNSUPPORTED;
-  const int workers = default_workers();
-  if (p.head_dim == 128) return launch_sk<128>(p, workers, min_tiles_of(split_keys), p.workspace, true, ctx);
-  if (p.head_dim == 64) return launch_sk<64>(p, workers, min_tiles_of(split_keys), p.workspace, true, ctx);
+  const int mt = min_tiles_of(split_keys);
+  if (p.kv_dtype == FA_I8) {
+    if (p.head_dim == 128) return launch_sk<128, false>(p, variant_workers<128, false>(), mt, p.workspace, true, ctx);
+    if (p.head_dim == 64) return launch_sk<64, false>(p, variant_workers<64, false>(), mt, p.workspace, true, ctx);
+  } else if (p.kv_dtype == FA_BF16) {
+    if (p.head_dim == 128) return launch_sk<128, true>(p, variant_workers<128, true>(), mt, p.workspace, true, ctx);
+    if (p.head_dim == 64) return launch_sk<64, true>(p, variant_workers<64, true>(), mt, p.workspace, true, ctx);
+  }
   return FA_ERR_UNSUPPORTED;
 }
 
@@ -751,8 +886,8 @@ fa_status launch_decode_noalloc(const fa_decode_params& p, int split_keys, long 
   fa_status st = noalloc_scratch(&scratch, &ctx.wd.word);
   if (st != FA_OK) return st;
   // (no note_variant here: its bookkeeping set may allocate host memory)
-  if (p.head_dim == 128) return launch_sk<128>(p, workers, min_tiles_of(split_keys), scratch, false, ctx);
-  if (p.head_dim == 64) return launch_sk<64>(p, workers, min_tiles_of(split_keys), scratch, false, ctx);
+  if (p.head_dim == 128) return launch_sk<128, false>(p, workers, min_tiles_of(split_keys), scratch, false, ctx);
+  if (p.head_dim == 64) return launch_sk<64, false>(p, workers, min_tiles_of(split_keys), scratch, false, ctx);
   return FA_ERR_UNSUPPORTED;
 }
 

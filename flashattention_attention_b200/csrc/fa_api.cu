@@ -170,7 +170,8 @@ fa_status fa_attention_fwd(const fa_fwd_params* p, fa_stream_t stream) {
     if (p->cu_seqlens_k != nullptr) return FA_ERR_INVALID;
   }
   if (p->q_dtype == FA_F32) {
-    if (p->kv_dtype != FA_F32) return FA_ERR_INVALID;
+    if (p->kv_dtype != FA_F32 && p->kv_dtype != FA_I8) return FA_ERR_INVALID;
+    if (p->kv_dtype == FA_I8 && (p->k_scales == nullptr || p->v_scales == nullptr)) return FA_ERR_INVALID;
     if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
     if (p->head_dim > 256) return FA_ERR_UNSUPPORTED;
   } else if (p->q_dtype == FA_BF16) {

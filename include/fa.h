@@ -108,10 +108,14 @@ FA_API fa_status fa_compress_kv(const void *x, fa_dtype x_dtype, int64_t rows, i
  * sequence (the mean of V; zeros when s_k = 0) -- SKaiNET-transformers
  * PR #419, Summary, "empty sliding-window bands reproduce the engine's
  * uniform softmax".
- * dtypes: q_dtype FA_F32 (then kv_dtype FA_F32, CUDA-core fp32 path) or
- * FA_BF16 (then kv_dtype FA_BF16, or FA_I8 with k_scales/v_scales
- * [batch*hkv, seqlen_k] dense or [hkv, total_k] varlen, one fp32 scale per
- * (token, kv-head) as fa_compress_kv writes them).  out has q's dtype.
+ * dtypes: q_dtype FA_F32 (CUDA-core fp32 path; kv_dtype FA_F32 or FA_I8) or
+ * FA_BF16 (tensor-core path; kv_dtype FA_BF16 or FA_I8).  FA_I8 K/V come
+ * with k_scales/v_scales [batch*hkv, seqlen_k] dense or [hkv, total_k]
+ * varlen, one fp32 scale per (token, kv-head) as fa_compress_kv writes them
+ * (16-byte aligned on the BF16 path).  The kernels dequantise c * s on chip
+ * (fkl_python PR #6, Summary): exactly in fp32 on the F32 path; on the BF16
+ * path c * s is formed exactly in fp32 and rounded once to bf16, the
+ * tensor-core operand type.  out has q's dtype.
  * head_dim: F32 path any multiple of 32 up to 256; BF16/I8 paths 64 or 128.
  */
 typedef struct {

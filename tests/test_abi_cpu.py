@@ -156,13 +156,14 @@ def test_decode_rejects_bad_arguments(fa):
 
 
 def test_workspace_size_formula(fa):
-    # tile plan (int32 [B+1], 256-byte padded), then one (d + 2)-float record per
-    # (sequence, q-head) and per (worker warp, head of a group of at most 8);
-    # without a GPU the library assumes 148 SMs: 148 * 2 CTAs * 4 warps
+    # tile plan (int32 prefix [B+1] and per-segment counters [B*hq], 256-byte
+    # padded), then one (d + 2)-float record per (sequence, q-head) and per
+    # (worker warp, head of a group of at most 8); without a GPU the library
+    # assumes 148 SMs: 148 * 2 CTAs * 4 warps
     workers = 148 * 2 * 4
-    plan = lambda b: ((b + 1) * 4 + 255) // 256 * 256
-    assert fa.decode_workspace_size(16, 32, 32768, 128) == plan(16) + (16 * 32 + workers * 8) * 130 * 4
-    assert fa.decode_workspace_size(1, 2, 256, 64) == plan(1) + (1 * 2 + workers * 2) * 66 * 4
+    plan = lambda b, hq: ((b + 1 + b * hq) * 4 + 255) // 256 * 256
+    assert fa.decode_workspace_size(16, 32, 32768, 128) == plan(16, 32) + (16 * 32 + workers * 8) * 130 * 4
+    assert fa.decode_workspace_size(1, 2, 256, 64) == plan(1, 2) + (1 * 2 + workers * 2) * 66 * 4
     assert fa.decode_workspace_size(0, 1, 1, 64) == 0
 
 

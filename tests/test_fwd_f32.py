@@ -110,3 +110,41 @@ def test_empty_band_rows_are_mean_of_v():
     for h in range(2):
         np.testing.assert_allclose(got[h, :30], np.broadcast_to(2 * v[h].double().numpy().mean(0), (30, 64)),
                                    atol=1e-6)
+
+
+I8_CASES = [
+    # B, hq, hkv, s_q, s_k, d, causal, window
+    (1, 2, 2, 64, 64, 64, True, 0),
+    (1, 8, 2, 100, 100, 128, True, 17),   # GQA + window
+    (2, 4, 2, 33, 127, 32, False, 0),     # ragged 33/127
+    (2, 2, 1, 90, 40, 64, True, 0),       # s_q > s_k: empty rows get the mean of dequantised V
+]
+
+
+@pytest.mark.parametrize("case", I8_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_int8_kv_exact_vs_dequantised_oracle(case):
+    """fkl_python PR #6, Verification, 'FA int8-KV exact vs dequantized
+    oracle': fp32 queries over an int8 cache made by fa_compress_kv from fp32
+    K/V (codes and scales bit-exact with the oracle's quantiser) match the fp64
+    oracle run on the dequantised cache within the fp32 gate."""
+    from flashattention_attention_b200 import fa
+    B, hq, hkv, s_q, s_k, d, causal, window = case
+    rng = np.random.default_rng(50 + sum(case))
+    q = inputs.normal(rng, (B * hq, s_q, d), torch.float32)
+    k = inputs.normal(rng, (B * hkv, s_k, d), torch.float32)
+    v = inputs.normal(rng, (B * hkv, s_k, d), torch.float32)
+    kc, ks = fa.compress_kv(k.cuda())
+    vc, vs = fa.compress_kv(v.cuda())
+    rk, rks = oracle.compress_kv(k)
+    rv, rvs = oracle.compress_kv(v)
+    assert np.array_equal(kc.cpu().numpy(), rk) and np.array_equal(vc.cpu().numpy(), rv)
+    assert np.array_equal(ks.cpu().numpy().view(np.uint32), rks.view(np.uint32))
+    assert np.array_equal(vs.cpu().numpy().view(np.uint32), rvs.view(np.uint32))
+    out = fa.attention_fwd(q.cuda(), kc, vc, k_scales=ks, v_scales=vs, hq=hq, hkv=hkv, causal=causal,
+                           window=window, scale=0.3, epilogue=[("mul", 2.0), ("add", -1.0)])
+    torch.cuda.synchronize()
+    assert fa.check_device_error() == fa.FA_OK
+    ref = oracle.attention(q, oracle.dequantize(rk, rks), oracle.dequantize(rv, rvs), hq=hq, hkv=hkv,
+                           causal=causal, window=window, scale=0.3, epilogue=[("mul", 2.0), ("add", -1.0)])
+    # |Mul(2)| doubles the absolute error of the normalised output
+    check(out.cpu(), ref, tol=2 * TOL)
