@@ -101,57 +101,105 @@ def prefill_flops(w):
 
 # ---------------------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock, power and clock-event reasons of one GPU every
+    5 ms from a background thread through NVML (the data nvidia-smi prints),
+    and summarises the samples taken inside the marked timed region.  Falls
+    back to an `nvidia-smi -lms 20` child process when NVML is unavailable."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
         self.dev = device_index
+        self.samples = []   # (time, sm_mhz, max_mhz, power_w, [reasons])
+        self.window = None
+        self.stop = None
+        self.thread = None
         self.proc = None
         self.path = os.path.join("/tmp", f"fa_bench_clocks_{os.getpid()}.csv")
 
+    def _nvml_loop(self, nv, h):
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.perf_counter(), float(sm), float(mx), pw,
+                                     [n for n, bit in self.REASONS if rs & bit]))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+            ent = vis[self.dev] if self.dev < len(vis) else str(self.dev)
+            h = (nv.nvmlDeviceGetHandleByUUID(ent) if ent.startswith(("GPU-", "MIG-"))
+                 else nv.nvmlDeviceGetHandleByIndex(int(ent)))
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self.thread.start()
+        except Exception:
+            self.thread = None
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                     "-lms", "20"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            except OSError:
+                self.proc = None
+        time.sleep(0.3)
         return self
 
+    def mark(self, t0, t1):
+        """The timed region, as perf_counter() times."""
+        self.window = (t0, t1)
+
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+            try:
+                for line in open(self.path):
+                    f = [x.strip() for x in line.split(",")]
+                    if len(f) >= 7 and f[0].replace(".", "").isdigit():
+                        rs = [n for n, v in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                                 "sw_power_cap"), f[3:7]) if v.lower().startswith("active")]
+                        self.samples.append((None, float(f[0]), float(f[1]),
+                                             float(f[2]) if f[2].replace(".", "").isdigit() else 0.0, rs))
+            except OSError:
+                pass
 
     def summary(self):
-        rows = []
-        try:
-            for line in open(self.path):
-                f = [x.strip() for x in line.split(",")]
-                if len(f) >= 9 and f[1].replace(".", "").isdigit():
-                    rows.append(f)
-        except OSError:
-            pass
+        rows = self.samples
+        if self.window is not None and rows and rows[0][0] is not None:
+            t0, t1 = self.window
+            inside = [r for r in rows if t0 <= r[0] <= t1]
+            rows = inside or rows
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
-        busy = [r for r in rows if pw and float(r[3]) > 0.5 * max(pw)] or rows
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in busy for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
-        return {"sm_mhz": statistics.median(float(r[1]) for r in busy),
-                "sm_max_mhz": max(float(r[2]) for r in rows), "reasons": reasons,
-                "samples": len(busy), "power_w_max": max(pw) if pw else None}
+        reasons = sorted({n for r in rows for n in r[4]})
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": max(r[2] for r in rows),
+                "reasons": reasons, "samples": len(rows), "power_w_max": round(max(r[3] for r in rows), 1),
+                "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------- GPU arm
-def time_launches(fn, steps, warmup, torch, dist=None):
+def time_launches(fn, steps, warmup, torch, dist=None, clocks=None):
     """Warm up, then time exactly `steps` calls between barriers and
-    synchronisations with CUDA events on the current stream; max over ranks."""
+    synchronisations with CUDA events on the current stream; max over ranks.
+    `clocks` (a ClockSampler) is told the host-side span of the timed region."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
@@ -160,11 +208,14 @@ def time_launches(fn, steps, warmup, torch, dist=None):
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
     e0.record()
     for _ in range(steps):
         fn()
     e1.record()
     torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.mark(t0, time.perf_counter())
     if dist is not None:
         dist.barrier()
     ms = e0.elapsed_time(e1)
@@ -198,7 +249,7 @@ def gpu_arm(args, rank, world, dist):
         return res
     l0 = fa.kernel_launches()
     with ClockSampler(dev.index or 0) as clocks:
-        ms = time_launches(prefill, args.steps, args.warmup, torch, dist)
+        ms = time_launches(prefill, args.steps, args.warmup, torch, dist, clocks)
     launches = fa.kernel_launches() - l0 - args.warmup * 1
     clk = clocks.summary()
     assert fa.check_device_error() == fa.FA_OK

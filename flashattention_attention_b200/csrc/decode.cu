@@ -6,11 +6,12 @@
 //
 // Work decomposition (stream-K): the 32-key tiles of every (sequence, KV
 // head) segment are laid end to end, T tiles in all, and a persistent grid of
-// P warps ("workers", 4 per CTA, 2 CTAs per SM) takes equal contiguous ranges
-// [w*T/P, (w+1)*T/P).  Each worker streams its tiles -- K codes, V codes and
-// their fp32 scales -- through its own 3-stage TMA ring (128-byte swizzle,
-// bounded mbarrier waits), straight across segment boundaries, so the ring
-// never drains and every SM gets the same number of bytes.  When a worker's
+// P warps ("workers", 4 per CTA, 2 CTAs per SM; 1 for bf16 at d = 128) takes
+// equal contiguous ranges [w*T/P, (w+1)*T/P).  Each worker streams its tiles
+// -- K codes, V codes and their fp32 scales -- through its own 3-stage TMA
+// ring (128-byte swizzle, bounded mbarrier waits), straight across segment
+// boundaries, so the ring never drains and every SM gets the same number of
+// bytes.  When a worker's
 // range leaves a segment it writes its partial softmax state (m, l, O) for
 // the segment's G = hq/hkv query heads to record (segment + worker) and
 // counts itself done on the segment; the last worker to finish a segment
@@ -49,8 +50,7 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kTile = 32;    // keys per tile
-constexpr int kStages = 3;
-constexpr int kCtasPerSm = 2;  // int8 (and bf16 at d = 64); bf16 at d = 128 fits one
+constexpr int kMaxCtasPerSm = 2;  // int8 and bf16 at d = 64; bf16 at d = 128 fits one
 constexpr int kMaxWorkers = 4096;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -82,11 +82,15 @@ struct Geom {
   // swizzle of 64-dim chunks [32 rows x 128 B]
   static constexpr int kSwzMask = (kBF || D == 128) ? 0x70 : 0x30;
   static constexpr int kChunkBytes = kTile * 128;
-  static constexpr int kCtas = (kBF && D == 128) ? 1 : kCtasPerSm;
+  static constexpr int kStages = 3;
+  static constexpr int kCtas = (kBF && D == 128) ? 1 : 2;
   static constexpr int kSmem = kWarps * kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
 };
 static_assert(Geom<128, true>::kSmem <= 232448, "shared memory budget");
-static_assert(2 * Geom<128, false>::kSmem <= 232448 && 2 * Geom<64, true>::kSmem <= 232448, "two CTAs per SM");
+static_assert(2 * Geom<128, false>::kSmem <= 232448 && 2 * Geom<64, false>::kSmem <= 232448 &&
+                  2 * Geom<64, true>::kSmem <= 232448,
+              "CTAs per SM");
+static_assert(Geom<128, false>::kCtas <= kMaxCtasPerSm && Geom<64, true>::kCtas <= kMaxCtasPerSm, "workers");
 
 // TMA swizzle of a byte offset inside a tile whose base is aligned to the
 // swizzle period: bits [4,7) (128B) or [4,6) (64B) ^= bits [7,10) / [7,9).
@@ -290,6 +294,7 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
     decode_sk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const SkArgs A) {
   using G = Geom<D, kBF>;
+  constexpr int kStages = G::kStages;
   constexpr int kSteps = D / 16;      // k-steps of the S MMA
   constexpr int kChunks = D / 64;     // 16-byte chunks per thread per K row
   constexpr int kMT = D / 16;         // O^T m-tiles (dims)
@@ -695,21 +700,6 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
   if (cur_seg >= 0) finish(cur_seg);
 }
 
-// SMs of the current device (cached per device).
-int sm_count() {
-  static std::mutex mu;
-  static int counts[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  std::lock_guard<std::mutex> lk(mu);
-  if (counts[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    counts[dev] = n;
-  }
-  return counts[dev];
-}
-
 // plan (prefix [B+1]) and counters [B*hkv <= B*hq], 256-byte padded
 size_t plan_bytes(int batch, int hq) {
   return (static_cast<size_t>(batch + 1 + static_cast<size_t>(batch) * hq) * sizeof(int32_t) + 255) / 256 * 256;
@@ -779,9 +769,9 @@ fa_status launch_sk(const fa_decode_params& p, int n_workers, int min_tiles, voi
 
 // the most workers any variant runs (int8 and bf16 at d = 64: two CTAs per
 // SM); the workspace is sized for this many
-int default_workers() { return min(kMaxWorkers, sm_count() * kCtasPerSm * kWarps); }
+int default_workers() { return min(kMaxWorkers, device_sm_count() * kMaxCtasPerSm * kWarps); }
 template <int D, bool kBF>
-int variant_workers() { return min(kMaxWorkers, sm_count() * Geom<D, kBF>::kCtas * kWarps); }
+int variant_workers() { return min(kMaxWorkers, device_sm_count() * Geom<D, kBF>::kCtas * kWarps); }
 
 int min_tiles_of(int split_keys) { return split_keys > 0 ? split_keys / kTile : 0; }
 

@@ -32,6 +32,25 @@ long long watchdog_budget() {
   return g_budget;
 }
 
+}  // namespace
+
+// SMs of the current device (cached per device; 148 if the query fails).
+int device_sm_count() {
+  static std::mutex mu;
+  static int counts[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(mu);
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
+namespace {
+
 fa_status status_word(unsigned int** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;

@@ -36,6 +36,9 @@ fa_status encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int ran
                             const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
                             CUtensorMapSwizzle swizzle);
 
+// SMs of the current device (cached per device).
+int device_sm_count();
+
 inline fa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
 
 }  // namespace fa

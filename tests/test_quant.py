@@ -75,3 +75,28 @@ def test_full_decode_cache_rows(decode_workload):
         rows = torch.cat([t[b * w.hkv:(b + 1) * w.hkv, :w.lengths[b]].reshape(-1, w.d)
                           for b in range(w.batch)])
         assert_bit_exact(rows)
+
+
+def test_near_ties_fp32():
+    """Rows built so that most quotients x / s fall within a few ulps of a
+    half-integer (k + 0.5), where a quotient that is not the correctly
+    rounded one would flip the code; s takes random significands over many
+    binades (both the reciprocal-and-correction path and, for |s| beyond
+    2^60 or below 2^-60, the IEEE-division path)."""
+    rng = np.random.default_rng(11)
+    rows, d = 1 << 15, 128
+    expo = rng.integers(-70, 70, rows).astype(np.float64)
+    s_target = (1.0 + rng.random(rows)) * np.exp2(expo)
+    amax = (s_target * 127.0).astype(np.float32)
+    s = amax / np.float32(127.0)                               # what the quantiser computes
+    k = rng.integers(0, 127, (rows, d - 1)).astype(np.float32)
+    x = ((k + np.float32(0.5)) * s[:, None]).astype(np.float32)
+    step = rng.integers(-3, 4, (rows, d - 1))
+    for _ in range(3):
+        up, dn = step > 0, step < 0
+        x = np.where(up, np.nextafter(x, np.float32(np.inf)), np.where(dn, np.nextafter(x, np.float32(-np.inf)), x))
+        step = step - np.sign(step)
+    x = np.minimum(x, amax[:, None])
+    x *= np.where(rng.random((rows, d - 1)) < 0.5, np.float32(-1), np.float32(1))
+    full = np.concatenate([amax[:, None], x], axis=1).astype(np.float32)
+    assert_bit_exact(torch.from_numpy(full))
