@@ -42,6 +42,7 @@
 // scores are masked, and in a tile that holds such rows the V rows are zeroed
 // in shared memory before P V, so 0 * NaN never reaches O.
 #include <mutex>
+#include <type_traits>
 
 #include "internal.h"
 
@@ -59,7 +60,8 @@ struct SkArgs {
   const float* k_scales;    // [B*hkv, cap]
   const float* v_scales;
   const int32_t* seqlens;   // [B]
-  const int32_t* prefix;    // [B+1]: tiles (x hkv) before sequence b; prefix[B] = T
+  const int32_t* prefix;    // [B+1]: tiles (x hkv) before sequence b; prefix[B] = T (plan kernel)
+  int smem_prefix;          // 1: each CTA recomputes the prefix in shared memory (small batches)
   float* rec_o;             // [B*hkv + P][G][D]
   float* rec_ml;            // [B*hkv + P][G][2]
   int32_t* counters;        // [B*hkv]: workers done with each segment (zeroed by the plan)
@@ -85,6 +87,9 @@ struct Geom {
   static constexpr int kStages = 3;
   static constexpr int kCtas = (kBF && D == 128) ? 1 : 2;
   static constexpr int kSmem = kWarps * kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  // sequences whose tile prefix fits in the shared memory the CTAs per SM
+  // leave over (228 KB per SM, 1 KB reserved per CTA, 256 B margin)
+  static constexpr int kPrefixCap = ((233472 / kCtas) - 1024 - kSmem - 256) / 4 - 1;
 };
 static_assert(Geom<128, true>::kSmem <= 232448, "shared memory budget");
 static_assert(2 * Geom<128, false>::kSmem <= 232448 && 2 * Geom<64, false>::kSmem <= 232448 &&
@@ -128,6 +133,16 @@ __device__ __forceinline__ uint32_t i8x2_to_f16x2_even(uint32_t w) {
 }
 // fp16x2 of the signed bytes 1 and 3 of w (exact).
 __device__ __forceinline__ uint32_t i8x2_to_f16x2_odd(uint32_t w) { return i8x2_to_f16x2_even(w >> 8); }
+
+// fp16x2 pairs 1152 + c of the signed bytes of w: bytes 0, 2 -> even and
+// 1, 3 -> odd (exact; the caller removes the bias).  byte ^ 0x80 = c + 128
+// becomes the low mantissa byte of 1024 (fp16 0x6400).
+__device__ __forceinline__ void i8x4_to_f16x2_biased(uint32_t w, uint32_t& even, uint32_t& odd) {
+  const uint32_t x = w ^ 0x80808080u;
+  even = prmt(x, 0x64646464u, 0x4240);
+  odd = prmt(x, 0x64646464u, 0x4341);
+}
+constexpr float kCodeBias = 1152.0f;
 
 // Four 8x8 b16 matrices; lane l gives the row address of matrix l / 8, row l % 8.
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
@@ -182,6 +197,14 @@ __device__ __forceinline__ int tiles_of(int L, int window) {
   return L > t_begin ? (L - t_begin + kTile - 1) / kTile : 0;
 }
 
+// Programmatic dependent launch: the plan kernel lets the decode kernel
+// start at once; the decode kernel waits for the plan's completion (its
+// zeroed counters) only where it first needs them.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // The worker whose range [w*T/P, (w+1)*T/P) holds tile x.
 __device__ __forceinline__ int worker_of(long long x, long long T, long long P) {
   return static_cast<int>((x * P + P - 1) / T);
@@ -203,6 +226,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
                                                            int32_t* __restrict__ prefix,
                                                            int32_t* __restrict__ counters,
                                                            __nv_bfloat16* __restrict__ out, Epilogue epi) {
+  griddep_launch_dependents();
   __shared__ int32_t warp_sums[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nthreads = blockDim.x;
@@ -252,30 +276,30 @@ struct Cursor {
   int64_t kv_row0;  // cache row of key 0 of (b, g)
 };
 
-__device__ __forceinline__ int seq_tiles(const SkArgs& A, int b) {
-  return (A.prefix[b + 1] - A.prefix[b]) / A.hkv;
+__device__ __forceinline__ int seq_tiles(const SkArgs& A, const int32_t* pre, int b) {
+  return (pre[b + 1] - pre[b]) / A.hkv;
 }
 __device__ __forceinline__ void set_segment(const SkArgs& A, Cursor& c) {
   int k_lo;
   key_range(clamp_len(A.seqlens[c.b], A.cap), A.window, k_lo, c.t_begin);
   c.kv_row0 = (static_cast<int64_t>(c.b) * A.hkv + c.g) * A.cap;
 }
-__device__ __forceinline__ Cursor locate(const SkArgs& A, long long x) {
+__device__ __forceinline__ Cursor locate(const SkArgs& A, const int32_t* pre, long long x) {
   int lo = 0, hi = A.batch - 1;  // largest b with prefix[b] <= x
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (A.prefix[mid] <= x) lo = mid; else hi = mid - 1;
+    if (pre[mid] <= x) lo = mid; else hi = mid - 1;
   }
   Cursor c;
   c.b = lo;
-  c.Tb = seq_tiles(A, lo);
-  const long long y = x - A.prefix[lo];
+  c.Tb = seq_tiles(A, pre, lo);
+  const long long y = x - pre[lo];
   c.g = static_cast<int>(y / c.Tb);
   c.t = static_cast<int>(y % c.Tb);
   set_segment(A, c);
   return c;
 }
-__device__ __forceinline__ void advance(const SkArgs& A, Cursor& c) {
+__device__ __forceinline__ void advance(const SkArgs& A, const int32_t* pre, Cursor& c) {
   if (++c.t < c.Tb) return;
   c.t = 0;
   if (++c.g < A.hkv) {
@@ -285,7 +309,7 @@ __device__ __forceinline__ void advance(const SkArgs& A, Cursor& c) {
   c.g = 0;
   do {
     ++c.b;
-  } while (c.b < A.batch && (c.Tb = seq_tiles(A, c.b)) == 0);
+  } while (c.b < A.batch && (c.Tb = seq_tiles(A, pre, c.b)) == 0);
   if (c.b < A.batch) set_segment(A, c);
 }
 
@@ -303,6 +327,9 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kStages * G::kStageBytes);
   __shared__ int abort_flag;
 
+  int32_t* s_pre = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 256);
+  __shared__ int32_t warp_sums[kWarps];
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, qq = lane & 3;
   if (threadIdx.x == 0) abort_flag = 0;
@@ -310,9 +337,37 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[warp * kStages + s], 1);
     fence_barrier_init();
   }
+  // the tile prefix over sequences: computed here for small batches (no
+  // dependence on the plan kernel until the first counter), else the plan's
+  const int32_t* pre = A.prefix;
+  if (A.smem_prefix) {
+    int32_t carry = 0;
+    for (int b0 = 0; b0 < A.batch; b0 += kWarps * 32) {
+      const int b = b0 + static_cast<int>(threadIdx.x);
+      const int32_t own = b < A.batch ? tiles_of(clamp_len(A.seqlens[b], A.cap), A.window) * A.hkv : 0;
+      int32_t incl = own;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      if (lane == 31) warp_sums[warp] = incl;
+      __syncthreads();
+      int32_t before = carry;
+      for (int v = 0; v < warp; ++v) before += warp_sums[v];
+      if (b < A.batch) s_pre[b] = before + incl - own;
+      for (int v = warp; v < kWarps; ++v) before += warp_sums[v];
+      carry = before;  // the same in every thread: the running total
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) s_pre[A.batch] = carry;
+    pre = s_pre;
+  } else {
+    griddep_wait();
+  }
   __syncthreads();
 
-  const long long T = A.prefix[A.batch];
+  const long long T = pre[A.batch];
   const long long P = effective_workers(A, T);
   const long long w = static_cast<long long>(blockIdx.x) * kWarps + warp;
   if (T == 0 || w >= P) return;
@@ -322,7 +377,7 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
 
   auto stage_ptr = [&](int s) { return smem + (warp * kStages + s) * G::kStageBytes; };
   // issue cursor (lane 0 runs it kStages tiles ahead of the compute cursor)
-  Cursor ic = locate(A, t_first);
+  Cursor ic = locate(A, pre, t_first);
   auto issue = [&](int i) {
     const int s = i % kStages;
     const int key0 = ic.t_begin + ic.t * kTile;
@@ -342,7 +397,7 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
       bulk_load(st + G::kScaleOff, A.k_scales + kv_row0 + key0, kTile * 4, bar);
       bulk_load(st + G::kScaleOff + kTile * 4, A.v_scales + kv_row0 + key0, kTile * 4, bar);
     }
-    advance(A, ic);
+    advance(A, pre, ic);
   };
   if (lane == 0) {
     for (int i = 0; i < min(kStages, my_tiles); ++i) issue(i);
@@ -351,6 +406,7 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
   // ---- per-segment state
   uint32_t qb0[kSteps], qb1[kSteps];
   float qs0 = 0.f, qs1 = 0.f;
+  float cb0 = 0.f, cb1 = 0.f;  // int8: 1152 * sum of the (prescaled fp16) q of heads 2qq, 2qq+1
   float o[kMT][4];
   float m_run[2], l_run[2];
   auto reset = [&]() {
@@ -395,14 +451,26 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
     if (amax > 0.f) frexpf(amax, &ex);
     const int kexp = amax > 0.f ? 15 - ex : 0;  // largest |q| * 2^kexp in [2^14, 2^15)
     const float qs_own = ldexpf(A.scale_log2, -kexp);
+    // K codes enter the MMA as 1152 + c, so every score of head n carries
+    // 1152 * (sum over dims of its fp16 q); the sum of these fp16 values is
+    // exact in fp64
+    double qsum = 0.0;
 #pragma unroll
     for (int ks = 0; ks < kSteps; ++ks) {
       qb0[ks] = pack_f16x2(ldexpf(qv[4 * ks + 0], kexp), ldexpf(qv[4 * ks + 2], kexp));
       qb1[ks] = pack_f16x2(ldexpf(qv[4 * ks + 1], kexp), ldexpf(qv[4 * ks + 3], kexp));
+      const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&qb0[ks]));
+      const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&qb1[ks]));
+      qsum += (static_cast<double>(f0.x) + f0.y) + (static_cast<double>(f1.x) + f1.y);
     }
-    // logit multipliers of this thread's two score columns (heads 2qq, 2qq+1)
+    qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
+    qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
+    const float cb_own = static_cast<float>(qsum * static_cast<double>(kCodeBias));
+    // logit multipliers and biases of this thread's two score columns (heads 2qq, 2qq+1)
     qs0 = __shfl_sync(0xffffffffu, qs_own, (2 * qq) * 4);
     qs1 = __shfl_sync(0xffffffffu, qs_own, (2 * qq + 1) * 4);
+    cb0 = __shfl_sync(0xffffffffu, cb_own, (2 * qq) * 4);
+    cb1 = __shfl_sync(0xffffffffu, cb_own, (2 * qq + 1) * 4);
   };
   // partial state of segment `seg` -> record (seg + w)
   auto finalize = [&](int seg) {
@@ -457,8 +525,8 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
   // The last worker done with a segment merges every record of it.
   auto segment_workers = [&](int seg, int& w_lo, int& w_hi) {
     const int b = seg / A.hkv, g = seg % A.hkv;
-    const int Tb = seq_tiles(A, b);
-    const long long a = A.prefix[b] + static_cast<long long>(g) * Tb;
+    const int Tb = seq_tiles(A, pre, b);
+    const long long a = pre[b] + static_cast<long long>(g) * Tb;
     w_lo = worker_of(a, T, P);
     w_hi = worker_of(a + Tb - 1, T, P);
   };
@@ -467,7 +535,10 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
     __threadfence();  // each lane's record stores are visible device-wide ...
     __syncwarp();     // ... before lane 0 counts the warp done
     int prev = 0;
-    if (lane == 0) prev = atomicAdd(&A.counters[seg], 1);
+    if (lane == 0) {
+      griddep_wait();  // the plan kernel has zeroed the counters
+      prev = atomicAdd(&A.counters[seg], 1);
+    }
     prev = __shfl_sync(0xffffffffu, prev, 0);
     int w_lo, w_hi;
     segment_workers(seg, w_lo, w_hi);
@@ -518,7 +589,7 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
     }
   };
 
-  Cursor cc = locate(A, t_first);
+  Cursor cc = locate(A, pre, t_first);
   int cur_seg = -1;
   int seg_t_begin = 0, k_lo = 0, key_end = 0;
   for (int i = 0; i < my_tiles; ++i) {
@@ -576,74 +647,94 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
         const uint4& B4 = kb[ks / 4];
         const uint32_t wa = (ks % 4 == 0) ? A4.x : (ks % 4 == 1) ? A4.y : (ks % 4 == 2) ? A4.z : A4.w;
         const uint32_t wb = (ks % 4 == 0) ? B4.x : (ks % 4 == 1) ? B4.y : (ks % 4 == 2) ? B4.z : B4.w;
-        mma16816(sc[mt], i8x2_to_f16x2_even(wa), i8x2_to_f16x2_even(wb), i8x2_to_f16x2_odd(wa),
-                 i8x2_to_f16x2_odd(wb), qb0[ks], qb1[ks]);
+        uint32_t ae, ao, be, bo;
+        i8x4_to_f16x2_biased(wa, ae, ao);
+        i8x4_to_f16x2_biased(wb, be, bo);
+        mma16816(sc[mt], ae, be, ao, bo, qb0[ks], qb1[ks]);
       }
     }
 
-    // ---- online softmax (per head column), masks by key position
-    float x[2][4];
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int kl = 16 * mt + gq + 8 * hf;
-        const int key = key0 + kl;
-        const bool ok = key >= k_lo && key < key_end;
-        const float kscale = kBF ? 1.f : ksc[kl];
-        x[mt][2 * hf + 0] = ok ? sc[mt][2 * hf + 0] * kscale * qs0 : -INFINITY;
-        x[mt][2 * hf + 1] = ok ? sc[mt][2 * hf + 1] * kscale * qs1 : -INFINITY;
-        mx0 = fmaxf(mx0, x[mt][2 * hf + 0]);
-        mx1 = fmaxf(mx1, x[mt][2 * hf + 1]);
-      }
-    }
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-    }
-    // the running maxima move only when a tile raises them, and the O
-    // rescale runs only when some head of the warp moved
-    const bool up0 = mx0 > m_run[0], up1 = mx1 > m_run[1];
-    if (__any_sync(0xffffffffu, up0 || up1)) {
-      const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
-      const float r0 = mn0 == -INFINITY ? 0.f : mn0, r1 = mn1 == -INFINITY ? 0.f : mn1;
-      const float al0 = ex2_approx(m_run[0] - r0), al1 = ex2_approx(m_run[1] - r1);
-      m_run[0] = mn0;
-      m_run[1] = mn1;
-      l_run[0] *= al0;
-      l_run[1] *= al1;
-#pragma unroll
-      for (int m = 0; m < kMT; ++m) {
-        o[m][0] *= al0; o[m][2] *= al0;
-        o[m][1] *= al1; o[m][3] *= al1;
-      }
-    }
-    const float ref0 = m_run[0] == -INFINITY ? 0.f : m_run[0];
-    const float ref1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
+    // ---- online softmax (per head column); only a tile that reaches past
+    // the band's ends masks by key position (warp-uniform choice)
     uint32_t pb[2][2];  // [mt][b0/b1] P' operand fragments
+    auto softmax = [&](auto masked_tag) {
+      constexpr bool kMasked = decltype(masked_tag)::value;
+      float x[2][4];
+      float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      uint32_t packed[2];
+      for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int kl = 16 * mt + gq + 8 * hf;
-        const int key = key0 + kl;
-        const bool ok = key >= k_lo && key < key_end;
-        const float p0 = ex2_approx(x[mt][2 * hf + 0] - ref0);
-        const float p1 = ex2_approx(x[mt][2 * hf + 1] - ref1);
-        l_run[0] += p0;
-        l_run[1] += p1;
-        if constexpr (kBF) {
-          packed[hf] = pack_bf16x2(ok ? p0 : 0.f, ok ? p1 : 0.f);
-        } else {
-          const float vscale = ok ? vsc[kl] : 0.f;
-          packed[hf] = pack_f16x2(ok ? p0 * vscale : 0.f, ok ? p1 * vscale : 0.f);
+        for (int hf = 0; hf < 2; ++hf) {
+          const int kl = 16 * mt + gq + 8 * hf;
+          const int key = key0 + kl;
+          const bool ok = !kMasked || (key >= k_lo && key < key_end);
+          float x0, x1;
+          if constexpr (kBF) {
+            x0 = sc[mt][2 * hf + 0] * qs0;
+            x1 = sc[mt][2 * hf + 1] * qs1;
+          } else {
+            const float kscale = ksc[kl];
+            x0 = (sc[mt][2 * hf + 0] - cb0) * (kscale * qs0);
+            x1 = (sc[mt][2 * hf + 1] - cb1) * (kscale * qs1);
+          }
+          x[mt][2 * hf + 0] = ok ? x0 : -INFINITY;
+          x[mt][2 * hf + 1] = ok ? x1 : -INFINITY;
+          mx0 = fmaxf(mx0, x[mt][2 * hf + 0]);
+          mx1 = fmaxf(mx1, x[mt][2 * hf + 1]);
         }
       }
-      pb[mt][0] = transpose8x8(packed[0]);  // (head gq; keys 2qq, 2qq+1)
-      pb[mt][1] = transpose8x8(packed[1]);  // (head gq; keys 8+2qq, 8+2qq+1)
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      // the running maxima move only when a tile raises them, and the O
+      // rescale runs only when some head of the warp moved
+      const bool up0 = mx0 > m_run[0], up1 = mx1 > m_run[1];
+      if (__any_sync(0xffffffffu, up0 || up1)) {
+        const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+        const float r0 = mn0 == -INFINITY ? 0.f : mn0, r1 = mn1 == -INFINITY ? 0.f : mn1;
+        const float al0 = ex2_approx(m_run[0] - r0), al1 = ex2_approx(m_run[1] - r1);
+        m_run[0] = mn0;
+        m_run[1] = mn1;
+        l_run[0] *= al0;
+        l_run[1] *= al1;
+#pragma unroll
+        for (int m = 0; m < kMT; ++m) {
+          o[m][0] *= al0; o[m][2] *= al0;
+          o[m][1] *= al1; o[m][3] *= al1;
+        }
+      }
+      const float ref0 = m_run[0] == -INFINITY ? 0.f : m_run[0];
+      const float ref1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        uint32_t packed[2];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int kl = 16 * mt + gq + 8 * hf;
+          const int key = key0 + kl;
+          const bool ok = !kMasked || (key >= k_lo && key < key_end);
+          const float p0 = ex2_approx(x[mt][2 * hf + 0] - ref0);
+          const float p1 = ex2_approx(x[mt][2 * hf + 1] - ref1);
+          l_run[0] += p0;
+          l_run[1] += p1;
+          if constexpr (kBF) {
+            packed[hf] = kMasked ? pack_bf16x2(ok ? p0 : 0.f, ok ? p1 : 0.f) : pack_bf16x2(p0, p1);
+          } else {
+            const float vscale = ok ? vsc[kl] : 0.f;
+            packed[hf] = pack_f16x2(p0 * vscale, p1 * vscale);
+          }
+        }
+        pb[mt][0] = transpose8x8(packed[0]);  // (head gq; keys 2qq, 2qq+1)
+        pb[mt][1] = transpose8x8(packed[1]);  // (head gq; keys 8+2qq, 8+2qq+1)
+      }
+    };
+    const bool interior = key0 >= k_lo && key0 + kTile <= key_end;
+    if (interior) {
+      softmax(std::false_type{});
+    } else {
+      softmax(std::true_type{});
     }
 
     // ---- O^T += V^T . P'
@@ -695,7 +786,7 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
       fence_proxy_async_smem();
       issue(i + kStages);
     }
-    advance(A, cc);
+    advance(A, pre, cc);
   }
   if (cur_seg >= 0) finish(cur_seg);
 }
@@ -761,10 +852,24 @@ fa_status launch_sk(const fa_decode_params& p, int n_workers, int min_tiles, voi
   plan<<<1, 1024, 0, ctx.stream>>>(p.cache_seqlens, p.batch, p.hq, p.hkv, p.capacity, p.window,
                                    reinterpret_cast<int32_t*>(base), A.counters, A.out, A.epi);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem) != cudaSuccess)
+  A.smem_prefix = p.batch <= G::kPrefixCap ? 1 : 0;
+  const size_t smem = G::kSmem + (A.smem_prefix ? (static_cast<size_t>(p.batch) + 1) * 4 : 0);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           G::kSmem + (G::kPrefixCap + 1) * 4) != cudaSuccess)
     return FA_ERR_CUDA;
-  kern<<<n_workers / kWarps, kWarps * 32, G::kSmem, ctx.stream>>>(tmk, tmv, A);
-  return cuda_status(cudaGetLastError());
+  // programmatic dependent launch: the decode kernel starts while the plan
+  // kernel runs and waits for it only before touching the counters
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(n_workers / kWarps));
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = ctx.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, tmk, tmv, A));
 }
 
 // the most workers any variant runs (int8 and bf16 at d = 64: two CTAs per
