@@ -14,7 +14,10 @@ from typing import Optional, Sequence, Tuple
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libfa.so")
+# FA_LIBRARY may name another build of the same library (e.g. one compiled
+# with different tuning constants); by default the in-tree build is loaded.
+_LIB_PATH = os.environ.get("FA_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib",
+                                                          "libfa.so")
 if not os.path.exists(_LIB_PATH):
     raise ImportError(f"libfa.so not built ({_LIB_PATH}); run __graft_entry__.build() "
                       "or python flashattention_attention_b200/build.py")
