@@ -51,7 +51,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "prefill_tc_kernel<128,bf16>": ["prefill_tc.cu", "umma.cuh", "device.cuh", "layout.cuh"],
     "decode_sk_kernel<128>": ["decode.cu", "device.cuh"],
-    "compress_kernel": ["quant.cu"],
+    "compress_rows8_kernel<bf16,16>": ["quant.cu", "device.cuh"],
 }
 
 
@@ -386,10 +386,10 @@ def decode_and_quant(args, dev, peaks, world, dist, result):
         quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
         result["quantiser"] = {"rows": quant_rows, "value": round(quant_gbs * world, 1), "unit": "GB/s",
                                "us_per_step": round(quant_ms * 1e3, 2), "bytes_per_step": quant_bytes,
-                               "roofline": {"bound": "hbm", "kernel": "compress_kernel",
+                               "roofline": {"bound": "hbm", "kernel": "compress_rows8_kernel<bf16,16>",
                                             "achieved": round(quant_gbs, 1), "peak": peaks["hbm_gbs"],
                                             "unit": "GB/s", "frac": round(quant_gbs / peaks["hbm_gbs"], 4),
-                                            "traffic": measured_traffic("compress_kernel")}}
+                                            "traffic": measured_traffic("compress_rows8_kernel<bf16,16>")}}
         del rows, codes, scales
     if args.only in ("all", "decode"):
         kc, ks = fa.compress_kv(dw.k.to(dev))
