@@ -417,6 +417,7 @@ def decode_and_quant(args, dev, peaks, world, dist, result):
                                          "unit": "GB/s", "frac": round(dec_gbs / peaks["hbm_gbs"], 4),
                                          "frac_of_nominal_8000": round(dec_gbs / 8000.0, 4),
                                          "traffic": measured_traffic("decode_sk_kernel<128>")}}
+        result["decode_step_graph"] = decode_step_graph(args, dw, dq, dout, ws, kc, vc, ks, vs, peaks, world, dist)
         del kc, vc, ks, vs
         torch.cuda.empty_cache()
         # the same decode over an uncompressed bf16 cache (2 * 2d bytes per key and KV head)
@@ -437,6 +438,56 @@ def decode_and_quant(args, dev, peaks, world, dist, result):
         torch.cuda.empty_cache()
     assert fa.check_device_error() == fa.FA_OK
     return result
+
+
+def decode_step_graph(args, dw, dq, dout, ws, kc, vc, ks, vs, peaks, world, dist):
+    """One decode step of the int8-KV workload as a captured CUDA graph: append
+    the step's new K/V rows at the device-side cur_pos (quantised on the way
+    in), decode over cache_seqlens = cur_pos + 1, advance cur_pos.  Each
+    replay is a new step (the cache grows by one token per sequence)."""
+    import numpy as np
+    import torch
+    from flashattention_attention_b200 import fa
+    rng = np.random.default_rng(5)
+    rows = dw.batch * dw.hkv
+    kn = torch.from_numpy(rng.standard_normal((rows, dw.d)).astype(np.float32)).bfloat16().cuda()
+    vn = torch.from_numpy(rng.standard_normal((rows, dw.d)).astype(np.float32)).bfloat16().cuda()
+    lens0 = torch.tensor(dw.lengths, dtype=torch.int32)
+    cur = lens0.cuda()
+    lens = lens0.cuda()
+
+    def step():
+        fa.kv_append(kn, vn, kc, vc, cur, hkv=dw.hkv, k_scales=ks, v_scales=vs, cache_seqlens=lens)
+        fa.attention_decode(dq, kc, vc, lens, hq=dw.hq, hkv=dw.hkv, k_scales=ks, v_scales=vs,
+                            max_seqlen=dw.cache_capacity, workspace=ws, out=dout)
+        cur.add_(1)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    steps = max(20, args.steps)
+    if int(lens0.max()) + 1 + steps + args.warmup + 1 > dw.cache_capacity:
+        steps = dw.cache_capacity - int(lens0.max()) - args.warmup - 2
+    start = int(cur[0].item()) - dw.lengths[0]  # steps already taken (warm-up on the side stream)
+    ms = time_launches(graph.replay, steps, args.warmup, torch, dist)
+    assert fa.check_device_error() == fa.FA_OK
+    # bytes: each timed step reads every cached key (codes + scales) once, Q, and
+    # writes O, plus the append (bf16 rows in, codes + scales out)
+    first = start + args.warmup
+    keys = sum((sum(dw.lengths) + dw.batch * (first + s + 1)) for s in range(steps)) / steps
+    step_bytes = keys * dw.hkv * 2 * (dw.d + 4) + 2 * dq.numel() * 2 + 2 * rows * (2 * dw.d + dw.d + 4)
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    del graph
+    return {"workload": dw.name + "_append_decode_graph", "value": round(gbs * world, 1), "unit": "GB/s",
+            "us_per_step": round(ms * 1e3, 2), "bytes_per_step": int(step_bytes),
+            "launches_per_step": "append + plan + decode + position advance, one graph replay",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4)}}
 
 
 # ---------------------------------------------------------------------------- CPU oracle

@@ -17,6 +17,9 @@ namespace fa {
 
 // Status bits in the per-device word.
 constexpr unsigned kStatusTimeout = 1u;
+// A device-side argument (e.g. a cache slot read from device memory) was out
+// of range; the kernel skipped the work it named.
+constexpr unsigned kStatusRange = 4u;
 
 struct Watchdog {
   unsigned int* word;       // device status word (never null)

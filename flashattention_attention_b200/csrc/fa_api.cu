@@ -274,6 +274,34 @@ fa_status fa_attention_decode_noalloc(const fa_decode_params* p, fa_stream_t str
   return launch_decode_noalloc(*p, split, watchdog_budget(), reinterpret_cast<cudaStream_t>(stream));
 }
 
+fa_status fa_kv_append(const fa_kv_append_params* p, fa_stream_t stream) {
+  if (p == nullptr) return FA_ERR_INVALID;
+  if (p->batch < 0 || p->hkv < 1 || p->capacity < 1) return FA_ERR_INVALID;
+  if (p->head_dim < 16 || p->head_dim > 1024 || p->head_dim % 16 != 0) return FA_ERR_INVALID;
+  if (p->x_dtype != FA_BF16 && p->x_dtype != FA_F32) return FA_ERR_INVALID;
+  if (p->cache_dtype != FA_I8 && p->cache_dtype != FA_BF16) return FA_ERR_INVALID;
+  if (static_cast<int64_t>(p->batch) * p->hkv == 0) return FA_OK;
+  if (p->k_new == nullptr || p->v_new == nullptr || p->k_cache == nullptr || p->v_cache == nullptr ||
+      p->cur_pos == nullptr)
+    return FA_ERR_INVALID;
+  if (!aligned16(p->k_new) || !aligned16(p->v_new) || !aligned16(p->k_cache) || !aligned16(p->v_cache) ||
+      !aligned16(p->cur_pos) || (p->cache_seqlens != nullptr && !aligned16(p->cache_seqlens)))
+    return FA_ERR_INVALID;
+  if (p->cache_dtype == FA_I8 &&
+      (p->k_scales == nullptr || p->v_scales == nullptr || !aligned16(p->k_scales) || !aligned16(p->v_scales)))
+    return FA_ERR_INVALID;
+  if (p->cache_seqlens != nullptr) {
+    // every warp of sequence b reads cur_pos[b] while one writes cache_seqlens[b]
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(p->cur_pos), a1 = a0 + 4ull * p->batch;
+    const uintptr_t b0 = reinterpret_cast<uintptr_t>(p->cache_seqlens), b1 = b0 + 4ull * p->batch;
+    if (a0 < b1 && b0 < a1) return FA_ERR_INVALID;
+  }
+  LaunchCtx ctx;
+  fa_status st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  return launch_kv_append(*p, ctx);
+}
+
 fa_status fa_check_device_error(fa_stream_t stream) {
   unsigned int* word = nullptr;
   fa_status st = status_word(&word);
@@ -286,6 +314,7 @@ fa_status fa_check_device_error(fa_stream_t stream) {
     if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
   }
   if (host & kStatusTimeout) return FA_ERR_TIMEOUT;
+  if (host & kStatusRange) return FA_ERR_INVALID;
   return FA_OK;
 }
 

@@ -21,6 +21,7 @@ void note_variant(const void* kernel_fn);
 
 fa_status launch_compress(const void* x, int x_dtype, int64_t rows, int d, int8_t* codes, float* scales,
                           const LaunchCtx& ctx);
+fa_status launch_kv_append(const fa_kv_append_params& p, const LaunchCtx& ctx);
 fa_status launch_attn_f32(const fa_fwd_params& p, const LaunchCtx& ctx);
 fa_status launch_empty_rows(const fa_fwd_params& p, const LaunchCtx& ctx);
 fa_status launch_prefill_tc(const fa_fwd_params& p, const LaunchCtx& ctx);

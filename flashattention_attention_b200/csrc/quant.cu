@@ -288,6 +288,107 @@ fa_status launch_dtype(const void* x, int64_t rows, int d, int8_t* codes, float*
   return launch_typed<T, 8, 1>(x, rows, d, codes, scales, ctx);
 }
 
+// ---------------------------------------------------------------- cache append
+// One new token per sequence: rows u = b * hkv + g of k_new / v_new go to
+// cache row u * capacity + cur_pos[b] (quantised exactly as compress_kernel
+// does, or stored as bf16).  One warp per (K or V, u) row; lane layout and
+// arithmetic as in compress_kernel.  A slot outside [0, capacity) is not
+// written and is reported in the status word.
+struct AppendArgs {
+  const void* k_new;
+  const void* v_new;
+  void* k_cache;
+  void* v_cache;
+  float* k_scales;
+  float* v_scales;
+  const int32_t* cur_pos;
+  int32_t* seqlens;  // optional: seqlens[b] = cur_pos[b] + 1
+  int batch, hkv, d, capacity, cache_i8;
+  Watchdog wd;
+};
+
+template <typename T, int kChunks>
+__global__ void __launch_bounds__(kWarpsPerCta * 32) kv_append_kernel(const AppendArgs A) {
+  using V = Vec4<T>;
+  const int lane = threadIdx.x & 31;
+  const int64_t units = static_cast<int64_t>(A.batch) * A.hkv;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
+  if (w >= 2 * units) return;
+  const bool is_v = w >= units;
+  const int64_t u = is_v ? w - units : w;
+  const int b = static_cast<int>(u / A.hkv);
+  const int pos = A.cur_pos[b];
+  if (pos < 0 || pos >= A.capacity) {
+    if (lane == 0) record_status(A.wd, kStatusRange);
+    return;
+  }
+  if (A.seqlens != nullptr && !is_v && u % A.hkv == 0 && lane == 0) A.seqlens[b] = pos + 1;
+  const T* src = static_cast<const T*>(is_v ? A.v_new : A.k_new) + u * A.d;
+  const int64_t row = u * A.capacity + pos;
+  float v[kChunks][4];
+  float amax = 0.0f;
+#pragma unroll
+  for (int c = 0; c < kChunks; ++c) {
+    const int col = c * 128 + lane * 4;
+    if (col < A.d) {
+      V::widen(V::load(src + col), v[c]);
+    } else {
+      v[c][0] = v[c][1] = v[c][2] = v[c][3] = 0.0f;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(v[c][e]));
+  }
+  if (!A.cache_i8) {
+    // bf16 cache: the row as bf16 (exact for bf16 input, RNE for fp32)
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(is_v ? A.v_cache : A.k_cache) + row * A.d;
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) {
+      const int col = c * 128 + lane * 4;
+      if (col < A.d) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(v[c][0], v[c][1]);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(v[c][2], v[c][3]);
+        *reinterpret_cast<uint2*>(dst + col) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+      }
+    }
+    return;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float s = __fdiv_rn(amax, 127.0f);
+  const bool fast = s >= 0x1p-60f && s <= 0x1p60f;  // warp-uniform
+  const float y = fast ? __frcp_rn(s) : 0.0f;
+  int8_t* codes = static_cast<int8_t*>(is_v ? A.v_cache : A.k_cache) + row * A.d;
+#pragma unroll
+  for (int c = 0; c < kChunks; ++c) {
+    const int col = c * 128 + lane * 4;
+    if (col < A.d) {
+      const uint32_t packed = fast ? quantise4_fast(v[c], s, y) : quantise4_div(v[c], s);
+      *reinterpret_cast<uint32_t*>(codes + col) = packed;
+    }
+  }
+  if (lane == 0) (is_v ? A.v_scales : A.k_scales)[row] = s;
+}
+
+template <typename T, int kChunks>
+fa_status launch_append_typed(const AppendArgs& A, const LaunchCtx& ctx) {
+  const int64_t rows = 2LL * A.batch * A.hkv;
+  const int64_t blocks = (rows + kWarpsPerCta - 1) / kWarpsPerCta;
+  if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  auto kern = kv_append_kernel<T, kChunks>;
+  note_variant(reinterpret_cast<const void*>(kern));
+  kern<<<static_cast<unsigned>(blocks), kWarpsPerCta * 32, 0, ctx.stream>>>(A);
+  return cuda_status(cudaGetLastError());
+}
+
+template <typename T>
+fa_status launch_append_dtype(const AppendArgs& A, const LaunchCtx& ctx) {
+  if (A.d <= 128) return launch_append_typed<T, 1>(A, ctx);
+  if (A.d <= 256) return launch_append_typed<T, 2>(A, ctx);
+  if (A.d <= 512) return launch_append_typed<T, 4>(A, ctx);
+  return launch_append_typed<T, 8>(A, ctx);
+}
+
 }  // namespace
 
 fa_status launch_compress(const void* x, int x_dtype, int64_t rows, int d, int8_t* codes, float* scales,
@@ -295,6 +396,31 @@ fa_status launch_compress(const void* x, int x_dtype, int64_t rows, int d, int8_
   if (rows == 0) return FA_OK;
   if (x_dtype == FA_BF16) return launch_dtype<__nv_bfloat16>(x, rows, d, codes, scales, ctx);
   return launch_dtype<float>(x, rows, d, codes, scales, ctx);
+}
+
+}  // namespace fa
+
+namespace fa {
+
+fa_status launch_kv_append(const fa_kv_append_params& p, const LaunchCtx& ctx) {
+  AppendArgs A;
+  A.k_new = p.k_new;
+  A.v_new = p.v_new;
+  A.k_cache = p.k_cache;
+  A.v_cache = p.v_cache;
+  A.k_scales = p.k_scales;
+  A.v_scales = p.v_scales;
+  A.cur_pos = p.cur_pos;
+  A.seqlens = p.cache_seqlens;
+  A.batch = p.batch;
+  A.hkv = p.hkv;
+  A.d = p.head_dim;
+  A.capacity = p.capacity;
+  A.cache_i8 = p.cache_dtype == FA_I8 ? 1 : 0;
+  A.wd = ctx.wd;
+  if (static_cast<int64_t>(p.batch) * p.hkv == 0) return FA_OK;
+  if (p.x_dtype == FA_BF16) return launch_append_dtype<__nv_bfloat16>(A, ctx);
+  return launch_append_dtype<float>(A, ctx);
 }
 
 }  // namespace fa

@@ -60,6 +60,15 @@ class DecodeParams(ctypes.Structure):
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class KvAppendParams(ctypes.Structure):
+    _fields_ = [("k_new", ctypes.c_void_p), ("v_new", ctypes.c_void_p), ("x_dtype", ctypes.c_int32),
+                ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("k_scales", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
+                ("cache_dtype", ctypes.c_int32), ("cur_pos", ctypes.c_void_p),
+                ("cache_seqlens", ctypes.c_void_p), ("batch", ctypes.c_int32), ("hkv", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("capacity", ctypes.c_int32)]
+
+
 lib.fa_compress_kv.restype = ctypes.c_int
 lib.fa_compress_kv.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int32,
                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
@@ -69,6 +78,8 @@ lib.fa_decode_workspace_size.restype = ctypes.c_size_t
 lib.fa_decode_workspace_size.argtypes = [ctypes.c_int32] * 4
 lib.fa_attention_decode.restype = ctypes.c_int
 lib.fa_attention_decode.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_void_p]
+lib.fa_kv_append.restype = ctypes.c_int
+lib.fa_kv_append.argtypes = [ctypes.POINTER(KvAppendParams), ctypes.c_void_p]
 lib.fa_status_string.restype = ctypes.c_char_p
 lib.fa_status_string.argtypes = [ctypes.c_int]
 lib.fa_check_device_error.restype = ctypes.c_int
@@ -224,8 +235,32 @@ def attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
     return out
 
 
+def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              cur_pos: torch.Tensor, *, hkv: int, k_scales=None, v_scales=None, cache_seqlens=None,
+              stream=None) -> None:
+    """Write one new token per sequence (k_new, v_new [B*hkv, d]) into the
+    caches [B*hkv, cap, d] at slot cur_pos[b] (device int32 [B]); an int8
+    cache is quantised on the way in (scales required), a bf16 one stored
+    as bf16.  cache_seqlens (device int32 [B]), if given, becomes cur_pos + 1.
+    Layouts and semantics as fa_kv_append in fa.h."""
+    for name, t in (("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache), ("v_cache", v_cache),
+                    ("cur_pos", cur_pos)):
+        _contig_cuda(t, name)
+    p = KvAppendParams()
+    p.k_new, p.v_new, p.x_dtype = k_new.data_ptr(), v_new.data_ptr(), _DT[k_new.dtype]
+    p.k_cache, p.v_cache, p.cache_dtype = k_cache.data_ptr(), v_cache.data_ptr(), _DT[k_cache.dtype]
+    p.k_scales = None if k_scales is None else k_scales.data_ptr()
+    p.v_scales = None if v_scales is None else v_scales.data_ptr()
+    p.cur_pos = cur_pos.data_ptr()
+    p.cache_seqlens = None if cache_seqlens is None else cache_seqlens.data_ptr()
+    p.batch, p.hkv = cur_pos.numel(), hkv
+    p.head_dim, p.capacity = k_cache.shape[-1], k_cache.shape[1]
+    _check(lib.fa_kv_append(ctypes.byref(p), _stream(stream)), "fa_kv_append")
+
+
 def check_device_error(stream=None) -> int:
-    """Synchronise and return (then clear) the device status: FA_OK or FA_ERR_TIMEOUT."""
+    """Synchronise and return (then clear) the device status: FA_OK,
+    FA_ERR_TIMEOUT, or FA_ERR_INVALID (a device-side argument was out of range)."""
     return int(lib.fa_check_device_error(_stream(stream)))
 
 

@@ -193,6 +193,50 @@ FA_API size_t fa_decode_workspace_size(int32_t batch, int32_t hq, int32_t capaci
 FA_API fa_status fa_attention_decode(const fa_decode_params *p, fa_stream_t stream);
 
 /*
+ * fa_kv_append -- write one new token per sequence into a decode KV cache,
+ * quantising on the way in (FlashRT QKV Cache RoPE, Kernels:
+ * "decode_k_norm_rope_kvwrite_devpos_bf16 ... selects the cache slot from a
+ * CUDA int32 cur_pos tensor for graph-friendly decode"; here without the norm
+ * and rotation, and with the int8 cache of fkl_python PR #6, Summary,
+ * "compressed int8 KV cache (per-token, one fp32 scale/token)").
+ *   k_new, v_new  [batch*hkv, d] x_dtype (FA_BF16 or FA_F32): the new token's
+ *                 K and V rows, row u = b * hkv + g
+ *   k_cache, v_cache [batch*hkv, capacity, d] cache_dtype: FA_I8 codes (with
+ *                 k_scales, v_scales [batch*hkv, capacity] fp32) or FA_BF16
+ *   cur_pos       device int32 [batch]: the slot written for sequence b
+ *   cache_seqlens optional device int32 [batch] (NULL: untouched): set to
+ *                 cur_pos[b] + 1, the length a following fa_attention_decode
+ *                 attends to; it must not overlap cur_pos
+ * Row u of K goes to cache row u * capacity + cur_pos[b] as int8 codes and
+ * scale computed exactly as fa_compress_kv computes them (bit-identical), or
+ * as bf16 (exact for bf16 input, round to nearest even for fp32).  Nothing
+ * else in the caches changes.  Because the slot is read on the device, one
+ * captured CUDA graph can append and decode step after step while a kernel
+ * (or copy) in the same graph advances cur_pos.  A cur_pos[b] outside
+ * [0, capacity) skips sequence b's rows (and its cache_seqlens entry) and is
+ * reported by fa_check_device_error as FA_ERR_INVALID.  As with every entry
+ * point, the first call on a device allocates the status word: make it
+ * before any stream capture.
+ * Requirements: 16 <= d <= 1024, d % 16 == 0; pointers 16-byte aligned;
+ * capacity >= 1.  batch * hkv = 0 enqueues nothing.
+ */
+typedef struct {
+    const void *k_new;
+    const void *v_new;
+    int32_t x_dtype;      /* fa_dtype: FA_BF16 or FA_F32 */
+    void *k_cache;
+    void *v_cache;
+    float *k_scales;      /* FA_I8 cache only, else NULL */
+    float *v_scales;
+    int32_t cache_dtype;  /* fa_dtype: FA_I8 or FA_BF16 */
+    const int32_t *cur_pos;
+    int32_t *cache_seqlens;
+    int32_t batch, hkv, head_dim, capacity;
+} fa_kv_append_params;
+
+FA_API fa_status fa_kv_append(const fa_kv_append_params *p, fa_stream_t stream);
+
+/*
  * fa_attention_decode_noalloc -- fa_attention_decode for callers that cannot
  * allocate device memory when they call.  The paper has no counterpart: this
  * entry point exists for callers such as a plug-in inside a serving runtime
@@ -232,7 +276,9 @@ FA_API const char *fa_status_string(fa_status s);
 /*
  * Synchronises `stream`, then reads and clears the current device's status
  * word: FA_ERR_TIMEOUT if a bounded wait in any kernel gave up since the last
- * check, FA_ERR_CUDA if the synchronisation itself failed, else FA_OK.
+ * check, FA_ERR_INVALID if a kernel skipped work because a device-side
+ * argument was out of range (fa_kv_append's cur_pos), FA_ERR_CUDA if the
+ * synchronisation itself failed, else FA_OK.
  */
 FA_API fa_status fa_check_device_error(fa_stream_t stream);
 

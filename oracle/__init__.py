@@ -19,7 +19,11 @@ Definitions followed:
     query head h reads KV head h // (hq // hkv);
   * int8 KV: fkl_python PR #6, Summary ("compress_kv(): per-token int8
     quantization (one fp32 scale/token)"); the oracle attends over the
-    dequantised cache c * s.
+    dequantised cache c * s;
+  * cache append at a device-side slot: FlashRT QKV Cache RoPE, Kernels
+    ("... selects the cache slot from a CUDA int32 cur_pos tensor"): row
+    b*hkv + g of the new token goes to slot cur_pos[b] of its cache row,
+    compressed as compress_kv does; nothing else changes.
 
 Every function is pinned by ``tests/test_oracle.py`` against closed forms,
 invariants, torch's fp64 scaled_dot_product_attention, pure-Python brute force
@@ -198,6 +202,40 @@ def compress_kv(x):
     if rows:
         _load().oracle_compress_kv(_ptr(x32), rows, d, _ptr(codes), _ptr(scales))
     return codes, scales
+
+
+def kv_append(cache, scales, new, cur_pos, hkv: int, seqlens=None):
+    """The cache after appending one token per sequence (plain definition).
+
+    cache: [B*hkv, cap, d] int8 codes (with scales [B*hkv, cap] fp32) or a
+    float cache (scales None, the row stored as given); new: [B*hkv, d];
+    cur_pos: [B] slots.  Returns (cache, scales, seqlens) as new arrays: row
+    u = b*hkv + g of `new` written at [u, cur_pos[b]] (compressed by
+    compress_kv for an int8 cache), seqlens[b] = cur_pos[b] + 1.  A slot
+    outside [0, cap) leaves sequence b untouched (and its seqlens entry).
+    """
+    def host(a):
+        return a.detach().cpu().numpy() if hasattr(a, "detach") else np.asarray(a)
+    c = host(cache).copy()
+    sc = None if scales is None else host(scales).copy()
+    x = host(new) if not hasattr(new, "detach") else new.detach().cpu().float().numpy()
+    pos = np.asarray(host(cur_pos), dtype=np.int64)
+    sl = None if seqlens is None else np.asarray(host(seqlens), dtype=np.int32).copy()
+    cap = c.shape[1]
+    for u in range(c.shape[0]):
+        b = u // hkv
+        p = int(pos[b])
+        if p < 0 or p >= cap:
+            continue
+        if sc is not None:
+            codes, s = compress_kv(np.asarray(x[u], dtype=np.float32)[None, :])
+            c[u, p] = codes[0]
+            sc[u, p] = s[0]
+        else:
+            c[u, p] = x[u]
+        if sl is not None:
+            sl[b] = p + 1
+    return c, sc, sl
 
 
 def dequantize(codes, scales) -> np.ndarray:

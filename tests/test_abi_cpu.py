@@ -171,3 +171,39 @@ def test_status_strings(fa):
     for s in range(6):
         assert fa.lib.fa_status_string(s)
     assert fa.lib.fa_status_string(99) == b"unknown status"
+
+
+def append_call(fa, **kw):
+    """fa_kv_append through the C ABI with fake (never dereferenced) pointers;
+    every case here must be rejected on the host before any CUDA call."""
+    p = fa.KvAppendParams()
+    p.k_new, p.v_new, p.x_dtype = 0x10000, 0x20000, fa.FA_BF16
+    p.k_cache, p.v_cache, p.cache_dtype = 0x30000, 0x40000, fa.FA_I8
+    p.k_scales, p.v_scales = 0x50000, 0x60000
+    p.cur_pos, p.cache_seqlens = 0x70000, 0x80000
+    p.batch, p.hkv, p.head_dim, p.capacity = 4, 2, 128, 64
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return fa.lib.fa_kv_append(ctypes.byref(p), None)
+
+
+def test_kv_append_rejects_bad_arguments(fa):
+    assert fa.lib.fa_kv_append(None, None) == fa.FA_ERR_INVALID
+    assert append_call(fa, head_dim=8) == fa.FA_ERR_INVALID            # below 16
+    assert append_call(fa, head_dim=136) == fa.FA_ERR_INVALID          # not a multiple of 16
+    assert append_call(fa, head_dim=2048) == fa.FA_ERR_INVALID
+    assert append_call(fa, x_dtype=fa.FA_I8) == fa.FA_ERR_INVALID      # new rows must be float
+    assert append_call(fa, cache_dtype=fa.FA_F32) == fa.FA_ERR_INVALID
+    assert append_call(fa, k_scales=None) == fa.FA_ERR_INVALID         # int8 cache needs scales
+    assert append_call(fa, cur_pos=None) == fa.FA_ERR_INVALID
+    assert append_call(fa, k_new=0x10004) == fa.FA_ERR_INVALID         # 16-byte alignment
+    assert append_call(fa, capacity=0) == fa.FA_ERR_INVALID
+    assert append_call(fa, hkv=0) == fa.FA_ERR_INVALID
+    assert append_call(fa, batch=-1) == fa.FA_ERR_INVALID
+    # cache_seqlens overlapping cur_pos (one warp writes what others read)
+    assert append_call(fa, cache_seqlens=0x70000) == fa.FA_ERR_INVALID
+    assert append_call(fa, cache_seqlens=0x70000 + 16, batch=8) == fa.FA_ERR_INVALID
+
+
+def test_kv_append_empty_batch_is_a_noop(fa):
+    assert append_call(fa, batch=0) == fa.FA_OK

@@ -383,3 +383,38 @@ def test_workload_lengths():
     assert w == [6974, 5230, 4203, 2234, 2544, 367, 646, 167]
     lens = np.random.default_rng(0).integers(1024, 32769, 16)
     assert int(lens.sum()) == 272568
+
+
+# ---------------------------------------------------------------- cache append
+def test_kv_append_writes_exactly_the_slots():
+    """FlashRT QKV Cache RoPE, Kernels (a single-slot cache write at a
+    device-side cur_pos): only rows (b*hkv + g, cur_pos[b]) change, each
+    within half a quantisation step of the new row, and the lengths become
+    cur_pos + 1; an out-of-range slot leaves its sequence untouched."""
+    rng = np.random.default_rng(21)
+    B, hkv, cap, d = 4, 3, 16, 32
+    cache = rng.integers(-127, 128, (B * hkv, cap, d)).astype(np.int8)
+    scales = rng.random((B * hkv, cap)).astype(np.float32)
+    new = rng.standard_normal((B * hkv, d)).astype(np.float32)
+    pos = np.array([0, cap - 1, 7, cap])  # the last one is out of range
+    lens = np.array([5, 5, 5, 5], dtype=np.int32)
+    c2, s2, l2 = oracle.kv_append(cache, scales, new, pos, hkv, seqlens=lens)
+    changed = np.argwhere((c2 != cache).any(axis=2) | (s2 != scales))
+    expect = {(b * hkv + g, int(pos[b])) for b in range(B - 1) for g in range(hkv)}
+    assert {tuple(x) for x in changed} <= expect
+    for u, p_ in expect:
+        s_ = float(s2[u, p_])
+        assert s_ == pytest.approx(np.abs(new[u]).max() / 127.0, rel=1e-6)
+        err = np.abs(new[u].astype(np.float64) - c2[u, p_].astype(np.float64) * s_)
+        assert err.max() <= s_ / 2 * (1 + 1e-6)
+    assert list(l2) == [1, cap, 8, 5]
+    assert np.array_equal(c2[(B - 1) * hkv:], cache[(B - 1) * hkv:])
+
+
+def test_kv_append_float_cache_stores_the_row():
+    rng = np.random.default_rng(22)
+    cache = np.zeros((2, 4, 16), dtype=np.float32)
+    new = rng.standard_normal((2, 16)).astype(np.float32)
+    c2, s2, l2 = oracle.kv_append(cache, None, new, np.array([2]), 2)
+    assert s2 is None and l2 is None
+    assert np.array_equal(c2[:, 2], new) and not c2[:, [0, 1, 3]].any()
