@@ -417,6 +417,8 @@ def decode_and_quant(args, dev, peaks, world, dist, result):
                                          "unit": "GB/s", "frac": round(dec_gbs / peaks["hbm_gbs"], 4),
                                          "frac_of_nominal_8000": round(dec_gbs / 8000.0, 4),
                                          "traffic": measured_traffic("decode_sk_kernel<128>")}}
+        result["decode_paged"] = decode_paged(args, dw, dq, dout, ws, kc, vc, ks, vs, lens, maxlen, dec_bytes,
+                                              peaks, world, dist)
         result["decode_step_graph"] = decode_step_graph(args, dw, dq, dout, ws, kc, vc, ks, vs, peaks, world, dist)
         del kc, vc, ks, vs
         torch.cuda.empty_cache()
@@ -438,6 +440,42 @@ def decode_and_quant(args, dev, peaks, world, dist, result):
         torch.cuda.empty_cache()
     assert fa.check_device_error() == fa.FA_OK
     return result
+
+
+def decode_paged(args, dw, dq, dout, ws, kc, vc, ks, vs, lens, maxlen, dec_bytes, peaks, world, dist):
+    """The int8-KV decode over the same cache cut into 256-token pages that a
+    random permutation scatters over a pool, read through a block table (the
+    same keys and bytes as the dense decode)."""
+    import torch
+    from flashattention_attention_b200 import fa
+    P = 256
+    B, hkv, cap, d = dw.batch, dw.hkv, dw.cache_capacity, dw.d
+    mp = cap // P
+    perm = torch.randperm(B * mp, generator=torch.Generator().manual_seed(3)).cuda()
+
+    def pool_of(t, tail):
+        src = t.view(B, hkv, mp, P, *tail).transpose(1, 2).reshape(B * mp, hkv, P, *tail)
+        pool = torch.empty_like(src)
+        pool[perm] = src
+        return pool
+
+    kp, vp = pool_of(kc, (d,)), pool_of(vc, (d,))
+    ksp, vsp = pool_of(ks, ()), pool_of(vs, ())
+    table = perm.view(B, mp).to(torch.int32).contiguous()
+
+    def decode():
+        fa.attention_decode_paged(dq, kp, vp, lens, table, hq=dw.hq, hkv=hkv, k_scales=ksp, v_scales=vsp,
+                                  max_seqlen=maxlen, workspace=ws, out=dout)
+
+    ms = time_launches(decode, max(20, args.steps), args.warmup, torch, dist)
+    assert fa.check_device_error() == fa.FA_OK
+    gbs = dec_bytes / (ms * 1e-3) / 1e9
+    del kp, vp, ksp, vsp
+    torch.cuda.empty_cache()
+    return {"workload": dw.name + "_paged256_shuffled", "value": round(gbs * world, 1), "unit": "GB/s",
+            "us_per_step": round(ms * 1e3, 2), "bytes_per_step": dec_bytes,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4)}}
 
 
 def decode_step_graph(args, dw, dq, dout, ws, kc, vc, ks, vs, peaks, world, dist):

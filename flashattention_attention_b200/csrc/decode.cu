@@ -68,6 +68,10 @@ struct SkArgs {
   __nv_bfloat16* out;       // [B*hq, D]
   Epilogue epi;
   int batch, hq, hkv, group, cap, window;
+  // paged cache (null table: dense [B*hkv, cap, d]): pool [num_pages, hkv,
+  // page_size, d]; key j of sequence b lives in page block_table[b*max_pages + j/page_size]
+  const int32_t* block_table;
+  int max_pages, page_size, num_pages;
   int n_workers;            // P (launched warps)
   int min_tiles;            // > 0: at least this many tiles per worker
   float scale_log2;
@@ -313,6 +317,36 @@ __device__ __forceinline__ void advance(const SkArgs& A, const int32_t* pre, Cur
   if (c.b < A.batch) set_segment(A, c);
 }
 
+// Cache row of the 32-key tile starting at key0 of segment (c.b, c.g).  For a
+// paged cache the issuing lane keeps the page of its current (sequence,
+// logical page) -- every KV head of a sequence shares it, and a page spans
+// page_size / 32 tiles -- and loads the next page's id as soon as it enters
+// a page, so the table read is off the issue path.  A page id outside the
+// pool is reported and replaced by page 0, so no load leaves the pool (that
+// sequence's result is then meaningless).
+struct PageCursor {
+  int b = -1, lp = -1, pg = 0, next = -1;
+};
+__device__ __forceinline__ int page_id(const SkArgs& A, int b, int lp) {
+  return lp < A.max_pages ? __ldg(A.block_table + static_cast<int64_t>(b) * A.max_pages + lp) : 0;
+}
+__device__ __forceinline__ int64_t tile_row(const SkArgs& A, const Cursor& c, int key0, PageCursor& pc) {
+  if (A.block_table == nullptr) return c.kv_row0 + key0;
+  const int lp = key0 / A.page_size;
+  if (c.b != pc.b || lp != pc.lp) {
+    int pg = (c.b == pc.b && lp == pc.lp + 1) ? pc.next : page_id(A, c.b, lp);
+    if (pg < 0 || pg >= A.num_pages) {
+      record_status(A.wd, kStatusRange);
+      pg = 0;
+    }
+    pc.b = c.b;
+    pc.lp = lp;
+    pc.pg = pg;
+    pc.next = page_id(A, c.b, lp + 1);  // consumed page_size / 32 tiles later
+  }
+  return (static_cast<int64_t>(pc.pg) * A.hkv + c.g) * A.page_size + key0 % A.page_size;
+}
+
 template <int D, bool kBF>
 __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
     decode_sk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -378,24 +412,25 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
   auto stage_ptr = [&](int s) { return smem + (warp * kStages + s) * G::kStageBytes; };
   // issue cursor (lane 0 runs it kStages tiles ahead of the compute cursor)
   Cursor ic = locate(A, pre, t_first);
+  PageCursor ipc;
   auto issue = [&](int i) {
     const int s = i % kStages;
     const int key0 = ic.t_begin + ic.t * kTile;
-    const int64_t kv_row0 = ic.kv_row0;
+    const int64_t row = tile_row(A, ic, key0, ipc);
     uint8_t* st = stage_ptr(s);
     uint64_t* bar = &bars[warp * kStages + s];
     mbar_expect_tx(bar, 2 * G::kTileBytes + G::kScaleBytes);
     if constexpr (kBF) {
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_2d(st + c * G::kChunkBytes, &tm_k, bar, 64 * c, static_cast<int>(kv_row0 + key0));
-        tma_load_2d(st + G::kTileBytes + c * G::kChunkBytes, &tm_v, bar, 64 * c, static_cast<int>(kv_row0 + key0));
+        tma_load_2d(st + c * G::kChunkBytes, &tm_k, bar, 64 * c, static_cast<int>(row));
+        tma_load_2d(st + G::kTileBytes + c * G::kChunkBytes, &tm_v, bar, 64 * c, static_cast<int>(row));
       }
     } else {
-      tma_load_2d(st, &tm_k, bar, 0, static_cast<int>(kv_row0 + key0));
-      tma_load_2d(st + G::kTileBytes, &tm_v, bar, 0, static_cast<int>(kv_row0 + key0));
-      bulk_load(st + G::kScaleOff, A.k_scales + kv_row0 + key0, kTile * 4, bar);
-      bulk_load(st + G::kScaleOff + kTile * 4, A.v_scales + kv_row0 + key0, kTile * 4, bar);
+      tma_load_2d(st, &tm_k, bar, 0, static_cast<int>(row));
+      tma_load_2d(st + G::kTileBytes, &tm_v, bar, 0, static_cast<int>(row));
+      bulk_load(st + G::kScaleOff, A.k_scales + row, kTile * 4, bar);
+      bulk_load(st + G::kScaleOff + kTile * 4, A.v_scales + row, kTile * 4, bar);
     }
     advance(A, pre, ic);
   };
@@ -802,10 +837,12 @@ size_t records_bytes(int batch, int hq, int hkv, int d, int n_workers) {
 
 // Launch plan + stream-K kernel + merge into `ws` (plan, then records).
 template <int D, bool kBF>
-fa_status launch_sk(const fa_decode_params& p, int n_workers, int min_tiles, void* ws, bool count_variants,
-                    const LaunchCtx& ctx) {
+fa_status launch_sk(const fa_decode_params& p, const fa_kv_pages* pages, int n_workers, int min_tiles, void* ws,
+                    bool count_variants, const LaunchCtx& ctx) {
   using G = Geom<D, kBF>;
-  const uint64_t rows = static_cast<uint64_t>(p.batch) * p.hkv * p.capacity;
+  const uint64_t rows = pages != nullptr
+                            ? static_cast<uint64_t>(pages->num_pages) * p.hkv * pages->page_size
+                            : static_cast<uint64_t>(p.batch) * p.hkv * p.capacity;
   CUtensorMap tmk, tmv;
   const uint64_t dims[2] = {static_cast<uint64_t>(D), rows};
   const uint64_t strides[1] = {static_cast<uint64_t>(D) * (kBF ? 2 : 1)};
@@ -837,6 +874,10 @@ fa_status launch_sk(const fa_decode_params& p, int n_workers, int min_tiles, voi
   A.hkv = p.hkv;
   A.group = group;
   A.cap = p.capacity;
+  A.block_table = pages != nullptr ? pages->block_table : nullptr;
+  A.max_pages = pages != nullptr ? pages->max_pages : 1;
+  A.page_size = pages != nullptr ? pages->page_size : p.capacity;
+  A.num_pages = pages != nullptr ? pages->num_pages : p.batch;
   A.window = p.window;
   A.n_workers = n_workers;
   A.min_tiles = min_tiles;
@@ -891,14 +932,14 @@ size_t decode_workspace_bytes(int batch, int hq, int head_dim) {
          (static_cast<size_t>(batch) * hq + workers * g) * (static_cast<size_t>(head_dim) + 2) * sizeof(float);
 }
 
-fa_status launch_decode(const fa_decode_params& p, int split_keys, const LaunchCtx& ctx) {
+fa_status launch_decode(const fa_decode_params& p, const fa_kv_pages* pages, int split_keys, const LaunchCtx& ctx) {
   const int mt = min_tiles_of(split_keys);
   if (p.kv_dtype == FA_I8) {
-    if (p.head_dim == 128) return launch_sk<128, false>(p, variant_workers<128, false>(), mt, p.workspace, true, ctx);
-    if (p.head_dim == 64) return launch_sk<64, false>(p, variant_workers<64, false>(), mt, p.workspace, true, ctx);
+    if (p.head_dim == 128) return launch_sk<128, false>(p, pages, variant_workers<128, false>(), mt, p.workspace, true, ctx);
+    if (p.head_dim == 64) return launch_sk<64, false>(p, pages, variant_workers<64, false>(), mt, p.workspace, true, ctx);
   } else if (p.kv_dtype == FA_BF16) {
-    if (p.head_dim == 128) return launch_sk<128, true>(p, variant_workers<128, true>(), mt, p.workspace, true, ctx);
-    if (p.head_dim == 64) return launch_sk<64, true>(p, variant_workers<64, true>(), mt, p.workspace, true, ctx);
+    if (p.head_dim == 128) return launch_sk<128, true>(p, pages, variant_workers<128, true>(), mt, p.workspace, true, ctx);
+    if (p.head_dim == 64) return launch_sk<64, true>(p, pages, variant_workers<64, true>(), mt, p.workspace, true, ctx);
   }
   return FA_ERR_UNSUPPORTED;
 }
@@ -981,8 +1022,8 @@ fa_status launch_decode_noalloc(const fa_decode_params& p, int split_keys, long 
   fa_status st = noalloc_scratch(&scratch, &ctx.wd.word);
   if (st != FA_OK) return st;
   // (no note_variant here: its bookkeeping set may allocate host memory)
-  if (p.head_dim == 128) return launch_sk<128, false>(p, workers, min_tiles_of(split_keys), scratch, false, ctx);
-  if (p.head_dim == 64) return launch_sk<64, false>(p, workers, min_tiles_of(split_keys), scratch, false, ctx);
+  if (p.head_dim == 128) return launch_sk<128, false>(p, nullptr, workers, min_tiles_of(split_keys), scratch, false, ctx);
+  if (p.head_dim == 64) return launch_sk<64, false>(p, nullptr, workers, min_tiles_of(split_keys), scratch, false, ctx);
   return FA_ERR_UNSUPPORTED;
 }
 

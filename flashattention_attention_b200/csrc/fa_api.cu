@@ -219,7 +219,10 @@ size_t fa_decode_workspace_size(int32_t batch, int32_t hq, int32_t capacity, int
   return decode_workspace_bytes(batch, hq, head_dim);
 }
 
-fa_status fa_attention_decode(const fa_decode_params* p, fa_stream_t stream) {
+namespace {
+// Host checks shared by the decode entry points (everything but the
+// workspace); FA_OK means launchable, or a no-op when batch == 0.
+fa_status decode_args(const fa_decode_params* p) {
   if (p == nullptr) return FA_ERR_INVALID;
   if (p->batch < 0 || p->hq <= 0 || p->hkv <= 0 || p->hq % p->hkv != 0) return FA_ERR_INVALID;
   if (p->capacity <= 0 || p->capacity % 32 != 0) return FA_ERR_INVALID;
@@ -241,12 +244,38 @@ fa_status fa_attention_decode(const fa_decode_params* p, fa_stream_t stream) {
     if (p->k_scales == nullptr || p->v_scales == nullptr) return FA_ERR_INVALID;
     if (!aligned16(p->k_scales) || !aligned16(p->v_scales)) return FA_ERR_INVALID;
   }
+  return FA_OK;
+}
+}  // namespace
+
+fa_status fa_attention_decode(const fa_decode_params* p, fa_stream_t stream) {
+  fa_status st = decode_args(p);
+  if (st != FA_OK || p->batch == 0) return st;
   const size_t need = fa_decode_workspace_size(p->batch, p->hq, p->capacity, p->head_dim);
   if (p->workspace == nullptr || p->workspace_bytes < need || !aligned16(p->workspace)) return FA_ERR_WORKSPACE;
   LaunchCtx ctx;
-  fa_status st = make_ctx(stream, &ctx);
+  st = make_ctx(stream, &ctx);
   if (st != FA_OK) return st;
-  return launch_decode(*p, p->split_keys, ctx);
+  return launch_decode(*p, nullptr, p->split_keys, ctx);
+}
+
+fa_status fa_attention_decode_paged(const fa_decode_params* p, const fa_kv_pages* pages, fa_stream_t stream) {
+  fa_status st = decode_args(p);
+  if (st != FA_OK) return st;
+  if (pages == nullptr || pages->max_pages < 1 || pages->num_pages < 1 || pages->page_size < 32 ||
+      pages->page_size % 32 != 0)
+    return FA_ERR_INVALID;
+  if (static_cast<int64_t>(pages->max_pages) * pages->page_size != p->capacity) return FA_ERR_INVALID;
+  if (static_cast<int64_t>(pages->num_pages) * p->hkv * pages->page_size >= (int64_t(1) << 31))
+    return FA_ERR_UNSUPPORTED;
+  if (p->batch == 0) return FA_OK;
+  if (pages->block_table == nullptr || !aligned16(pages->block_table)) return FA_ERR_INVALID;
+  const size_t need = fa_decode_workspace_size(p->batch, p->hq, p->capacity, p->head_dim);
+  if (p->workspace == nullptr || p->workspace_bytes < need || !aligned16(p->workspace)) return FA_ERR_WORKSPACE;
+  LaunchCtx ctx;
+  st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  return launch_decode(*p, pages, p->split_keys, ctx);
 }
 
 fa_status fa_attention_decode_noalloc(const fa_decode_params* p, fa_stream_t stream) {
@@ -274,7 +303,8 @@ fa_status fa_attention_decode_noalloc(const fa_decode_params* p, fa_stream_t str
   return launch_decode_noalloc(*p, split, watchdog_budget(), reinterpret_cast<cudaStream_t>(stream));
 }
 
-fa_status fa_kv_append(const fa_kv_append_params* p, fa_stream_t stream) {
+namespace {
+fa_status kv_append_args(const fa_kv_append_params* p) {
   if (p == nullptr) return FA_ERR_INVALID;
   if (p->batch < 0 || p->hkv < 1 || p->capacity < 1) return FA_ERR_INVALID;
   if (p->head_dim < 16 || p->head_dim > 1024 || p->head_dim % 16 != 0) return FA_ERR_INVALID;
@@ -296,10 +326,31 @@ fa_status fa_kv_append(const fa_kv_append_params* p, fa_stream_t stream) {
     const uintptr_t b0 = reinterpret_cast<uintptr_t>(p->cache_seqlens), b1 = b0 + 4ull * p->batch;
     if (a0 < b1 && b0 < a1) return FA_ERR_INVALID;
   }
+  return FA_OK;
+}
+}  // namespace
+
+fa_status fa_kv_append(const fa_kv_append_params* p, fa_stream_t stream) {
+  fa_status st = kv_append_args(p);
+  if (st != FA_OK || static_cast<int64_t>(p->batch) * p->hkv == 0) return st;
   LaunchCtx ctx;
-  fa_status st = make_ctx(stream, &ctx);
+  st = make_ctx(stream, &ctx);
   if (st != FA_OK) return st;
-  return launch_kv_append(*p, ctx);
+  return launch_kv_append(*p, nullptr, ctx);
+}
+
+fa_status fa_kv_append_paged(const fa_kv_append_params* p, const fa_kv_pages* pages, fa_stream_t stream) {
+  fa_status st = kv_append_args(p);
+  if (st != FA_OK) return st;
+  if (pages == nullptr || pages->max_pages < 1 || pages->num_pages < 1 || pages->page_size < 1)
+    return FA_ERR_INVALID;
+  if (static_cast<int64_t>(pages->max_pages) * pages->page_size != p->capacity) return FA_ERR_INVALID;
+  if (static_cast<int64_t>(p->batch) * p->hkv == 0) return FA_OK;
+  if (pages->block_table == nullptr || !aligned16(pages->block_table)) return FA_ERR_INVALID;
+  LaunchCtx ctx;
+  st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  return launch_kv_append(*p, pages, ctx);
 }
 
 fa_status fa_check_device_error(fa_stream_t stream) {

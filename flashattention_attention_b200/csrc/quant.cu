@@ -290,10 +290,12 @@ fa_status launch_dtype(const void* x, int64_t rows, int d, int8_t* codes, float*
 
 // ---------------------------------------------------------------- cache append
 // One new token per sequence: rows u = b * hkv + g of k_new / v_new go to
-// cache row u * capacity + cur_pos[b] (quantised exactly as compress_kernel
-// does, or stored as bf16).  One warp per (K or V, u) row; lane layout and
-// arithmetic as in compress_kernel.  A slot outside [0, capacity) is not
-// written and is reported in the status word.
+// cache row u * capacity + cur_pos[b] (dense) or to token cur_pos[b] %
+// page_size of page block_table[b][cur_pos[b] / page_size] (paged),
+// quantised exactly as compress_kernel does, or stored as bf16.  One warp per
+// (K or V, u) row; lane layout and arithmetic as in compress_kernel.  A slot
+// outside [0, capacity), or a page outside the pool, is not written and is
+// reported in the status word.
 struct AppendArgs {
   const void* k_new;
   const void* v_new;
@@ -304,6 +306,9 @@ struct AppendArgs {
   const int32_t* cur_pos;
   int32_t* seqlens;  // optional: seqlens[b] = cur_pos[b] + 1
   int batch, hkv, d, capacity, cache_i8;
+  // paged caches (null table: dense): pool [num_pages, hkv, page_size, d]
+  const int32_t* block_table;
+  int max_pages, page_size, num_pages;
   Watchdog wd;
 };
 
@@ -322,9 +327,17 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) kv_append_kernel(const Appe
     if (lane == 0) record_status(A.wd, kStatusRange);
     return;
   }
+  int64_t row = u * A.capacity + pos;
+  if (A.block_table != nullptr) {
+    const int pg = A.block_table[static_cast<int64_t>(b) * A.max_pages + pos / A.page_size];
+    if (pg < 0 || pg >= A.num_pages) {
+      if (lane == 0) record_status(A.wd, kStatusRange);
+      return;
+    }
+    row = (static_cast<int64_t>(pg) * A.hkv + (u % A.hkv)) * A.page_size + pos % A.page_size;
+  }
   if (A.seqlens != nullptr && !is_v && u % A.hkv == 0 && lane == 0) A.seqlens[b] = pos + 1;
   const T* src = static_cast<const T*>(is_v ? A.v_new : A.k_new) + u * A.d;
-  const int64_t row = u * A.capacity + pos;
   float v[kChunks][4];
   float amax = 0.0f;
 #pragma unroll
@@ -402,8 +415,12 @@ fa_status launch_compress(const void* x, int x_dtype, int64_t rows, int d, int8_
 
 namespace fa {
 
-fa_status launch_kv_append(const fa_kv_append_params& p, const LaunchCtx& ctx) {
+fa_status launch_kv_append(const fa_kv_append_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx) {
   AppendArgs A;
+  A.block_table = pages != nullptr ? pages->block_table : nullptr;
+  A.max_pages = pages != nullptr ? pages->max_pages : 1;
+  A.page_size = pages != nullptr ? pages->page_size : p.capacity;
+  A.num_pages = pages != nullptr ? pages->num_pages : p.batch;
   A.k_new = p.k_new;
   A.v_new = p.v_new;
   A.k_cache = p.k_cache;

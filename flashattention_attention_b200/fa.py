@@ -60,6 +60,11 @@ class DecodeParams(ctypes.Structure):
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class KvPages(ctypes.Structure):
+    _fields_ = [("block_table", ctypes.c_void_p), ("max_pages", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
+
+
 class KvAppendParams(ctypes.Structure):
     _fields_ = [("k_new", ctypes.c_void_p), ("v_new", ctypes.c_void_p), ("x_dtype", ctypes.c_int32),
                 ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
@@ -78,8 +83,12 @@ lib.fa_decode_workspace_size.restype = ctypes.c_size_t
 lib.fa_decode_workspace_size.argtypes = [ctypes.c_int32] * 4
 lib.fa_attention_decode.restype = ctypes.c_int
 lib.fa_attention_decode.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_void_p]
+lib.fa_attention_decode_paged.restype = ctypes.c_int
+lib.fa_attention_decode_paged.argtypes = [ctypes.POINTER(DecodeParams), ctypes.POINTER(KvPages), ctypes.c_void_p]
 lib.fa_kv_append.restype = ctypes.c_int
 lib.fa_kv_append.argtypes = [ctypes.POINTER(KvAppendParams), ctypes.c_void_p]
+lib.fa_kv_append_paged.restype = ctypes.c_int
+lib.fa_kv_append_paged.argtypes = [ctypes.POINTER(KvAppendParams), ctypes.POINTER(KvPages), ctypes.c_void_p]
 lib.fa_status_string.restype = ctypes.c_char_p
 lib.fa_status_string.argtypes = [ctypes.c_int]
 lib.fa_check_device_error.restype = ctypes.c_int
@@ -235,6 +244,36 @@ def attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
     return out
 
 
+def attention_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                           cache_seqlens: torch.Tensor, block_table: torch.Tensor, *, hq: int, hkv: int,
+                           k_scales=None, v_scales=None, window: int = 0, scale: Optional[float] = None,
+                           epilogue: Sequence[Tuple[str, float]] = (), max_seqlen: int = 0,
+                           split_keys: int = 0, workspace: Optional[torch.Tensor] = None,
+                           out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """s_q = 1 decode over page pools k_pages/v_pages [num_pages, hkv, page_size, d]
+    (int8 with scales [num_pages, hkv, page_size], or bf16) through a device
+    int32 block_table [B, max_pages]; as fa_attention_decode_paged in fa.h."""
+    for name, t in (("q", q), ("k_pages", k_pages), ("v_pages", v_pages), ("cache_seqlens", cache_seqlens),
+                    ("block_table", block_table)):
+        _contig_cuda(t, name)
+    num_pages, _, page_size, d = k_pages.shape
+    max_pages = block_table.shape[1]
+    capacity = max_pages * page_size
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        nbytes = decode_workspace_size(cache_seqlens.numel(), hq, capacity, d)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    p = decode_params(q, k_pages, v_pages, cache_seqlens, out, workspace, hq=hq, hkv=hkv,
+                      k_scales=k_scales, v_scales=v_scales, window=window, scale=scale,
+                      epilogue=epilogue, max_seqlen=max_seqlen, split_keys=split_keys)
+    p.capacity = capacity
+    pg = KvPages(block_table.data_ptr(), max_pages, page_size, num_pages)
+    _check(lib.fa_attention_decode_paged(ctypes.byref(p), ctypes.byref(pg), _stream(stream)),
+           "fa_attention_decode_paged")
+    return out
+
+
 def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
               cur_pos: torch.Tensor, *, hkv: int, k_scales=None, v_scales=None, cache_seqlens=None,
               stream=None) -> None:
@@ -243,6 +282,24 @@ def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v
     cache is quantised on the way in (scales required), a bf16 one stored
     as bf16.  cache_seqlens (device int32 [B]), if given, becomes cur_pos + 1.
     Layouts and semantics as fa_kv_append in fa.h."""
+    p = _append_params(k_new, v_new, k_cache, v_cache, cur_pos, hkv, k_scales, v_scales, cache_seqlens)
+    _check(lib.fa_kv_append(ctypes.byref(p), _stream(stream)), "fa_kv_append")
+
+
+def kv_append_paged(k_new: torch.Tensor, v_new: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                    cur_pos: torch.Tensor, block_table: torch.Tensor, *, hkv: int, k_scales=None,
+                    v_scales=None, cache_seqlens=None, stream=None) -> None:
+    """kv_append into page pools [num_pages, hkv, page_size, d] through a
+    device int32 block_table [B, max_pages]; as fa_kv_append_paged in fa.h."""
+    _contig_cuda(block_table, "block_table")
+    p = _append_params(k_new, v_new, k_pages, v_pages, cur_pos, hkv, k_scales, v_scales, cache_seqlens)
+    num_pages, _, page_size, d = k_pages.shape
+    p.head_dim, p.capacity = d, block_table.shape[1] * page_size
+    pg = KvPages(block_table.data_ptr(), block_table.shape[1], page_size, num_pages)
+    _check(lib.fa_kv_append_paged(ctypes.byref(p), ctypes.byref(pg), _stream(stream)), "fa_kv_append_paged")
+
+
+def _append_params(k_new, v_new, k_cache, v_cache, cur_pos, hkv, k_scales, v_scales, cache_seqlens):
     for name, t in (("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache), ("v_cache", v_cache),
                     ("cur_pos", cur_pos)):
         _contig_cuda(t, name)
@@ -255,7 +312,7 @@ def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v
     p.cache_seqlens = None if cache_seqlens is None else cache_seqlens.data_ptr()
     p.batch, p.hkv = cur_pos.numel(), hkv
     p.head_dim, p.capacity = k_cache.shape[-1], k_cache.shape[1]
-    _check(lib.fa_kv_append(ctypes.byref(p), _stream(stream)), "fa_kv_append")
+    return p
 
 
 def check_device_error(stream=None) -> int:

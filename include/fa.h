@@ -193,6 +193,36 @@ FA_API size_t fa_decode_workspace_size(int32_t batch, int32_t hq, int32_t capaci
 FA_API fa_status fa_attention_decode(const fa_decode_params *p, fa_stream_t stream);
 
 /*
+ * fa_attention_decode_paged -- fa_attention_decode over a paged cache, so a
+ * serving loop hands the kernel its cache pages in place instead of copying
+ * each sequence's prefix into a contiguous buffer (SKaiNET-transformers
+ * PR #419, Summary: the positional KV caches "hand the kernel copy-free views
+ * instead of copying the whole prefix per layer per token").
+ *   k_cache, v_cache  page pools [num_pages, hkv, page_size, d] (FA_I8 codes
+ *                     with k_scales, v_scales [num_pages, hkv, page_size], or FA_BF16)
+ *   block_table       device int32 [batch, max_pages]: key j of sequence b
+ *                     is token j % page_size of page block_table[b][j / page_size]
+ * Everything else as fa_attention_decode, with p->capacity the logical
+ * capacity max_pages * page_size (cache_seqlens <= capacity) and the same
+ * workspace size.  Only the pages holding attended keys are read; other
+ * table entries may hold anything.  page_size is a multiple of 32 and
+ * num_pages * hkv * page_size < 2^31.  A page id outside [0, num_pages) is
+ * reported by fa_check_device_error as FA_ERR_INVALID; the kernel reads page
+ * 0 in its place (never outside the pool) and that sequence's output is
+ * meaningless.  Results equal fa_attention_decode's on the same keys bit for
+ * bit (same split, same arithmetic).
+ */
+typedef struct {
+    const int32_t *block_table;
+    int32_t max_pages;   /* row length of block_table */
+    int32_t page_size;   /* tokens per page, multiple of 32 */
+    int32_t num_pages;   /* pages in each pool */
+} fa_kv_pages;
+
+FA_API fa_status fa_attention_decode_paged(const fa_decode_params *p, const fa_kv_pages *pages,
+                                           fa_stream_t stream);
+
+/*
  * fa_kv_append -- write one new token per sequence into a decode KV cache,
  * quantising on the way in (FlashRT QKV Cache RoPE, Kernels:
  * "decode_k_norm_rope_kvwrite_devpos_bf16 ... selects the cache slot from a
@@ -237,6 +267,17 @@ typedef struct {
 FA_API fa_status fa_kv_append(const fa_kv_append_params *p, fa_stream_t stream);
 
 /*
+ * fa_kv_append_paged -- fa_kv_append into page pools [num_pages, hkv,
+ * page_size, d] (scales [num_pages, hkv, page_size]) through the block table
+ * of fa_attention_decode_paged: the slot cur_pos[b] is token cur_pos[b] %
+ * page_size of page block_table[b][cur_pos[b] / page_size]; p->capacity is
+ * max_pages * page_size.  A page id outside [0, num_pages) skips that
+ * sequence's rows and is reported like an out-of-range slot.
+ */
+FA_API fa_status fa_kv_append_paged(const fa_kv_append_params *p, const fa_kv_pages *pages,
+                                    fa_stream_t stream);
+
+/*
  * fa_attention_decode_noalloc -- fa_attention_decode for callers that cannot
  * allocate device memory when they call.  The paper has no counterpart: this
  * entry point exists for callers such as a plug-in inside a serving runtime
@@ -276,8 +317,8 @@ FA_API const char *fa_status_string(fa_status s);
 /*
  * Synchronises `stream`, then reads and clears the current device's status
  * word: FA_ERR_TIMEOUT if a bounded wait in any kernel gave up since the last
- * check, FA_ERR_INVALID if a kernel skipped work because a device-side
- * argument was out of range (fa_kv_append's cur_pos), FA_ERR_CUDA if the
+ * check, FA_ERR_INVALID if a kernel met a device-side argument out of range
+ * (fa_kv_append's cur_pos, a paged decode's page id), FA_ERR_CUDA if the
  * synchronisation itself failed, else FA_OK.
  */
 FA_API fa_status fa_check_device_error(fa_stream_t stream);

@@ -207,3 +207,52 @@ def test_kv_append_rejects_bad_arguments(fa):
 
 def test_kv_append_empty_batch_is_a_noop(fa):
     assert append_call(fa, batch=0) == fa.FA_OK
+
+
+def test_decode_paged_rejects_bad_arguments(fa):
+    import torch
+    q = FakeTensor(0x10000, (8, 128), torch.bfloat16)
+    kp = FakeTensor(0x20000, (16, 2, 64, 128), torch.int8)
+    lens = FakeTensor(0x30000, (2,), torch.int32)
+    o = FakeTensor(0x40000, (8, 128), torch.bfloat16)
+    ws = FakeTensor(0x50000, (1 << 24,), torch.uint8)
+    sc = FakeTensor(0x60000, (16, 2, 64), torch.float32)
+    p = fa.decode_params(q, kp, kp, lens, o, ws, hq=4, hkv=2, k_scales=sc, v_scales=sc)
+
+    def call(**kw):
+        pg = fa.KvPages(0x70000, 4, 64, 16)
+        p.capacity = 256
+        for k, v in kw.items():
+            if hasattr(pg, k):
+                setattr(pg, k, v)
+            else:
+                setattr(p, k, v)
+        return fa.lib.fa_attention_decode_paged(ctypes.byref(p), ctypes.byref(pg), None)
+
+    assert fa.lib.fa_attention_decode_paged(ctypes.byref(p), None, None) == fa.FA_ERR_INVALID
+    assert call(page_size=48) == fa.FA_ERR_INVALID           # not a multiple of 32
+    assert call(capacity=512) == fa.FA_ERR_INVALID           # capacity != max_pages * page_size
+    assert call(block_table=None) == fa.FA_ERR_INVALID
+    assert call(block_table=0x70004) == fa.FA_ERR_INVALID    # alignment
+    assert call(num_pages=0) == fa.FA_ERR_INVALID
+    assert call(num_pages=1 << 24) == fa.FA_ERR_UNSUPPORTED  # pool rows past 2^31
+    assert call(workspace_bytes=16) == fa.FA_ERR_WORKSPACE
+
+
+def test_kv_append_paged_rejects_bad_arguments(fa):
+    def call(**kw):
+        p = fa.KvAppendParams()
+        p.k_new, p.v_new, p.x_dtype = 0x10000, 0x20000, fa.FA_BF16
+        p.k_cache, p.v_cache, p.cache_dtype = 0x30000, 0x40000, fa.FA_I8
+        p.k_scales, p.v_scales = 0x50000, 0x60000
+        p.cur_pos, p.cache_seqlens = 0x70000, 0x80000
+        p.batch, p.hkv, p.head_dim, p.capacity = 4, 2, 128, 256
+        pg = fa.KvPages(0x90000, 4, 64, 16)
+        for k, v in kw.items():
+            setattr(pg if hasattr(pg, k) else p, k, v)
+        return fa.lib.fa_kv_append_paged(ctypes.byref(p), ctypes.byref(pg), None)
+    assert call(capacity=512) == fa.FA_ERR_INVALID        # capacity != max_pages * page_size
+    assert call(block_table=None) == fa.FA_ERR_INVALID
+    assert call(num_pages=0) == fa.FA_ERR_INVALID
+    assert call(head_dim=8) == fa.FA_ERR_INVALID
+    assert call(batch=0) == fa.FA_OK
