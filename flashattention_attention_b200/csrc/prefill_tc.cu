@@ -7,6 +7,11 @@
 // attention/README.md, References: the FlashAttention paper and the online
 // softmax trick), so the score matrix never leaves the SM.
 //
+// Persistent CTAs (one per SM) walk work items in longest-first order; the
+// next item's Q, first K/V tiles and first S MMAs run under the current
+// item's last softmax, PV and epilogue (its Q is reloaded once the current
+// item's S MMAs have read it, its first PV waits until O has been read out).
+//
 // CTA work tile: two 128-row Q tiles = the same 128 query rows of two query
 // heads of one GQA group (SKaiNET-transformers PR #419, Summary: one task per
 // GQA group).  Both tiles see the same mask, so they walk the same key range
@@ -40,7 +45,7 @@
 // round once to bf16, the tensor-core operand type, write it in the operand
 // layout and fence it to the async proxy.  The softmax is then the bf16 one.
 // That variant runs 16 warps and rebalances registers with setmaxnreg
-// (softmax 200, the rest 56).
+// (softmax 192, the rest 64).
 #include "internal.h"
 #include "layout.cuh"
 #include "umma.cuh"
@@ -124,6 +129,55 @@ __device__ __forceinline__ uint2 dequant4_bf16(uint32_t w, float2 s2) {
   return make_uint2(pack_bf16x2(y01.x, y01.y), pack_bf16x2(y23.x, y23.y));
 }
 
+// One work item: 128 query rows of one head pair (or one head), in the
+// longest-first order (highest q-block first, then sequence, then head pair).
+struct Item {
+  Seq sq;
+  int b, h0, g, i0, j_lo, n_iter;
+  int q_plane, q_prow, k_plane, k_prow0;  // TMA coordinates
+};
+// False for an item with no row or no visible key (the empty-band kernel
+// writes such rows).
+__device__ __forceinline__ bool item_of(const PrefillArgs& A, int item, Item& w) {
+  const int n_pairs = A.two_tiles ? A.hq / 2 : A.hq;
+  const int per_qb = A.batch * n_pairs;
+  const int qb = A.n_qblocks - 1 - item / per_qb;
+  const int rem = item % per_qb;
+  w.b = rem / n_pairs;
+  const int pair = rem % n_pairs;
+  w.h0 = A.two_tiles ? 2 * pair : pair;
+  w.g = w.h0 / A.group;
+  w.sq = seq_of(A.L, w.b, w.h0, w.g);
+  w.i0 = qb * kBM;
+  if (w.i0 >= w.sq.s_q) return false;
+  const int i_last = min(w.i0 + kBM, w.sq.s_q) - 1;
+  int lo_first, hi_first, lo_last, hi_last;
+  band_of(A.L, w.i0, w.sq.s_q, w.sq.s_k, lo_first, hi_first);
+  band_of(A.L, i_last, w.sq.s_q, w.sq.s_k, lo_last, hi_last);
+  const int k_lo = max(0, lo_first);
+  const int k_hi = min(w.sq.s_k, hi_last);
+  w.j_lo = k_lo / kBN;
+  w.n_iter = k_hi > k_lo ? (k_hi + kBN - 1) / kBN - w.j_lo : 0;
+  if (w.n_iter == 0) return false;
+  // dense planes are (b*h + h), varlen planes are h with the sequence
+  // starting at cu[b] inside the plane
+  const bool varlen = A.L.cu_q != nullptr;
+  w.q_plane = varlen ? w.h0 : w.b * A.hq + w.h0;
+  w.q_prow = (varlen ? A.L.cu_q[w.b] : 0) + w.i0;
+  w.k_plane = varlen ? w.g : w.b * A.hkv + w.g;
+  w.k_prow0 = varlen ? A.L.cu_k[w.b] : 0;
+  return true;
+}
+
+// The k-th item of CTA c among G persistent CTAs: rounds of G items in the
+// longest-first order, walked forwards in even rounds and backwards in odd
+// ones, so each CTA's total stays close to the others' (a plain stride gives
+// CTA 0 the longest item of every round).
+__device__ __forceinline__ int item_at(int c, int G, int k) {
+  const int round = k, base = round * G;
+  return (round & 1) ? base + (G - 1 - c) : base + c;
+}
+
 template <int D, bool kI8>
 __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -145,38 +199,16 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
   uint64_t* drain = o_done + 2;
   uint64_t* kraw_full = drain + 1;   // [KS] int8 variant: TMA landed the int8 K tile
   uint64_t* vraw_full = kraw_full + KS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(vraw_full + VS);
+  uint64_t* q_empty = vraw_full + VS;  // every S MMA of an item has read Q
+  uint64_t* o_free = q_empty + 1;       // [2] the softmax warps have read O_t out
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 2);
   __shared__ int abort_flag;
 
-  // ---- work tile: longest (highest q-block) first, then sequence, then head pair
-  const int n_pairs = A.two_tiles ? A.hq / 2 : A.hq;
-  const int per_qb = A.batch * n_pairs;
-  const int qb = A.n_qblocks - 1 - static_cast<int>(blockIdx.x) / per_qb;
-  const int rem = static_cast<int>(blockIdx.x) % per_qb;
-  const int b = rem / n_pairs, pair = rem % n_pairs;
-  const int h0 = A.two_tiles ? 2 * pair : pair;
+  // Persistent CTAs: CTA c takes one item per round of gridDim.x items of the
+  // longest-first order (item_at); every role walks the same sequence, with
+  // the K/V ring and every barrier phase counted across items.
+  const int n_items = A.n_qblocks * A.batch * (A.two_tiles ? A.hq / 2 : A.hq);
   const int ntile = A.two_tiles ? 2 : 1;
-  const int g = h0 / A.group;
-  const Seq sq = seq_of(A.L, b, h0, g);
-  const int i0 = qb * kBM;
-  if (i0 >= sq.s_q) return;
-  const int i_last = min(i0 + kBM, sq.s_q) - 1;
-  int lo_first, hi_first, lo_last, hi_last;
-  band_of(A.L, i0, sq.s_q, sq.s_k, lo_first, hi_first);
-  band_of(A.L, i_last, sq.s_q, sq.s_k, lo_last, hi_last);
-  const int k_lo = max(0, lo_first);
-  const int k_hi = min(sq.s_k, hi_last);
-  const int j_lo = k_lo / kBN;
-  const int n_iter = k_hi > k_lo ? (k_hi + kBN - 1) / kBN - j_lo : 0;
-  if (n_iter == 0) return;  // no row of this tile sees a key: the empty-band kernel writes them
-
-  // TMA coordinates: dense planes are (b*h + h), varlen planes are h with the
-  // sequence starting at cu[b] inside the plane.
-  const bool varlen = A.L.cu_q != nullptr;
-  const int q_plane = varlen ? h0 : b * A.hq + h0;
-  const int q_prow = (varlen ? A.L.cu_q[b] : 0) + i0;
-  const int k_plane = varlen ? g : b * A.hkv + g;
-  const int k_prow0 = varlen ? A.L.cu_k[b] : 0;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -200,6 +232,9 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       mbar_init(o_done + t, 1);
     }
     mbar_init(drain, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(o_free, kBM);
+    mbar_init(o_free + 1, kBM);
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
@@ -213,44 +248,55 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
 
   // Roles split by warpgroup first: warpgroups 0-1 softmax, 2-3 the rest.
   // int8 variant registers: 512 threads launched at 128; warpgroups 0-1 take
-  // 200, warpgroups 2-3 give back down to 56: 256*200 + 256*56 = 512*128.
+  // 192, warpgroups 2-3 give back down to 64: 256*192 + 256*64 = 512*128.
   if (warp >= 8) {
-  if constexpr (kI8) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+  if constexpr (kI8) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
-      mbar_expect_tx(q_full, ntile * G::kQBytes);
-      for (int t = 0; t < ntile; ++t)
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + t * G::kQBytes + c * kChunkBytes, &tm_q, q_full, 64 * c, q_prow, q_plane + t);
-      for (int it = 0; it < n_iter; ++it) {
-        int s = it % KS, u = it / KS;
-        const int krow = k_prow0 + (j_lo + it) * kBN;
-        if (u > 0 && !wait_parity(k_empty + s, (u - 1) & 1, A.wd, &abort_flag)) break;
-        if constexpr (kI8) {
-          mbar_expect_tx(kraw_full + s, G::kI8Bytes);
-          tma_load_3d(smem + G::k_stage(s), &tm_k, kraw_full + s, 0, krow, k_plane);
-        } else {
-          mbar_expect_tx(k_full + s, G::kKVBytes);
+      int base = 0, done = 0;  // K/V tiles and items before this one
+      bool ok = true;
+      for (int k = 0, item; ok && (item = item_at(blockIdx.x, gridDim.x, k)) < n_items; ++k) {
+        Item w;
+        if (!item_of(A, item, w)) continue;
+        // Q of this item once every S MMA of the previous one has read its Q
+        if (done > 0 && !wait_parity(q_empty, (done - 1) & 1, A.wd, &abort_flag)) break;
+        mbar_expect_tx(q_full, ntile * G::kQBytes);
+        for (int t = 0; t < ntile; ++t)
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem + G::kKOff + s * G::kKVBytes + c * kChunkBytes, &tm_k, k_full + s, 64 * c, krow,
-                        k_plane);
+            tma_load_3d(smem + t * G::kQBytes + c * kChunkBytes, &tm_q, q_full, 64 * c, w.q_prow, w.q_plane + t);
+        for (int it = 0; it < w.n_iter; ++it) {
+          const int gi = base + it;
+          int s = gi % KS, u = gi / KS;
+          const int krow = w.k_prow0 + (w.j_lo + it) * kBN;
+          if (u > 0 && !(ok = wait_parity(k_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
+          if constexpr (kI8) {
+            mbar_expect_tx(kraw_full + s, G::kI8Bytes);
+            tma_load_3d(smem + G::k_stage(s), &tm_k, kraw_full + s, 0, krow, w.k_plane);
+          } else {
+            mbar_expect_tx(k_full + s, G::kKVBytes);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(smem + G::kKOff + s * G::kKVBytes + c * kChunkBytes, &tm_k, k_full + s, 64 * c, krow,
+                          w.k_plane);
+          }
+          s = gi % VS;
+          u = gi / VS;
+          if (u > 0 && !(ok = wait_parity(v_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
+          if constexpr (kI8) {
+            mbar_expect_tx(vraw_full + s, G::kI8Bytes);
+            tma_load_3d(smem + G::v_stage(s), &tm_v, vraw_full + s, 0, krow, w.k_plane);
+          } else {
+            mbar_expect_tx(v_full + s, G::kKVBytes);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(smem + G::kVOff + s * G::kKVBytes + c * kChunkBytes, &tm_v, v_full + s, 64 * c, krow,
+                          w.k_plane);
+          }
         }
-        s = it % VS;
-        u = it / VS;
-        if (u > 0 && !wait_parity(v_empty + s, (u - 1) & 1, A.wd, &abort_flag)) break;
-        if constexpr (kI8) {
-          mbar_expect_tx(vraw_full + s, G::kI8Bytes);
-          tma_load_3d(smem + G::v_stage(s), &tm_v, vraw_full + s, 0, krow, k_plane);
-        } else {
-          mbar_expect_tx(v_full + s, G::kKVBytes);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem + G::kVOff + s * G::kKVBytes + c * kChunkBytes, &tm_v, v_full + s, 64 * c, krow,
-                        k_plane);
-        }
+        base += w.n_iter;
+        ++done;
       }
     }
   } else if (warp == kMmaWarp) {
@@ -284,38 +330,53 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
                  (accumulate || k > 0) ? 1u : 0u);
         }
       };
-      // PV for step `j` of tile t, each half as soon as the softmax wrote it
+      int base = 0, done = 0;  // K/V tiles and items before the current one
+      // PV for step j (of the current item) of tile t, each half as soon as
+      // the softmax wrote it; an item's first PV overwrites O_t, so it also
+      // waits until the previous item's O_t has been read out
       auto issue_pv = [&](int t, int j) -> bool {
-        const int vs = j % VS;
-        if (!wait_parity(p_full + 2 * t, j & 1, A.wd, &abort_flag)) return false;
-        if (t == 0 && !wait_parity(v_full + vs, (j / VS) & 1, A.wd, &abort_flag)) return false;
+        const int gj = base + j;
+        const int vs = gj % VS;
+        if (j == 0 && done > 0 && !wait_parity(o_free + t, (done - 1) & 1, A.wd, &abort_flag)) return false;
+        if (!wait_parity(p_full + 2 * t, gj & 1, A.wd, &abort_flag)) return false;
+        if (t == 0 && !wait_parity(v_full + vs, (gj / VS) & 1, A.wd, &abort_flag)) return false;
         tc_fence_after();
         issue_pv_half(t, vs, 0, j > 0);
-        if (!wait_parity(p_full + 2 * t + 1, j & 1, A.wd, &abort_flag)) return false;
+        if (!wait_parity(p_full + 2 * t + 1, gj & 1, A.wd, &abort_flag)) return false;
         tc_fence_after();
         issue_pv_half(t, vs, 1, true);
         return true;
       };
-      bool ok = wait_parity(q_full, 0, A.wd, &abort_flag);
-      for (int it = 0; ok && it < n_iter; ++it) {
-        const int s = it % KS;
-        if (!(ok = wait_parity(k_full + s, (it / KS) & 1, A.wd, &abort_flag))) break;
-        tc_fence_after();
-        for (int t = 0; t < ntile; ++t) {
-          if (it > 0) {
-            if (!(ok = issue_pv(t, it - 1))) break;
-            if (t == ntile - 1) mma_commit(v_empty + (it - 1) % VS);
+      bool ok = true;
+      for (int k = 0, item; ok && (item = item_at(blockIdx.x, gridDim.x, k)) < n_items; ++k) {
+        Item w;
+        if (!item_of(A, item, w)) continue;
+        if (!(ok = wait_parity(q_full, done & 1, A.wd, &abort_flag))) break;
+        for (int it = 0; ok && it < w.n_iter; ++it) {
+          const int gi = base + it;
+          const int s = gi % KS;
+          if (!(ok = wait_parity(k_full + s, (gi / KS) & 1, A.wd, &abort_flag))) break;
+          tc_fence_after();
+          for (int t = 0; t < ntile; ++t) {
+            if (it > 0) {
+              if (!(ok = issue_pv(t, it - 1))) break;
+              if (t == ntile - 1) mma_commit(v_empty + (gi - 1) % VS);
+            }
+            issue_s(t, s);
+            mma_commit(s_full + t);
           }
-          issue_s(t, s);
-          mma_commit(s_full + t);
+          if (ok) mma_commit(k_empty + s);
         }
-        if (ok) mma_commit(k_empty + s);
-      }
-      if (ok) {
+        if (!ok) break;
+        mma_commit(q_empty);  // Q is free once this item's S MMAs complete
         for (int t = 0; t < ntile; ++t) {
-          if (!(ok = issue_pv(t, n_iter - 1))) break;
+          if (!(ok = issue_pv(t, w.n_iter - 1))) break;
           mma_commit(o_done + t);
         }
+        if (!ok) break;
+        mma_commit(v_empty + (base + w.n_iter - 1) % VS);
+        base += w.n_iter;
+        ++done;
       }
       // every MMA this thread issued has completed before TMEM is released
       mma_commit(drain);
@@ -326,7 +387,6 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
     // thread r rewrites row r of each int8 K and V tile as bf16 in the
     // 128-byte-swizzled K-major (K) / MN-major (V) operand layout
     const int r = static_cast<int>(threadIdx.x) - kConvWarp0 * 32;
-    const int64_t scale_row0 = static_cast<int64_t>(k_plane) * A.k_plane_rows + k_prow0;
     auto convert_row = [&](const uint8_t* src_tile, uint8_t* dst_tile, float sc) {
       const float2 s2 = make_float2(sc, sc);
 #pragma unroll
@@ -341,43 +401,56 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
         *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ (r & 7)) * 16)) = make_uint4(y2.x, y2.y, y3.x, y3.y);
       }
     };
-    for (int it = 0; it < n_iter; ++it) {
-      const int s = it % KS, sv = it % VS;
-      const uint32_t ph = (it / KS) & 1, phv = (it / VS) & 1;
-      // this thread's key row: its two scales, loaded ahead of the waits (0
-      // past the sequence end, so those rows become zeros; the softmax masks them)
-      const int key = (j_lo + it) * kBN + r;
-      float ksc = 0.f, vsc = 0.f;
-      if (key < sq.s_k) {
-        ksc = __ldg(A.k_scales + scale_row0 + key);
-        vsc = __ldg(A.v_scales + scale_row0 + key);
+    int base = 0;
+    bool ok = true;
+    for (int k = 0, item; ok && (item = item_at(blockIdx.x, gridDim.x, k)) < n_items; ++k) {
+      Item w;
+      if (!item_of(A, item, w)) continue;
+      const int64_t scale_row0 = static_cast<int64_t>(w.k_plane) * A.k_plane_rows + w.k_prow0;
+      for (int it = 0; it < w.n_iter; ++it) {
+        const int gi = base + it;
+        const int s = gi % KS, sv = gi % VS;
+        const uint32_t ph = (gi / KS) & 1, phv = (gi / VS) & 1;
+        // this thread's key row: its two scales, loaded ahead of the waits (0
+        // past the sequence end, so those rows become zeros; the softmax masks them)
+        const int key = (w.j_lo + it) * kBN + r;
+        float ksc = 0.f, vsc = 0.f;
+        if (key < w.sq.s_k) {
+          ksc = __ldg(A.k_scales + scale_row0 + key);
+          vsc = __ldg(A.v_scales + scale_row0 + key);
+        }
+        if (!(ok = __all_sync(0xffffffffu, wait_parity(kraw_full + s, ph, A.wd, &abort_flag)))) break;
+        convert_row(smem + G::k_stage(s), smem + G::kKOff + s * G::kKVBytes, ksc);
+        fence_proxy_async_smem();
+        mbar_arrive(k_full + s);
+        if (!(ok = __all_sync(0xffffffffu, wait_parity(vraw_full + sv, phv, A.wd, &abort_flag)))) break;
+        convert_row(smem + G::v_stage(sv), smem + G::kVOff + sv * G::kKVBytes, vsc);
+        fence_proxy_async_smem();
+        mbar_arrive(v_full + sv);
       }
-      if (!__all_sync(0xffffffffu, wait_parity(kraw_full + s, ph, A.wd, &abort_flag))) break;
-      convert_row(smem + G::k_stage(s), smem + G::kKOff + s * G::kKVBytes, ksc);
-      fence_proxy_async_smem();
-      mbar_arrive(k_full + s);
-      if (!__all_sync(0xffffffffu, wait_parity(vraw_full + sv, phv, A.wd, &abort_flag))) break;
-      convert_row(smem + G::v_stage(sv), smem + G::kVOff + sv * G::kKVBytes, vsc);
-      fence_proxy_async_smem();
-      mbar_arrive(v_full + sv);
+      base += w.n_iter;
     }
   }
   } else {
-  if constexpr (kI8) asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+  if constexpr (kI8) asm volatile("setmaxnreg.inc.sync.aligned.u32 192;" ::: "memory");
   if (warp / 4 < ntile) {
     // ------------------------------------------------------------ softmax
     const int t = warp / 4, quarter = warp % 4;
     const int r = quarter * 32 + lane;
-    const int i = i0 + r;
-    int lo, hi;
-    band_of(A.L, i, sq.s_q, sq.s_k, lo, hi);
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_tm = tmem + lane_base + t * kBN;
     const uint32_t o_tm = tmem + lane_base + 256 + t * D;
-    float m_used = -INFINITY, l = 0.f;
+    int base = 0, done = 0;  // K/V tiles and items before the current one
     bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
-      ok = __all_sync(0xffffffffu, wait_parity(s_full + t, it & 1, A.wd, &abort_flag));
+    for (int k = 0, item; ok && (item = item_at(blockIdx.x, gridDim.x, k)) < n_items; ++k) {
+    Item w;
+    if (!item_of(A, item, w)) continue;
+    const int i = w.i0 + r;
+    int lo, hi;
+    band_of(A.L, i, w.sq.s_q, w.sq.s_k, lo, hi);
+    float m_used = -INFINITY, l = 0.f;
+    for (int it = 0; it < w.n_iter; ++it) {
+      ok = __all_sync(0xffffffffu, wait_parity(s_full + t, (base + it) & 1, A.wd, &abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t raw[4][32];
@@ -386,7 +459,7 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       tmem_ld32(s_tm + 64, raw[2]);
       tmem_ld32(s_tm + 96, raw[3]);
       tmem_wait_ld();
-      const int kb = (j_lo + it) * kBN;
+      const int kb = (w.j_lo + it) * kBN;
       if (!(kb >= lo && kb + kBN <= hi)) {
         // boundary tile: keys outside this row's band become -inf (the
         // softmax scale is positive, so masking before it is the same)
@@ -461,30 +534,37 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       lacc[0] = add2(lacc[0], lacc[1]);
       l = l * alpha + (lacc[0].x + lacc[0].y);
     }
-    if (ok) ok = __all_sync(0xffffffffu, wait_parity(o_done + t, 0, A.wd, &abort_flag));
-    if (ok) {
-      tc_fence_after();
-      const bool store = i < sq.s_q && lo < hi;
-      const float inv_l = 1.f / l;
-      __nv_bfloat16* orow = A.out + (sq.q_row0 + static_cast<int64_t>(t) * A.L.q_hstride + i) * D;
+    if (ok) ok = __all_sync(0xffffffffu, wait_parity(o_done + t, done & 1, A.wd, &abort_flag));
+    if (!ok) break;
+    tc_fence_after();
+    const bool store = i < w.sq.s_q && lo < hi;
+    const float inv_l = 1.f / l;
+    __nv_bfloat16* orow = A.out + (w.sq.q_row0 + static_cast<int64_t>(t) * A.L.q_hstride + i) * D;
 #pragma unroll
-      for (int oc = 0; oc < D / 32; ++oc) {
-        uint32_t o[32];
-        tmem_ld32(o_tm + oc * 32, o);
-        tmem_wait_ld();
-        float y[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) y[e] = __uint_as_float(o[e]) * inv_l;
-        apply_epilogue_vec(y, A.epi);
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + oc * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        }
+    for (int oc = 0; oc < D / 32; ++oc) {
+      uint32_t o[32];
+      tmem_ld32(o_tm + oc * 32, o);
+      tmem_wait_ld();
+      if (oc == D / 32 - 1) {
+        // O_t is in registers: the next item's first PV may overwrite it
+        tc_fence_before();
+        mbar_arrive(o_free + t);
       }
+      float y[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) y[e] = __uint_as_float(o[e]) * inv_l;
+      apply_epilogue_vec(y, A.epi);
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
+      if (store) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + oc * 32);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+      }
+    }
+    base += w.n_iter;
+    ++done;
     }
   }
   }
@@ -557,9 +637,12 @@ fa_status launch_tc(const fa_fwd_params& p, const LaunchCtx& ctx) {
   A.epi = make_epilogue(p.epilogue, p.n_epilogue);
   A.wd = ctx.wd;
   const long long n_pairs = A.two_tiles ? p.hq / 2 : p.hq;
-  const long long grid = static_cast<long long>(A.n_qblocks) * p.batch * n_pairs;
-  if (grid == 0) return FA_OK;
-  if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  const long long items = static_cast<long long>(A.n_qblocks) * p.batch * n_pairs;
+  if (items == 0) return FA_OK;
+  if (items > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  // persistent: one CTA per SM (the shared memory allows no second), each
+  // walking its share of the items
+  const long long grid = items < device_sm_count() ? items : device_sm_count();
   auto kern = prefill_tc_kernel<D, kI8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem) != cudaSuccess)
     return FA_ERR_CUDA;
