@@ -218,12 +218,18 @@ def time_launches(fn, steps, warmup, torch, dist=None, clocks=None):
         clocks.mark(t0, time.perf_counter())
     if dist is not None:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, torch, "cuda")
     return ms / steps
+
+
+def max_over_ranks(x: float, dist, torch, device) -> float:
+    """The largest of every rank's x (the job is as slow as its slowest
+    rank); x itself without a process group."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def gpu_arm(args, rank, world, dist):
