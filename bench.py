@@ -302,11 +302,48 @@ def gpu_arm(args, rank, world, dist):
         "clocks": clk,
     }
     if args.only == "all":
+        result["gqa_causal_prefill_paged"] = paged_prefill(args, w, flops_tiles, peaks, world, dist, dev)
         other_prefills(args, dev, peaks, world, dist, result)
         decode_and_quant(args, dev, peaks, world, dist, result)
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, flops_tiles, flops_exact, args.cpu_seconds)
     return result
+
+
+def paged_prefill(args, w, flops_tiles, peaks, world, dist, dev):
+    """The causal GQA prefill with K/V read from 256-token pages that a random
+    permutation scatters over a pool (dense queries, per-sequence key counts)."""
+    import torch
+    from flashattention_attention_b200 import fa
+    P = 256
+    B, hkv, S, d = w.batch, w.hkv, w.seqlen_k, w.d
+    mp = S // P
+    perm = torch.randperm(B * mp, generator=torch.Generator().manual_seed(4)).to(dev)
+
+    def pool_of(t):
+        src = t.to(dev).view(B, hkv, mp, P, d).transpose(1, 2).reshape(B * mp, hkv, P, d)
+        pool = torch.empty_like(src)
+        pool[perm] = src
+        return pool
+
+    kp, vp = pool_of(w.k), pool_of(w.v)
+    table = perm.view(B, mp).to(torch.int32).contiguous()
+    cu_k = torch.arange(0, (B + 1) * S, S, dtype=torch.int32, device=dev)
+    q = w.q.to(dev)
+    out = torch.empty_like(q)
+
+    def step():
+        fa.attention_fwd_paged(q, kp, vp, cu_k, table, hq=w.hq, hkv=hkv, causal=True, out=out)
+
+    ms = time_launches(step, max(20, args.steps // 2), args.warmup, torch, dist)
+    assert fa.check_device_error() == fa.FA_OK
+    tf = flops_tiles / (ms * 1e-3) / 1e12
+    del kp, vp, q, out
+    torch.cuda.empty_cache()
+    return {"workload": w.name + "_paged256_shuffled", "value": round(tf * world, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "flops_per_step": flops_tiles,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4)}}
 
 
 def varlen_flops(w):

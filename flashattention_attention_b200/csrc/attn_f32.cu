@@ -167,7 +167,13 @@ __global__ void __launch_bounds__(128)
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     float sum = 0.f;
     for (int j = 0; j < sq.s_k; ++j) {
-      const int64_t row = sq.k_row0 + j;
+      int64_t row = sq.k_row0 + j;
+      if (L.block_table != nullptr) {
+        int plane, prow;
+        bool bad;
+        paged_key(L, b, g, j, plane, prow, bad);  // a bad page id is reported by the prefill kernel
+        row = static_cast<int64_t>(plane) * L.page_size + prow;
+      }
       float x;
       if constexpr (sizeof(TV) == 1) {
         x = static_cast<float>(v[row * d + c]) * v_scales[row];
@@ -214,14 +220,16 @@ fa_status launch_attn_f32(const fa_fwd_params& p, const LaunchCtx& ctx) {
   }
 }
 
-fa_status launch_empty_rows(const fa_fwd_params& p, const LaunchCtx& ctx) {
+fa_status launch_empty_rows(const fa_fwd_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx) {
   if (!p.causal) return FA_OK;
-  // Dense inputs with s_q <= s_k have no empty row; varlen is decided per
-  // sequence on the device.
-  if (p.cu_seqlens_q == nullptr && p.seqlen_q <= p.seqlen_k) return FA_OK;
-  if (p.cu_seqlens_q != nullptr && (p.cu_seqlens_k == nullptr || p.cu_seqlens_k == p.cu_seqlens_q))
-    return FA_OK;
-  const SeqLayout L = SeqLayout::from(p);
+  // Dense inputs with s_q <= s_k have no empty row; varlen and paged keys
+  // are decided per sequence on the device.
+  if (pages == nullptr) {
+    if (p.cu_seqlens_q == nullptr && p.seqlen_q <= p.seqlen_k) return FA_OK;
+    if (p.cu_seqlens_q != nullptr && (p.cu_seqlens_k == nullptr || p.cu_seqlens_k == p.cu_seqlens_q))
+      return FA_OK;
+  }
+  const SeqLayout L = pages != nullptr ? SeqLayout::paged(p, *pages) : SeqLayout::from(p);
   const Epilogue epi = make_epilogue(p.epilogue, p.n_epilogue);
   dim3 grid(p.hq, p.batch);
   if (p.q_dtype == FA_F32 && p.kv_dtype == FA_I8) {

@@ -209,9 +209,41 @@ fa_status fa_attention_fwd(const fa_fwd_params* p, fa_stream_t stream) {
   LaunchCtx ctx;
   fa_status st = make_ctx(stream, &ctx);
   if (st != FA_OK) return st;
-  st = (p->q_dtype == FA_F32) ? launch_attn_f32(*p, ctx) : launch_prefill_tc(*p, ctx);
+  st = (p->q_dtype == FA_F32) ? launch_attn_f32(*p, ctx) : launch_prefill_tc(*p, nullptr, ctx);
   if (st != FA_OK) return st;
-  return launch_empty_rows(*p, ctx);
+  return launch_empty_rows(*p, nullptr, ctx);
+}
+
+fa_status fa_attention_fwd_paged(const fa_fwd_params* p, const fa_kv_pages* pages, fa_stream_t stream) {
+  if (p == nullptr || pages == nullptr) return FA_ERR_INVALID;
+  if (p->batch < 0 || p->hq <= 0 || p->hkv <= 0 || p->hq % p->hkv != 0) return FA_ERR_INVALID;
+  if (!epilogue_ok(p->epilogue, p->n_epilogue)) return FA_ERR_INVALID;
+  if (!std::isfinite(p->softmax_scale)) return FA_ERR_INVALID;
+  if (p->q_dtype != FA_BF16 || (p->kv_dtype != FA_BF16 && p->kv_dtype != FA_I8)) return FA_ERR_INVALID;
+  if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
+  if (p->head_dim != 64 && p->head_dim != 128) return FA_ERR_UNSUPPORTED;
+  if (p->kv_dtype == FA_I8 && (p->k_scales == nullptr || p->v_scales == nullptr || !aligned16(p->k_scales) ||
+                               !aligned16(p->v_scales)))
+    return FA_ERR_INVALID;
+  if (pages->max_pages < 1 || pages->num_pages < 1 || pages->page_size < 128 || pages->page_size % 128 != 0)
+    return FA_ERR_INVALID;
+  if (static_cast<int64_t>(pages->num_pages) * p->hkv >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  const bool varlen = p->cu_seqlens_q != nullptr;
+  if (varlen ? (p->total_q < 0 || p->max_seqlen_q < 0) : p->seqlen_q < 0) return FA_ERR_INVALID;
+  const bool empty = p->batch == 0 || (varlen ? p->total_q == 0 : p->seqlen_q == 0);
+  if (empty) return FA_OK;
+  if (p->q == nullptr || p->k == nullptr || p->v == nullptr || p->out == nullptr || p->cu_seqlens_k == nullptr ||
+      pages->block_table == nullptr)
+    return FA_ERR_INVALID;
+  if (!aligned16(p->q) || !aligned16(p->k) || !aligned16(p->v) || !aligned16(p->out) ||
+      !aligned16(pages->block_table))
+    return FA_ERR_INVALID;
+  LaunchCtx ctx;
+  fa_status st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  st = launch_prefill_tc(*p, pages, ctx);
+  if (st != FA_OK) return st;
+  return launch_empty_rows(*p, pages, ctx);
 }
 
 size_t fa_decode_workspace_size(int32_t batch, int32_t hq, int32_t capacity, int32_t head_dim) {

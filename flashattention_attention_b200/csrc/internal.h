@@ -23,8 +23,8 @@ fa_status launch_compress(const void* x, int x_dtype, int64_t rows, int d, int8_
                           const LaunchCtx& ctx);
 fa_status launch_kv_append(const fa_kv_append_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx);
 fa_status launch_attn_f32(const fa_fwd_params& p, const LaunchCtx& ctx);
-fa_status launch_empty_rows(const fa_fwd_params& p, const LaunchCtx& ctx);
-fa_status launch_prefill_tc(const fa_fwd_params& p, const LaunchCtx& ctx);
+fa_status launch_empty_rows(const fa_fwd_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx);
+fa_status launch_prefill_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx);
 fa_status launch_decode(const fa_decode_params& p, const fa_kv_pages* pages, int split_keys, const LaunchCtx& ctx);
 size_t decode_workspace_bytes(int batch, int hq, int head_dim);
 int decode_noalloc_workers(int batch, int hq, int hkv, int head_dim);

@@ -169,6 +169,20 @@ __device__ __forceinline__ bool item_of(const PrefillArgs& A, int item, Item& w)
   return true;
 }
 
+// TMA plane and row of the 128-key tile starting at key0 of item w (paged:
+// through the block table; a page id outside the pool reads page 0 and is
+// reported).
+__device__ __forceinline__ void kv_tile(const PrefillArgs& A, const Item& w, int key0, int& plane, int& row) {
+  if (A.L.block_table == nullptr) {
+    plane = w.k_plane;
+    row = w.k_prow0 + key0;
+    return;
+  }
+  bool bad;
+  paged_key(A.L, w.b, w.g, key0, plane, row, bad);
+  if (bad) record_status(A.wd, kStatusRange);
+}
+
 // The k-th item of CTA c among G persistent CTAs: rounds of G items in the
 // longest-first order, walked forwards in even rounds and backwards in odd
 // ones, so each CTA's total stays close to the others' (a plain stride gives
@@ -271,28 +285,29 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
         for (int it = 0; it < w.n_iter; ++it) {
           const int gi = base + it;
           int s = gi % KS, u = gi / KS;
-          const int krow = w.k_prow0 + (w.j_lo + it) * kBN;
+          int kplane, krow;
+          kv_tile(A, w, (w.j_lo + it) * kBN, kplane, krow);
           if (u > 0 && !(ok = wait_parity(k_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
           if constexpr (kI8) {
             mbar_expect_tx(kraw_full + s, G::kI8Bytes);
-            tma_load_3d(smem + G::k_stage(s), &tm_k, kraw_full + s, 0, krow, w.k_plane);
+            tma_load_3d(smem + G::k_stage(s), &tm_k, kraw_full + s, 0, krow, kplane);
           } else {
             mbar_expect_tx(k_full + s, G::kKVBytes);
             for (int c = 0; c < D / 64; ++c)
               tma_load_3d(smem + G::kKOff + s * G::kKVBytes + c * kChunkBytes, &tm_k, k_full + s, 64 * c, krow,
-                          w.k_plane);
+                          kplane);
           }
           s = gi % VS;
           u = gi / VS;
           if (u > 0 && !(ok = wait_parity(v_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
           if constexpr (kI8) {
             mbar_expect_tx(vraw_full + s, G::kI8Bytes);
-            tma_load_3d(smem + G::v_stage(s), &tm_v, vraw_full + s, 0, krow, w.k_plane);
+            tma_load_3d(smem + G::v_stage(s), &tm_v, vraw_full + s, 0, krow, kplane);
           } else {
             mbar_expect_tx(v_full + s, G::kKVBytes);
             for (int c = 0; c < D / 64; ++c)
               tma_load_3d(smem + G::kVOff + s * G::kKVBytes + c * kChunkBytes, &tm_v, v_full + s, 64 * c, krow,
-                          w.k_plane);
+                          kplane);
           }
         }
         base += w.n_iter;
@@ -406,18 +421,20 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
     for (int k = 0, item; ok && (item = item_at(blockIdx.x, gridDim.x, k)) < n_items; ++k) {
       Item w;
       if (!item_of(A, item, w)) continue;
-      const int64_t scale_row0 = static_cast<int64_t>(w.k_plane) * A.k_plane_rows + w.k_prow0;
       for (int it = 0; it < w.n_iter; ++it) {
         const int gi = base + it;
         const int s = gi % KS, sv = gi % VS;
         const uint32_t ph = (gi / KS) & 1, phv = (gi / VS) & 1;
         // this thread's key row: its two scales, loaded ahead of the waits (0
         // past the sequence end, so those rows become zeros; the softmax masks them)
-        const int key = (w.j_lo + it) * kBN + r;
+        const int key0 = (w.j_lo + it) * kBN;
         float ksc = 0.f, vsc = 0.f;
-        if (key < w.sq.s_k) {
-          ksc = __ldg(A.k_scales + scale_row0 + key);
-          vsc = __ldg(A.v_scales + scale_row0 + key);
+        if (key0 + r < w.sq.s_k) {
+          int kplane, krow;
+          kv_tile(A, w, key0, kplane, krow);
+          const int64_t at = static_cast<int64_t>(kplane) * A.k_plane_rows + krow + r;
+          ksc = __ldg(A.k_scales + at);
+          vsc = __ldg(A.v_scales + at);
         }
         if (!(ok = __all_sync(0xffffffffu, wait_parity(kraw_full + s, ph, A.wd, &abort_flag)))) break;
         convert_row(smem + G::k_stage(s), smem + G::kKOff + s * G::kKVBytes, ksc);
@@ -578,13 +595,15 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
 }
 
 template <int D, bool kI8>
-fa_status launch_tc(const fa_fwd_params& p, const LaunchCtx& ctx) {
+fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx) {
   using G = TcGeom<D, kI8>;
   const bool varlen = p.cu_seqlens_q != nullptr;
   const uint64_t q_rows = varlen ? p.total_q : p.seqlen_q;
-  const uint64_t k_rows = varlen ? p.total_k : p.seqlen_k;
+  // paged keys: planes of page_size rows, one per (page, KV head)
+  const uint64_t k_rows = pages != nullptr ? pages->page_size : (varlen ? p.total_k : p.seqlen_k);
   const uint64_t q_planes = varlen ? p.hq : static_cast<uint64_t>(p.batch) * p.hq;
-  const uint64_t k_planes = varlen ? p.hkv : static_cast<uint64_t>(p.batch) * p.hkv;
+  const uint64_t k_planes = pages != nullptr ? static_cast<uint64_t>(pages->num_pages) * p.hkv
+                                             : (varlen ? p.hkv : static_cast<uint64_t>(p.batch) * p.hkv);
   if (k_rows == 0) return FA_OK;  // no keys anywhere: only the empty-band kernel writes
   CUtensorMap tq, tk, tv;
   {
@@ -617,7 +636,7 @@ fa_status launch_tc(const fa_fwd_params& p, const LaunchCtx& ctx) {
     if (st != FA_OK) return st;
   }
   PrefillArgs A;
-  A.L = SeqLayout::from(p);
+  A.L = pages != nullptr ? SeqLayout::paged(p, *pages) : SeqLayout::from(p);
   A.out = static_cast<__nv_bfloat16*>(p.out);
   A.k_scales = p.k_scales;
   A.v_scales = p.v_scales;
@@ -653,14 +672,14 @@ fa_status launch_tc(const fa_fwd_params& p, const LaunchCtx& ctx) {
 
 }  // namespace
 
-fa_status launch_prefill_tc(const fa_fwd_params& p, const LaunchCtx& ctx) {
+fa_status launch_prefill_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx) {
   if (p.kv_dtype == FA_I8) {
-    if (p.head_dim == 128) return launch_tc<128, true>(p, ctx);
-    if (p.head_dim == 64) return launch_tc<64, true>(p, ctx);
+    if (p.head_dim == 128) return launch_tc<128, true>(p, pages, ctx);
+    if (p.head_dim == 64) return launch_tc<64, true>(p, pages, ctx);
     return FA_ERR_UNSUPPORTED;
   }
-  if (p.head_dim == 128) return launch_tc<128, false>(p, ctx);
-  if (p.head_dim == 64) return launch_tc<64, false>(p, ctx);
+  if (p.head_dim == 128) return launch_tc<128, false>(p, pages, ctx);
+  if (p.head_dim == 64) return launch_tc<64, false>(p, pages, ctx);
   return FA_ERR_UNSUPPORTED;
 }
 

@@ -83,6 +83,8 @@ lib.fa_decode_workspace_size.restype = ctypes.c_size_t
 lib.fa_decode_workspace_size.argtypes = [ctypes.c_int32] * 4
 lib.fa_attention_decode.restype = ctypes.c_int
 lib.fa_attention_decode.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_void_p]
+lib.fa_attention_fwd_paged.restype = ctypes.c_int
+lib.fa_attention_fwd_paged.argtypes = [ctypes.POINTER(FwdParams), ctypes.POINTER(KvPages), ctypes.c_void_p]
 lib.fa_attention_decode_paged.restype = ctypes.c_int
 lib.fa_attention_decode_paged.argtypes = [ctypes.POINTER(DecodeParams), ctypes.POINTER(KvPages), ctypes.c_void_p]
 lib.fa_kv_append.restype = ctypes.c_int
@@ -195,6 +197,44 @@ def attention_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, hq: int,
                    epilogue=epilogue, k_scales=k_scales, v_scales=v_scales, cu_seqlens_q=cu_seqlens_q,
                    cu_seqlens_k=cu_seqlens_k, max_seqlen_q=max_seqlen_q, max_seqlen_k=max_seqlen_k)
     _check(lib.fa_attention_fwd(ctypes.byref(p), _stream(stream)), "fa_attention_fwd")
+    return out
+
+
+def attention_fwd_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                        cu_seqlens_k: torch.Tensor, block_table: torch.Tensor, *, hq: int, hkv: int,
+                        causal: bool = False, window: int = 0, scale: Optional[float] = None,
+                        epilogue: Sequence[Tuple[str, float]] = (), k_scales=None, v_scales=None,
+                        cu_seqlens_q=None, max_seqlen_q=None, out: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """Prefill over page pools k_pages/v_pages [num_pages, hkv, page_size, d]
+    (int8 with scales [num_pages, hkv, page_size], or bf16) through a device
+    int32 block_table [B, max_pages]; q dense [B*hq, s_q, d] or varlen
+    [hq, total_q, d] with cu_seqlens_q.  As fa_attention_fwd_paged in fa.h."""
+    for name, t in (("q", q), ("k_pages", k_pages), ("v_pages", v_pages), ("cu_seqlens_k", cu_seqlens_k),
+                    ("block_table", block_table)):
+        _contig_cuda(t, name)
+    if out is None:
+        out = torch.empty_like(q)
+    p = FwdParams()
+    p.q, p.k, p.v, p.out = q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), out.data_ptr()
+    p.k_scales = None if k_scales is None else k_scales.data_ptr()
+    p.v_scales = None if v_scales is None else v_scales.data_ptr()
+    p.q_dtype, p.kv_dtype = _DT[q.dtype], _DT[k_pages.dtype]
+    p.hq, p.hkv, p.head_dim = hq, hkv, q.shape[-1]
+    p.batch = cu_seqlens_k.numel() - 1
+    p.cu_seqlens_k = cu_seqlens_k.data_ptr()
+    if cu_seqlens_q is None:
+        p.seqlen_q = q.shape[1]
+    else:
+        p.cu_seqlens_q = cu_seqlens_q.data_ptr()
+        p.total_q = q.shape[1]
+        p.max_seqlen_q = int(max_seqlen_q)
+    p.causal, p.window = int(bool(causal)), int(window)
+    p.softmax_scale = float(scale if scale is not None else 1.0 / math.sqrt(q.shape[-1]))
+    p.n_epilogue = _fill_epilogue(p.epilogue, epilogue)
+    num_pages, _, page_size, _ = k_pages.shape
+    pg = KvPages(block_table.data_ptr(), block_table.shape[1], page_size, num_pages)
+    _check(lib.fa_attention_fwd_paged(ctypes.byref(p), ctypes.byref(pg), _stream(stream)), "fa_attention_fwd_paged")
     return out
 
 

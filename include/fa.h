@@ -223,6 +223,30 @@ FA_API fa_status fa_attention_decode_paged(const fa_decode_params *p, const fa_k
                                            fa_stream_t stream);
 
 /*
+ * fa_attention_fwd_paged -- fa_attention_fwd with K/V read from page pools
+ * through a block table (SKaiNET-transformers PR #419, Summary: copy-free
+ * K/V views for prefill as well as decode): e.g. a chunk of new queries per
+ * sequence attending to that sequence's whole cached prefix, without copying
+ * the prefix out of its pages.
+ *   q, out   dense [batch*hq, seqlen_q, d] (cu_seqlens_q NULL) or varlen
+ *            [hq, total_q, d] with cu_seqlens_q / max_seqlen_q, as for
+ *            fa_attention_fwd; bf16
+ *   k, v     page pools [num_pages, hkv, page_size, d] (FA_BF16, or FA_I8
+ *            codes with k_scales, v_scales [num_pages, hkv, page_size])
+ *   cu_seqlens_k  device int32 [batch+1]: sequence b has
+ *            cu_seqlens_k[b+1] - cu_seqlens_k[b] keys, key j in token
+ *            j % page_size of page block_table[b][j / page_size]
+ * Masks, GQA, the empty-band rule and the epilogue as fa_attention_fwd
+ * (query i of a sequence with s_q queries and s_k keys sits at key position
+ * i + s_k - s_q).  page_size is a multiple of 128 (a 128-key tile never
+ * crosses a page); seqlen_k, total_k and max_seqlen_k are not used.  A page id
+ * outside [0, num_pages) reads page 0 and is reported by
+ * fa_check_device_error as FA_ERR_INVALID.  Results equal fa_attention_fwd's
+ * on the same keys in a contiguous layout bit for bit.
+ */
+FA_API fa_status fa_attention_fwd_paged(const fa_fwd_params *p, const fa_kv_pages *pages, fa_stream_t stream);
+
+/*
  * fa_kv_append -- write one new token per sequence into a decode KV cache,
  * quantising on the way in (FlashRT QKV Cache RoPE, Kernels:
  * "decode_k_norm_rope_kvwrite_devpos_bf16 ... selects the cache slot from a
@@ -318,7 +342,7 @@ FA_API const char *fa_status_string(fa_status s);
  * Synchronises `stream`, then reads and clears the current device's status
  * word: FA_ERR_TIMEOUT if a bounded wait in any kernel gave up since the last
  * check, FA_ERR_INVALID if a kernel met a device-side argument out of range
- * (fa_kv_append's cur_pos, a paged decode's page id), FA_ERR_CUDA if the
+ * (fa_kv_append's cur_pos, a paged call's page id), FA_ERR_CUDA if the
  * synchronisation itself failed, else FA_OK.
  */
 FA_API fa_status fa_check_device_error(fa_stream_t stream);

@@ -256,3 +256,24 @@ def test_kv_append_paged_rejects_bad_arguments(fa):
     assert call(num_pages=0) == fa.FA_ERR_INVALID
     assert call(head_dim=8) == fa.FA_ERR_INVALID
     assert call(batch=0) == fa.FA_OK
+
+
+def test_fwd_paged_rejects_bad_arguments(fa):
+    def call(**kw):
+        p = fa.FwdParams()
+        p.q, p.k, p.v, p.out = 0x10000, 0x20000, 0x30000, 0x40000
+        p.q_dtype, p.kv_dtype = fa.FA_BF16, fa.FA_BF16
+        p.batch, p.hq, p.hkv, p.head_dim, p.seqlen_q = 2, 4, 2, 128, 64
+        p.cu_seqlens_k = 0x50000
+        p.causal, p.softmax_scale = 1, 0.125
+        pg = fa.KvPages(0x60000, 4, 128, 8)
+        for k, v in kw.items():
+            setattr(pg if hasattr(pg, k) else p, k, v)
+        return fa.lib.fa_attention_fwd_paged(ctypes.byref(p), ctypes.byref(pg), None)
+    assert call(page_size=64) == fa.FA_ERR_INVALID          # not a multiple of 128
+    assert call(cu_seqlens_k=None) == fa.FA_ERR_INVALID      # per-sequence key counts required
+    assert call(block_table=None) == fa.FA_ERR_INVALID
+    assert call(q_dtype=fa.FA_F32, kv_dtype=fa.FA_F32) == fa.FA_ERR_INVALID   # tensor-core path only
+    assert call(head_dim=96) == fa.FA_ERR_UNSUPPORTED
+    assert call(kv_dtype=fa.FA_I8) == fa.FA_ERR_INVALID       # int8 needs scales
+    assert call(seqlen_q=0) == fa.FA_OK                       # nothing to do

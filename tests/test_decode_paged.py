@@ -158,3 +158,126 @@ def test_paged_append_then_decode_equals_dense(int8):
     tab = table.cpu().numpy()
     expect = {(int(tab[b, L // page_size]), g, L % page_size) for b, L in enumerate(lengths) for g in range(hkv)}
     assert {tuple(x) for x in changed} <= expect
+
+
+def paginate_varlen(x, scales, lens, hkv, page_size, rng, extra=3):
+    """Pages of a varlen [hkv, total, d] tensor (sequence b owns rows
+    cu[b]..cu[b+1]-1 of every head plane) over a shuffled pool; returns the
+    pool, its scale pool and the block table."""
+    B = len(lens)
+    need = [max(1, -(-int(L) // page_size)) for L in lens]
+    max_pages = max(need) + 1
+    num_pages = sum(need) + extra
+    order = rng.permutation(num_pages)
+    d = x.shape[-1]
+    pool = torch.zeros((num_pages, hkv, page_size, d), dtype=x.dtype)
+    spool = None if scales is None else torch.zeros((num_pages, hkv, page_size), dtype=torch.float32)
+    table = np.full((B, max_pages), -1, dtype=np.int32)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    k = 0
+    for b in range(B):
+        for lp in range(need[b]):
+            pg = int(order[k])
+            k += 1
+            table[b, lp] = pg
+            a, e = cu[b] + lp * page_size, min(cu[b] + (lp + 1) * page_size, cu[b + 1])
+            if e > a:
+                pool[pg, :, :e - a] = x[:, a:e]
+                if scales is not None:
+                    spool[pg, :, :e - a] = scales[:, a:e]
+    return pool, spool, torch.from_numpy(table)
+
+
+@pytest.mark.parametrize("int8", [False, True])
+@pytest.mark.parametrize("d,page_size,window", [(128, 128, 0), (128, 256, 0), (64, 128, 200)])
+def test_paged_prefill_equals_varlen(int8, d, page_size, window):
+    """Chunked prefill over a paged cache: each sequence's new queries (fewer
+    than its keys, bottom-right causal) attend to its whole prefix read from
+    shuffled pages; bit-identical to the contiguous varlen prefill, and the
+    oracle's within the bf16 gate."""
+    fa = _fa()
+    rng = np.random.default_rng(50 + d + page_size + window + int8)
+    hq, hkv = 8, 2
+    k_lens = [700, 129, 1024, 40]
+    q_lens = [64, 129, 300, 40]
+    cu_k = torch.tensor(np.concatenate([[0], np.cumsum(k_lens)]), dtype=torch.int32)
+    cu_q = torch.tensor(np.concatenate([[0], np.cumsum(q_lens)]), dtype=torch.int32)
+    tk, tq = int(cu_k[-1]), int(cu_q[-1])
+    k = torch.from_numpy(rng.standard_normal((hkv, tk, d)).astype(np.float32)).bfloat16()
+    v = torch.from_numpy(rng.standard_normal((hkv, tk, d)).astype(np.float32)).bfloat16()
+    q = torch.from_numpy(rng.standard_normal((hq, tq, d)).astype(np.float32)).bfloat16().cuda()
+    if int8:
+        kc, ks = (t.cpu() for t in fa.compress_kv(k.cuda()))
+        vc, vs = (t.cpu() for t in fa.compress_kv(v.cuda()))
+    else:
+        kc, ks, vc, vs = k, None, v, None
+    kp, ksp, table = paginate_varlen(kc, ks, k_lens, hkv, page_size, rng)
+    vp, vsp, _ = paginate_varlen(vc, vs, k_lens, hkv, page_size, np.random.default_rng(0))
+    # V in K's pages
+    vp = torch.zeros_like(kp)
+    vsp = None if vs is None else torch.zeros_like(ksp)
+    cu = np.concatenate([[0], np.cumsum(k_lens)])
+    for b in range(len(k_lens)):
+        for lp in range(table.shape[1]):
+            pg = int(table[b, lp])
+            if pg < 0:
+                continue
+            a, e = cu[b] + lp * page_size, min(cu[b] + (lp + 1) * page_size, cu[b + 1])
+            if e > a:
+                vp[pg, :, :e - a] = vc[:, a:e]
+                if vs is not None:
+                    vsp[pg, :, :e - a] = vs[:, a:e]
+    cuda = lambda t: None if t is None else t.cuda()
+    # the gate bounds the attention output; an epilogue with gain 2 would
+    # double the int8 path's operand rounding (c * s to bf16) before it, so
+    # the int8 cases take the long-context int8 workload's own Mul(0.5)
+    epi = [("mul", 0.5)] if int8 else [("mul", 2.0), ("add", 0.5)]
+    ref_gpu = fa.attention_fwd(q, cuda(kc), cuda(vc), hq=hq, hkv=hkv, causal=True, window=window, epilogue=epi,
+                               k_scales=cuda(ks), v_scales=cuda(vs), cu_seqlens_q=cu_q.cuda(),
+                               cu_seqlens_k=cu_k.cuda(), max_seqlen_q=max(q_lens), max_seqlen_k=max(k_lens))
+    paged = fa.attention_fwd_paged(q, cuda(kp), cuda(vp), cu_k.cuda(), cuda(table), hq=hq, hkv=hkv, causal=True,
+                                   window=window, epilogue=epi, k_scales=cuda(ksp), v_scales=cuda(vsp),
+                                   cu_seqlens_q=cu_q.cuda(), max_seqlen_q=max(q_lens))
+    assert fa.check_device_error() == fa.FA_OK
+    assert torch.equal(ref_gpu, paged)
+    kref = oracle.dequantize(kc, ks) if int8 else kc.float().numpy()
+    vref = oracle.dequantize(vc, vs) if int8 else vc.float().numpy()
+    ref = oracle.attention(q.cpu(), kref, vref, hq=hq, hkv=hkv, causal=True, window=window, epilogue=epi,
+                           cu_seqlens_q=cu_q.numpy(), cu_seqlens_k=cu_k.numpy())
+    assert_close_bf16(paged.float().cpu().numpy(), ref)
+
+
+def test_paged_prefill_dense_queries_and_empty_band():
+    """Dense queries [B*hq, s_q, d] over paged keys, with one sequence holding
+    fewer keys than queries: its first s_q - s_k rows see no key and get the
+    mean of V (the empty-band rule), read through the pages."""
+    fa = _fa()
+    rng = np.random.default_rng(61)
+    B, hq, hkv, d, s_q, page_size = 3, 4, 2, 128, 200, 128
+    k_lens = [300, 150, 130]  # sequences 1, 2: the first 50 and 70 query rows see no key
+    cu_k = torch.tensor(np.concatenate([[0], np.cumsum(k_lens)]), dtype=torch.int32)
+    tk = int(cu_k[-1])
+    k = torch.from_numpy(rng.standard_normal((hkv, tk, d)).astype(np.float32)).bfloat16()
+    v = torch.from_numpy(rng.standard_normal((hkv, tk, d)).astype(np.float32)).bfloat16()
+    q = torch.from_numpy(rng.standard_normal((B * hq, s_q, d)).astype(np.float32)).bfloat16().cuda()
+    kp, _, table = paginate_varlen(k, None, k_lens, hkv, page_size, rng)
+    vp = torch.zeros_like(kp)
+    cu = cu_k.numpy()
+    for b in range(B):
+        for lp in range(table.shape[1]):
+            pg = int(table[b, lp])
+            if pg < 0:
+                continue
+            a, e = cu[b] + lp * page_size, min(cu[b] + (lp + 1) * page_size, cu[b + 1])
+            if e > a:
+                vp[pg, :, :e - a] = v[:, a:e]
+    out = fa.attention_fwd_paged(q, kp.cuda(), vp.cuda(), cu_k.cuda(), table.cuda(), hq=hq, hkv=hkv, causal=True)
+    assert fa.check_device_error() == fa.FA_OK
+    # oracle: per sequence, dense q against that sequence's keys
+    qh = q.cpu().reshape(B, hq, s_q, d)
+    for b in range(B):
+        kb = k[:, cu[b]:cu[b + 1]].float().numpy()
+        vb = v[:, cu[b]:cu[b + 1]].float().numpy()
+        ref = oracle.attention(qh[b].float().numpy(), kb, vb, hq=hq, hkv=hkv, causal=True)
+        got = out.cpu().reshape(B, hq, s_q, d)[b].float().numpy()
+        assert_close_bf16(got, ref, what=f"sequence {b}")
