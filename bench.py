@@ -253,6 +253,10 @@ def gpu_arm(args, rank, world, dist):
         res = {}
         other_prefills(args, dev, peaks, world, dist, res)
         return res
+    if args.only == "ring":
+        res = {}
+        ring_rank_steps(args, dev, peaks, world, dist, res)
+        return res
     l0 = fa.kernel_launches()
     with ClockSampler(dev.index or 0) as clocks:
         ms = time_launches(prefill, args.steps, args.warmup, torch, dist, clocks)
@@ -304,6 +308,7 @@ def gpu_arm(args, rank, world, dist):
     if args.only == "all":
         result["gqa_causal_prefill_paged"] = paged_prefill(args, w, flops_tiles, peaks, world, dist, dev)
         other_prefills(args, dev, peaks, world, dist, result)
+        ring_rank_steps(args, dev, peaks, world, dist, result)
         decode_and_quant(args, dev, peaks, world, dist, result)
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, flops_tiles, flops_exact, args.cpu_seconds)
@@ -408,6 +413,72 @@ def int8_long_prefill(args, dev, peaks, world, dist, result, steps):
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None}}
     del q, kc, vc, ks, vs, out
+    torch.cuda.empty_cache()
+
+
+def ring_rank_steps(args, dev, peaks, world, dist, result):
+    """The device work of the busiest rank of a 4-way context-parallel causal
+    prefill (the last one: its own block causal, three earlier blocks in full),
+    run through ring.attend_blocks (one fa_attention_fwd_acc per block, the
+    merge inside the kernel's epilogue) on blocks already in this GPU's
+    memory, i.e. without the block transfers.  For comparison: the same steps
+    as partial results merged by the separate merge kernel, and that merge
+    kernel alone (HBM-bound)."""
+    import torch
+    from flashattention_attention_b200 import fa, inputs, ring
+    w = inputs.ring_cp_last_rank()
+    R, blk = w.seqlen_k // w.seqlen_q, w.seqlen_q
+    rank = R - 1
+    q = w.q.to(dev)
+    kb = [w.k[:, b * blk:(b + 1) * blk].contiguous().to(dev) for b in range(R)]
+    vb = [w.v[:, b * blk:(b + 1) * blk].contiguous().to(dev) for b in range(R)]
+    blocks = [((rank - s) % R, kb[(rank - s) % R], vb[(rank - s) % R]) for s in range(R)]
+    steps = max(10, args.steps // 4)
+
+    def step():
+        ring.attend_blocks(q, blocks, rank=rank, n_blocks=R, hq=w.hq, hkv=w.hkv, causal=True)
+
+    l0 = fa.kernel_launches()
+    ms = time_launches(step, steps, args.warmup, torch, dist)
+    launches = (fa.kernel_launches() - l0) / (steps + args.warmup)
+    per = w.batch * w.hq * 4 * w.d * TILE * TILE
+    flops = per * (band_tiles(blk, blk, True, 0)[0] + (R - 1) * band_tiles(blk, blk, False, 0)[0])
+    tf = flops / (ms * 1e-3) / 1e12
+
+    acc_o = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    acc_l = torch.empty(q.shape[:-1], dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+
+    def unfused():
+        acc_o.zero_()
+        acc_l.fill_(float("-inf"))
+        for b, k, v in blocks:
+            if b <= rank:
+                o, lse = fa.attention_fwd_lse(q, k, v, hq=w.hq, hkv=w.hkv, causal=b == rank)
+                fa.attention_merge(acc_o, acc_l, o, lse)
+        fa.attention_merge(acc_o, acc_l, out=out)
+
+    ms_unfused = time_launches(unfused, steps, args.warmup, torch, dist)
+    o, lse = fa.attention_fwd_lse(q, kb[0], vb[0], hq=w.hq, hkv=w.hkv)
+    ms_merge = time_launches(lambda: fa.attention_merge(acc_o, acc_l, o, lse), steps, args.warmup, torch, dist)
+    assert fa.check_device_error() == fa.FA_OK
+    rows = q.shape[0] * q.shape[1]
+    # o_acc read + written (fp32), o_part read (bf16), lse_acc read + written, lse_part read
+    merge_bytes = rows * w.d * (4 + 4 + 2) + rows * 3 * 4
+    gbs = merge_bytes / (ms_merge * 1e-3) / 1e9
+    result["ring_cp4_last_rank"] = {
+        "workload": w.name, "value": round(tf * world, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+        "flops_per_step": flops, "flops_counting": "128x128 tiles intersecting each block's band",
+        "transfers": "not timed (blocks resident; one GPU)", "launches_per_step": launches,
+        "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel<128,bf16> (accumulate)",
+                     "achieved": round(tf, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(tf / peaks["bf16_tflops"], 4)},
+        "unfused_lse_then_merge": {"ms": round(ms_unfused, 4),
+                                   "achieved": round(flops / (ms_unfused * 1e-3) / 1e12, 2), "unit": "TFLOP/s"},
+        "merge_kernel": {"ms": round(ms_merge, 4), "bytes": merge_bytes,
+                         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                                      "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4)}}}
+    del q, kb, vb, blocks, o, lse, acc_o, acc_l, out
     torch.cuda.empty_cache()
 
 
@@ -640,7 +711,7 @@ def main():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "quant", "prefill_int8", "varlen"],
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "quant", "prefill_int8", "varlen", "ring"],
                     help="time one part only (used for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:

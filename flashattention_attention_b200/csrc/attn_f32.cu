@@ -14,10 +14,12 @@
 // kernel sees the dequantised cache itself.
 //
 // empty_rows_kernel: rows whose band is empty (causal with s_q > s_k leaves
-// rows i < s_q - s_k without keys) get uniform weights over all s_k keys,
-// i.e. the mean of V (SKaiNET-transformers PR #419, Summary: "empty
-// sliding-window bands reproduce the engine's uniform softmax"), then the
-// epilogue.  The main kernels skip those rows.
+// rows i < s_q - s_k without keys; s_k = 0 leaves every row without keys)
+// get uniform weights over all s_k keys, i.e. the mean of V, zeros for s_k =
+// 0 (SKaiNET-transformers PR #419, Summary: "empty sliding-window bands
+// reproduce the engine's uniform softmax"), then the epilogue.  The main
+// kernels skip those rows.  Partial results (an lse output) or an
+// accumulator to merge into give such rows no weight instead.
 #include "internal.h"
 #include "layout.cuh"
 
@@ -157,13 +159,40 @@ __global__ void __launch_bounds__(128)
 template <typename TV, typename TO>
 __global__ void __launch_bounds__(128)
     empty_rows_kernel(const TV* __restrict__ v, const float* __restrict__ v_scales, TO* __restrict__ out,
-                      SeqLayout L, int hq, int hkv, int d, Epilogue epi) {
+                      RowSink sink, SeqLayout L, int hq, int hkv, int d, Epilogue epi) {
   const int b = blockIdx.y, h = blockIdx.x;
   const int g = h / (hq / hkv);
   const Seq sq = seq_of(L, b, h, g);
-  if (!L.causal) return;
-  const int n_empty = min(sq.s_q, sq.s_q - sq.s_k);
+  // rows i < n_empty have no visible key (a window never empties a row that
+  // the causal mask leaves a key)
+  const int n_empty = sq.s_k == 0 ? sq.s_q : (L.causal ? min(sq.s_q, sq.s_q - sq.s_k) : 0);
   if (n_empty <= 0) return;
+  if (sink.acc_o != nullptr) {
+    // merging nothing: the accumulator stays (or starts empty); the last
+    // step writes it out
+    for (int i = 0; i < n_empty; ++i) {
+      const int64_t row = sq.q_row0 + i;
+      for (int c = threadIdx.x; c < d; c += blockDim.x) {
+        const float a = sink.first ? 0.f : sink.acc_o[row * d + c];
+        if (sink.last) {
+          out[row * d + c] = static_cast<TO>(apply_epilogue(a, epi));
+        } else if (sink.first) {
+          sink.acc_o[row * d + c] = 0.f;
+        }
+      }
+      if (threadIdx.x == 0 && sink.first && !sink.last) sink.acc_lse[row] = -INFINITY;
+    }
+    return;
+  }
+  if (sink.lse != nullptr) {
+    // partial results: rows without keys carry no weight (lse = -inf)
+    const TO zero = static_cast<TO>(apply_epilogue(0.f, epi));
+    for (int i = 0; i < n_empty; ++i) {
+      for (int c = threadIdx.x; c < d; c += blockDim.x) out[(sq.q_row0 + i) * d + c] = zero;
+      if (threadIdx.x == 0) sink.lse[sq.q_row0 + i] = -INFINITY;
+    }
+    return;
+  }
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     float sum = 0.f;
     for (int j = 0; j < sq.s_k; ++j) {
@@ -220,12 +249,15 @@ fa_status launch_attn_f32(const fa_fwd_params& p, const LaunchCtx& ctx) {
   }
 }
 
-fa_status launch_empty_rows(const fa_fwd_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx) {
-  if (!p.causal) return FA_OK;
-  // Dense inputs with s_q <= s_k have no empty row; varlen and paged keys
-  // are decided per sequence on the device.
+fa_status launch_empty_rows(const fa_fwd_params& p, const fa_kv_pages* pages, const RowSink& sink,
+                            const LaunchCtx& ctx) {
+  // Rows lose every key only to the causal mask with s_q > s_k, or when
+  // s_k = 0.  Dense inputs decide it here; varlen self-attention (one
+  // cu_seqlens for both) has s_q = s_k per sequence, so the diagonal (or,
+  // without the causal mask, every key) stays visible; separate varlen key
+  // counts and paged keys are decided per sequence on the device.
   if (pages == nullptr) {
-    if (p.cu_seqlens_q == nullptr && p.seqlen_q <= p.seqlen_k) return FA_OK;
+    if (p.cu_seqlens_q == nullptr && p.seqlen_k > 0 && (!p.causal || p.seqlen_q <= p.seqlen_k)) return FA_OK;
     if (p.cu_seqlens_q != nullptr && (p.cu_seqlens_k == nullptr || p.cu_seqlens_k == p.cu_seqlens_q))
       return FA_OK;
   }
@@ -236,22 +268,22 @@ fa_status launch_empty_rows(const fa_fwd_params& p, const fa_kv_pages* pages, co
     auto kern = empty_rows_kernel<int8_t, float>;
     note_variant(reinterpret_cast<const void*>(kern));
     kern<<<grid, 128, 0, ctx.stream>>>(static_cast<const int8_t*>(p.v), p.v_scales, static_cast<float*>(p.out),
-                                       L, p.hq, p.hkv, p.head_dim, epi);
+                                       sink, L, p.hq, p.hkv, p.head_dim, epi);
   } else if (p.q_dtype == FA_F32) {
     auto kern = empty_rows_kernel<float, float>;
     note_variant(reinterpret_cast<const void*>(kern));
     kern<<<grid, 128, 0, ctx.stream>>>(static_cast<const float*>(p.v), nullptr, static_cast<float*>(p.out),
-                                       L, p.hq, p.hkv, p.head_dim, epi);
+                                       sink, L, p.hq, p.hkv, p.head_dim, epi);
   } else if (p.kv_dtype == FA_I8) {
     auto kern = empty_rows_kernel<int8_t, __nv_bfloat16>;
     note_variant(reinterpret_cast<const void*>(kern));
     kern<<<grid, 128, 0, ctx.stream>>>(static_cast<const int8_t*>(p.v), p.v_scales,
-                                       static_cast<__nv_bfloat16*>(p.out), L, p.hq, p.hkv, p.head_dim, epi);
+                                       static_cast<__nv_bfloat16*>(p.out), sink, L, p.hq, p.hkv, p.head_dim, epi);
   } else {
     auto kern = empty_rows_kernel<__nv_bfloat16, __nv_bfloat16>;
     note_variant(reinterpret_cast<const void*>(kern));
     kern<<<grid, 128, 0, ctx.stream>>>(static_cast<const __nv_bfloat16*>(p.v), nullptr,
-                                       static_cast<__nv_bfloat16*>(p.out), L, p.hq, p.hkv, p.head_dim, epi);
+                                       static_cast<__nv_bfloat16*>(p.out), sink, L, p.hq, p.hkv, p.head_dim, epi);
   }
   return cuda_status(cudaGetLastError());
 }

@@ -176,12 +176,18 @@ fa_status fa_compress_kv(const void* x, fa_dtype x_dtype, int64_t rows, int32_t 
   return launch_compress(x, x_dtype, rows, d, codes, scales, ctx);
 }
 
-fa_status fa_attention_fwd(const fa_fwd_params* p, fa_stream_t stream) {
+namespace {
+// Host checks of fa_attention_fwd's parameters; *launch is false when the
+// call has nothing to do.  need_out = false lets out be NULL.
+fa_status fwd_args(const fa_fwd_params* p, bool* launch, bool need_out = true) {
+  *launch = false;
   if (p == nullptr) return FA_ERR_INVALID;
   if (p->batch < 0 || p->hq <= 0 || p->hkv <= 0 || p->hq % p->hkv != 0) return FA_ERR_INVALID;
   if (!epilogue_ok(p->epilogue, p->n_epilogue)) return FA_ERR_INVALID;
   if (!std::isfinite(p->softmax_scale)) return FA_ERR_INVALID;
   const bool varlen = p->cu_seqlens_q != nullptr;
+  // with no key anywhere K, V and their scales are never read and may be NULL
+  const bool no_keys = varlen ? (p->cu_seqlens_k != nullptr && p->total_k == 0) : p->seqlen_k == 0;
   if (varlen) {
     if (p->total_q < 0 || p->total_k < 0 || p->max_seqlen_q < 0 || p->max_seqlen_k < 0) return FA_ERR_INVALID;
   } else {
@@ -190,13 +196,15 @@ fa_status fa_attention_fwd(const fa_fwd_params* p, fa_stream_t stream) {
   }
   if (p->q_dtype == FA_F32) {
     if (p->kv_dtype != FA_F32 && p->kv_dtype != FA_I8) return FA_ERR_INVALID;
-    if (p->kv_dtype == FA_I8 && (p->k_scales == nullptr || p->v_scales == nullptr)) return FA_ERR_INVALID;
+    if (p->kv_dtype == FA_I8 && !no_keys && (p->k_scales == nullptr || p->v_scales == nullptr))
+      return FA_ERR_INVALID;
     if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
     if (p->head_dim > 256) return FA_ERR_UNSUPPORTED;
   } else if (p->q_dtype == FA_BF16) {
     if (p->kv_dtype != FA_BF16 && p->kv_dtype != FA_I8) return FA_ERR_INVALID;
     if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
-    if (p->kv_dtype == FA_I8 && (p->k_scales == nullptr || p->v_scales == nullptr)) return FA_ERR_INVALID;
+    if (p->kv_dtype == FA_I8 && !no_keys && (p->k_scales == nullptr || p->v_scales == nullptr))
+      return FA_ERR_INVALID;
     if (p->kv_dtype == FA_I8 && (!aligned16(p->k_scales) || !aligned16(p->v_scales))) return FA_ERR_INVALID;
     if (p->head_dim != 64 && p->head_dim != 128) return FA_ERR_UNSUPPORTED;
   } else {
@@ -204,14 +212,86 @@ fa_status fa_attention_fwd(const fa_fwd_params* p, fa_stream_t stream) {
   }
   const bool empty = p->batch == 0 || (varlen ? p->total_q == 0 : p->seqlen_q == 0);
   if (empty) return FA_OK;
-  if (p->q == nullptr || p->k == nullptr || p->v == nullptr || p->out == nullptr) return FA_ERR_INVALID;
-  if (!aligned16(p->q) || !aligned16(p->k) || !aligned16(p->v) || !aligned16(p->out)) return FA_ERR_INVALID;
+  if (p->q == nullptr || (!no_keys && (p->k == nullptr || p->v == nullptr)) || (need_out && p->out == nullptr))
+    return FA_ERR_INVALID;
+  if (!aligned16(p->q) || !aligned16(p->k) || !aligned16(p->v) || (p->out != nullptr && !aligned16(p->out)))
+    return FA_ERR_INVALID;
+  *launch = true;
+  return FA_OK;
+}
+}  // namespace
+
+fa_status fa_attention_fwd(const fa_fwd_params* p, fa_stream_t stream) {
+  bool launch = false;
+  fa_status st = fwd_args(p, &launch);
+  if (st != FA_OK || !launch) return st;
+  LaunchCtx ctx;
+  st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  st = (p->q_dtype == FA_F32) ? launch_attn_f32(*p, ctx) : launch_prefill_tc(*p, nullptr, RowSink{}, ctx);
+  if (st != FA_OK) return st;
+  return launch_empty_rows(*p, nullptr, RowSink{}, ctx);
+}
+
+fa_status fa_attention_fwd_lse(const fa_fwd_params* p, float* lse, fa_stream_t stream) {
+  bool launch = false;
+  fa_status st = fwd_args(p, &launch);
+  if (st != FA_OK) return st;
+  if (p->q_dtype != FA_BF16) return FA_ERR_UNSUPPORTED;  // the fp32 path has no lse output
+  if (!launch) return FA_OK;
+  if (lse == nullptr || !aligned16(lse)) return FA_ERR_INVALID;
+  LaunchCtx ctx;
+  st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  RowSink sink;
+  sink.lse = lse;
+  st = launch_prefill_tc(*p, nullptr, sink, ctx);
+  if (st != FA_OK) return st;
+  return launch_empty_rows(*p, nullptr, sink, ctx);
+}
+
+fa_status fa_attention_fwd_acc(const fa_fwd_params* p, float* o_acc, float* lse_acc, int32_t flags,
+                               fa_stream_t stream) {
+  if ((flags & ~(FA_ACC_FIRST | FA_ACC_LAST)) != 0) return FA_ERR_INVALID;
+  const bool last = (flags & FA_ACC_LAST) != 0;
+  bool launch = false;
+  fa_status st = fwd_args(p, &launch, last);
+  if (st != FA_OK) return st;
+  if (p->q_dtype != FA_BF16) return FA_ERR_UNSUPPORTED;  // the tensor-core path only
+  if (!launch) return FA_OK;
+  if (o_acc == nullptr || lse_acc == nullptr || !aligned16(o_acc) || !aligned16(lse_acc)) return FA_ERR_INVALID;
+  LaunchCtx ctx;
+  st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  RowSink sink;
+  sink.acc_o = o_acc;
+  sink.acc_lse = lse_acc;
+  sink.first = (flags & FA_ACC_FIRST) != 0;
+  sink.last = last;
+  fa_fwd_params q = *p;
+  if (!last) q.out = nullptr;  // not written
+  st = launch_prefill_tc(q, nullptr, sink, ctx);
+  if (st != FA_OK) return st;
+  return launch_empty_rows(q, nullptr, sink, ctx);
+}
+
+fa_status fa_attention_merge(const fa_merge_params* p, fa_stream_t stream) {
+  if (p == nullptr || p->rows < 0) return FA_ERR_INVALID;
+  if (p->head_dim < 32 || p->head_dim > 256 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
+  if (!epilogue_ok(p->epilogue, p->n_epilogue)) return FA_ERR_INVALID;
+  if (p->o_part != nullptr && p->part_dtype != FA_BF16 && p->part_dtype != FA_F32) return FA_ERR_INVALID;
+  if (p->out != nullptr && p->out_dtype != FA_BF16 && p->out_dtype != FA_F32) return FA_ERR_INVALID;
+  if (p->rows == 0) return FA_OK;
+  if (p->o_acc == nullptr || p->lse_acc == nullptr || (p->o_part != nullptr && p->lse_part == nullptr))
+    return FA_ERR_INVALID;
+  if (!aligned16(p->o_acc) || !aligned16(p->lse_acc) || (p->o_part && !aligned16(p->o_part)) ||
+      (p->lse_part && !aligned16(p->lse_part)) || (p->out && !aligned16(p->out)))
+    return FA_ERR_INVALID;
   LaunchCtx ctx;
   fa_status st = make_ctx(stream, &ctx);
   if (st != FA_OK) return st;
-  st = (p->q_dtype == FA_F32) ? launch_attn_f32(*p, ctx) : launch_prefill_tc(*p, nullptr, ctx);
-  if (st != FA_OK) return st;
-  return launch_empty_rows(*p, nullptr, ctx);
+  return launch_merge(p->o_acc, p->lse_acc, p->o_part, p->part_dtype, p->lse_part, p->rows, p->head_dim, p->out,
+                      p->out_dtype, p->epilogue, p->n_epilogue, ctx);
 }
 
 fa_status fa_attention_fwd_paged(const fa_fwd_params* p, const fa_kv_pages* pages, fa_stream_t stream) {
@@ -241,9 +321,9 @@ fa_status fa_attention_fwd_paged(const fa_fwd_params* p, const fa_kv_pages* page
   LaunchCtx ctx;
   fa_status st = make_ctx(stream, &ctx);
   if (st != FA_OK) return st;
-  st = launch_prefill_tc(*p, pages, ctx);
+  st = launch_prefill_tc(*p, pages, RowSink{}, ctx);
   if (st != FA_OK) return st;
-  return launch_empty_rows(*p, pages, ctx);
+  return launch_empty_rows(*p, pages, RowSink{}, ctx);
 }
 
 size_t fa_decode_workspace_size(int32_t batch, int32_t hq, int32_t capacity, int32_t head_dim) {

@@ -23,8 +23,25 @@ fa_status launch_compress(const void* x, int x_dtype, int64_t rows, int d, int8_
                           const LaunchCtx& ctx);
 fa_status launch_kv_append(const fa_kv_append_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx);
 fa_status launch_attn_f32(const fa_fwd_params& p, const LaunchCtx& ctx);
-fa_status launch_empty_rows(const fa_fwd_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx);
-fa_status launch_prefill_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx);
+
+// How the tensor-core prefill hands over its rows: the normalised output
+// (all null), that output with its per-row log-sum-exp (lse), or merged into
+// an fp32 accumulator (acc_o, acc_lse; see fa_attention_fwd_acc).
+struct RowSink {
+  float* lse = nullptr;
+  float* acc_o = nullptr;
+  float* acc_lse = nullptr;
+  int first = 0;  // the accumulator holds nothing yet and is not read
+  int last = 0;   // the merged rows go to out; the accumulator is left as it was
+};
+
+fa_status launch_empty_rows(const fa_fwd_params& p, const fa_kv_pages* pages, const RowSink& sink,
+                            const LaunchCtx& ctx);
+fa_status launch_prefill_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowSink& sink,
+                            const LaunchCtx& ctx);
+fa_status launch_merge(float* o_acc, float* lse_acc, const void* o_part, int part_dtype, const float* lse_part,
+                       int64_t rows, int d, void* out, int out_dtype, const fa_epi_op* epi, int n_epi,
+                       const LaunchCtx& ctx);
 fa_status launch_decode(const fa_decode_params& p, const fa_kv_pages* pages, int split_keys, const LaunchCtx& ctx);
 size_t decode_workspace_bytes(int batch, int hq, int head_dim);
 int decode_noalloc_workers(int batch, int hq, int hkv, int head_dim);

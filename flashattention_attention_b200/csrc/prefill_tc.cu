@@ -28,6 +28,14 @@
 // P (bf16, two per 32-bit column) overwrites the first 64 columns of its S
 // tile and is the A operand of O += P V straight from TMEM.
 //
+// Result modes: the normalised output (epilogue applied, bf16); that output
+// with each row's log-sum-exp (a partial result over the given keys); or,
+// for a result built up over several key blocks (the ring steps of a
+// context-parallel prefill -- kernbench2 commit message, ADR-0060 (long
+// context): an online-softmax merge at every ring step), merged in the
+// epilogue into an fp32 accumulator (o, lse) that the softmax warps
+// prefetch into L2 when an item starts, so no separate merge pass runs.
+//
 // MMA issue order per key tile j (ping-pong between the two Q tiles):
 //   PV0(j-1), S0(j), PV1(j-1), S1(j)
 // so the tensor core works on one tile while the other tile's softmax runs.
@@ -95,6 +103,11 @@ static_assert(TcGeom<64, true>::kSmem <= 232448, "shared memory budget");
 struct PrefillArgs {
   SeqLayout L;
   __nv_bfloat16* out;
+  float* lse;  // optional [rows of out]: log-sum-exp of the scaled scores (partial results)
+  float* acc_o;    // optional fp32 [rows of out, D] accumulator merged into (with acc_lse)
+  float* acc_lse;
+  int acc_first;   // the accumulator holds nothing yet: not read
+  int acc_last;    // merged rows go to out (epilogue applied); the accumulator is not written
   const float* k_scales;  // int8 variant: one fp32 scale per K / V row
   const float* v_scales;
   int64_t k_plane_rows;   // rows per K plane (the scales share K's row numbering)
@@ -465,6 +478,14 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
     const int i = w.i0 + r;
     int lo, hi;
     band_of(A.L, i, w.sq.s_q, w.sq.s_k, lo, hi);
+    const int64_t out_row = w.sq.q_row0 + static_cast<int64_t>(t) * A.L.q_hstride + i;
+    if (A.acc_o != nullptr && !A.acc_first && i < w.sq.s_q) {
+      // the accumulator row is read in this item's epilogue: start it towards L2
+      const char* arow = reinterpret_cast<const char*>(A.acc_o + out_row * D);
+#pragma unroll
+      for (int c = 0; c < D * 4; c += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(arow + c));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(A.acc_lse + out_row));
+    }
     float m_used = -INFINITY, l = 0.f;
     for (int it = 0; it < w.n_iter; ++it) {
       ok = __all_sync(0xffffffffu, wait_parity(s_full + t, (base + it) & 1, A.wd, &abort_flag));
@@ -554,9 +575,30 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
     if (ok) ok = __all_sync(0xffffffffu, wait_parity(o_done + t, done & 1, A.wd, &abort_flag));
     if (!ok) break;
     tc_fence_after();
-    const bool store = i < w.sq.s_q && lo < hi;
-    const float inv_l = 1.f / l;
-    __nv_bfloat16* orow = A.out + (w.sq.q_row0 + static_cast<int64_t>(t) * A.L.q_hstride + i) * D;
+    const bool has_keys = lo < hi;
+    const bool acc = A.acc_o != nullptr;
+    // with lse (partial results) a row without keys is the epilogue of 0 with
+    // lse = -inf; otherwise (and always when accumulating) the empty-band
+    // kernel writes it
+    const bool store = i < w.sq.s_q && (has_keys || (A.lse != nullptr && !acc));
+    float inv_l = has_keys ? 1.f / l : 0.f;
+    float w_acc = 0.f;  // accumulate mode: o_new = w_acc * o_acc + inv_l * O
+    if (store && (A.lse != nullptr || acc)) {
+      const float lse_part = has_keys ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+      if (A.lse != nullptr) A.lse[out_row] = lse_part;
+      if (acc) {
+        // merge by log-sum-exp: lse = log(e^lse_acc + e^lse_part), each side
+        // weighted by e^(its lse - lse); this row has keys, so lse_part is finite
+        const float la = A.acc_first ? -INFINITY : A.acc_lse[out_row];
+        const float mx = fmaxf(la, lse_part);
+        const float ea = expf(la - mx), eb = expf(lse_part - mx), sum = ea + eb;
+        w_acc = ea / sum;
+        inv_l *= eb / sum;
+        if (!A.acc_last) A.acc_lse[out_row] = mx + logf(sum);
+      }
+    }
+    __nv_bfloat16* orow = A.out != nullptr ? A.out + out_row * D : nullptr;
+    float* arow = acc ? A.acc_o + out_row * D : nullptr;
 #pragma unroll
     for (int oc = 0; oc < D / 32; ++oc) {
       uint32_t o[32];
@@ -570,6 +612,25 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       float y[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) y[e] = __uint_as_float(o[e]) * inv_l;
+      if (acc && store && w_acc != 0.f) {
+        const float4* src = reinterpret_cast<const float4*>(arow + oc * 32);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 a = src[v];
+          y[4 * v] = fmaf(a.x, w_acc, y[4 * v]);
+          y[4 * v + 1] = fmaf(a.y, w_acc, y[4 * v + 1]);
+          y[4 * v + 2] = fmaf(a.z, w_acc, y[4 * v + 2]);
+          y[4 * v + 3] = fmaf(a.w, w_acc, y[4 * v + 3]);
+        }
+      }
+      if (acc && !A.acc_last) {
+        if (store) {
+          float4* dst = reinterpret_cast<float4*>(arow + oc * 32);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) dst[v] = make_float4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
+        }
+        continue;
+      }
       apply_epilogue_vec(y, A.epi);
       uint32_t pk[16];
 #pragma unroll
@@ -595,7 +656,7 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
 }
 
 template <int D, bool kI8>
-fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx) {
+fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowSink& sink, const LaunchCtx& ctx) {
   using G = TcGeom<D, kI8>;
   const bool varlen = p.cu_seqlens_q != nullptr;
   const uint64_t q_rows = varlen ? p.total_q : p.seqlen_q;
@@ -638,6 +699,11 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const Laun
   PrefillArgs A;
   A.L = pages != nullptr ? SeqLayout::paged(p, *pages) : SeqLayout::from(p);
   A.out = static_cast<__nv_bfloat16*>(p.out);
+  A.lse = sink.lse;
+  A.acc_o = sink.acc_o;
+  A.acc_lse = sink.acc_lse;
+  A.acc_first = sink.first;
+  A.acc_last = sink.last;
   A.k_scales = p.k_scales;
   A.v_scales = p.v_scales;
   A.k_plane_rows = static_cast<int64_t>(k_rows);
@@ -672,14 +738,15 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const Laun
 
 }  // namespace
 
-fa_status launch_prefill_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const LaunchCtx& ctx) {
+fa_status launch_prefill_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowSink& sink,
+                            const LaunchCtx& ctx) {
   if (p.kv_dtype == FA_I8) {
-    if (p.head_dim == 128) return launch_tc<128, true>(p, pages, ctx);
-    if (p.head_dim == 64) return launch_tc<64, true>(p, pages, ctx);
+    if (p.head_dim == 128) return launch_tc<128, true>(p, pages, sink, ctx);
+    if (p.head_dim == 64) return launch_tc<64, true>(p, pages, sink, ctx);
     return FA_ERR_UNSUPPORTED;
   }
-  if (p.head_dim == 128) return launch_tc<128, false>(p, pages, ctx);
-  if (p.head_dim == 64) return launch_tc<64, false>(p, pages, ctx);
+  if (p.head_dim == 128) return launch_tc<128, false>(p, pages, sink, ctx);
+  if (p.head_dim == 64) return launch_tc<64, false>(p, pages, sink, ctx);
   return FA_ERR_UNSUPPORTED;
 }
 

@@ -28,6 +28,7 @@ FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_W
 FA_F32, FA_BF16, FA_I8 = 0, 1, 2
 FA_EPI_MUL, FA_EPI_ADD = 1, 2
 FA_MAX_EPILOGUE = 8
+FA_ACC_FIRST, FA_ACC_LAST = 1, 2
 
 
 class EpiOp(ctypes.Structure):
@@ -60,6 +61,13 @@ class DecodeParams(ctypes.Structure):
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class MergeParams(ctypes.Structure):
+    _fields_ = [("o_acc", ctypes.c_void_p), ("lse_acc", ctypes.c_void_p), ("o_part", ctypes.c_void_p),
+                ("part_dtype", ctypes.c_int32), ("lse_part", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("head_dim", ctypes.c_int32), ("out", ctypes.c_void_p), ("out_dtype", ctypes.c_int32),
+                ("n_epilogue", ctypes.c_int32), ("epilogue", EpiOp * FA_MAX_EPILOGUE)]
+
+
 class KvPages(ctypes.Structure):
     _fields_ = [("block_table", ctypes.c_void_p), ("max_pages", ctypes.c_int32),
                 ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
@@ -83,6 +91,13 @@ lib.fa_decode_workspace_size.restype = ctypes.c_size_t
 lib.fa_decode_workspace_size.argtypes = [ctypes.c_int32] * 4
 lib.fa_attention_decode.restype = ctypes.c_int
 lib.fa_attention_decode.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_void_p]
+lib.fa_attention_fwd_lse.restype = ctypes.c_int
+lib.fa_attention_fwd_lse.argtypes = [ctypes.POINTER(FwdParams), ctypes.c_void_p, ctypes.c_void_p]
+lib.fa_attention_fwd_acc.restype = ctypes.c_int
+lib.fa_attention_fwd_acc.argtypes = [ctypes.POINTER(FwdParams), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                     ctypes.c_void_p]
+lib.fa_attention_merge.restype = ctypes.c_int
+lib.fa_attention_merge.argtypes = [ctypes.POINTER(MergeParams), ctypes.c_void_p]
 lib.fa_attention_fwd_paged.restype = ctypes.c_int
 lib.fa_attention_fwd_paged.argtypes = [ctypes.POINTER(FwdParams), ctypes.POINTER(KvPages), ctypes.c_void_p]
 lib.fa_attention_decode_paged.restype = ctypes.c_int
@@ -197,6 +212,81 @@ def attention_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, hq: int,
                    epilogue=epilogue, k_scales=k_scales, v_scales=v_scales, cu_seqlens_q=cu_seqlens_q,
                    cu_seqlens_k=cu_seqlens_k, max_seqlen_q=max_seqlen_q, max_seqlen_k=max_seqlen_k)
     _check(lib.fa_attention_fwd(ctypes.byref(p), _stream(stream)), "fa_attention_fwd")
+    return out
+
+
+def attention_fwd_lse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, hq: int, hkv: int,
+                      causal: bool = False, window: int = 0, scale: Optional[float] = None,
+                      k_scales=None, v_scales=None, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None,
+                      max_seqlen_k=None, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                      stream=None):
+    """Partial attention result (bf16 path): (out, lse) with lse the natural
+    log-sum-exp of each row's scaled scores (-inf and out = 0 for a row
+    without keys).  As fa_attention_fwd_lse in fa.h; no epilogue."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _contig_cuda(t, name)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    p = fwd_params(q, k, v, out, hq=hq, hkv=hkv, causal=causal, window=window, scale=scale, epilogue=(),
+                   k_scales=k_scales, v_scales=v_scales, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
+                   max_seqlen_q=max_seqlen_q, max_seqlen_k=max_seqlen_k)
+    _check(lib.fa_attention_fwd_lse(ctypes.byref(p), _ptr(lse), _stream(stream)), "fa_attention_fwd_lse")
+    return out, lse
+
+
+def attention_fwd_acc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o_acc: torch.Tensor,
+                      lse_acc: torch.Tensor, *, hq: int, hkv: int, causal: bool = False, window: int = 0,
+                      scale: Optional[float] = None, first: bool = False, last: bool = False,
+                      out: Optional[torch.Tensor] = None, epilogue: Sequence[Tuple[str, float]] = (),
+                      k_scales=None, v_scales=None, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None,
+                      max_seqlen_k=None, stream=None) -> Optional[torch.Tensor]:
+    """Attention of q over these keys merged into the fp32 accumulator
+    (o_acc [..., d] like q, lse_acc [...]) in the kernel's epilogue.  first:
+    the accumulator is empty and not read; last: the merged rows go to `out`
+    (allocated in q's dtype if None) after the epilogue and are returned,
+    the accumulator is left as it was.  As fa_attention_fwd_acc in fa.h."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o_acc", o_acc), ("lse_acc", lse_acc)):
+        _contig_cuda(t, name)
+    if o_acc.dtype != torch.float32 or lse_acc.dtype != torch.float32:
+        raise ValueError("the accumulator is fp32")
+    if o_acc.shape != q.shape or lse_acc.shape != q.shape[:-1]:
+        raise ValueError("o_acc must have q's shape and lse_acc q's shape without the last dim")
+    if last and out is None:
+        out = torch.empty_like(q)
+    p = fwd_params(q, k, v, out if last else q, hq=hq, hkv=hkv, causal=causal, window=window, scale=scale,
+                   epilogue=epilogue, k_scales=k_scales, v_scales=v_scales, cu_seqlens_q=cu_seqlens_q,
+                   cu_seqlens_k=cu_seqlens_k, max_seqlen_q=max_seqlen_q, max_seqlen_k=max_seqlen_k)
+    if not last:
+        p.out = None
+    flags = (FA_ACC_FIRST if first else 0) | (FA_ACC_LAST if last else 0)
+    _check(lib.fa_attention_fwd_acc(ctypes.byref(p), _ptr(o_acc), _ptr(lse_acc), flags, _stream(stream)),
+           "fa_attention_fwd_acc")
+    return out if last else None
+
+
+def attention_merge(o_acc: torch.Tensor, lse_acc: torch.Tensor, o_part: Optional[torch.Tensor] = None,
+                    lse_part: Optional[torch.Tensor] = None, *, out: Optional[torch.Tensor] = None,
+                    epilogue: Sequence[Tuple[str, float]] = (), stream=None) -> Optional[torch.Tensor]:
+    """Fold the partial result (o_part, lse_part) into the fp32 accumulator
+    (o_acc [..., d], lse_acc [...]) in place; with `out`, also write the
+    merged rows after the epilogue.  As fa_attention_merge in fa.h."""
+    _contig_cuda(o_acc, "o_acc")
+    _contig_cuda(lse_acc, "lse_acc")
+    p = MergeParams()
+    p.o_acc, p.lse_acc = o_acc.data_ptr(), lse_acc.data_ptr()
+    if o_part is not None:
+        _contig_cuda(o_part, "o_part")
+        _contig_cuda(lse_part, "lse_part")
+        p.o_part, p.part_dtype, p.lse_part = o_part.data_ptr(), _DT[o_part.dtype], lse_part.data_ptr()
+    p.head_dim = o_acc.shape[-1]
+    p.rows = o_acc.numel() // p.head_dim
+    if out is not None:
+        _contig_cuda(out, "out")
+        p.out, p.out_dtype = out.data_ptr(), _DT[out.dtype]
+    p.n_epilogue = _fill_epilogue(p.epilogue, epilogue)
+    _check(lib.fa_attention_merge(ctypes.byref(p), _stream(stream)), "fa_attention_merge")
     return out
 
 

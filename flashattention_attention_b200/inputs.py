@@ -128,6 +128,15 @@ def gqa_causal_prefill(seed=0, batch=4, s=4096) -> Workload:
                          dtype=torch.bfloat16, causal=True, seed=seed)
 
 
+def ring_cp_last_rank(seed=0, batch=4, block=4096, ranks=4) -> Workload:
+    """The last rank of a `ranks`-way context-parallel causal prefill: its
+    query block q [batch*32, block, 128] and the K/V of all ranks
+    [batch*8, ranks*block, 128] (block r = positions r*block..), bf16."""
+    return dense_prefill(f"ring_cp{ranks}_last_rank_b{batch}_hq32_hkv8_block{block}_d128_bf16",
+                         batch=batch, hq=32, hkv=8, s_q=block, s_k=ranks * block, d=128,
+                         dtype=torch.bfloat16, causal=True, seed=seed)
+
+
 def int8kv_decode(seed=0, batch=16, lo=1024, hi=32768, capacity=32768) -> Workload:
     """s_q=1 decode, B=16, Hq=32, Hkv=8, d=128, cache lengths U[1024, 32768]."""
     lengths = np.random.default_rng(seed).integers(lo, hi + 1, batch)

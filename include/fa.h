@@ -117,6 +117,8 @@ FA_API fa_status fa_compress_kv(const void *x, fa_dtype x_dtype, int64_t rows, i
  * path c * s is formed exactly in fp32 and rounded once to bf16, the
  * tensor-core operand type.  out has q's dtype.
  * head_dim: F32 path any multiple of 32 up to 256; BF16/I8 paths 64 or 128.
+ * A problem without keys (seqlen_k = 0, or varlen total_k = 0 with
+ * cu_seqlens_k given) reads no K or V: k, v and the scales may be NULL.
  */
 typedef struct {
     const void *q;
@@ -245,6 +247,72 @@ FA_API fa_status fa_attention_decode_paged(const fa_decode_params *p, const fa_k
  * on the same keys in a contiguous layout bit for bit.
  */
 FA_API fa_status fa_attention_fwd_paged(const fa_fwd_params *p, const fa_kv_pages *pages, fa_stream_t stream);
+
+/*
+ * fa_attention_fwd_lse -- fa_attention_fwd (bf16 tensor-core path) that also
+ * returns, per output row, the natural log-sum-exp of the row's scaled
+ * scores over its visible keys: a partial result that fa_attention_merge can
+ * combine with others over disjoint key sets (the per-step (m, l, O) state
+ * of a split or ring computation -- kernbench2 commit message, ADR-0060 (long context)).
+ *   lse  [batch*hq*seqlen_q] fp32 (dense) or [hq*total_q] (varlen), the row
+ *        numbering of out
+ * A row without visible keys gets out = the epilogue applied to 0 and
+ * lse = -inf (no uniform fallback: such a row weighs nothing in a merge).
+ * Partial results meant for merging should carry no epilogue.
+ */
+FA_API fa_status fa_attention_fwd_lse(const fa_fwd_params *p, float *lse, fa_stream_t stream);
+
+/*
+ * fa_attention_fwd_acc -- fa_attention_fwd_lse and fa_attention_merge in one
+ * pass: the attention of q over this call's keys is merged, row by row, into
+ * an fp32 accumulator inside the kernel's epilogue, so a result built up over
+ * several key blocks (the steps of a ring / context-parallel prefill --
+ * kernbench2 commit message, ADR-0060 (long context): an online-softmax
+ * merge at every ring step) costs no separate merge pass.
+ *   o_acc   [rows of out, head_dim] fp32 (out's row numbering), 16-byte aligned
+ *   lse_acc [rows of out] fp32: natural log-sum-exp of the scaled scores seen
+ *           so far (-inf: none), 16-byte aligned
+ *   flags   FA_ACC_FIRST: the accumulator holds nothing yet and is not read
+ *           (it is written as if it had been o = 0, lse = -inf);
+ *           FA_ACC_LAST: the merged rows are written to p->out, after the
+ *           epilogue, instead of back to the accumulator (left unchanged)
+ * p->out is used only with FA_ACC_LAST (may be NULL otherwise), and the
+ * epilogue applies only there.  A row without visible keys merges nothing.
+ * BF16 path (q FA_BF16, K/V FA_BF16 or FA_I8) only: other q types give
+ * FA_ERR_UNSUPPORTED.
+ */
+#define FA_ACC_FIRST 1
+#define FA_ACC_LAST 2
+FA_API fa_status fa_attention_fwd_acc(const fa_fwd_params *p, float *o_acc, float *lse_acc, int32_t flags,
+                                      fa_stream_t stream);
+
+/*
+ * fa_attention_merge -- fold a partial attention result into an accumulator:
+ *   lse = log(e^lse_acc + e^lse_part)
+ *   o_acc = o_acc e^(lse_acc - lse) + o_part e^(lse_part - lse)
+ * per row (lse_acc = -inf and o_acc = 0 start an empty accumulator; two
+ * empty rows stay empty).  o_part NULL merges nothing (only writes out).
+ *   o_acc     [rows, head_dim] fp32, updated in place;  lse_acc [rows] fp32
+ *   o_part    [rows, head_dim] part_dtype (FA_BF16 or FA_F32);  lse_part [rows]
+ *   out       optional [rows, head_dim] out_dtype (FA_BF16 or FA_F32): the
+ *             merged rows after the epilogue (the last merge of a sequence)
+ * head_dim a multiple of 32 up to 256; pointers 16-byte aligned.
+ */
+typedef struct {
+    float *o_acc;
+    float *lse_acc;
+    const void *o_part;
+    int32_t part_dtype;
+    const float *lse_part;
+    int64_t rows;
+    int32_t head_dim;
+    void *out;
+    int32_t out_dtype;
+    int32_t n_epilogue;
+    fa_epi_op epilogue[FA_MAX_EPILOGUE];
+} fa_merge_params;
+
+FA_API fa_status fa_attention_merge(const fa_merge_params *p, fa_stream_t stream);
 
 /*
  * fa_kv_append -- write one new token per sequence into a decode KV cache,

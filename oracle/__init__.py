@@ -23,7 +23,11 @@ Definitions followed:
   * cache append at a device-side slot: FlashRT QKV Cache RoPE, Kernels
     ("... selects the cache slot from a CUDA int32 cur_pos tensor"): row
     b*hkv + g of the new token goes to slot cur_pos[b] of its cache row,
-    compressed as compress_kv does; nothing else changes.
+    compressed as compress_kv does; nothing else changes;
+  * partial results over disjoint key sets and their merge: kernbench2
+    commit message, ADR-0060 (long context: an online-softmax merge of the
+    per-step (m, l, O) state at every ring step), written with the
+    log-sum-exp lse = m + log l.
 
 Every function is pinned by ``tests/test_oracle.py`` against closed forms,
 invariants, torch's fp64 scaled_dot_product_attention, pure-Python brute force
@@ -160,6 +164,76 @@ def attention(q, k, v, *, hq: int, hkv: int, causal: bool = False, window: int =
         _run(q, k, v, out, batch, hq, hkv, d, 0, tq, cq[:-1], np.diff(cq), 0, tk,
              ck[:-1], np.diff(ck), scale, causal, window, epilogue, rows)
     return out
+
+
+def attention_lse(q, k, v, *, hq: int, hkv: int, causal: bool = False, window: int = 0,
+                  scale: Optional[float] = None, cu_seqlens_q=None, cu_seqlens_k=None):
+    """Partial attention result: (o, lse) in fp64, numpy, one (sequence,
+    head) score matrix at a time.  lse[row] = log of the sum of exp(scale *
+    q.k) over the row's visible keys, o[row] the softmax-weighted mean of
+    their values; a row with no visible key has lse = -inf and o = 0 (it
+    weighs nothing when partial results over disjoint key sets are merged).
+    Layouts, masks and the GQA map as attention(); no epilogue.
+    """
+    qf, kf, vf = _f64(q), _f64(k), _f64(v)
+    d = qf.shape[-1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    group = hq // hkv
+    o = np.zeros_like(qf)
+    lse = np.full(qf.shape[:-1], -np.inf)
+    if cu_seqlens_q is None:
+        batch = qf.shape[0] // hq
+        spans = [((b * hq, 0, qf.shape[1]), (b * hkv, 0, kf.shape[1])) for b in range(batch)]
+    else:
+        cq, ck = np.asarray(cu_seqlens_q), np.asarray(cu_seqlens_k)
+        spans = [((0, int(cq[b]), int(cq[b + 1] - cq[b])), (0, int(ck[b]), int(ck[b + 1] - ck[b])))
+                 for b in range(len(cq) - 1)]
+    for (qp, q0, s_q), (kp, k0, s_k) in spans:
+        i = np.arange(s_q)[:, None]
+        j = np.arange(s_k)[None, :]
+        pos = i + s_k - s_q
+        vis = np.ones((s_q, s_k), dtype=bool)
+        if causal:
+            vis &= j <= pos
+        if window > 0:
+            vis &= j > pos - window
+        for h in range(hq):
+            g = h // group
+            qs = qf[qp + h, q0:q0 + s_q] if cu_seqlens_q is None else qf[h, q0:q0 + s_q]
+            ks = kf[kp + g, k0:k0 + s_k] if cu_seqlens_q is None else kf[g, k0:k0 + s_k]
+            vs = vf[kp + g, k0:k0 + s_k] if cu_seqlens_q is None else vf[g, k0:k0 + s_k]
+            x = np.where(vis, scale * (qs @ ks.T), -np.inf)
+            m = x.max(axis=1, initial=-np.inf)
+            has = np.isfinite(m)
+            w = np.exp(x - np.where(has, m, 0.0)[:, None])
+            l = w.sum(axis=1)
+            rows = np.where(has)[0]
+            out = np.zeros((s_q, d))
+            out[rows] = (w[rows] @ vs) / l[rows, None]
+            ls = np.full(s_q, -np.inf)
+            ls[rows] = m[rows] + np.log(l[rows])
+            if cu_seqlens_q is None:
+                o[qp + h, q0:q0 + s_q] = out
+                lse[qp + h, q0:q0 + s_q] = ls
+            else:
+                o[h, q0:q0 + s_q] = out
+                lse[h, q0:q0 + s_q] = ls
+    return o, lse
+
+
+def merge(o_a, lse_a, o_b, lse_b):
+    """The partial result over the union of two disjoint key sets:
+    lse = log(e^lse_a + e^lse_b), o = o_a e^(lse_a - lse) + o_b e^(lse_b - lse)
+    (fp64; rows empty in both stay o = 0, lse = -inf)."""
+    oa, ob = _f64(o_a), _f64(o_b)
+    la, lb = np.asarray(lse_a, dtype=np.float64), np.asarray(lse_b, dtype=np.float64)
+    lse = np.logaddexp(la, lb)
+    fin = np.isfinite(lse)
+    safe = np.where(fin, lse, 0.0)  # rows empty on both sides get weight 0
+    wa = np.where(fin, np.exp(la - safe), 0.0)
+    wb = np.where(fin, np.exp(lb - safe), 0.0)
+    return oa * wa[..., None] + ob * wb[..., None], lse
 
 
 def decode(q, k_cache, v_cache, cache_seqlens, *, hq: int, hkv: int, window: int = 0,

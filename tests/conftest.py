@@ -41,7 +41,7 @@ def pytest_sessionstart(session):
 
 
 def assert_close_bf16(got, ref, atol=2e-2, rel_l2=5e-3, what=""):
-    """Spec tolerance for bf16 outputs: max abs <= 2e-2 and relative
+    """The bf16 output gate: max abs <= 2e-2 and relative
     L2 <= 5e-3 against the fp64 oracle run on the same bf16 inputs."""
     import numpy as np
     g = np.asarray(got, dtype=np.float64)

@@ -277,3 +277,69 @@ def test_fwd_paged_rejects_bad_arguments(fa):
     assert call(head_dim=96) == fa.FA_ERR_UNSUPPORTED
     assert call(kv_dtype=fa.FA_I8) == fa.FA_ERR_INVALID       # int8 needs scales
     assert call(seqlen_q=0) == fa.FA_OK                       # nothing to do
+
+
+def test_fwd_lse_rejects_bad_arguments(fa):
+    import torch
+    lse = 0x50000
+    assert fa.lib.fa_attention_fwd_lse(None, lse, None) == fa.FA_ERR_INVALID
+    p = fwd(fa)
+    assert fa.lib.fa_attention_fwd_lse(ctypes.byref(p), None, None) == fa.FA_ERR_INVALID  # no lse buffer
+    assert fa.lib.fa_attention_fwd_lse(ctypes.byref(p), 0x50004, None) == fa.FA_ERR_INVALID  # misaligned lse
+    p = fwd(fa, q=FakeTensor(0x10000, (4, 64, 128), torch.float32), k=FakeTensor(0x20000, (2, 64, 128), torch.float32),
+            v=FakeTensor(0x30000, (2, 64, 128), torch.float32), out=FakeTensor(0x40000, (4, 64, 128), torch.float32))
+    assert fa.lib.fa_attention_fwd_lse(ctypes.byref(p), lse, None) == fa.FA_ERR_UNSUPPORTED  # fp32: no lse output
+    p = fwd(fa)
+    p.hq = 3
+    assert fa.lib.fa_attention_fwd_lse(ctypes.byref(p), lse, None) == fa.FA_ERR_INVALID
+    p = fwd(fa)
+    p.seqlen_q = 0
+    p.q = p.k = p.v = p.out = None
+    assert fa.lib.fa_attention_fwd_lse(ctypes.byref(p), None, None) == fa.FA_OK  # empty problem
+
+
+def test_merge_rejects_bad_arguments(fa):
+    assert fa.lib.fa_attention_merge(None, None) == fa.FA_ERR_INVALID
+
+    def params(**kw):
+        p = fa.MergeParams()
+        p.o_acc, p.lse_acc, p.o_part, p.lse_part = 0x10000, 0x20000, 0x30000, 0x40000
+        p.part_dtype, p.rows, p.head_dim = fa.FA_BF16, 10, 128
+        for key, val in kw.items():
+            setattr(p, key, val)
+        return fa.lib.fa_attention_merge(ctypes.byref(p), None)
+
+    assert params(head_dim=48) == fa.FA_ERR_INVALID
+    assert params(head_dim=288) == fa.FA_ERR_INVALID
+    assert params(rows=-1) == fa.FA_ERR_INVALID
+    assert params(part_dtype=fa.FA_I8) == fa.FA_ERR_INVALID
+    assert params(out=0x50000, out_dtype=fa.FA_I8) == fa.FA_ERR_INVALID
+    assert params(lse_part=None) == fa.FA_ERR_INVALID
+    assert params(o_acc=None) == fa.FA_ERR_INVALID
+    assert params(o_acc=0x10008) == fa.FA_ERR_INVALID
+    assert params(n_epilogue=9) == fa.FA_ERR_INVALID
+    assert params(rows=0, o_acc=None, lse_acc=None) == fa.FA_OK
+
+
+def test_fwd_acc_rejects_bad_arguments(fa):
+    import torch
+    acc, lse = 0x60000, 0x70000
+    call = lambda p, a=acc, l=lse, f=0: fa.lib.fa_attention_fwd_acc(ctypes.byref(p) if p is not None else None,
+                                                                    a, l, f, None)
+    assert call(None) == fa.FA_ERR_INVALID
+    p = fwd(fa)
+    assert call(p, f=4) == fa.FA_ERR_INVALID                  # unknown flag
+    assert call(p, a=None) == fa.FA_ERR_INVALID               # no accumulator
+    assert call(p, l=0x70008) == fa.FA_ERR_INVALID            # misaligned lse_acc
+    p.out = None
+    assert call(p, f=fa.FA_ACC_LAST) == fa.FA_ERR_INVALID     # the last step writes out
+    p = fwd(fa, q=FakeTensor(0x10000, (4, 64, 128), torch.float32), k=FakeTensor(0x20000, (2, 64, 128), torch.float32),
+            v=FakeTensor(0x30000, (2, 64, 128), torch.float32), out=FakeTensor(0x40000, (4, 64, 128), torch.float32))
+    assert call(p) == fa.FA_ERR_UNSUPPORTED                   # fp32 path
+    p = fwd(fa)
+    p.head_dim = 96
+    assert call(p) == fa.FA_ERR_UNSUPPORTED
+    p = fwd(fa)
+    p.seqlen_q = 0
+    p.q = p.k = p.v = p.out = None
+    assert call(p, a=None, l=None, f=3) == fa.FA_OK           # empty problem

@@ -1,7 +1,7 @@
 """GPU parity of fa_attention_decode over a bf16 KV cache against the fp64
 oracle on the same bf16 values (the decode step of fkl_python PR #6,
 Verification, "FA decode step s_q=1 vs s_k=256", with an uncompressed cache;
-spec gate for bf16 outputs: max abs <= 2e-2 and relative L2 <= 5e-3).
+bf16 output gate: max abs <= 2e-2 and relative L2 <= 5e-3).
 Cache rows outside the attended band may hold any bytes, NaN and Inf
 included; they must not reach the result."""
 import numpy as np

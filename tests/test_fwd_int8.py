@@ -1,7 +1,7 @@
 """GPU parity of the tensor-core prefill over an int8 KV cache (codes +
 per-token fp32 scales made by fa_compress_kv) against the fp64 oracle on the
 dequantised cache (fkl_python PR #6, Verification: "FA int8-KV exact vs
-dequantized oracle"; spec gate: max abs <= 2e-2, relative L2 <= 5e-3;
+dequantized oracle"; bf16 output gate: max abs <= 2e-2, relative L2 <= 5e-3;
 codes and scales bit-exact)."""
 import numpy as np
 import pytest

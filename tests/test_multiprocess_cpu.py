@@ -66,3 +66,91 @@ def test_reference_arm_under_torchrun_world2():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def _ring_main(rank, world, port, out_dir, causal):
+    import datetime
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from flashattention_attention_b200 import ring
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        B, hq, hkv, S, d = 2, 4, 2, 24 * world, 16
+        rng = np.random.default_rng(7)
+        q = torch.from_numpy(rng.standard_normal((B * hq, S, d)))
+        k = torch.from_numpy(rng.standard_normal((B * hkv, S, d)))
+        v = torch.from_numpy(rng.standard_normal((B * hkv, S, d)))
+        blk = S // world
+        sl = slice(rank * blk, (rank + 1) * blk)
+
+        calls = []
+
+        def step(q, k, v, acc, *, hq, hkv, causal, scale, first, last, epilogue):
+            calls.append((first, last, acc is None))
+            o, lse = oracle.attention_lse(q.numpy(), k.numpy(), v.numpy(), hq=hq, hkv=hkv, causal=causal, scale=scale)
+            if acc is not None:
+                o, lse = oracle.merge(acc[0], acc[1], o, lse)
+            out = None
+            if last:
+                out = o.copy()
+                for op, val in epilogue:
+                    out = out * val if op == "mul" else out + val
+                out = torch.from_numpy(out)
+            return (o, lse), out
+
+        out = ring.ring_attention_fwd(q[:, sl].contiguous(), k[:, sl].contiguous(), v[:, sl].contiguous(), hq=hq,
+                                      hkv=hkv, causal=causal, epilogue=[("mul", 2.0), ("add", 0.5)],
+                                      group=dist.group.WORLD, step=step)
+        n = rank + 1 if causal else world
+        assert calls == [(c == 0, c == n - 1, c == 0) for c in range(n)], calls
+        ref = oracle.attention(q.numpy(), k.numpy(), v.numpy(), hq=hq, hkv=hkv, causal=causal,
+                               epilogue=[("mul", 2.0), ("add", 0.5)])[:, sl]
+        err = float(np.abs(out.numpy() - ref).max())
+        with open(os.path.join(out_dir, f"ring{rank}.txt"), "w") as f:
+            f.write(repr(err))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ring_schedule_pairs_every_send_with_a_receive():
+    """Every transfer of ring_schedule has its receive on the next rank, and
+    rank r attends to exactly blocks 0..r (causal) or all blocks, each once."""
+    sys.path.insert(0, ROOT)
+    from flashattention_attention_b200.ring import ring_schedule
+    for world in range(1, 9):
+        for causal in (False, True):
+            held = list(range(world))  # block held by each rank
+            seen = [[] for _ in range(world)]
+            for s in range(world):
+                for r in range(world):
+                    seen[r].append(held[r])
+                sched = [ring_schedule(r, world, causal, s) for r in range(world)]
+                for r in range(world):
+                    assert sched[r][0] == sched[(r + 1) % world][1], (world, causal, s, r)
+                held = [held[(r - 1) % world] if sched[r][1] else held[r] for r in range(world)]
+            for r in range(world):
+                want = list(range(r + 1)) if causal else list(range(world))
+                got = [b for b in seen[r][:len(want)]]
+                assert sorted(got) == want, (world, causal, r, seen[r])
+            if causal and world > 1:
+                n_sends = sum(ring_schedule(r, world, True, s)[0] for r in range(world) for s in range(world))
+                assert n_sends == world * (world - 1) // 2
+
+
+@pytest.mark.parametrize("world,causal", [(2, True), (2, False), (3, True), (4, True)])
+def test_ring_schedule_gloo(tmp_path, world, causal):
+    """The ring schedule of ring_attention_fwd (blocks passed to the next
+    rank while each step computes, future blocks skipped under causal
+    masking, the diagonal block causal, partial results merged) over gloo
+    ranks with the oracle's per-step computations: every rank's block equals
+    the oracle's attention over the whole sequence."""
+    port = _free_port()
+    mp.start_processes(_ring_main, args=(world, port, str(tmp_path), causal), nprocs=world, join=True,
+                       start_method="spawn")
+    errs = [float(open(tmp_path / f"ring{r}.txt").read()) for r in range(world)]
+    assert max(errs) < 1e-12, errs

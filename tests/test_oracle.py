@@ -418,3 +418,58 @@ def test_kv_append_float_cache_stores_the_row():
     c2, s2, l2 = oracle.kv_append(cache, None, new, np.array([2]), 2)
     assert s2 is None and l2 is None
     assert np.array_equal(c2[:, 2], new) and not c2[:, [0, 1, 3]].any()
+
+
+# ---------------------------------------------------------------- partial results and merge
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+def test_attention_lse_matches_attention_and_logsumexp():
+    """The numpy partial-result oracle against the C oracle (outputs of rows
+    with keys) and torch.logsumexp of the masked fp64 scores (lse)."""
+    import torch
+    rng = np.random.default_rng(70)
+    hq, hkv, s_q, s_k, d = 4, 2, 37, 53, 32
+    q, k, v = _rand(rng, hq, s_q, d), _rand(rng, hkv, s_k, d), _rand(rng, hkv, s_k, d)
+    for causal, window in ((False, 0), (True, 0), (True, 9), (False, 7)):
+        o, lse = oracle.attention_lse(q, k, v, hq=hq, hkv=hkv, causal=causal, window=window)
+        ref = oracle.attention(q, k, v, hq=hq, hkv=hkv, causal=causal, window=window)
+        fin = np.isfinite(lse)
+        assert np.allclose(o[fin], ref[fin], rtol=1e-12, atol=1e-12)
+        for h in range(hq):
+            x = torch.tensor(q[h] @ k[h // 2].T / np.sqrt(d))
+            i = torch.arange(s_q)[:, None] + s_k - s_q
+            j = torch.arange(s_k)[None, :]
+            vis = torch.ones(s_q, s_k, dtype=torch.bool)
+            if causal:
+                vis &= j <= i
+            if window > 0:
+                vis &= j > i - window
+            want = torch.logsumexp(x.masked_fill(~vis, float("-inf")), dim=1).numpy()
+            assert np.allclose(lse[h], want, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_lse_empty_rows():
+    rng = np.random.default_rng(71)
+    q, k, v = _rand(rng, 2, 10, 16), _rand(rng, 2, 4, 16), _rand(rng, 2, 4, 16)
+    o, lse = oracle.attention_lse(q, k, v, hq=2, hkv=2, causal=True)
+    assert np.all(np.isneginf(lse[:, :6])) and not o[:, :6].any()  # rows i < s_q - s_k see no key
+    assert np.all(np.isfinite(lse[:, 6:]))
+
+
+def test_merge_of_disjoint_key_sets_is_attention_over_their_union():
+    """Splitting the keys into blocks, attending to each and merging gives
+    attention over all keys (the identity the ring and split schedules rely
+    on), for any split and order, with empty blocks weighing nothing."""
+    rng = np.random.default_rng(72)
+    hq, hkv, s, d = 4, 2, 48, 16
+    q, k, v = _rand(rng, hq, s, d), _rand(rng, hkv, s, d), _rand(rng, hkv, s, d)
+    full_o, full_lse = oracle.attention_lse(q, k, v, hq=hq, hkv=hkv)
+    cuts = [0, 5, 20, 20, 48]  # includes an empty block
+    acc_o, acc_lse = np.zeros_like(full_o), np.full(full_lse.shape, -np.inf)
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        po, pl = oracle.attention_lse(q, k[:, a:b], v[:, a:b], hq=hq, hkv=hkv)
+        acc_o, acc_lse = oracle.merge(acc_o, acc_lse, po, pl)
+    assert np.allclose(acc_o, full_o, rtol=1e-12, atol=1e-12)
+    assert np.allclose(acc_lse, full_lse, rtol=1e-12, atol=1e-12)
