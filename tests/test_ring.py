@@ -41,19 +41,21 @@ def test_fwd_lse_matches_oracle(d, causal, s_q, s_k):
     assert not out.float()[torch.from_numpy(~fin)].any()
 
 
-def test_merge_matches_oracle_and_writes_the_final_output():
+@pytest.mark.parametrize("d,part_dtype", [(128, torch.bfloat16), (96, torch.float32), (256, torch.bfloat16),
+                                          (32, torch.float32)])
+def test_merge_matches_oracle_and_writes_the_final_output(d, part_dtype):
     fa = _fa()
-    rng = np.random.default_rng(80)
-    rows, d = 1000, 128
+    rng = np.random.default_rng(80 + d)
+    rows = 1001
     acc = torch.from_numpy(rng.standard_normal((rows, d)).astype(np.float32))
     lacc = torch.from_numpy(rng.standard_normal(rows).astype(np.float32))
-    part = _bf(rng, rows, d)
+    part = torch.from_numpy(rng.standard_normal((rows, d)).astype(np.float32)).to(part_dtype)
     lpart = torch.from_numpy(rng.standard_normal(rows).astype(np.float32))
     lacc[:10] = float("-inf")   # empty accumulator rows take the partial
     lpart[5:15] = float("-inf")  # empty partial rows leave the accumulator (rows 5-9: both empty)
     acc[:10] = 0
     g_acc, g_lacc = acc.cuda(), lacc.cuda()
-    out = torch.empty((rows, d), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((rows, d), dtype=part_dtype, device="cuda")
     fa.attention_merge(g_acc, g_lacc, part.cuda(), lpart.cuda(), out=out, epilogue=[("mul", 2.0)])
     assert fa.check_device_error() == fa.FA_OK
     ro, rl = oracle.merge(acc.double().numpy(), lacc.double().numpy(), part.double().numpy(), lpart.double().numpy())
@@ -61,7 +63,14 @@ def test_merge_matches_oracle_and_writes_the_final_output():
     gl = g_lacc.cpu().numpy()
     assert np.array_equal(np.isneginf(gl), np.isneginf(rl)) and np.allclose(gl[np.isfinite(rl)], rl[np.isfinite(rl)],
                                                                             rtol=1e-5, atol=1e-5)
-    assert_close_bf16(out.float().cpu().numpy(), 2.0 * ro)
+    # out is the merged fp32 row (the one stored in the accumulator) after the
+    # epilogue, rounded once to the output type
+    assert torch.equal(out, (2.0 * g_acc).to(part_dtype))
+    # finalise only (no partial): out = epilogue(accumulator), accumulator untouched
+    before = g_acc.clone()
+    fa.attention_merge(g_acc, g_lacc, out=out, epilogue=[("add", 1.0)])
+    assert torch.equal(g_acc, before)
+    assert torch.equal(out, (before + 1.0).to(part_dtype))
 
 
 def _epi(y, epilogue):
