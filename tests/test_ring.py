@@ -221,3 +221,30 @@ def test_ring_steps_on_one_gpu_equal_full_attention(n_blocks):
     # the driver itself with a one-process ring
     one = ring.ring_attention_fwd(q, k, v, hq=hq, hkv=hkv, causal=True, epilogue=epi)
     assert torch.equal(one, full)  # one block, first and last: the plain kernel's arithmetic
+
+
+def test_full_size_ring_last_rank_sampled():
+    """The bench's ring line at full size: the last rank of a 4-way causal
+    ring (B=4, Hq=32, Hkv=8, block 4096, d=128: queries at positions
+    12288..16383 over 16384 keys), run through ring.attend_blocks exactly as
+    timed, checked on sampled rows the oracle computes one by one."""
+    from flashattention_attention_b200 import inputs, ring
+    fa = _fa()
+    w = inputs.ring_cp_last_rank()
+    R, blk = w.seqlen_k // w.seqlen_q, w.seqlen_q
+    q = w.q.cuda()
+    kb = [w.k[:, b * blk:(b + 1) * blk].contiguous().cuda() for b in range(R)]
+    vb = [w.v[:, b * blk:(b + 1) * blk].contiguous().cuda() for b in range(R)]
+    blocks = [((R - 1 - s) % R, kb[(R - 1 - s) % R], vb[(R - 1 - s) % R]) for s in range(R)]
+    got = ring.attend_blocks(q, blocks, rank=R - 1, n_blocks=R, hq=w.hq, hkv=w.hkv, causal=True)
+    assert fa.check_device_error() == fa.FA_OK
+    rng = np.random.default_rng(5)
+    rows = {(int(b), int(h), int(i)) for b, h, i in zip(rng.integers(0, w.batch, 120), rng.integers(0, w.hq, 120),
+                                                          rng.integers(0, blk, 120))}
+    rows |= {(0, 0, 0), (0, 0, blk - 1), (w.batch - 1, w.hq - 1, 0), (w.batch - 1, w.hq - 1, blk - 1)}
+    rows = sorted(rows)
+    ref = oracle.attention(w.q, w.k, w.v, hq=w.hq, hkv=w.hkv, causal=True, rows=rows)
+    idx = np.array([(b * w.hq + h, i) for b, h, i in rows])
+    g = got.float().cpu().numpy()[idx[:, 0], idx[:, 1]]
+    assert_close_bf16(g, ref[idx[:, 0], idx[:, 1]], what="full-size ring sample")
+    assert torch.isfinite(got.float()).all()
