@@ -27,7 +27,11 @@ Definitions followed:
   * partial results over disjoint key sets and their merge: kernbench2
     commit message, ADR-0060 (long context: an online-softmax merge of the
     per-step (m, l, O) state at every ring step), written with the
-    log-sum-exp lse = m + log l.
+    log-sum-exp lse = m + log l;
+  * TurboQuant KV compression (rotation, Beta(d/2, d/2) Lloyd-Max codebook,
+    bit-packing): the C attention library's README, "TurboQuant KV Cache
+    Compression" -- in ``oracle/turboquant.py`` (numpy, fp64), pinned by
+    ``tests/test_turboquant_oracle.py``.
 
 Every function is pinned by ``tests/test_oracle.py`` against closed forms,
 invariants, torch's fp64 scaled_dot_product_attention, pure-Python brute force
