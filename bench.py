@@ -257,6 +257,10 @@ def gpu_arm(args, rank, world, dist):
         res = {}
         ring_rank_steps(args, dev, peaks, world, dist, res)
         return res
+    if args.only == "tq":
+        res = {}
+        turboquant_decode(args, dev, peaks, world, dist, res)
+        return res
     l0 = fa.kernel_launches()
     with ClockSampler(dev.index or 0) as clocks:
         ms = time_launches(prefill, args.steps, args.warmup, torch, dist, clocks)
@@ -310,6 +314,7 @@ def gpu_arm(args, rank, world, dist):
         other_prefills(args, dev, peaks, world, dist, result)
         ring_rank_steps(args, dev, peaks, world, dist, result)
         decode_and_quant(args, dev, peaks, world, dist, result)
+        turboquant_decode(args, dev, peaks, world, dist, result)
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, flops_tiles, flops_exact, args.cpu_seconds)
     return result
@@ -479,6 +484,55 @@ def ring_rank_steps(args, dev, peaks, world, dist, result):
                          "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                                       "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4)}}}
     del q, kb, vb, blocks, o, lse, acc_o, acc_l, out
+    torch.cuda.empty_cache()
+
+
+def turboquant_decode(args, dev, peaks, world, dist, result):
+    """The decode workload's cache (B=16, Hq=32, Hkv=8, d=128, lengths
+    U[1024, 32768]) compressed TurboQuant K4/V2; one decode step timed (the
+    split kernel and the merge + inverse rotation), and the compression of
+    the whole cache."""
+    import torch
+    from flashattention_attention_b200 import fa, inputs
+    w = inputs.int8kv_decode()
+    s = inputs.rotation_signs(w.d, 0).to(dev)
+    lk, lv = fa.tq_codebook(w.d, 4).to(dev), fa.tq_codebook(w.d, 2).to(dev)
+    k, v = w.k.to(dev), w.v.to(dev)
+    kc, kn = fa.tq_compress(k, s, lk, 4)
+    vc, vn = fa.tq_compress(v, s, lv, 2)
+    steps = max(20, args.steps // 2)
+    rows = k.shape[0] * k.shape[1]
+    ms_c = time_launches(lambda: fa.tq_compress(k, s, lk, 4, codes=kc, norms=kn), max(10, steps // 4), args.warmup,
+                         torch, dist)
+    c_bytes = rows * (w.d * 2 + w.d * 4 // 8 + 4)
+    del k, v
+    torch.cuda.empty_cache()
+    q = w.q.reshape(-1, w.d).to(dev)
+    lens = torch.tensor(w.lengths, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    ws = torch.empty(fa.tq_decode_workspace_size(w.batch, w.hq, w.d, kc.shape[1]), dtype=torch.uint8, device=dev)
+
+    def step():
+        fa.tq_attention_decode(q, kc, kn, vc, vn, lens, hq=w.hq, hkv=w.hkv, k_bits=4, v_bits=2, k_levels=lk,
+                               v_levels=lv, signs=s, out=out, workspace=ws)
+
+    ms = time_launches(step, steps, args.warmup, torch, dist)
+    assert fa.check_device_error() == fa.FA_OK
+    keys = int(sum(w.lengths))
+    per_key = (w.d * 4 // 8 + 4) + (w.d * 2 // 8 + 4)
+    dec_bytes = keys * w.hkv * per_key + 2 * q.numel() * 2
+    gbs = dec_bytes / (ms * 1e-3) / 1e9
+    cgbs = c_bytes / (ms_c * 1e-3) / 1e9
+    result["turboquant_k4v2_decode"] = {
+        "workload": w.name + "_tq_k4v2", "value": round(gbs * world, 1), "unit": "GB/s",
+        "us_per_step": round(ms * 1e3, 2), "bytes_per_step": dec_bytes,
+        "bytes_counting": "K (d/2 + 4) and V (d/4 + 4) bytes per (key, KV head), q and out",
+        "roofline": {"bound": "hbm", "kernel": "tq_decode_kernel<128,4,2,4> + tq_merge_kernel<128>",
+                     "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs / peaks["hbm_gbs"], 4)},
+        "compress_k4": {"us": round(ms_c * 1e3, 2), "rows": rows, "bytes": c_bytes, "achieved": round(cgbs, 1),
+                        "unit": "GB/s", "frac": round(cgbs / peaks["hbm_gbs"], 4)}}
+    del kc, kn, vc, vn, q, out, ws
     torch.cuda.empty_cache()
 
 
@@ -711,7 +765,7 @@ def main():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "quant", "prefill_int8", "varlen", "ring"],
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "quant", "prefill_int8", "varlen", "ring", "tq"],
                     help="time one part only (used for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:

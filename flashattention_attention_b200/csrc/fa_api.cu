@@ -465,6 +465,55 @@ fa_status fa_kv_append_paged(const fa_kv_append_params* p, const fa_kv_pages* pa
   return launch_kv_append(*p, pages, ctx);
 }
 
+fa_status fa_tq_codebook(int32_t head_dim, int32_t bits, float* levels) {
+  if (levels == nullptr || head_dim < 4 || head_dim > (1 << 20) || head_dim % 2 != 0) return FA_ERR_INVALID;
+  if (bits < 1 || bits > 8) return FA_ERR_INVALID;
+  return tq_codebook_host(head_dim, bits, levels);
+}
+
+fa_status fa_tq_compress(const fa_tq_compress_params* p, fa_stream_t stream) {
+  if (p == nullptr || p->rows < 0) return FA_ERR_INVALID;
+  if (p->x_dtype != FA_BF16 && p->x_dtype != FA_F32) return FA_ERR_INVALID;
+  if (p->head_dim != 64 && p->head_dim != 128) return FA_ERR_UNSUPPORTED;
+  if (p->bits < 2 || p->bits > 4) return FA_ERR_UNSUPPORTED;
+  if (p->rows == 0) return FA_OK;
+  if (p->x == nullptr || p->signs == nullptr || p->levels == nullptr || p->codes == nullptr || p->norms == nullptr)
+    return FA_ERR_INVALID;
+  if (!aligned16(p->x) || !aligned16(p->signs) || !aligned16(p->levels) || !aligned16(p->codes) ||
+      !aligned16(p->norms))
+    return FA_ERR_INVALID;
+  LaunchCtx ctx;
+  fa_status st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  return launch_tq_compress(*p, ctx);
+}
+
+size_t fa_tq_decode_workspace_size(int32_t batch, int32_t hq, int32_t head_dim, int32_t capacity) {
+  if (batch <= 0 || hq <= 0 || head_dim <= 0 || capacity <= 0) return 0;
+  return static_cast<size_t>(batch) * hq * tq_decode_splits(capacity) * (head_dim + 2) * sizeof(float);
+}
+
+fa_status fa_tq_attention_decode(const fa_tq_decode_params* p, fa_stream_t stream) {
+  if (p == nullptr || p->batch < 0 || p->hq <= 0 || p->hkv <= 0 || p->hq % p->hkv != 0) return FA_ERR_INVALID;
+  if (p->head_dim != 64 && p->head_dim != 128) return FA_ERR_UNSUPPORTED;
+  if (p->k_bits < 2 || p->k_bits > 4 || p->v_bits < 2 || p->v_bits > 4) return FA_ERR_UNSUPPORTED;
+  const int group = p->hq / p->hkv;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return FA_ERR_UNSUPPORTED;
+  if (p->capacity < 1 || !std::isfinite(p->softmax_scale)) return FA_ERR_INVALID;
+  if (!epilogue_ok(p->epilogue, p->n_epilogue)) return FA_ERR_INVALID;
+  if (p->batch == 0) return FA_OK;
+  const void* ptrs[] = {p->q, p->k_codes, p->k_norms, p->v_codes, p->v_norms, p->k_levels,
+                        p->v_levels, p->signs, p->cache_seqlens, p->out};
+  for (const void* q : ptrs)
+    if (q == nullptr || !aligned16(q)) return FA_ERR_INVALID;
+  const size_t need = fa_tq_decode_workspace_size(p->batch, p->hq, p->head_dim, p->capacity);
+  if (p->workspace == nullptr || !aligned16(p->workspace) || p->workspace_bytes < need) return FA_ERR_WORKSPACE;
+  LaunchCtx ctx;
+  fa_status st = make_ctx(stream, &ctx);
+  if (st != FA_OK) return st;
+  return launch_tq_decode(*p, static_cast<float*>(p->workspace), ctx);
+}
+
 fa_status fa_check_device_error(fa_stream_t stream) {
   unsigned int* word = nullptr;
   fa_status st = status_word(&word);

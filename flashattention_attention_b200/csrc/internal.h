@@ -43,6 +43,12 @@ fa_status launch_merge(float* o_acc, float* lse_acc, const void* o_part, int par
                        int64_t rows, int d, void* out, int out_dtype, const fa_epi_op* epi, int n_epi,
                        const LaunchCtx& ctx);
 fa_status launch_decode(const fa_decode_params& p, const fa_kv_pages* pages, int split_keys, const LaunchCtx& ctx);
+// TurboQuant: keys per split of the decode, its split count, launchers and the host codebook
+constexpr int kTqSplitKeys = 2048;
+int tq_decode_splits(int capacity);
+fa_status launch_tq_compress(const fa_tq_compress_params& p, const LaunchCtx& ctx);
+fa_status launch_tq_decode(const fa_tq_decode_params& p, float* part, const LaunchCtx& ctx);
+fa_status tq_codebook_host(int d, int bits, float* levels);
 size_t decode_workspace_bytes(int batch, int hq, int head_dim);
 int decode_noalloc_workers(int batch, int hq, int hkv, int head_dim);
 fa_status launch_decode_noalloc(const fa_decode_params& p, int split_keys, long long budget, cudaStream_t stream);

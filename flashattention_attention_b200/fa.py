@@ -68,6 +68,23 @@ class MergeParams(ctypes.Structure):
                 ("n_epilogue", ctypes.c_int32), ("epilogue", EpiOp * FA_MAX_EPILOGUE)]
 
 
+class TqCompressParams(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("x_dtype", ctypes.c_int32), ("rows", ctypes.c_int64),
+                ("head_dim", ctypes.c_int32), ("bits", ctypes.c_int32), ("signs", ctypes.c_void_p),
+                ("levels", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("norms", ctypes.c_void_p)]
+
+
+class TqDecodeParams(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k_codes", ctypes.c_void_p), ("k_norms", ctypes.c_void_p),
+                ("v_codes", ctypes.c_void_p), ("v_norms", ctypes.c_void_p), ("k_levels", ctypes.c_void_p),
+                ("v_levels", ctypes.c_void_p), ("signs", ctypes.c_void_p), ("cache_seqlens", ctypes.c_void_p),
+                ("batch", ctypes.c_int32), ("hq", ctypes.c_int32), ("hkv", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("capacity", ctypes.c_int32), ("k_bits", ctypes.c_int32),
+                ("v_bits", ctypes.c_int32), ("softmax_scale", ctypes.c_float), ("out", ctypes.c_void_p),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("n_epilogue", ctypes.c_int32), ("epilogue", EpiOp * FA_MAX_EPILOGUE)]
+
+
 class KvPages(ctypes.Structure):
     _fields_ = [("block_table", ctypes.c_void_p), ("max_pages", ctypes.c_int32),
                 ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
@@ -106,6 +123,14 @@ lib.fa_kv_append.restype = ctypes.c_int
 lib.fa_kv_append.argtypes = [ctypes.POINTER(KvAppendParams), ctypes.c_void_p]
 lib.fa_kv_append_paged.restype = ctypes.c_int
 lib.fa_kv_append_paged.argtypes = [ctypes.POINTER(KvAppendParams), ctypes.POINTER(KvPages), ctypes.c_void_p]
+lib.fa_tq_codebook.restype = ctypes.c_int
+lib.fa_tq_codebook.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]
+lib.fa_tq_compress.restype = ctypes.c_int
+lib.fa_tq_compress.argtypes = [ctypes.POINTER(TqCompressParams), ctypes.c_void_p]
+lib.fa_tq_decode_workspace_size.restype = ctypes.c_size_t
+lib.fa_tq_decode_workspace_size.argtypes = [ctypes.c_int32] * 4
+lib.fa_tq_attention_decode.restype = ctypes.c_int
+lib.fa_tq_attention_decode.argtypes = [ctypes.POINTER(TqDecodeParams), ctypes.c_void_p]
 lib.fa_status_string.restype = ctypes.c_char_p
 lib.fa_status_string.argtypes = [ctypes.c_int]
 lib.fa_check_device_error.restype = ctypes.c_int
@@ -461,3 +486,70 @@ def kernel_variants_used() -> int:
 
 def kernel_launches() -> int:
     return int(lib.fa_kernel_launches())
+
+
+# --- TurboQuant KV cache -------------------------------------------------------
+
+def tq_codebook(head_dim: int, bits: int) -> torch.Tensor:
+    """The 2^bits Lloyd-Max levels (fp32, CPU) of the Beta(head_dim/2,
+    head_dim/2) law in u-space.  As fa_tq_codebook in fa.h."""
+    out = (ctypes.c_float * (1 << bits))()
+    _check(lib.fa_tq_codebook(head_dim, bits, ctypes.cast(out, ctypes.c_void_p)), "fa_tq_codebook")
+    return torch.tensor(list(out), dtype=torch.float32)
+
+
+def tq_compress(x: torch.Tensor, signs: torch.Tensor, levels: torch.Tensor, bits: int,
+                codes: Optional[torch.Tensor] = None, norms: Optional[torch.Tensor] = None, stream=None):
+    """(codes uint8 [..., d*bits/8], norms fp32 [...]) of rows x [..., d]
+    (bf16 or fp32).  signs / levels: fp32 CUDA tensors.  As fa_tq_compress."""
+    for name, t in (("x", x), ("signs", signs), ("levels", levels)):
+        _contig_cuda(t, name)
+    d = x.shape[-1]
+    if codes is None:
+        codes = torch.empty(x.shape[:-1] + (d * bits // 8,), dtype=torch.uint8, device=x.device)
+    if norms is None:
+        norms = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    p = TqCompressParams()
+    p.x, p.x_dtype, p.rows, p.head_dim, p.bits = x.data_ptr(), _DT[x.dtype], x.numel() // d if d else 0, d, bits
+    p.signs, p.levels, p.codes, p.norms = signs.data_ptr(), levels.data_ptr(), codes.data_ptr(), norms.data_ptr()
+    _check(lib.fa_tq_compress(ctypes.byref(p), _stream(stream)), "fa_tq_compress")
+    return codes, norms
+
+
+def tq_decode_workspace_size(batch: int, hq: int, head_dim: int, capacity: int) -> int:
+    return int(lib.fa_tq_decode_workspace_size(batch, hq, head_dim, capacity))
+
+
+def tq_attention_decode(q: torch.Tensor, k_codes: torch.Tensor, k_norms: torch.Tensor, v_codes: torch.Tensor,
+                        v_norms: torch.Tensor, cache_seqlens: torch.Tensor, *, hq: int, hkv: int, k_bits: int,
+                        v_bits: int, k_levels: torch.Tensor, v_levels: torch.Tensor, signs: torch.Tensor,
+                        scale: Optional[float] = None, epilogue: Sequence[Tuple[str, float]] = (),
+                        out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """One decode step over a TurboQuant cache: q [B*hq, d] (or [B*hq, 1, d])
+    bf16, codes [B*hkv, capacity, d*bits/8], norms [B*hkv, capacity].  As
+    fa_tq_attention_decode in fa.h."""
+    for name, t in (("q", q), ("k_codes", k_codes), ("k_norms", k_norms), ("v_codes", v_codes),
+                    ("v_norms", v_norms), ("cache_seqlens", cache_seqlens), ("k_levels", k_levels),
+                    ("v_levels", v_levels), ("signs", signs)):
+        _contig_cuda(t, name)
+    d = q.shape[-1]
+    batch = cache_seqlens.numel()
+    cap = k_codes.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    need = tq_decode_workspace_size(batch, hq, d, cap)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    p = TqDecodeParams()
+    p.q, p.k_codes, p.k_norms, p.v_codes, p.v_norms = (q.data_ptr(), k_codes.data_ptr(), k_norms.data_ptr(),
+                                                       v_codes.data_ptr(), v_norms.data_ptr())
+    p.k_levels, p.v_levels, p.signs, p.cache_seqlens = (k_levels.data_ptr(), v_levels.data_ptr(), signs.data_ptr(),
+                                                        cache_seqlens.data_ptr())
+    p.batch, p.hq, p.hkv, p.head_dim, p.capacity, p.k_bits, p.v_bits = batch, hq, hkv, d, cap, k_bits, v_bits
+    p.softmax_scale = float(scale if scale is not None else 1.0 / math.sqrt(d))
+    p.out, p.workspace, p.workspace_bytes = out.data_ptr(), workspace.data_ptr(), workspace.numel()
+    p.n_epilogue = _fill_epilogue(p.epilogue, epilogue)
+    _check(lib.fa_tq_attention_decode(ctypes.byref(p), _stream(stream)), "fa_tq_attention_decode")
+    return out
+

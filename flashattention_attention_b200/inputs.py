@@ -160,3 +160,10 @@ def int8kv_long_prefill(seed=0, s=16384) -> Workload:
     return dense_prefill(f"int8kv_causal_prefill_b1_hq64_hkv8_s{s}_d128", batch=1, hq=64,
                          hkv=8, s_q=s, s_k=s, d=128, dtype=torch.bfloat16, causal=True,
                          epilogue=[("mul", 0.5)], seed=seed, kv_int8=True)
+
+
+def rotation_signs(d: int, seed: int = 0) -> torch.Tensor:
+    """The random +-1 signs of a TurboQuant rotation (fp32 [d]), drawn from
+    numpy's PCG64 with the given seed (the method's random draw, passed in)."""
+    return torch.from_numpy(np.random.default_rng(seed).choice(np.array([-1.0, 1.0], np.float32), d))
+

@@ -407,6 +407,97 @@ FA_API fa_status fa_attention_decode_noalloc(const fa_decode_params *p, fa_strea
 FA_API const char *fa_status_string(fa_status s);
 
 /*
+ * TurboQuant KV cache compression (the C attention library's README,
+ * "TurboQuant KV Cache Compression"): a K or V row x of head size d is
+ * rotated, y = H (s * x) / sqrt(d) with H the Sylvester-ordered Hadamard
+ * matrix and s random +-1 signs applied before it, normalised by its L2
+ * norm, u = y / ||x||, and each u_i replaced by the b-bit index of the
+ * nearest level of the Lloyd-Max quantiser of the Beta(d/2, d/2) law of
+ * (u + 1) / 2 (a tie goes to the lower level); the codes are bit-packed,
+ * channel i at bits [i b, i b + b) of the row's little-endian bit stream,
+ * beside one fp32 norm per row.  A row reads back as
+ * x_hat = s * (H (||x|| level[code])) / sqrt(d).  K4/V2 at d = 64 is 56
+ * bytes per token and KV head against 512 in fp32 (the page's 9.14x).
+ *
+ * fa_tq_codebook -- host function: the 2^bits levels in u-space, ascending
+ * and antisymmetric, into levels[] (host memory).  4 <= head_dim <= 2^20,
+ * head_dim even; 1 <= bits <= 8.  Computed in double by Lloyd's iteration
+ * on a 2^20-interval quadrature of the density (1 - u^2)^(d/2 - 1).
+ */
+FA_API fa_status fa_tq_codebook(int32_t head_dim, int32_t bits, float *levels);
+
+/*
+ * fa_tq_compress -- rows of K or V into packed codes and norms.
+ *   x       [rows, head_dim] x_dtype (FA_BF16 or FA_F32)
+ *   signs   device [head_dim] fp32, each +1 or -1 (the rotation)
+ *   levels  device [2^bits] fp32 (fa_tq_codebook(head_dim, bits))
+ *   codes   [rows, head_dim * bits / 8] uint8;  norms [rows] fp32
+ * head_dim 64 or 128; bits 2, 3 or 4; every pointer 16-byte aligned; the
+ * decisions are taken in fp32 (a value within rounding of a cell edge may
+ * land on either side).  rows = 0 enqueues nothing.
+ */
+typedef struct {
+    const void *x;
+    int32_t x_dtype;
+    int64_t rows;
+    int32_t head_dim;
+    int32_t bits;
+    const float *signs;
+    const float *levels;
+    uint8_t *codes;
+    float *norms;
+} fa_tq_compress_params;
+
+FA_API fa_status fa_tq_compress(const fa_tq_compress_params *p, fa_stream_t stream);
+
+/*
+ * fa_tq_attention_decode -- s_q = 1 attention of every query head over a
+ * TurboQuant cache, without rebuilding K or V: scores are
+ * ||k|| (R q) . level[code] with R the rotation, the V side is accumulated
+ * in the rotated basis and rotated back once per output row.
+ *   q          [batch*hq, head_dim] bf16;  out [batch*hq, head_dim] bf16
+ *   k_codes    [batch*hkv, capacity, head_dim*k_bits/8] uint8, k_norms
+ *              [batch*hkv, capacity] fp32 (fa_tq_compress of the K rows);
+ *              v_codes / v_norms likewise with v_bits
+ *   k_levels, v_levels  device [2^bits] fp32;  signs device [head_dim] fp32
+ *              (one rotation for K and V)
+ *   cache_seqlens device int32 [batch]: keys 0 .. L_b - 1 are attended; a
+ *              value outside [0, capacity] is clamped and reported by
+ *              fa_check_device_error as FA_ERR_INVALID; L_b = 0 gives the
+ *              epilogue of 0
+ *   workspace  device, >= fa_tq_decode_workspace_size() bytes (partials of
+ *              the key splits), 16-byte aligned
+ * head_dim 64 or 128; k_bits, v_bits 2..4; hq / hkv in {1, 2, 4, 8}.
+ */
+typedef struct {
+    const void *q;
+    const uint8_t *k_codes;
+    const float *k_norms;
+    const uint8_t *v_codes;
+    const float *v_norms;
+    const float *k_levels;
+    const float *v_levels;
+    const float *signs;
+    const int32_t *cache_seqlens;
+    int32_t batch;
+    int32_t hq;
+    int32_t hkv;
+    int32_t head_dim;
+    int32_t capacity;
+    int32_t k_bits;
+    int32_t v_bits;
+    float softmax_scale;
+    void *out;
+    void *workspace;
+    size_t workspace_bytes;
+    int32_t n_epilogue;
+    fa_epi_op epilogue[FA_MAX_EPILOGUE];
+} fa_tq_decode_params;
+
+FA_API size_t fa_tq_decode_workspace_size(int32_t batch, int32_t hq, int32_t head_dim, int32_t capacity);
+FA_API fa_status fa_tq_attention_decode(const fa_tq_decode_params *p, fa_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's status
  * word: FA_ERR_TIMEOUT if a bounded wait in any kernel gave up since the last
  * check, FA_ERR_INVALID if a kernel met a device-side argument out of range

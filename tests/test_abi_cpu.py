@@ -343,3 +343,62 @@ def test_fwd_acc_rejects_bad_arguments(fa):
     p.seqlen_q = 0
     p.q = p.k = p.v = p.out = None
     assert call(p, a=None, l=None, f=3) == fa.FA_OK           # empty problem
+
+
+@pytest.mark.parametrize("d,bits", [(64, 2), (64, 4), (128, 2), (128, 3), (128, 4)])
+def test_tq_codebook_host_function_matches_the_oracle(fa, d, bits):
+    """fa_tq_codebook runs on the host: its levels (own quadrature and Lloyd
+    iteration in the library) against the oracle's (incomplete-beta path)."""
+    import numpy as np
+    from oracle import turboquant as tq
+    lv = fa.tq_codebook(d, bits).numpy()
+    assert np.array_equal(lv, -lv[::-1])  # exactly antisymmetric
+    assert np.abs(lv - tq.codebook(d, bits)).max() < 1e-7
+
+
+def test_tq_rejects_bad_arguments(fa):
+    buf = (ctypes.c_float * 16)()
+    assert fa.lib.fa_tq_codebook(128, 4, None) == fa.FA_ERR_INVALID
+    assert fa.lib.fa_tq_codebook(127, 4, ctypes.cast(buf, ctypes.c_void_p)) == fa.FA_ERR_INVALID
+    assert fa.lib.fa_tq_codebook(128, 9, ctypes.cast(buf, ctypes.c_void_p)) == fa.FA_ERR_INVALID
+    assert fa.lib.fa_tq_compress(None, None) == fa.FA_ERR_INVALID
+
+    def comp(**kw):
+        p = fa.TqCompressParams()
+        p.x, p.x_dtype, p.rows, p.head_dim, p.bits = 0x1000, fa.FA_BF16, 10, 128, 4
+        p.signs, p.levels, p.codes, p.norms = 0x2000, 0x3000, 0x4000, 0x5000
+        for k, v in kw.items():
+            setattr(p, k, v)
+        return fa.lib.fa_tq_compress(ctypes.byref(p), None)
+
+    assert comp(head_dim=96) == fa.FA_ERR_UNSUPPORTED
+    assert comp(bits=5) == fa.FA_ERR_UNSUPPORTED
+    assert comp(x_dtype=fa.FA_I8) == fa.FA_ERR_INVALID
+    assert comp(codes=None) == fa.FA_ERR_INVALID
+    assert comp(x=0x1008) == fa.FA_ERR_INVALID
+    assert comp(rows=-1) == fa.FA_ERR_INVALID
+    assert comp(rows=0, x=None) == fa.FA_OK
+
+    def dec(**kw):
+        p = fa.TqDecodeParams()
+        p.q, p.k_codes, p.k_norms, p.v_codes, p.v_norms = 0x1000, 0x2000, 0x3000, 0x4000, 0x5000
+        p.k_levels, p.v_levels, p.signs, p.cache_seqlens, p.out = 0x6000, 0x7000, 0x8000, 0x9000, 0xa000
+        p.batch, p.hq, p.hkv, p.head_dim, p.capacity, p.k_bits, p.v_bits = 2, 8, 2, 128, 4096, 4, 2
+        p.softmax_scale = 0.1
+        p.workspace = 0xb000
+        p.workspace_bytes = fa.tq_decode_workspace_size(2, 8, 128, 4096)
+        for k, v in kw.items():
+            setattr(p, k, v)
+        return fa.lib.fa_tq_attention_decode(ctypes.byref(p), None)
+
+    assert fa.tq_decode_workspace_size(2, 8, 128, 4096) == 2 * 8 * 2 * 130 * 4  # two 2048-key splits
+    assert dec(hq=6) == fa.FA_ERR_UNSUPPORTED          # group of 3
+    assert dec(hq=7) == fa.FA_ERR_INVALID              # hq % hkv != 0
+    assert dec(head_dim=96) == fa.FA_ERR_UNSUPPORTED
+    assert dec(v_bits=1) == fa.FA_ERR_UNSUPPORTED
+    assert dec(capacity=0) == fa.FA_ERR_INVALID
+    assert dec(softmax_scale=float("inf")) == fa.FA_ERR_INVALID
+    assert dec(signs=None) == fa.FA_ERR_INVALID
+    assert dec(workspace_bytes=16) == fa.FA_ERR_WORKSPACE
+    assert dec(n_epilogue=9) == fa.FA_ERR_INVALID
+    assert dec(batch=0) == fa.FA_OK
