@@ -115,9 +115,11 @@ __global__ void __launch_bounds__(256)
   constexpr int LB = E * B;            // code bits per lane
   constexpr int MAXC = (32 + LB - 1) / LB + 1;  // lanes feeding one word
   const int lane = threadIdx.x & 31;
-  float edge[NL - 1];
-#pragma unroll
-  for (int k = 0; k < NL - 1; ++k) edge[k] = 0.5f * (levels[k] + levels[k + 1]);
+  // cell edges, with a sentinel so the binary search below reads edge[c + h - 1]
+  __shared__ float edge[NL];
+  if (threadIdx.x < NL - 1) edge[threadIdx.x] = 0.5f * (levels[threadIdx.x] + levels[threadIdx.x + 1]);
+  if (threadIdx.x == NL - 1) edge[NL - 1] = INFINITY;
+  __syncthreads();
   float sg[E];
 #pragma unroll
   for (int i = 0; i < E; ++i) sg[i] = signs[lane * E + i];
@@ -141,9 +143,10 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int i = 0; i < E; ++i) {
       const float u = v[i] * inv;
+      // the number of edges below u, by binary search (edges ascending)
       uint32_t c = 0;
 #pragma unroll
-      for (int k = 0; k < NL - 1; ++k) c += (u > edge[k]) ? 1u : 0u;
+      for (int h = NL / 2; h > 0; h >>= 1) c += (u > edge[c + h - 1]) ? h : 0u;
       val |= c << (i * B);
     }
     // word w of the row gathers the code bits of lanes l0 .. l0 + MAXC - 1
@@ -187,10 +190,16 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   constexpr int KW = D * KB / 32;   // 32-bit words of a packed K row
   constexpr int KROW = D * KB / 8;  // bytes of a packed K row
   constexpr int VROW = D * VB / 8;
-  constexpr int LVB = E * VB;       // V code bits per lane
-  __shared__ __align__(16) float qr[G][D];
-  __shared__ float klut[1 << KB];
-  __shared__ float vlut[1 << VB];
+  constexpr int LVB = E * VB;       // V code bits per lane (its E channels)
+  constexpr int VU2 = VROW / 8;     // 8-byte words of a 32-key V block per lane
+  constexpr int GP = (G + 1) / 2;   // head pairs
+  // queries interleaved by head: one vector load gives a channel of every head
+  __shared__ __align__(16) float qr[D][G];
+  // V pair table: entry c is (level[c & m], level[c >> b]) for two consecutive
+  // b-bit codes read as one 2b-bit field
+  __shared__ float klut[1 << KB];  // one code per read: distinct entries, distinct banks
+  __shared__ __align__(8) float2 vtab[1 << (2 * VB)];
+  __shared__ __align__(16) uint2 vblk[kDecodeWarps][32 * VU2];  // a warp's staged V codes
   __shared__ float s_m[kDecodeWarps][G], s_l[kDecodeWarps][G];
   __shared__ __align__(16) float s_o[kDecodeWarps][G][D];
 
@@ -205,7 +214,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   const int k0 = split * A.split_keys;
   const int k1 = min(len, k0 + A.split_keys);
   if (threadIdx.x < (1 << KB)) klut[threadIdx.x] = A.k_levels[threadIdx.x];
-  if (threadIdx.x < (1 << VB)) vlut[threadIdx.x] = A.v_levels[threadIdx.x];
+  for (int c = threadIdx.x; c < (1 << (2 * VB)); c += blockDim.x)
+    vtab[c] = make_float2(A.v_levels[c & ((1 << VB) - 1)], A.v_levels[c >> VB]);
   // rotated, pre-scaled queries: qr = scale log2(e) H (s * q) / sqrt(d)
   for (int gi = warp; gi < G; gi += kDecodeWarps) {
     const int h = g * G + gi;
@@ -216,30 +226,35 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     warp_fwht<E>(v, lane);
     const float sc = A.scale_log2 * rsqrtf(static_cast<float>(D));
 #pragma unroll
-    for (int i = 0; i < E; ++i) qr[gi][lane * E + i] = v[i] * sc;
+    for (int i = 0; i < E; ++i) qr[lane * E + i][gi] = v[i] * sc;
   }
   __syncthreads();
 
-  float m[G], lsum[G], o[G][E];
+  float m[G], lsum[G];
+  float2 o[GP][E];  // heads (2p, 2p + 1) of channel e of this lane
 #pragma unroll
   for (int gi = 0; gi < G; ++gi) {
     m[gi] = -INFINITY;
     lsum[gi] = 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) o[gi][e] = 0.f;
   }
+#pragma unroll
+  for (int pi = 0; pi < GP; ++pi)
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[pi][e] = make_float2(0.f, 0.f);
   const int64_t plane = static_cast<int64_t>(b) * A.hkv + g;
   const uint8_t* kc = A.kc + plane * A.cap * KROW;
   const uint8_t* vc = A.vc + plane * A.cap * VROW;
   const float* kn = A.kn + plane * A.cap;
   const float* vn = A.vn + plane * A.cap;
 
-  for (int c0 = k0 + warp * 32; c0 < k1; c0 += kDecodeWarps * 32) {
-    // scores: one key per lane
-    const int key = c0 + lane;
-    float s[G];
+  // one chunk's operands: this lane's K row and both norms of its key, and
+  // its share of the chunk's packed V rows (rows past the end read as 0)
+  auto load_chunk = [&](int c, uint32_t (&kw)[KW], float& nk, float& nv, uint2 (&vr)[VU2]) {
+    const int key = c + lane;
+    const int n = k1 - c;
+    nk = 0.f;
+    nv = 0.f;
     if (key < k1) {
-      uint32_t kw[KW];
       if constexpr (KROW % 16 == 0) {
         const uint4* src = reinterpret_cast<const uint4*>(kc + static_cast<int64_t>(key) * KROW);
 #pragma unroll
@@ -255,61 +270,109 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
           kw[2 * t] = u.x; kw[2 * t + 1] = u.y;
         }
       }
-      float acc[G];
-#pragma unroll
-      for (int gi = 0; gi < G; ++gi) acc[gi] = 0.f;
-#pragma unroll
-      for (int i = 0; i < D; i += 4) {
-        float lev[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) lev[t] = klut[code_at<KB, KW>(kw, (i + t) * KB)];
-#pragma unroll
-        for (int gi = 0; gi < G; ++gi) {
-          const float4 qv = *reinterpret_cast<const float4*>(&qr[gi][i]);
-          acc[gi] = fmaf(qv.x, lev[0], acc[gi]);
-          acc[gi] = fmaf(qv.y, lev[1], acc[gi]);
-          acc[gi] = fmaf(qv.z, lev[2], acc[gi]);
-          acc[gi] = fmaf(qv.w, lev[3], acc[gi]);
-        }
-      }
-      const float nk = kn[key];
-#pragma unroll
-      for (int gi = 0; gi < G; ++gi) s[gi] = acc[gi] * nk;
+      nk = kn[key];
+      nv = vn[key];
     } else {
 #pragma unroll
-      for (int gi = 0; gi < G; ++gi) s[gi] = -INFINITY;
+      for (int t = 0; t < KW; ++t) kw[t] = 0u;
     }
-    // online softmax, per head, over this warp's 32 keys
+    const uint2* vsrc = reinterpret_cast<const uint2*>(vc + static_cast<int64_t>(c) * VROW);
+#pragma unroll
+    for (int t = 0; t < VU2; ++t) {
+      const int idx = t * 32 + lane;
+      vr[t] = (idx * 8) / VROW < n ? vsrc[idx] : make_uint2(0u, 0u);
+    }
+  };
+
+  int c0 = k0 + warp * 32;
+  uint32_t kw[KW];
+  float nk = 0.f, nv = 0.f;
+  uint2 vr[VU2];
+  if (c0 < k1) load_chunk(c0, kw, nk, nv, vr);
+  for (; c0 < k1; c0 += kDecodeWarps * 32) {
+    __syncwarp();
+#pragma unroll
+    for (int t = 0; t < VU2; ++t) vblk[warp][t * 32 + lane] = vr[t];
+    const float nk_c = nk, nv_c = nv;
+    uint32_t kw_c[KW];
+#pragma unroll
+    for (int t = 0; t < KW; ++t) kw_c[t] = kw[t];
+    // the next chunk's loads fly while this one computes
+    const int c1 = c0 + kDecodeWarps * 32;
+    if (c1 < k1) load_chunk(c1, kw, nk, nv, vr);
+
+    // scores: one key per lane, two channels per table read
+    const int key = c0 + lane;
+    float acc[G];
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) acc[gi] = 0.f;
+#pragma unroll
+    for (int i = 0; i < D; ++i) {
+      const float lv = klut[code_at<KB, KW>(kw_c, i * KB)];
+      if constexpr (G == 1) {
+        acc[0] = fmaf(qr[i][0], lv, acc[0]);
+      } else if constexpr (G == 2) {
+        const float2 q2 = *reinterpret_cast<const float2*>(&qr[i][0]);
+        const float2 a = fma2(q2, make_float2(lv, lv), make_float2(acc[0], acc[1]));
+        acc[0] = a.x;
+        acc[1] = a.y;
+      } else {
+        // four heads per 16-byte broadcast read of the rotated queries
+#pragma unroll
+        for (int g4 = 0; g4 < G; g4 += 4) {
+          const float4 q4 = *reinterpret_cast<const float4*>(&qr[i][g4]);
+          const float2 a = fma2(make_float2(q4.x, q4.y), make_float2(lv, lv), make_float2(acc[g4], acc[g4 + 1]));
+          const float2 c = fma2(make_float2(q4.z, q4.w), make_float2(lv, lv), make_float2(acc[g4 + 2], acc[g4 + 3]));
+          acc[g4] = a.x;
+          acc[g4 + 1] = a.y;
+          acc[g4 + 2] = c.x;
+          acc[g4 + 3] = c.y;
+        }
+      }
+    }
+    // online softmax, per head, over this warp's 32 keys; p carries ||v||
     float p[G];
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
-      const float m_new = fmaxf(m[gi], warp_max(s[gi]));
+      const float s = key < k1 ? acc[gi] * nk_c : -INFINITY;
+      const float m_new = fmaxf(m[gi], warp_max(s));
       const float alpha = m[gi] == -INFINITY ? 0.f : exp2f(m[gi] - m_new);
-      p[gi] = s[gi] == -INFINITY ? 0.f : exp2f(s[gi] - m_new);
-      lsum[gi] = lsum[gi] * alpha + p[gi];
+      const float pe = s == -INFINITY ? 0.f : exp2f(s - m_new);
+      lsum[gi] = lsum[gi] * alpha + pe;
       m[gi] = m_new;
+      p[gi] = pe * nv_c;
+      if (alpha != 1.f) {
 #pragma unroll
-      for (int e = 0; e < E; ++e) o[gi][e] *= alpha;
+        for (int e = 0; e < E; ++e) {
+          if (gi % 2 == 0) o[gi / 2][e].x *= alpha;
+          else o[gi / 2][e].y *= alpha;
+        }
+      }
     }
+    __syncwarp();
     // V: the lanes over the channels, one key at a time
     const int n = min(32, k1 - c0);
     const int bitpos = lane * LVB;
-    const int nbytes = ((bitpos & 7) + LVB + 7) >> 3;
+    const uint32_t* vw = reinterpret_cast<const uint32_t*>(vblk[warp]) + (bitpos >> 5);
+    const int sh = bitpos & 31;
+    const bool two = sh + LVB > 32;  // this lane's bits cross into the next word
     for (int j = 0; j < n; ++j) {
-      const int64_t vrow = static_cast<int64_t>(c0 + j);
-      const uint8_t* vp = vc + vrow * VROW + (bitpos >> 3);
-      uint32_t bits = 0;
-      for (int t = 0; t < nbytes; ++t) bits |= static_cast<uint32_t>(vp[t]) << (8 * t);
-      bits >>= (bitpos & 7);
+      const uint32_t w0 = vw[j * (VROW / 4)];
+      const uint32_t w1 = two ? vw[j * (VROW / 4) + 1] : 0u;
+      const uint32_t bits = __funnelshift_r(w0, w1, sh);
       float lev[E];
 #pragma unroll
-      for (int e = 0; e < E; ++e) lev[e] = vlut[(bits >> (e * VB)) & ((1u << VB) - 1u)];
-      const float nv = vn[vrow];
+      for (int e = 0; e < E; e += 2) {
+        const float2 t = vtab[(bits >> (e * VB)) & ((1u << (2 * VB)) - 1u)];
+        lev[e] = t.x;
+        lev[e + 1] = t.y;
+      }
 #pragma unroll
-      for (int gi = 0; gi < G; ++gi) {
-        const float pj = __shfl_sync(0xffffffffu, p[gi], j) * nv;
+      for (int pi = 0; pi < GP; ++pi) {
+        const float p0 = __shfl_sync(0xffffffffu, p[2 * pi], j);
+        const float p1 = (2 * pi + 1 < G) ? __shfl_sync(0xffffffffu, p[(2 * pi + 1) % G], j) : 0.f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) o[gi][e] = fmaf(pj, lev[e], o[gi][e]);
+        for (int e = 0; e < E; ++e) o[pi][e] = fma2(make_float2(p0, p1), make_float2(lev[e], lev[e]), o[pi][e]);
       }
     }
   }
@@ -323,7 +386,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
       s_l[warp][gi] = l;
     }
 #pragma unroll
-    for (int e = 0; e < E; ++e) s_o[warp][gi][lane * E + e] = o[gi][e];
+    for (int e = 0; e < E; ++e) s_o[warp][gi][lane * E + e] = gi % 2 == 0 ? o[gi / 2][e].x : o[gi / 2][e].y;
   }
   __syncthreads();
   for (int idx = threadIdx.x; idx < G * (D + 2); idx += blockDim.x) {
