@@ -22,6 +22,8 @@
 // key per lane, the V update with the lanes over the channels), and
 // tq_merge_kernel (one warp per output row: the split merge, the inverse
 // rotation, the epilogue, the bf16 store).
+#include <cuda_fp16.h>
+
 #include <cmath>
 #include <vector>
 
@@ -183,27 +185,89 @@ struct TqArgs {
   Watchdog wd;
 };
 
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// D (fp32) += A (16x16 fp16, row) . B (16x8 fp16, col)
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four B-bit codes, one per nibble of `nib`, to fp16 pairs {level[c0],
+// level[c1]} and {level[c2], level[c3]}.  The codebook is antisymmetric:
+// with P the upper half of the levels (positive, ascending), a code c in the
+// upper half reads P[c - half] and one in the lower half -P[half - 1 - c].
+// pl / ph hold the low / high bytes of P[0..7] (fp16), so one byte permute
+// per byte plane looks up four codes; the sign bit is ORed in after.
+template <int B>
+__device__ __forceinline__ void dequant4(uint32_t nib, const uint32_t (&pl)[2], const uint32_t (&ph)[2],
+                                         uint32_t& h01, uint32_t& h23) {
+  constexpr uint32_t kHalf = 1u << (B - 1);
+  const uint32_t pos = (nib >> (B - 1)) & 0x1111u;
+  const uint32_t neg = pos ^ 0x1111u;
+  const uint32_t j = (nib & (0x1111u * (kHalf - 1))) ^ (neg * (kHalf - 1));
+  const uint32_t lo = prmt(pl[0], pl[1], j);
+  const uint32_t hi = prmt(ph[0], ph[1], j);
+  h01 = prmt(lo, hi, 0x5140u) | ((neg & 0x1u) << 15) | ((neg & 0x10u) << 27);
+  h23 = prmt(lo, hi, 0x7362u) | ((neg & 0x100u) << 7) | ((neg & 0x1000u) << 19);
+}
+
+// The 4B bits of four consecutive B-bit codes, one code per nibble.
+template <int B>
+__device__ __forceinline__ uint32_t to_nibbles(uint32_t f) {
+  if constexpr (B == 4) {
+    return f;
+  } else if constexpr (B == 3) {
+    return (f & 0x7u) | ((f & 0x38u) << 1) | ((f & 0x1c0u) << 2) | ((f & 0xe00u) << 3);
+  } else {
+    return (f & 0x3u) | ((f & 0xcu) << 2) | ((f & 0x30u) << 4) | ((f & 0xc0u) << 6);
+  }
+}
+
+// Split-K decode over one (sequence, KV head, key split).  Per warp and
+// 32-key chunk:
+//   S^T [32 keys x 8 heads] = K_hat . (R q)^T on mma.sync m16n8k16 (keys on
+//     M, the group's heads on N, channels on K).  Channels are summed over,
+//     so their order inside a k-step is free: thread (g, t) takes channels
+//     [t d/4, t d/4 + d/4) of its rows, four per k-step, and the rotated
+//     queries' B fragments (fp16, registers) use the same order.  A
+//     fragments come from the packed codes by byte permutes (dequant4).
+//   online softmax per head on the S fragments; p ||v|| goes to shared memory
+//   O_rot [channels x heads] += sum_j p_j ||v_j|| level[code_j] with the lanes
+//     over the channels (one broadcast read of a key's p for all heads).
 template <int D, int KB, int VB, int G>
 __global__ void __launch_bounds__(kDecodeWarps * 32)
     tq_decode_kernel(TqArgs A) {
   constexpr int E = D / 32;
-  constexpr int KW = D * KB / 32;   // 32-bit words of a packed K row
   constexpr int KROW = D * KB / 8;  // bytes of a packed K row
   constexpr int VROW = D * VB / 8;
   constexpr int LVB = E * VB;       // V code bits per lane (its E channels)
   constexpr int VU2 = VROW / 8;     // 8-byte words of a 32-key V block per lane
   constexpr int GP = (G + 1) / 2;   // head pairs
-  // queries interleaved by head: one vector load gives a channel of every head
+  constexpr int KS = D / 16;        // k-steps of the score MMA
+  constexpr int SB = D * KB / 32;   // bytes of a thread's quarter of a K row
+  constexpr int SW = (SB + 3) / 4;
+  constexpr int PG = G < 4 ? G : 4 * ((G + 3) / 4);  // p row stride (16-byte rows from 4 heads up)
   __shared__ __align__(16) float qr[D][G];
-  // V pair table: entry c is (level[c & m], level[c >> b]) for two consecutive
-  // b-bit codes read as one 2b-bit field
-  __shared__ float klut[1 << KB];  // one code per read: distinct entries, distinct banks
-  __shared__ __align__(8) float2 vtab[1 << (2 * VB)];
+  __shared__ __align__(8) float2 vtab[1 << (2 * VB)];  // V pair table: (level[c & m], level[c >> b])
   __shared__ __align__(16) uint2 vblk[kDecodeWarps][32 * VU2];  // a warp's staged V codes
+  __shared__ __align__(16) float ps[kDecodeWarps][32][PG];      // p ||v|| per key and head
   __shared__ float s_m[kDecodeWarps][G], s_l[kDecodeWarps][G];
   __shared__ __align__(16) float s_o[kDecodeWarps][G][D];
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gq = lane >> 2, tq = lane & 3;  // fragment row group and column pair
   const int bg = blockIdx.y, split = blockIdx.x;
   const int b = bg / A.hkv, g = bg % A.hkv;
   int len = A.seqlens[b];
@@ -213,9 +277,17 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   }
   const int k0 = split * A.split_keys;
   const int k1 = min(len, k0 + A.split_keys);
-  if (threadIdx.x < (1 << KB)) klut[threadIdx.x] = A.k_levels[threadIdx.x];
   for (int c = threadIdx.x; c < (1 << (2 * VB)); c += blockDim.x)
     vtab[c] = make_float2(A.v_levels[c & ((1 << VB) - 1)], A.v_levels[c >> VB]);
+  // the upper half of the K levels as fp16 byte planes (8 entries, zero-padded)
+  uint32_t pl[2] = {0u, 0u}, ph[2] = {0u, 0u};
+#pragma unroll
+  for (int jj = 0; jj < (1 << (KB - 1)); ++jj) {
+    const __half hv = __float2half_rn(A.k_levels[(1 << (KB - 1)) + jj]);
+    const uint32_t bits = *reinterpret_cast<const uint16_t*>(&hv);
+    pl[jj / 4] |= (bits & 0xffu) << (8 * (jj % 4));
+    ph[jj / 4] |= (bits >> 8) << (8 * (jj % 4));
+  }
   // rotated, pre-scaled queries: qr = scale log2(e) H (s * q) / sqrt(d)
   for (int gi = warp; gi < G; gi += kDecodeWarps) {
     const int h = g * G + gi;
@@ -229,14 +301,19 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     for (int i = 0; i < E; ++i) qr[lane * E + i][gi] = v[i] * sc;
   }
   __syncthreads();
-
-  float m[G], lsum[G];
-  float2 o[GP][E];  // heads (2p, 2p + 1) of channel e of this lane
+  // B fragments: head gq (zero past the group), channels t d/4 + 4 ks + 0..3
+  uint32_t qb[KS][2];
 #pragma unroll
-  for (int gi = 0; gi < G; ++gi) {
-    m[gi] = -INFINITY;
-    lsum[gi] = 0.f;
+  for (int ks = 0; ks < KS; ++ks) {
+    const int ch = tq * (D / 4) + 4 * ks;
+    const bool on = gq < G;
+    const int hh = on ? gq : 0;
+    qb[ks][0] = on ? pack_h2(qr[ch][hh], qr[ch + 1][hh]) : 0u;
+    qb[ks][1] = on ? pack_h2(qr[ch + 2][hh], qr[ch + 3][hh]) : 0u;
   }
+
+  float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};  // heads 2 tq, 2 tq + 1
+  float2 o[GP][E];  // heads (2p, 2p + 1) of channel e of this lane
 #pragma unroll
   for (int pi = 0; pi < GP; ++pi)
 #pragma unroll
@@ -247,34 +324,42 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   const float* kn = A.kn + plane * A.cap;
   const float* vn = A.vn + plane * A.cap;
 
-  // one chunk's operands: this lane's K row and both norms of its key, and
-  // its share of the chunk's packed V rows (rows past the end read as 0)
-  auto load_chunk = [&](int c, uint32_t (&kw)[KW], float& nk, float& nv, uint2 (&vr)[VU2]) {
-    const int key = c + lane;
+  // one chunk's operands: the quarter K rows of this thread's four keys
+  // (16 mt + gq + 8 r), their norms, and its share of the packed V rows
+  auto load_chunk = [&](int c, uint32_t (&kw)[4][SW], float (&nk)[4], float (&nv)[4], uint2 (&vr)[VU2]) {
     const int n = k1 - c;
-    nk = 0.f;
-    nv = 0.f;
-    if (key < k1) {
-      if constexpr (KROW % 16 == 0) {
-        const uint4* src = reinterpret_cast<const uint4*>(kc + static_cast<int64_t>(key) * KROW);
 #pragma unroll
-        for (int t = 0; t < KW / 4; ++t) {
-          const uint4 u = src[t];
-          kw[4 * t] = u.x; kw[4 * t + 1] = u.y; kw[4 * t + 2] = u.z; kw[4 * t + 3] = u.w;
-        }
-      } else {  // 24-byte rows (d = 64, 3 bits): 8-byte loads
-        const uint2* src = reinterpret_cast<const uint2*>(kc + static_cast<int64_t>(key) * KROW);
+    for (int r4 = 0; r4 < 4; ++r4) {
+      const int kk = 16 * (r4 >> 1) + gq + 8 * (r4 & 1);
+      nk[r4] = 0.f;
+      nv[r4] = 0.f;
 #pragma unroll
-        for (int t = 0; t < KW / 2; ++t) {
-          const uint2 u = src[t];
-          kw[2 * t] = u.x; kw[2 * t + 1] = u.y;
+      for (int t = 0; t < SW; ++t) kw[r4][t] = 0u;
+      if (kk < n) {
+        const uint8_t* src = kc + static_cast<int64_t>(c + kk) * KROW + tq * SB;
+        if constexpr (SB % 16 == 0) {
+#pragma unroll
+          for (int t = 0; t < SW / 4; ++t) {
+            const uint4 u = reinterpret_cast<const uint4*>(src)[t];
+            kw[r4][4 * t] = u.x; kw[r4][4 * t + 1] = u.y; kw[r4][4 * t + 2] = u.z; kw[r4][4 * t + 3] = u.w;
+          }
+        } else if constexpr (SB % 8 == 0) {
+#pragma unroll
+          for (int t = 0; t < SW / 2; ++t) {
+            const uint2 u = reinterpret_cast<const uint2*>(src)[t];
+            kw[r4][2 * t] = u.x; kw[r4][2 * t + 1] = u.y;
+          }
+        } else if constexpr (SB % 4 == 0) {
+#pragma unroll
+          for (int t = 0; t < SW; ++t) kw[r4][t] = reinterpret_cast<const uint32_t*>(src)[t];
+        } else {  // 6-byte quarters (d = 64, 3 bits): 2-byte loads
+          const uint16_t* h = reinterpret_cast<const uint16_t*>(src);
+          kw[r4][0] = static_cast<uint32_t>(h[0]) | (static_cast<uint32_t>(h[1]) << 16);
+          kw[r4][1] = h[2];
         }
+        nk[r4] = kn[c + kk];
+        nv[r4] = vn[c + kk];
       }
-      nk = kn[key];
-      nv = vn[key];
-    } else {
-#pragma unroll
-      for (int t = 0; t < KW; ++t) kw[t] = 0u;
     }
     const uint2* vsrc = reinterpret_cast<const uint2*>(vc + static_cast<int64_t>(c) * VROW);
 #pragma unroll
@@ -285,69 +370,85 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   };
 
   int c0 = k0 + warp * 32;
-  uint32_t kw[KW];
-  float nk = 0.f, nv = 0.f;
+  uint32_t kw[4][SW];
+  float nk[4], nv[4];
   uint2 vr[VU2];
   if (c0 < k1) load_chunk(c0, kw, nk, nv, vr);
   for (; c0 < k1; c0 += kDecodeWarps * 32) {
-    __syncwarp();
+    __syncwarp();  // the previous chunk's reads of vblk and ps are done
 #pragma unroll
     for (int t = 0; t < VU2; ++t) vblk[warp][t * 32 + lane] = vr[t];
-    const float nk_c = nk, nv_c = nv;
-    uint32_t kw_c[KW];
+    uint32_t kc4[4][SW];
+    float nk4[4], nv4[4];
 #pragma unroll
-    for (int t = 0; t < KW; ++t) kw_c[t] = kw[t];
+    for (int r4 = 0; r4 < 4; ++r4) {
+      nk4[r4] = nk[r4];
+      nv4[r4] = nv[r4];
+#pragma unroll
+      for (int t = 0; t < SW; ++t) kc4[r4][t] = kw[r4][t];
+    }
     // the next chunk's loads fly while this one computes
     const int c1 = c0 + kDecodeWarps * 32;
     if (c1 < k1) load_chunk(c1, kw, nk, nv, vr);
 
-    // scores: one key per lane, two channels per table read
-    const int key = c0 + lane;
-    float acc[G];
+    // scores on the tensor cores: two 16-key tiles
+    float sacc[2][4];
 #pragma unroll
-    for (int gi = 0; gi < G; ++gi) acc[gi] = 0.f;
+    for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-    for (int i = 0; i < D; ++i) {
-      const float lv = klut[code_at<KB, KW>(kw_c, i * KB)];
-      if constexpr (G == 1) {
-        acc[0] = fmaf(qr[i][0], lv, acc[0]);
-      } else if constexpr (G == 2) {
-        const float2 q2 = *reinterpret_cast<const float2*>(&qr[i][0]);
-        const float2 a = fma2(q2, make_float2(lv, lv), make_float2(acc[0], acc[1]));
-        acc[0] = a.x;
-        acc[1] = a.y;
-      } else {
-        // four heads per 16-byte broadcast read of the rotated queries
+      for (int t = 0; t < 4; ++t) sacc[mt][t] = 0.f;
 #pragma unroll
-        for (int g4 = 0; g4 < G; g4 += 4) {
-          const float4 q4 = *reinterpret_cast<const float4*>(&qr[i][g4]);
-          const float2 a = fma2(make_float2(q4.x, q4.y), make_float2(lv, lv), make_float2(acc[g4], acc[g4 + 1]));
-          const float2 c = fma2(make_float2(q4.z, q4.w), make_float2(lv, lv), make_float2(acc[g4 + 2], acc[g4 + 3]));
-          acc[g4] = a.x;
-          acc[g4 + 1] = a.y;
-          acc[g4 + 2] = c.x;
-          acc[g4 + 3] = c.y;
-        }
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        dequant4<KB>(to_nibbles<KB>(code_at<4 * KB, SW>(kc4[2 * mt], 4 * ks * KB)), pl, ph, a0, a2);
+        dequant4<KB>(to_nibbles<KB>(code_at<4 * KB, SW>(kc4[2 * mt + 1], 4 * ks * KB)), pl, ph, a1, a3);
+        mma_f16(sacc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
       }
     }
-    // online softmax, per head, over this warp's 32 keys; p carries ||v||
-    float p[G];
+    // online softmax for heads 2 tq, 2 tq + 1 over the chunk's 32 keys
+    float sv[2][4];
+    float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int gi = 0; gi < G; ++gi) {
-      const float s = key < k1 ? acc[gi] * nk_c : -INFINITY;
-      const float m_new = fmaxf(m[gi], warp_max(s));
-      const float alpha = m[gi] == -INFINITY ? 0.f : exp2f(m[gi] - m_new);
-      const float pe = s == -INFINITY ? 0.f : exp2f(s - m_new);
-      lsum[gi] = lsum[gi] * alpha + pe;
-      m[gi] = m_new;
-      p[gi] = pe * nv_c;
-      if (alpha != 1.f) {
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-          if (gi % 2 == 0) o[gi / 2][e].x *= alpha;
-          else o[gi / 2][e].y *= alpha;
-        }
+      for (int t = 0; t < 4; ++t) {
+        const int r4 = 2 * mt + (t >> 1);
+        const int kk = 16 * mt + gq + 8 * (t >> 1);
+        const float x = c0 + kk < k1 ? sacc[mt][t] * nk4[r4] : -INFINITY;
+        sv[mt][t] = x;
+        tmax[t & 1] = fmaxf(tmax[t & 1], x);
       }
+    float alpha2[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float mx = tmax[hh];
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float m_new = fmaxf(m2[hh], mx);
+      alpha2[hh] = m2[hh] == -INFINITY ? 0.f : exp2f(m2[hh] - m_new);
+      m2[hh] = m_new;
+      l2[hh] *= alpha2[hh];
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int hh = t & 1;
+        const int r4 = 2 * mt + (t >> 1);
+        const int kk = 16 * mt + gq + 8 * (t >> 1);
+        const float pe = sv[mt][t] == -INFINITY ? 0.f : exp2f(sv[mt][t] - m2[hh]);
+        l2[hh] += pe;
+        const int h = 2 * tq + hh;
+        if (h < G) ps[warp][kk][h] = pe * nv4[r4];
+      }
+    // the O rows of every head take their alpha (held by lane h / 2)
+#pragma unroll
+    for (int pi = 0; pi < GP; ++pi) {
+      const float a0 = __shfl_sync(0xffffffffu, alpha2[0], pi);
+      const float a1 = __shfl_sync(0xffffffffu, alpha2[1], pi);
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[pi][e] = make_float2(o[pi][e].x * a0, o[pi][e].y * a1);
     }
     __syncwarp();
     // V: the lanes over the channels, one key at a time
@@ -367,27 +468,46 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
         lev[e] = t.x;
         lev[e + 1] = t.y;
       }
+      float pj[2 * GP];
+      if constexpr (G >= 4) {
 #pragma unroll
-      for (int pi = 0; pi < GP; ++pi) {
-        const float p0 = __shfl_sync(0xffffffffu, p[2 * pi], j);
-        const float p1 = (2 * pi + 1 < G) ? __shfl_sync(0xffffffffu, p[(2 * pi + 1) % G], j) : 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) o[pi][e] = fma2(make_float2(p0, p1), make_float2(lev[e], lev[e]), o[pi][e]);
+        for (int g4 = 0; g4 < G; g4 += 4) {
+          const float4 p4 = *reinterpret_cast<const float4*>(&ps[warp][j][g4]);
+          pj[g4] = p4.x; pj[g4 + 1] = p4.y; pj[g4 + 2] = p4.z; pj[g4 + 3] = p4.w;
+        }
+      } else if constexpr (G == 2) {
+        const float2 p2 = *reinterpret_cast<const float2*>(&ps[warp][j][0]);
+        pj[0] = p2.x; pj[1] = p2.y;
+      } else {
+        pj[0] = ps[warp][j][0];
+        pj[1] = 0.f;
       }
+#pragma unroll
+      for (int pi = 0; pi < GP; ++pi)
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          o[pi][e] = fma2(make_float2(pj[2 * pi], pj[2 * pi + 1]), make_float2(lev[e], lev[e]), o[pi][e]);
     }
   }
 
-  // the four warps' states merge into this split's partial
+  // this warp's state: m and l of head 2 tq + hh sit in the lanes of column
+  // pair tq (l summed over them); O in the lanes over the channels
 #pragma unroll
-  for (int gi = 0; gi < G; ++gi) {
-    const float l = warp_sum(lsum[gi]);
-    if (lane == 0) {
-      s_m[warp][gi] = m[gi];
-      s_l[warp][gi] = l;
+  for (int hh = 0; hh < 2; ++hh) {
+    float l = l2[hh];
+    l += __shfl_xor_sync(0xffffffffu, l, 4);
+    l += __shfl_xor_sync(0xffffffffu, l, 8);
+    l += __shfl_xor_sync(0xffffffffu, l, 16);
+    const int h = 2 * tq + hh;
+    if (gq == 0 && h < G) {
+      s_m[warp][h] = m2[hh];
+      s_l[warp][h] = l;
     }
+  }
+#pragma unroll
+  for (int gi = 0; gi < G; ++gi)
 #pragma unroll
     for (int e = 0; e < E; ++e) s_o[warp][gi][lane * E + e] = gi % 2 == 0 ? o[gi / 2][e].x : o[gi / 2][e].y;
-  }
   __syncthreads();
   for (int idx = threadIdx.x; idx < G * (D + 2); idx += blockDim.x) {
     const int gi = idx / (D + 2), c = idx % (D + 2);
