@@ -143,3 +143,49 @@ def test_quality_in_the_range_the_page_reports():
     assert 0.92 <= c42 <= 0.955, c42   # the page: about 0.94
     assert 0.985 <= c44 <= 0.995, c44  # the page: about 0.99
     assert c42 < c43 < c44
+
+
+def _plant(monkeypatch, name, fn):
+    monkeypatch.setattr(tq, name, fn)
+    tq._codebook_cached.cache_clear()
+
+
+_REAL = {n: getattr(tq, n) for n in ("fwht", "rotate", "_codebook", "pack", "dequantize", "edges_of")}
+
+PLANTS = {
+    # butterfly outputs swapped: H with its rows reordered
+    "fwht_swapped": ("fwht", lambda x: _REAL["fwht"](x)[..., ::-1].copy(),
+                     lambda mp: test_fwht_is_the_sylvester_hadamard_matrix(8)),
+    # signs applied after the transform instead of before it
+    "signs_after_H": ("rotate", lambda x, s: _REAL["fwht"](np.asarray(x, np.float64)) * np.asarray(s, np.float64)
+                      / np.sqrt(np.asarray(x).shape[-1]),
+                      lambda mp: test_rotation_is_orthonormal_with_the_signs_first()),
+    # the quantiles the iteration starts from, not the Lloyd-Max fixed point
+    "no_lloyd_iteration": ("_codebook", lambda d, b: _REAL["_codebook"](d, b, iters=1),
+                           lambda mp: test_codebook_meets_the_lloyd_max_conditions(64, 4)),
+    # a uniform codebook of the right range
+    "uniform_levels": ("_codebook", lambda d, b: np.linspace(-3, 3, 1 << b) / np.sqrt(d + 1),
+                       lambda mp: test_large_d_codebook_is_the_gaussian_lloyd_max_quantiser(2)),
+    # cell edges at the levels themselves instead of the midpoints
+    "edges_at_levels": ("edges_of", lambda lv: np.asarray(lv, np.float64)[1:],
+                        lambda mp: test_codes_are_the_nearest_level()),
+    # most significant bit first within each code
+    "msb_first": ("pack", lambda c, b: _REAL["pack"](np.sum(((np.asarray(c, np.uint8)[..., None] >> np.arange(b))
+                                                            & 1) << np.arange(b)[::-1], -1).astype(np.uint8), b),
+                  lambda mp: test_bit_packing_is_lsb_first()),
+    # the inverse rotation without the signs
+    "unrotate_without_signs": ("dequantize", lambda p, n, s, b, lv, d: _REAL["dequantize"](p, n, np.ones(d), b, lv, d),
+                               lambda mp: test_quality_in_the_range_the_page_reports()),
+}
+
+
+@pytest.mark.parametrize("plant", sorted(PLANTS))
+def test_a_planted_mistake_fails_a_pin(monkeypatch, plant):
+    """Each plausible mistake, planted in the oracle, makes its pin fail."""
+    name, wrong, pin = PLANTS[plant]
+    _plant(monkeypatch, name, wrong)
+    try:
+        with pytest.raises(AssertionError):
+            pin(monkeypatch)
+    finally:
+        tq._codebook_cached.cache_clear()
