@@ -127,44 +127,74 @@ __global__ void __launch_bounds__(256)
   for (int i = 0; i < E; ++i) sg[i] = signs[lane * E + i];
   const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
-       row += warps) {
-    float v[E];
-    load_row<E>(x + row * D + lane * E, v);
-    float ss = 0.f;
+  // two rows per iteration: their independent chains interleave
+  for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row0 < rows;
+       row0 += 2 * warps) {
+    const int64_t rr[2] = {row0, row0 + warps};
+    const bool live1 = rr[1] < rows;
+    float v[2][E];
+    load_row<E>(x + rr[0] * D + lane * E, v[0]);
+    if (live1) {
+      load_row<E>(x + rr[1] * D + lane * E, v[1]);
+    } else {
 #pragma unroll
-    for (int i = 0; i < E; ++i) {
-      v[i] *= sg[i];
-      ss = fmaf(v[i], v[i], ss);
+      for (int i = 0; i < E; ++i) v[1][i] = 0.f;
     }
-    ss = warp_sum(ss);
-    warp_fwht<E>(v, lane);
-    const float norm = sqrtf(ss);
-    const float inv = norm > 0.f ? inv_sqrt_d / norm : 0.f;
-    uint32_t val = 0;
+    float ss[2] = {0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < E; ++i) {
-      const float u = v[i] * inv;
-      // the number of edges below u, by binary search (edges ascending)
-      uint32_t c = 0;
+    for (int r = 0; r < 2; ++r)
 #pragma unroll
-      for (int h = NL / 2; h > 0; h >>= 1) c += (u > edge[c + h - 1]) ? h : 0u;
-      val |= c << (i * B);
+      for (int i = 0; i < E; ++i) {
+        v[r][i] *= sg[i];
+        ss[r] = fmaf(v[r][i], v[r][i], ss[r]);
+      }
+#pragma unroll
+    for (int h = 16; h > 0; h >>= 1) {
+      ss[0] += __shfl_xor_sync(0xffffffffu, ss[0], h);
+      ss[1] += __shfl_xor_sync(0xffffffffu, ss[1], h);
     }
-    // word w of the row gathers the code bits of lanes l0 .. l0 + MAXC - 1
+    warp_fwht<E>(v[0], lane);
+    warp_fwht<E>(v[1], lane);
+    uint32_t val[2];
+    float norm[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      norm[r] = sqrtf(ss[r]);
+      const float inv = norm[r] > 0.f ? inv_sqrt_d / norm[r] : 0.f;
+      val[r] = 0;
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        const float u = v[r][i] * inv;
+        // the number of edges below u, by binary search (edges ascending)
+        uint32_t c = 0;
+#pragma unroll
+        for (int h = NL / 2; h > 0; h >>= 1) c += (u > edge[c + h - 1]) ? h : 0u;
+        val[r] |= c << (i * B);
+      }
+    }
+    // word w of a row gathers the code bits of lanes l0 .. l0 + MAXC - 1
     const int w = lane;
     const int l0 = (32 * w) / LB;
-    uint32_t word = 0;
+    uint32_t word[2] = {0u, 0u};
 #pragma unroll
     for (int j = 0; j < MAXC; ++j) {
       const int src = min(l0 + j, 31);
-      const uint32_t t = __shfl_sync(0xffffffffu, val, src);
+      const uint32_t t0 = __shfl_sync(0xffffffffu, val[0], src);
+      const uint32_t t1 = __shfl_sync(0xffffffffu, val[1], src);
       const int shift = src * LB - 32 * w;
-      if (l0 + j <= 31 && shift < 32 && shift > -LB)
-        word |= shift >= 0 ? (t << shift) : (t >> (-shift));
+      if (l0 + j <= 31 && shift < 32 && shift > -LB) {
+        word[0] |= shift >= 0 ? (t0 << shift) : (t0 >> (-shift));
+        word[1] |= shift >= 0 ? (t1 << shift) : (t1 >> (-shift));
+      }
     }
-    if (w < W) reinterpret_cast<uint32_t*>(codes + row * (D * B / 8))[w] = word;
-    if (lane == 0) norms[row] = norm;
+    if (w < W) {
+      reinterpret_cast<uint32_t*>(codes + rr[0] * (D * B / 8))[w] = word[0];
+      if (live1) reinterpret_cast<uint32_t*>(codes + rr[1] * (D * B / 8))[w] = word[1];
+    }
+    if (lane == 0) {
+      norms[rr[0]] = norm[0];
+      if (live1) norms[rr[1]] = norm[1];
+    }
   }
 }
 
@@ -610,7 +640,7 @@ fa_status launch_compress_d(const fa_tq_compress_params& p, const LaunchCtx& ctx
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0) != cudaSuccess || per_sm < 1)
       return FA_ERR_CUDA;
-    const int64_t need = (p.rows + 7) / 8;
+    const int64_t need = (p.rows + 15) / 16;  // eight warps, two rows per warp per pass
     const int64_t cap = static_cast<int64_t>(per_sm) * device_sm_count();
     const unsigned grid = static_cast<unsigned>(need < cap ? need : cap);
     kern<<<grid, 256, 0, ctx.stream>>>(static_cast<const T*>(p.x), p.rows, p.signs, p.levels, p.codes, p.norms);

@@ -459,8 +459,10 @@ FA_API fa_status fa_tq_compress(const fa_tq_compress_params *p, fa_stream_t stre
  *   k_codes    [batch*hkv, capacity, head_dim*k_bits/8] uint8, k_norms
  *              [batch*hkv, capacity] fp32 (fa_tq_compress of the K rows);
  *              v_codes / v_norms likewise with v_bits
- *   k_levels, v_levels  device [2^bits] fp32;  signs device [head_dim] fp32
- *              (one rotation for K and V)
+ *   k_levels, v_levels  device [2^bits] fp32, ascending and antisymmetric
+ *              (level[n-1-i] = -level[i], as fa_tq_codebook returns them: the
+ *              K side is looked up from the upper half, mirrored for the
+ *              lower);  signs device [head_dim] fp32 (one rotation for K and V)
  *   cache_seqlens device int32 [batch]: keys 0 .. L_b - 1 are attended; a
  *              value outside [0, capacity] is clamped and reported by
  *              fa_check_device_error as FA_ERR_INVALID; L_b = 0 gives the
