@@ -767,9 +767,15 @@ def _cores():
 def cpu_baseline(w, flops_tiles, flops_exact, budget_s):
     """The oracle on the host cores over a bounded sample (about budget_s
     seconds of CPU work), scaled to the whole step by the exact pair count."""
-    dt, pairs = _oracle_sample(w, 64, 1)
-    n = int(min(4_000_000, max(64, 64 * budget_s / max(dt, 1e-4))))
-    dt, pairs = _oracle_sample(w, n, 2)
+    # calibrate on enough rows that fixed costs do not dominate, then size
+    # the sample to the budget (once more if it still came out short)
+    n = 1024
+    dt, pairs = _oracle_sample(w, n, 1)
+    for seed in (2, 3):
+        n = int(min(4_000_000, max(1024, n * budget_s / max(dt, 1e-4))))
+        dt, pairs = _oracle_sample(w, n, seed)
+        if dt >= 0.5 * budget_s:
+            break
     full_s = dt * flops_exact / (4 * w.d * pairs)
     return {"value": flops_tiles / full_s / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
             "sample": f"{n} random causal rows of one head plane ({pairs} visible pairs, {dt:.2f} s of fp64 "
@@ -779,13 +785,14 @@ def cpu_baseline(w, flops_tiles, flops_exact, budget_s):
 
 def reference_arm(args, world):
     """The oracle timed on host cores on this arm's workload, metric and unit;
-    each step is a bounded sample of 256 rows scaled by the exact pair count."""
+    each step is a bounded sample of 2048 rows (large enough that the call's
+    fixed costs do not dominate) scaled by the exact pair count."""
     from flashattention_attention_b200 import inputs
     w = inputs.gqa_causal_prefill()
     flops_tiles, flops_exact = prefill_flops(w)
     vals = []
     for s in range(args.warmup + args.steps):
-        dt, pairs = _oracle_sample(w, 256, 100 + s)
+        dt, pairs = _oracle_sample(w, 2048, 100 + s)
         if s >= args.warmup:
             vals.append(flops_tiles / (dt * flops_exact / (4 * w.d * pairs)) / 1e12)
     value = statistics.median(vals)
@@ -796,7 +803,7 @@ def reference_arm(args, world):
             "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "seq_len": w.seqlen_q,
                        "head_dim": w.d, "causal": True, "flops_per_step": flops_tiles},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
-                             "sample": "each step: 256 random causal rows of one head plane, fp64, scaled to "
+                             "sample": "each step: 2048 random causal rows of one head plane, fp64, scaled to "
                                        "the whole step by its exact pair count"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
