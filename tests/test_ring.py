@@ -248,3 +248,38 @@ def test_full_size_ring_last_rank_sampled():
     g = got.float().cpu().numpy()[idx[:, 0], idx[:, 1]]
     assert_close_bf16(g, ref[idx[:, 0], idx[:, 1]], what="full-size ring sample")
     assert torch.isfinite(got.float()).all()
+
+
+def test_fwd_acc_varlen_keys_in_two_sets():
+    """Varlen queries whose keys arrive as two packed sets with their own
+    per-sequence counts (cu_seqlens_k), merged in the epilogue, equal the
+    oracle's attention over each sequence's keys of both sets.  One sequence
+    has no keys in the first set."""
+    fa = _fa()
+    rng = np.random.default_rng(21)
+    hq, hkv, d = 4, 2, 128
+    q_lens, ka, kb = [100, 300, 1], [50, 0, 7], [130, 260, 200]
+    cu = lambda L: torch.tensor(np.concatenate([[0], np.cumsum(L)]), dtype=torch.int32)
+    q = _bf(rng, hq, sum(q_lens), d)
+    k1, v1 = _bf(rng, hkv, sum(ka), d), _bf(rng, hkv, sum(ka), d)
+    k2, v2 = _bf(rng, hkv, sum(kb), d), _bf(rng, hkv, sum(kb), d)
+    acc_o = torch.empty((hq, sum(q_lens), d), dtype=torch.float32, device="cuda")
+    acc_l = torch.empty((hq, sum(q_lens)), dtype=torch.float32, device="cuda")
+    epi = [("add", 0.25)]
+    common = dict(hq=hq, hkv=hkv, cu_seqlens_q=cu(q_lens).cuda(), max_seqlen_q=max(q_lens))
+    fa.attention_fwd_acc(q.cuda(), k1.cuda(), v1.cuda(), acc_o, acc_l, first=True, cu_seqlens_k=cu(ka).cuda(),
+                         max_seqlen_k=max(ka), **common)
+    out = fa.attention_fwd_acc(q.cuda(), k2.cuda(), v2.cuda(), acc_o, acc_l, last=True, epilogue=epi,
+                               cu_seqlens_k=cu(kb).cuda(), max_seqlen_k=max(kb), **common)
+    assert fa.check_device_error() == fa.FA_OK
+    # the oracle over each sequence's keys of both sets, concatenated per sequence
+    cq, ca_, cb_ = cu(q_lens).numpy(), cu(ka).numpy(), cu(kb).numpy()
+    ks, vs, ck = [], [], [0]
+    for b in range(len(q_lens)):
+        ks += [k1[:, ca_[b]:ca_[b + 1]], k2[:, cb_[b]:cb_[b + 1]]]
+        vs += [v1[:, ca_[b]:ca_[b + 1]], v2[:, cb_[b]:cb_[b + 1]]]
+        ck.append(ck[-1] + ka[b] + kb[b])
+    kc, vc = torch.cat(ks, dim=1), torch.cat(vs, dim=1)
+    ref = oracle.attention(q, kc, vc, hq=hq, hkv=hkv, epilogue=epi, cu_seqlens_q=cq,
+                           cu_seqlens_k=np.array(ck, dtype=np.int32))
+    assert_close_bf16(out.float().cpu().numpy(), ref)
