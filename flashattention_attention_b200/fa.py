@@ -176,6 +176,21 @@ def _fill_epilogue(arr, epilogue: Sequence[Tuple[str, float]]) -> int:
     return len(epilogue)
 
 
+def _shape(t, want, name: str):
+    """ValueError unless t has the shape `want` (None: any extent).  The C
+    ABI sees only pointers and sizes, so a tensor smaller than its sizes say
+    must be caught here, before a kernel reads past it."""
+    got = tuple(t.shape)
+    if len(got) != len(want) or any(w is not None and g != w for g, w in zip(got, want)):
+        shown = tuple("*" if w is None else w for w in want)
+        raise ValueError(f"{name} has shape {got}, expected {shown}")
+
+
+def _int32(t, name: str):
+    if t is not None and t.dtype != torch.int32:
+        raise ValueError(f"{name} must be int32")
+
+
 def _contig_cuda(t: torch.Tensor, name: str):
     if not t.is_cuda or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
@@ -201,6 +216,25 @@ def compress_kv(x: torch.Tensor, codes: Optional[torch.Tensor] = None,
 def fwd_params(q, k, v, out, *, hq, hkv, causal=False, window=0, scale=None, epilogue=(),
                k_scales=None, v_scales=None, cu_seqlens_q=None, cu_seqlens_k=None,
                max_seqlen_q=None, max_seqlen_k=None) -> FwdParams:
+    d = q.shape[-1]
+    if hq <= 0 or hkv <= 0:
+        raise ValueError("hq and hkv must be positive")
+    if cu_seqlens_q is None:
+        if len(q.shape) != 3 or q.shape[0] % hq:
+            raise ValueError(f"dense q must be [batch*hq, s_q, d]; got {tuple(q.shape)} with hq={hq}")
+        _shape(k, (q.shape[0] // hq * hkv, None, d), "k")
+    else:
+        _int32(cu_seqlens_q, "cu_seqlens_q")
+        _int32(cu_seqlens_k, "cu_seqlens_k")
+        _shape(q, (hq, None, d), "q")
+        _shape(k, (hkv, None, d), "k")
+        if cu_seqlens_k is not None:
+            _shape(cu_seqlens_k, (cu_seqlens_q.numel(),), "cu_seqlens_k")
+    _shape(v, tuple(k.shape), "v")
+    _shape(out, tuple(q.shape), "out")
+    for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        if t is not None:
+            _shape(t, tuple(k.shape[:2]), name)
     p = FwdParams()
     p.q, p.k, p.v, p.out = q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr()
     p.k_scales = None if k_scales is None else k_scales.data_ptr()
@@ -299,6 +333,14 @@ def attention_merge(o_acc: torch.Tensor, lse_acc: torch.Tensor, o_part: Optional
     merged rows after the epilogue.  As fa_attention_merge in fa.h."""
     _contig_cuda(o_acc, "o_acc")
     _contig_cuda(lse_acc, "lse_acc")
+    _shape(lse_acc, tuple(o_acc.shape[:-1]), "lse_acc")
+    if o_part is not None:
+        _shape(o_part, tuple(o_acc.shape), "o_part")
+        if lse_part is None:
+            raise ValueError("lse_part is required with o_part")
+        _shape(lse_part, tuple(lse_acc.shape), "lse_part")
+    if out is not None:
+        _shape(out, tuple(o_acc.shape), "out")
     p = MergeParams()
     p.o_acc, p.lse_acc = o_acc.data_ptr(), lse_acc.data_ptr()
     if o_part is not None:
@@ -315,6 +357,33 @@ def attention_merge(o_acc: torch.Tensor, lse_acc: torch.Tensor, o_part: Optional
     return out
 
 
+def _pool_shapes(k_pages, v_pages, k_scales, v_scales, hkv: int, d: int):
+    """Page pools [num_pages, hkv, page_size, d] and their scales
+    [num_pages, hkv, page_size]."""
+    _shape(k_pages, (None, hkv, None, d), "k_pages")
+    _shape(v_pages, tuple(k_pages.shape), "v_pages")
+    for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        if t is not None:
+            _shape(t, tuple(k_pages.shape[:3]), name)
+
+
+def _cache_shapes(q, k_cache, v_cache, k_scales, v_scales, cache_seqlens, out, hq: int, hkv: int):
+    """Decode operands: q [batch*hq, d] or [batch*hq, 1, d], dense caches
+    [batch*hkv, capacity, d] and scales [batch*hkv, capacity]."""
+    _int32(cache_seqlens, "cache_seqlens")
+    batch, d = cache_seqlens.numel(), q.shape[-1]
+    if q.numel() != batch * hq * d:
+        raise ValueError(f"q has shape {tuple(q.shape)}, expected batch*hq = {batch * hq} rows of {d}")
+    if k_cache is not None:
+        _shape(k_cache, (batch * hkv, None, d), "k_cache")
+        _shape(v_cache, tuple(k_cache.shape), "v_cache")
+        for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+            if t is not None:
+                _shape(t, tuple(k_cache.shape[:2]), name)
+    if out is not None:
+        _shape(out, tuple(q.shape), "out")
+
+
 def attention_fwd_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
                         cu_seqlens_k: torch.Tensor, block_table: torch.Tensor, *, hq: int, hkv: int,
                         causal: bool = False, window: int = 0, scale: Optional[float] = None,
@@ -328,6 +397,19 @@ def attention_fwd_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.T
     for name, t in (("q", q), ("k_pages", k_pages), ("v_pages", v_pages), ("cu_seqlens_k", cu_seqlens_k),
                     ("block_table", block_table)):
         _contig_cuda(t, name)
+    d = q.shape[-1]
+    _pool_shapes(k_pages, v_pages, k_scales, v_scales, hkv, d)
+    for name, t in (("cu_seqlens_k", cu_seqlens_k), ("block_table", block_table), ("cu_seqlens_q", cu_seqlens_q)):
+        _int32(t, name)
+    batch = cu_seqlens_k.numel() - 1
+    _shape(block_table, (batch, None), "block_table")
+    if cu_seqlens_q is None:
+        _shape(q, (batch * hq, None, d), "q")
+    else:
+        _shape(q, (hq, None, d), "q")
+        _shape(cu_seqlens_q, (batch + 1,), "cu_seqlens_q")
+    if out is not None:
+        _shape(out, tuple(q.shape), "out")
     if out is None:
         out = torch.empty_like(q)
     p = FwdParams()
@@ -387,6 +469,7 @@ def attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
     for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
                     ("cache_seqlens", cache_seqlens)):
         _contig_cuda(t, name)
+    _cache_shapes(q, k_cache, v_cache, k_scales, v_scales, cache_seqlens, out, hq, hkv)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
@@ -411,6 +494,10 @@ def attention_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torc
     for name, t in (("q", q), ("k_pages", k_pages), ("v_pages", v_pages), ("cache_seqlens", cache_seqlens),
                     ("block_table", block_table)):
         _contig_cuda(t, name)
+    _pool_shapes(k_pages, v_pages, k_scales, v_scales, hkv, q.shape[-1])
+    _cache_shapes(q, None, None, None, None, cache_seqlens, out, hq, hkv)
+    _int32(block_table, "block_table")
+    _shape(block_table, (cache_seqlens.numel(), None), "block_table")
     num_pages, _, page_size, d = k_pages.shape
     max_pages = block_table.shape[1]
     capacity = max_pages * page_size
@@ -437,6 +524,12 @@ def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v
     cache is quantised on the way in (scales required), a bf16 one stored
     as bf16.  cache_seqlens (device int32 [B]), if given, becomes cur_pos + 1.
     Layouts and semantics as fa_kv_append in fa.h."""
+    _append_shapes(k_new, v_new, cur_pos, cache_seqlens, hkv)
+    _shape(k_cache, (cur_pos.numel() * hkv, None, k_new.shape[-1]), "k_cache")
+    _shape(v_cache, tuple(k_cache.shape), "v_cache")
+    for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        if t is not None:
+            _shape(t, tuple(k_cache.shape[:2]), name)
     p = _append_params(k_new, v_new, k_cache, v_cache, cur_pos, hkv, k_scales, v_scales, cache_seqlens)
     _check(lib.fa_kv_append(ctypes.byref(p), _stream(stream)), "fa_kv_append")
 
@@ -447,11 +540,24 @@ def kv_append_paged(k_new: torch.Tensor, v_new: torch.Tensor, k_pages: torch.Ten
     """kv_append into page pools [num_pages, hkv, page_size, d] through a
     device int32 block_table [B, max_pages]; as fa_kv_append_paged in fa.h."""
     _contig_cuda(block_table, "block_table")
+    _append_shapes(k_new, v_new, cur_pos, cache_seqlens, hkv)
+    _pool_shapes(k_pages, v_pages, k_scales, v_scales, hkv, k_new.shape[-1])
+    _int32(block_table, "block_table")
+    _shape(block_table, (cur_pos.numel(), None), "block_table")
     p = _append_params(k_new, v_new, k_pages, v_pages, cur_pos, hkv, k_scales, v_scales, cache_seqlens)
     num_pages, _, page_size, d = k_pages.shape
     p.head_dim, p.capacity = d, block_table.shape[1] * page_size
     pg = KvPages(block_table.data_ptr(), block_table.shape[1], page_size, num_pages)
     _check(lib.fa_kv_append_paged(ctypes.byref(p), ctypes.byref(pg), _stream(stream)), "fa_kv_append_paged")
+
+
+def _append_shapes(k_new, v_new, cur_pos, cache_seqlens, hkv: int):
+    _int32(cur_pos, "cur_pos")
+    _int32(cache_seqlens, "cache_seqlens")
+    _shape(k_new, (cur_pos.numel() * hkv, None), "k_new")
+    _shape(v_new, tuple(k_new.shape), "v_new")
+    if cache_seqlens is not None:
+        _shape(cache_seqlens, (cur_pos.numel(),), "cache_seqlens")
 
 
 def _append_params(k_new, v_new, k_cache, v_cache, cur_pos, hkv, k_scales, v_scales, cache_seqlens):
@@ -505,10 +611,14 @@ def tq_compress(x: torch.Tensor, signs: torch.Tensor, levels: torch.Tensor, bits
     for name, t in (("x", x), ("signs", signs), ("levels", levels)):
         _contig_cuda(t, name)
     d = x.shape[-1]
+    _shape(signs, (d,), "signs")
+    _shape(levels, (1 << bits,), "levels")
     if codes is None:
         codes = torch.empty(x.shape[:-1] + (d * bits // 8,), dtype=torch.uint8, device=x.device)
     if norms is None:
         norms = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _shape(codes, tuple(x.shape[:-1]) + (d * bits // 8,), "codes")
+    _shape(norms, tuple(x.shape[:-1]), "norms")
     p = TqCompressParams()
     p.x, p.x_dtype, p.rows, p.head_dim, p.bits = x.data_ptr(), _DT[x.dtype], x.numel() // d if d else 0, d, bits
     p.signs, p.levels, p.codes, p.norms = signs.data_ptr(), levels.data_ptr(), codes.data_ptr(), norms.data_ptr()
@@ -535,7 +645,15 @@ def tq_attention_decode(q: torch.Tensor, k_codes: torch.Tensor, k_norms: torch.T
         _contig_cuda(t, name)
     d = q.shape[-1]
     batch = cache_seqlens.numel()
+    _cache_shapes(q, None, None, None, None, cache_seqlens, out, hq, hkv)
+    _shape(k_codes, (batch * hkv, None, d * k_bits // 8), "k_codes")
     cap = k_codes.shape[1]
+    _shape(v_codes, (batch * hkv, cap, d * v_bits // 8), "v_codes")
+    _shape(k_norms, (batch * hkv, cap), "k_norms")
+    _shape(v_norms, (batch * hkv, cap), "v_norms")
+    _shape(k_levels, (1 << k_bits,), "k_levels")
+    _shape(v_levels, (1 << v_bits,), "v_levels")
+    _shape(signs, (d,), "signs")
     if out is None:
         out = torch.empty_like(q)
     need = tq_decode_workspace_size(batch, hq, d, cap)

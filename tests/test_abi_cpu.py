@@ -402,3 +402,48 @@ def test_tq_rejects_bad_arguments(fa):
     assert dec(workspace_bytes=16) == fa.FA_ERR_WORKSPACE
     assert dec(n_epilogue=9) == fa.FA_ERR_INVALID
     assert dec(batch=0) == fa.FA_OK
+
+
+def test_binding_rejects_tensors_smaller_than_their_sizes_say(fa):
+    """The C ABI sees pointers and sizes only: the binding checks that every
+    tensor has the shape the sizes imply (and int32 index tensors), so a
+    kernel is never pointed past a tensor's end."""
+    import torch
+    F = FakeTensor
+    bf, i32, f32 = torch.bfloat16, torch.int32, torch.float32
+    q, k, o = F(0x1000, (4, 64, 128), bf), F(0x2000, (2, 64, 128), bf), F(0x3000, (4, 64, 128), bf)
+    fa.fwd_params(q, k, k, o, hq=4, hkv=2)  # consistent: accepted
+    with pytest.raises(ValueError):
+        fa.fwd_params(q, F(0x2000, (1, 64, 128), bf), k, o, hq=4, hkv=2)  # fewer K planes than batch*hkv
+    with pytest.raises(ValueError):
+        fa.fwd_params(q, k, F(0x2000, (2, 63, 128), bf), o, hq=4, hkv=2)  # V shorter than K
+    with pytest.raises(ValueError):
+        fa.fwd_params(q, k, k, F(0x3000, (4, 64, 64), bf), hq=4, hkv=2)   # out narrower than q
+    with pytest.raises(ValueError):
+        fa.fwd_params(q, k, k, o, hq=3, hkv=1)                             # batch*hq does not divide
+    with pytest.raises(ValueError):
+        fa.fwd_params(q, F(0x2000, (2, 64, 128), torch.int8), k, o, hq=4, hkv=2,
+                      k_scales=F(0x4000, (2, 32), f32))                     # scales of the wrong length
+    cu = F(0x5000, (3,), i32)
+    with pytest.raises(ValueError):
+        fa.fwd_params(F(0x1000, (4, 100, 128), bf), F(0x2000, (2, 90, 128), bf), F(0x2000, (2, 90, 128), bf),
+                      F(0x3000, (4, 100, 128), bf), hq=4, hkv=2, cu_seqlens_q=cu,
+                      cu_seqlens_k=F(0x6000, (4,), i32), max_seqlen_q=60)  # B + 1 entries differ
+    with pytest.raises(ValueError):
+        fa.fwd_params(F(0x1000, (4, 100, 128), bf), F(0x2000, (2, 90, 128), bf), F(0x2000, (2, 90, 128), bf),
+                      F(0x3000, (4, 100, 128), bf), hq=4, hkv=2, cu_seqlens_q=F(0x5000, (3,), torch.int64),
+                      max_seqlen_q=60)                                      # int64 offsets
+    lens = F(0x7000, (2,), i32)
+    fa._cache_shapes(F(0x1000, (8, 128), bf), F(0x2000, (4, 256, 128), bf), F(0x2000, (4, 256, 128), bf),
+                     None, None, lens, None, 4, 2)
+    with pytest.raises(ValueError):  # cache planes for one sequence only
+        fa._cache_shapes(F(0x1000, (8, 128), bf), F(0x2000, (2, 256, 128), bf), F(0x2000, (2, 256, 128), bf),
+                         None, None, lens, None, 4, 2)
+    with pytest.raises(ValueError):  # q rows for one sequence only
+        fa._cache_shapes(F(0x1000, (4, 128), bf), None, None, None, None, lens, None, 4, 2)
+    with pytest.raises(ValueError):  # float lengths
+        fa._cache_shapes(F(0x1000, (8, 128), bf), None, None, None, None, F(0x7000, (2,), f32), None, 4, 2)
+    with pytest.raises(ValueError):  # pools with the wrong KV head count
+        fa._pool_shapes(F(0x2000, (16, 3, 64, 128), bf), F(0x2000, (16, 3, 64, 128), bf), None, None, 2, 128)
+    with pytest.raises(ValueError):  # new rows for fewer sequences than cur_pos has
+        fa._append_shapes(F(0x1000, (2, 128), bf), F(0x1000, (2, 128), bf), F(0x7000, (2,), i32), None, 2)
