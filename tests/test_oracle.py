@@ -473,3 +473,39 @@ def test_merge_of_disjoint_key_sets_is_attention_over_their_union():
         acc_o, acc_lse = oracle.merge(acc_o, acc_lse, po, pl)
     assert np.allclose(acc_o, full_o, rtol=1e-12, atol=1e-12)
     assert np.allclose(acc_lse, full_lse, rtol=1e-12, atol=1e-12)
+
+
+_REAL_LSE, _REAL_MERGE = oracle.attention_lse, oracle.merge
+
+
+def _lse_log2_units(*a, **k):
+    o, lse = _REAL_LSE(*a, **k)
+    return o, lse * np.log2(np.e)
+
+
+def _merge_swapped(o_a, lse_a, o_b, lse_b):
+    # each side weighted by the other's share
+    o, lse = _REAL_MERGE(o_a, lse_a, o_b, lse_b)
+    la, lb = np.asarray(lse_a, np.float64), np.asarray(lse_b, np.float64)
+    fin = np.isfinite(lse)
+    safe = np.where(fin, lse, 0.0)
+    wa = np.where(fin, np.exp(lb - safe), 0.0)
+    wb = np.where(fin, np.exp(la - safe), 0.0)
+    return np.asarray(o_a, np.float64) * wa[..., None] + np.asarray(o_b, np.float64) * wb[..., None], lse
+
+
+def _merge_max_lse(o_a, lse_a, o_b, lse_b):
+    o, _ = _REAL_MERGE(o_a, lse_a, o_b, lse_b)
+    return o, np.maximum(np.asarray(lse_a, np.float64), np.asarray(lse_b, np.float64))
+
+
+@pytest.mark.parametrize("name,attr,wrong,pin", [
+    ("lse in log2 units", "attention_lse", _lse_log2_units, "test_attention_lse_matches_attention_and_logsumexp"),
+    ("merge weights swapped", "merge", _merge_swapped, "test_merge_of_disjoint_key_sets_is_attention_over_their_union"),
+    ("merged lse = max", "merge", _merge_max_lse, "test_merge_of_disjoint_key_sets_is_attention_over_their_union"),
+])
+def test_a_planted_partial_result_mistake_fails_a_pin(monkeypatch, name, attr, wrong, pin):
+    """Mistakes planted in the partial-result oracle fail its pins."""
+    monkeypatch.setattr(oracle, attr, wrong)
+    with pytest.raises(AssertionError):
+        globals()[pin]()
