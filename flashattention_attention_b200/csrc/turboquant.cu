@@ -85,17 +85,6 @@ __device__ __forceinline__ void warp_fwht(float (&v)[E], int lane) {
   }
 }
 
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-  for (int h = 16; h > 0; h >>= 1) x += __shfl_xor_sync(0xffffffffu, x, h);
-  return x;
-}
-__device__ __forceinline__ float warp_max(float x) {
-#pragma unroll
-  for (int h = 16; h > 0; h >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, h));
-  return x;
-}
-
 // b-bit code starting at bit `pos` of the little-endian word array w (pos
 // and B compile-time after unrolling; a code may straddle two words).
 template <int B, int NW>
