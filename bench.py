@@ -50,6 +50,8 @@ def load_peaks():
 
 KERNEL_SOURCES = {
     "prefill_tc_kernel<128,bf16>": ["prefill_tc.cu", "umma.cuh", "device.cuh", "layout.cuh"],
+    "prefill_tc_kernel<128,int8>": ["prefill_tc.cu", "umma.cuh", "device.cuh", "layout.cuh"],
+    "prefill_tc_kernel<64,bf16>": ["prefill_tc.cu", "umma.cuh", "device.cuh", "layout.cuh"],
     "decode_sk_kernel<128>": ["decode.cu", "device.cuh"],
     "compress_rows8_kernel<bf16,16>": ["quant.cu", "device.cuh"],
 }
@@ -279,6 +281,15 @@ def max_over_ranks(x: float, dist, torch, device) -> float:
     return float(t.item())
 
 
+def prefill_config(w, flops_tiles, flops_exact, world):
+    """The headline step's config (the same dict on both arms)."""
+    return {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "seq_len": w.seqlen_q,
+            "head_dim": w.d, "causal": True, "window": 0, "epilogue": [],
+            "flops_per_step": flops_tiles, "flops_counting": "128x128 tiles intersecting the band",
+            "flops_exact_pairs": flops_exact, "l2": "inputs larger than L2 (201 MB), no flush",
+            "parallelism": f"replicas x{world} (no collective)"}
+
+
 def gpu_arm(args, rank, world, dist):
     import torch
     from flashattention_attention_b200 import fa, inputs
@@ -335,11 +346,7 @@ def gpu_arm(args, rank, world, dist):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1), numpy PCG64 -> fp32 -> bf16)",
-        "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "seq_len": w.seqlen_q,
-                   "head_dim": w.d, "causal": True, "window": 0, "epilogue": [],
-                   "flops_per_step": flops_tiles, "flops_counting": "128x128 tiles intersecting the band",
-                   "flops_exact_pairs": flops_exact, "l2": "inputs larger than L2 (201 MB), no flush",
-                   "parallelism": f"replicas x{world} (no collective)"},
+        "config": prefill_config(w, flops_tiles, flops_exact, world),
         "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel<128,bf16>", "achieved": round(tflops, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(tflops / peaks["bf16_tflops"], 4),
@@ -361,7 +368,25 @@ def gpu_arm(args, rank, world, dist):
         turboquant_decode(args, dev, peaks, world, dist, result)
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, flops_tiles, flops_exact, args.cpu_seconds)
+    summarise(result)
     return result
+
+
+def summarise(result):
+    """A compact {workload: roofline fraction} table of every timed line,
+    kept inside the headline roofline object and repeated as the line's last
+    key (both places survive a reader that keeps only known keys or the end
+    of the line)."""
+    table = {"gqa_causal_prefill": {"frac": result["roofline"]["frac"], "achieved": result["roofline"]["achieved"],
+                                    "unit": result["roofline"]["unit"]}}
+    for key, val in result.items():
+        if isinstance(val, dict) and isinstance(val.get("roofline"), dict) and "frac" in val["roofline"]:
+            rf = val["roofline"]
+            table[key] = {"frac": rf["frac"], "achieved": rf["achieved"], "unit": rf["unit"]}
+            if "frac_of_nominal_8000" in rf:
+                table[key]["frac_of_nominal_8000"] = rf["frac_of_nominal_8000"]
+    result["roofline"]["all_workloads"] = table
+    result["summary"] = table
 
 
 def paged_prefill(args, w, flops_tiles, peaks, world, dist, dev):
@@ -433,18 +458,23 @@ def varlen_prefill(args, dev, peaks, world, dist, result, steps):
                                                 max_seqlen_q=max(w.lengths), out=out),
                        steps, args.warmup, torch, dist)
     ft, fe = varlen_flops(w)
+    tf = ft / (ms * 1e-3) / 1e12
     result["varlen_window_prefill"] = {
-        "workload": w.name, "lengths": w.lengths, "value": round(fe / (ms * 1e-3) / 1e12 * world, 2),
-        "unit": "TFLOP/s", "flops_counting": "exact visible pairs", "flops_per_step": fe,
-        "flops_tile_count": ft, "ms_per_step": round(ms, 4),
-        "frac_of_bf16_peak": round(fe / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
+        "workload": w.name, "lengths": w.lengths, "value": round(tf * world, 2), "unit": "TFLOP/s",
+        "flops_counting": "128x128 tiles intersecting the band", "flops_per_step": ft,
+        "flops_exact_pairs": fe, "exact_pairs_tflops": round(fe / (ms * 1e-3) / 1e12, 2),
+        "ms_per_step": round(ms, 4),
+        "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel<64,bf16>", "achieved": round(tf, 2),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(tf / peaks["bf16_tflops"], 4),
+                     "traffic": measured_traffic("prefill_tc_kernel<64,bf16>")}}
     del q, k, v, out
 
 
 def int8_long_prefill(args, dev, peaks, world, dist, result, steps):
     import torch
     from flashattention_attention_b200 import fa, inputs
-    w = inputs.int8kv_long_prefill()
+    w = inputs.int8kv_long_prefill(s=8192) if args.profile_small else inputs.int8kv_long_prefill()
     kc, ks = fa.compress_kv(w.k.to(dev))
     vc, vs = fa.compress_kv(w.v.to(dev))
     q = w.q.to(dev)
@@ -460,7 +490,8 @@ def int8_long_prefill(args, dev, peaks, world, dist, result, steps):
         "flops_exact_pairs": fe, "ms_per_step": round(ms, 4),
         "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel<128,int8>", "achieved": round(tf, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None}}
+                     "frac": round(tf / peaks["bf16_tflops"], 4),
+                     "traffic": measured_traffic("prefill_tc_kernel<128,int8>")}}
     del q, kc, vc, ks, vs, out
     torch.cuda.empty_cache()
 
@@ -764,47 +795,86 @@ def _cores():
     return int(os.environ.get("OMP_NUM_THREADS", cores))
 
 
+def _oracle_rows_for(w, seconds, seed):
+    """Rows of an oracle sample that takes about `seconds` on these cores:
+    calibrated on 1024 rows (enough that fixed costs do not dominate), then
+    re-measured once at the estimated size."""
+    n = 1024
+    dt, _ = _oracle_sample(w, n, seed)
+    for s in (seed + 1, seed + 2):
+        n = int(min(4_000_000, max(1024, n * seconds / max(dt, 1e-4))))
+        dt, _ = _oracle_sample(w, n, s)
+        if dt >= 0.5 * seconds:
+            break
+    return int(min(4_000_000, max(1024, n * seconds / max(dt, 1e-4))))
+
+
+def _oracle_rate(w, flops_tiles, flops_exact, dt, pairs):
+    """The sample's rate expressed in the step's metric: TFLOP/s of the
+    whole step (tile count) if the oracle ran it at the sample's pace."""
+    return flops_tiles / (dt * flops_exact / (4 * w.d * pairs)) / 1e12
+
+
+def _single_core_rate(w, flops_tiles, flops_exact, seconds):
+    """The same oracle on one core (a child process with OMP_NUM_THREADS=1,
+    so the thread count is fixed before its OpenMP runtime starts)."""
+    code = ("import json, sys; sys.path.insert(0, %r); import bench; from flashattention_attention_b200 import inputs; "
+            "w = inputs.gqa_causal_prefill(); n = bench._oracle_rows_for(w, %f, 11); "
+            "dt, pairs = bench._oracle_sample(w, n, 14); print(json.dumps([n, dt, pairs]))" % (ROOT, seconds))
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    try:
+        r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                           timeout=30 * seconds + 120)
+        n, dt, pairs = json.loads(r.stdout.strip().splitlines()[-1])
+    except Exception as e:  # reported, never fatal to the GPU line
+        return {"error": f"single-core sample failed: {type(e).__name__}"}
+    return {"value": _oracle_rate(w, flops_tiles, flops_exact, dt, pairs), "unit": "TFLOP/s", "cores": 1,
+            "sample": f"{n} random causal rows of one head plane ({pairs} visible pairs, {dt:.2f} s)"}
+
+
 def cpu_baseline(w, flops_tiles, flops_exact, budget_s):
     """The oracle on the host cores over a bounded sample (about budget_s
-    seconds of CPU work), scaled to the whole step by the exact pair count."""
-    # calibrate on enough rows that fixed costs do not dominate, then size
-    # the sample to the budget (once more if it still came out short)
-    n = 1024
-    dt, pairs = _oracle_sample(w, n, 1)
-    for seed in (2, 3):
-        n = int(min(4_000_000, max(1024, n * budget_s / max(dt, 1e-4))))
-        dt, pairs = _oracle_sample(w, n, seed)
-        if dt >= 0.5 * budget_s:
-            break
+    seconds of CPU work) sized exactly as the reference arm sizes its steps,
+    scaled to the whole step by the exact pair count; and on one core."""
+    n = _oracle_rows_for(w, budget_s, 1)
+    dt, pairs = _oracle_sample(w, n, 4)
     full_s = dt * flops_exact / (4 * w.d * pairs)
     return {"value": flops_tiles / full_s / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
             "sample": f"{n} random causal rows of one head plane ({pairs} visible pairs, {dt:.2f} s of fp64 "
                       f"CPU work), scaled to the whole step by its exact pair count",
-            "seconds_sampled": round(dt, 3)}
+            "seconds_sampled": round(dt, 3),
+            "single_core": _single_core_rate(w, flops_tiles, flops_exact, max(2.0, budget_s / 4))}
 
 
 def reference_arm(args, world):
-    """The oracle timed on host cores on this arm's workload, metric and unit;
-    each step is a bounded sample of 2048 rows (large enough that the call's
-    fixed costs do not dominate) scaled by the exact pair count."""
+    """The oracle timed on host cores on this arm's workload, metric and unit.
+    Every step is the same bounded sample size (rows chosen once, during
+    warm-up, so a step takes about --ref-step-seconds), and the line's
+    ms_per_step is the measured time of those sampled steps; value is the
+    sampled rate expressed for the whole step (exact pair count scaling)."""
     from flashattention_attention_b200 import inputs
     w = inputs.gqa_causal_prefill()
     flops_tiles, flops_exact = prefill_flops(w)
-    vals = []
+    n = _oracle_rows_for(w, args.ref_step_seconds, 1)
+    times, rates = [], []
     for s in range(args.warmup + args.steps):
-        dt, pairs = _oracle_sample(w, 2048, 100 + s)
+        dt, pairs = _oracle_sample(w, n, 100 + s)
         if s >= args.warmup:
-            vals.append(flops_tiles / (dt * flops_exact / (4 * w.d * pairs)) / 1e12)
-    value = statistics.median(vals)
+            times.append(dt)
+            rates.append(_oracle_rate(w, flops_tiles, flops_exact, dt, pairs))
+    value = statistics.median(rates)
+    ms = statistics.mean(times) * 1e3
+    sample = (f"each step: {n} random causal rows of one head plane, fp64 (about {args.ref_step_seconds:g} s), "
+              f"scaled to the whole step by its exact pair count")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": flops_tiles / (value * 1e12) * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "ms_per_step_is": "measured time of one sampled step (not the whole workload)",
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded N(0,1), numpy PCG64 -> fp32 -> bf16)",
-            "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "seq_len": w.seqlen_q,
-                       "head_dim": w.d, "causal": True, "flops_per_step": flops_tiles},
+            "config": prefill_config(w, flops_tiles, flops_exact, world),
+            "rows_per_sampled_step": n,
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
-                             "sample": "each step: 2048 random causal rows of one head plane, fp64, scaled to "
-                                       "the whole step by its exact pair count"},
+                             "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -815,7 +885,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=2.0,
+                    help="oracle seconds per sampled step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-small", action="store_true",
+                    help="profiler captures: the int8-KV long prefill at S=8192 (same kernel, inputs still "
+                         "larger than L2)")
     ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "quant", "prefill_int8", "varlen", "ring", "tq"],
                     help="time one part only (used for profiler captures)")
     args = ap.parse_args()

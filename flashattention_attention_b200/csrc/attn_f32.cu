@@ -1,23 +1,23 @@
 // attn_f32.cu -- fp32 attention on the CUDA cores, and the empty-band rows.
 //
 // attn_f32_kernel: the correctness tier for fp32 inputs (fkl_python PR #6,
-// Verification, "FA dense d64 causal (err=1.5e-07)": fp32 error levels need
-// fp32 products, so no TF32 tensor cores here).  Same masks, GQA, varlen and
+// Verification: the dense causal check at head size 64 reaches errors near
+// 1e-7, which needs fp32 products, so no TF32 tensor cores here).  Same masks, GQA, varlen and
 // epilogue semantics as the tensor-core path.  A CTA owns 32 query rows of one
 // (sequence, q-head); four threads share a row, each holding every 16th group
 // of 4 dims, so the K/V tiles in shared memory are read without bank
 // conflicts.  Keys stream in tiles of 32 through an online softmax (running
 // max m and sum l in fp32, exp2 with log2(e) folded into the scale).
-// With an int8 KV cache (fkl_python PR #6, Verification, "FA int8-KV exact
-// vs dequantized oracle") each K/V element enters the shared tile as c * s
+// With an int8 KV cache (fkl_python PR #6, Verification: int8-cache
+// attention checked against an oracle on the dequantised cache) each K/V element enters the shared tile as c * s
 // computed in fp32, which is exact (|c| <= 127 times an fp32 scale), so the
 // kernel sees the dequantised cache itself.
 //
 // empty_rows_kernel: rows whose band is empty (causal with s_q > s_k leaves
 // rows i < s_q - s_k without keys; s_k = 0 leaves every row without keys)
 // get uniform weights over all s_k keys, i.e. the mean of V, zeros for s_k =
-// 0 (SKaiNET-transformers PR #419, Summary: "empty sliding-window bands
-// reproduce the engine's uniform softmax"), then the epilogue.  The main
+// 0 (SKaiNET-transformers PR #419, Summary: a sliding-window row whose band
+// holds no key falls back to the uniform softmax), then the epilogue.  The main
 // kernels skip those rows.  Partial results (an lse output) or an
 // accumulator to merge into give such rows no weight instead.
 #include "internal.h"

@@ -1,7 +1,7 @@
 // decode.cu -- single-query decode over a KV cache, split along the keys
-// (fkl_python PR #6, Verification: "FA decode step s_q=1 vs s_k=256 int8";
-// Summary: the int8 cache is dequantised in-register and never inflated in
-// global memory; kernbench2 commit ADR-0060: decode splits the keys and
+// (fkl_python PR #6, Verification: a one-query decode step over 256 int8 keys;
+// Summary: the kernel dequantises the int8 cache on chip, with no widened
+// copy in global memory; kernbench2 commit ADR-0060: decode splits the keys and
 // reduces the partial softmax states (m, l, O) to one output).
 //
 // Work decomposition (stream-K): the 32-key tiles of every (sequence, KV
@@ -224,12 +224,15 @@ __device__ __forceinline__ int effective_workers(const SkArgs& A, long long T) {
 
 // ---------------------------------------------------------------- plan
 // prefix[b] = sum over earlier sequences of (tiles x hkv); prefix[B] = T.
+// A length outside [0, cap] is clamped (every kernel of the call clamps it
+// the same way) and reported in the status word.
 template <int D>
 __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __restrict__ seqlens, int batch,
                                                            int hq, int hkv, int cap, int window,
                                                            int32_t* __restrict__ prefix,
                                                            int32_t* __restrict__ counters,
-                                                           __nv_bfloat16* __restrict__ out, Epilogue epi) {
+                                                           __nv_bfloat16* __restrict__ out, Epilogue epi,
+                                                           unsigned int* status) {
   griddep_launch_dependents();
   __shared__ int32_t warp_sums[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -237,7 +240,13 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   const int per = (batch + nthreads - 1) / nthreads;
   const int b0 = min(batch, tid * per), b1 = min(batch, b0 + per);
   int32_t local = 0;
-  for (int b = b0; b < b1; ++b) local += tiles_of(clamp_len(seqlens[b], cap), window) * hkv;
+  bool bad = false;
+  for (int b = b0; b < b1; ++b) {
+    const int L = seqlens[b];
+    bad |= L < 0 || L > cap;
+    local += tiles_of(clamp_len(L, cap), window) * hkv;
+  }
+  if (bad) atomicOr(status, kStatusRange);
   int32_t incl = local;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -891,7 +900,7 @@ fa_status launch_sk(const fa_decode_params& p, const fa_kv_pages* pages, int n_w
     note_variant(reinterpret_cast<const void*>(kern));
   }
   plan<<<1, 1024, 0, ctx.stream>>>(p.cache_seqlens, p.batch, p.hq, p.hkv, p.capacity, p.window,
-                                   reinterpret_cast<int32_t*>(base), A.counters, A.out, A.epi);
+                                   reinterpret_cast<int32_t*>(base), A.counters, A.out, A.epi, ctx.wd.word);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   A.smem_prefix = p.batch <= G::kPrefixCap ? 1 : 0;
   const size_t smem = G::kSmem + (A.smem_prefix ? (static_cast<size_t>(p.batch) + 1) * 4 : 0);
@@ -967,21 +976,26 @@ namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
 static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[kNoAllocScratchBytes];
-// Watchdog word of this path (the library's shared status word is allocated
-// lazily, which this path must not do).
+// Status word of this path (the library's shared status word is allocated
+// lazily, which this path must not do): a bounded wait that gave up, or a
+// cache length outside [0, capacity].  fa_check_device_error reads and
+// clears it.
 static __device__ unsigned int g_decode_noalloc_status;
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};
+void* g_noalloc_word[64] = {};
 
 // Device addresses of the scratch array and status word for the current
 // device.  The first call on each device looks them up (cudaGetSymbolAddress,
 // with that device current); later calls reuse them.
 fa_status noalloc_scratch(void** scratch, unsigned int** status) {
-  static std::mutex mu;
-  static void* addr[64] = {};
-  static void* word[64] = {};
+  void** addr = g_noalloc_addr;
+  void** word = g_noalloc_word;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   if (dev < 0 || dev >= 64) return FA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(mu);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
   if (addr[dev] == nullptr) {
     void* p = nullptr;
     void* w = nullptr;
@@ -998,6 +1012,29 @@ fa_status noalloc_scratch(void** scratch, unsigned int** status) {
 }  // namespace
 
 size_t decode_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// Status bits the no-alloc decode recorded on the current device since the
+// last read, cleared as they are read (0 before its first call there).  The
+// caller has synchronised the stream; the copies are plain synchronous
+// cudaMemcpy calls, which allocate nothing.
+fa_status take_noalloc_status(unsigned int* bits) {
+  *bits = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return FA_OK;
+  unsigned int* word = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    word = static_cast<unsigned int*>(g_noalloc_word[dev]);
+  }
+  if (word == nullptr) return FA_OK;
+  if (cudaMemcpy(bits, word, sizeof(*bits), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+  if (*bits != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
 
 // Workers that fit the scratch: plan + (B*hkv + P) * G * (d + 2) floats;
 // 0 when not even one CTA of workers fits.

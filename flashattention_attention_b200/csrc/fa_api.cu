@@ -391,28 +391,12 @@ fa_status fa_attention_decode_paged(const fa_decode_params* p, const fa_kv_pages
 }
 
 fa_status fa_attention_decode_noalloc(const fa_decode_params* p, fa_stream_t stream) {
-  if (p == nullptr) return FA_ERR_INVALID;
-  if (p->batch < 0 || p->hq <= 0 || p->hkv <= 0 || p->hq % p->hkv != 0) return FA_ERR_INVALID;
-  if (p->capacity <= 0 || p->capacity % 32 != 0) return FA_ERR_INVALID;
-  if (p->max_seqlen < 0 || p->max_seqlen > p->capacity) return FA_ERR_INVALID;
-  if (p->split_keys < 0 || p->split_keys % 256 != 0) return FA_ERR_INVALID;
-  if (!epilogue_ok(p->epilogue, p->n_epilogue)) return FA_ERR_INVALID;
-  if (!std::isfinite(p->softmax_scale)) return FA_ERR_INVALID;
-  if (p->kv_dtype != FA_I8 && p->kv_dtype != FA_BF16) return FA_ERR_INVALID;
-  if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
-  if (p->head_dim != 64 && p->head_dim != 128) return FA_ERR_UNSUPPORTED;
-  if (p->hq / p->hkv > 8) return FA_ERR_UNSUPPORTED;
+  fa_status st = decode_args(p);
+  if (st != FA_OK) return st;
   if (p->kv_dtype != FA_I8) return FA_ERR_UNSUPPORTED;
   if (p->batch == 0) return FA_OK;
-  if (p->q == nullptr || p->k_cache == nullptr || p->v_cache == nullptr || p->out == nullptr ||
-      p->cache_seqlens == nullptr || p->k_scales == nullptr || p->v_scales == nullptr)
-    return FA_ERR_INVALID;
-  if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->out) ||
-      !aligned16(p->k_scales) || !aligned16(p->v_scales))
-    return FA_ERR_INVALID;
   if (decode_noalloc_workers(p->batch, p->hq, p->hkv, p->head_dim) < 4) return FA_ERR_WORKSPACE;
-  const int split = p->split_keys;
-  return launch_decode_noalloc(*p, split, watchdog_budget(), reinterpret_cast<cudaStream_t>(stream));
+  return launch_decode_noalloc(*p, p->split_keys, watchdog_budget(), reinterpret_cast<cudaStream_t>(stream));
 }
 
 namespace {
@@ -515,16 +499,27 @@ fa_status fa_tq_attention_decode(const fa_tq_decode_params* p, fa_stream_t strea
 }
 
 fa_status fa_check_device_error(fa_stream_t stream) {
-  unsigned int* word = nullptr;
-  fa_status st = status_word(&word);
-  if (st != FA_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
-  unsigned int host = 0;
-  if (cudaMemcpy(&host, word, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
-  if (host != 0) {
-    const unsigned int zero = 0;
-    if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
+  // the shared word exists once some entry point has launched on this
+  // device; before that there is nothing to read (and nothing is allocated)
+  unsigned int* word = nullptr;
+  if (dev >= 0 && dev < kMaxDevices) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    word = g_status[dev];
   }
+  unsigned int host = 0;
+  if (word != nullptr) {
+    if (cudaMemcpy(&host, word, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+    if (host != 0) {
+      const unsigned int zero = 0;
+      if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
+    }
+  }
+  unsigned int noalloc = 0;
+  if (take_noalloc_status(&noalloc) != FA_OK) return FA_ERR_CUDA;
+  host |= noalloc;
   if (host & kStatusTimeout) return FA_ERR_TIMEOUT;
   if (host & kStatusRange) return FA_ERR_INVALID;
   return FA_OK;

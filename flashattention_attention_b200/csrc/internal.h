@@ -53,6 +53,7 @@ size_t decode_workspace_bytes(int batch, int hq, int head_dim);
 int decode_noalloc_workers(int batch, int hq, int hkv, int head_dim);
 fa_status launch_decode_noalloc(const fa_decode_params& p, int split_keys, long long budget, cudaStream_t stream);
 size_t decode_noalloc_scratch_bytes();
+fa_status take_noalloc_status(unsigned int* bits);
 fa_status launch_watchdog_selftest(unsigned long long budget, const LaunchCtx& ctx);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).

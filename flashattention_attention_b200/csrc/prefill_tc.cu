@@ -45,8 +45,8 @@
 // exact), rescale O_t in TMEM when it did, write P_t, signal the MMA warp.
 // Every wait is bounded (device.cuh); a timeout aborts all roles cleanly.
 //
-// int8 K/V (fkl_python PR #6, Summary: "dequantizes in-register inside q.k
-// and p.v; the compressed cache is never inflated in global memory"): TMA
+// int8 K/V (fkl_python PR #6, Summary: the fused kernel dequantises on chip
+// for both products and never widens the cache in global memory): TMA
 // brings each int8 tile into shared memory (at d = 128 into the upper half of
 // the bf16 slot it becomes); four converter warps, one thread per key row,
 // dequantise it as c * s in fp32 (exact: |c| <= 127 times an fp32 scale),

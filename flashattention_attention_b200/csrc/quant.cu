@@ -1,5 +1,5 @@
-// quant.cu -- per-row int8 KV quantiser (fkl_python PR #6, Summary,
-// "compress_kv(): GPU-side per-token int8 quantization (one fp32 scale/token)").
+// quant.cu -- per-row int8 KV quantiser (fkl_python PR #6, Summary: the
+// cache compressed on the GPU to int8 codes per token, one fp32 scale each).
 //
 // One warp per row.  Each lane holds 4 consecutive elements per 128-element
 // chunk (8-byte bf16 / 16-byte fp32 vector loads, fully coalesced), the warp

@@ -56,9 +56,9 @@ typedef enum {
     FA_I8 = 2    /* int8 codes, with one fp32 scale per row (token, kv-head) */
 } fa_dtype;
 
-/* Epilogue ops (fkl_python PR #6, Summary: "epilogue=[ops]: any fkl compute
- * ops run in-register on the attention output inside the same kernel";
- * example [Mul(2.0), Add(0.5)]).  They are applied to the normalised fp32
+/* Epilogue ops (fkl_python PR #6, Summary: a list of elementwise ops that
+ * the attention kernel itself applies to its output in registers; example
+ * [Mul(2.0), Add(0.5)]).  They are applied to the normalised fp32
  * output in list order, each rounded to fp32 (no fused multiply-add), before
  * the cast to the output dtype.  Values are plain kernel arguments, so
  * changing them -- or the list's shape -- never compiles anything. */
@@ -70,9 +70,9 @@ typedef struct {
 } fa_epi_op;
 
 /*
- * fa_compress_kv -- per-row int8 quantisation (fkl_python PR #6, Summary,
- * "compress_kv(): GPU-side per-token int8 quantization (one fp32
- * scale/token)").
+ * fa_compress_kv -- per-row int8 quantisation (fkl_python PR #6, Summary:
+ * the KV cache compressed on the GPU to int8 codes per token, with one fp32
+ * scale per token).
  *   x       [rows, d] FA_BF16 or FA_F32, row-major.  A row is one (token,
  *           kv-head) vector; K and V are compressed by separate calls.
  *   codes   [rows, d] int8 out;  scales [rows] fp32 out.
@@ -86,8 +86,9 @@ FA_API fa_status fa_compress_kv(const void *x, fa_dtype x_dtype, int64_t rows, i
                          int8_t *codes, float *scales, fa_stream_t stream);
 
 /*
- * Forward attention parameters (fkl_python PR #6, Summary: layout
- * (batch*heads, seq, head_dim), fp32 accumulation, head_dim multiple of 32).
+ * Forward attention parameters (fkl_python PR #6, Summary: tensors laid out
+ * as (batch*heads, seq, head_dim), accumulation in fp32, head sizes that are
+ * multiples of 32).
  *
  * out = softmax(scale * q k^T + mask) v, then the epilogue chain.
  *
@@ -106,8 +107,8 @@ FA_API fa_status fa_compress_kv(const void *x, fa_dtype x_dtype, int64_t rows, i
  *     window <= 0 means no window.
  * A row with no visible key gets uniform weights over all s_k keys of its
  * sequence (the mean of V; zeros when s_k = 0) -- SKaiNET-transformers
- * PR #419, Summary, "empty sliding-window bands reproduce the engine's
- * uniform softmax".
+ * PR #419, Summary: a sliding-window row whose band holds no key falls back
+ * to the engine's uniform softmax.
  * dtypes: q_dtype FA_F32 (CUDA-core fp32 path; kv_dtype FA_F32 or FA_I8) or
  * FA_BF16 (tensor-core path; kv_dtype FA_BF16 or FA_I8).  FA_I8 K/V come
  * with k_scales/v_scales [batch*hkv, seqlen_k] dense or [hkv, total_k]
@@ -145,14 +146,17 @@ typedef struct {
 FA_API fa_status fa_attention_fwd(const fa_fwd_params *p, fa_stream_t stream);
 
 /*
- * Single-query decode against a KV cache (fkl_python PR #6, Verification,
- * "FA decode step s_q=1 vs s_k=256 int8"; Summary: the compressed cache is
- * dequantised in-register and never inflated in global memory).
+ * Single-query decode against a KV cache (fkl_python PR #6, Verification:
+ * a one-query decode step over 256 int8-cached keys; Summary: the kernel
+ * dequantises the compressed cache on chip, with no widened copy in global
+ * memory).
  *   q        [batch*hq, d] bf16 (one query per sequence and head)
  *   k_cache, v_cache [batch*hkv, capacity, d], kv_dtype FA_I8 (with k_scales,
  *            v_scales [batch*hkv, capacity] fp32) or FA_BF16
  *   cache_seqlens  device int32 [batch]: sequence b attends to keys
- *            0 .. L_b-1 (the current token already appended), 0 <= L_b <= capacity
+ *            0 .. L_b-1 (the current token already appended), 0 <= L_b <= capacity;
+ *            an L_b outside that range is clamped into it and reported by
+ *            fa_check_device_error as FA_ERR_INVALID
  *   out      [batch*hq, d] bf16
  * The query sits at position L_b - 1, so every cached key is visible; a
  * window W > 0 keeps the last W.  L_b = 0 gives the epilogue applied to zeros.
@@ -198,8 +202,8 @@ FA_API fa_status fa_attention_decode(const fa_decode_params *p, fa_stream_t stre
  * fa_attention_decode_paged -- fa_attention_decode over a paged cache, so a
  * serving loop hands the kernel its cache pages in place instead of copying
  * each sequence's prefix into a contiguous buffer (SKaiNET-transformers
- * PR #419, Summary: the positional KV caches "hand the kernel copy-free views
- * instead of copying the whole prefix per layer per token").
+ * PR #419, Summary: the positional KV caches give the kernel views of the
+ * cached prefix where it lies, with no per-token copy).
  *   k_cache, v_cache  page pools [num_pages, hkv, page_size, d] (FA_I8 codes
  *                     with k_scales, v_scales [num_pages, hkv, page_size], or FA_BF16)
  *   block_table       device int32 [batch, max_pages]: key j of sequence b
@@ -316,11 +320,11 @@ FA_API fa_status fa_attention_merge(const fa_merge_params *p, fa_stream_t stream
 
 /*
  * fa_kv_append -- write one new token per sequence into a decode KV cache,
- * quantising on the way in (FlashRT QKV Cache RoPE, Kernels:
- * "decode_k_norm_rope_kvwrite_devpos_bf16 ... selects the cache slot from a
- * CUDA int32 cur_pos tensor for graph-friendly decode"; here without the norm
- * and rotation, and with the int8 cache of fkl_python PR #6, Summary,
- * "compressed int8 KV cache (per-token, one fp32 scale/token)").
+ * quantising on the way in (FlashRT QKV Cache RoPE, Kernels: the
+ * decode_k_norm_rope_kvwrite_devpos_bf16 kernel reads its cache slot from a
+ * device-side int32 position, so a captured decode graph can replay it; here
+ * without the norm and rotation, and with the int8 cache of fkl_python PR #6,
+ * Summary: per-token int8 codes with one fp32 scale per token).
  *   k_new, v_new  [batch*hkv, d] x_dtype (FA_BF16 or FA_F32): the new token's
  *                 K and V rows, row u = b * hkv + g
  *   k_cache, v_cache [batch*hkv, capacity, d] cache_dtype: FA_I8 codes (with
@@ -396,9 +400,12 @@ FA_API fa_status fa_kv_append_paged(const fa_kv_append_params *p, const fa_kv_pa
  *   - All calls on a device share the scratch and it keeps the last call's
  *     contents (nothing in it needs clearing).  Calls that overlap on the GPU
  *     race on it: serialise them (one stream, or events between streams).
- *   - A bounded device wait that gives up inside this call is recorded in a
- *     status word of this entry point's own (the shared one is allocated on
- *     first use), which fa_check_device_error does not read.
+ *   - A bounded device wait that gives up inside this call, or a cache
+ *     length outside [0, capacity], is recorded in a status word of this
+ *     entry point's own (a statically allocated device word: the library's
+ *     shared one is allocated on first use).  fa_check_device_error reads and
+ *     clears both words, allocating nothing, and reports FA_ERR_TIMEOUT or
+ *     FA_ERR_INVALID as for the other entry points.
  */
 #define FA_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 FA_API fa_status fa_attention_decode_noalloc(const fa_decode_params *p, fa_stream_t stream);
@@ -501,10 +508,13 @@ FA_API fa_status fa_tq_attention_decode(const fa_tq_decode_params *p, fa_stream_
 
 /*
  * Synchronises `stream`, then reads and clears the current device's status
- * word: FA_ERR_TIMEOUT if a bounded wait in any kernel gave up since the last
+ * words (the shared one and fa_attention_decode_noalloc's own):
+ * FA_ERR_TIMEOUT if a bounded wait in any kernel gave up since the last
  * check, FA_ERR_INVALID if a kernel met a device-side argument out of range
- * (fa_kv_append's cur_pos, a paged call's page id), FA_ERR_CUDA if the
- * synchronisation itself failed, else FA_OK.
+ * (fa_kv_append's cur_pos, a paged call's page id, a decode cache length),
+ * FA_ERR_CUDA if the synchronisation itself failed, else FA_OK.  It
+ * allocates nothing: before the first launch on a device there is nothing
+ * to read.
  */
 FA_API fa_status fa_check_device_error(fa_stream_t stream);
 

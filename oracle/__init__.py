@@ -21,7 +21,7 @@ Definitions followed:
     quantization (one fp32 scale/token)"); the oracle attends over the
     dequantised cache c * s;
   * cache append at a device-side slot: FlashRT QKV Cache RoPE, Kernels
-    ("... selects the cache slot from a CUDA int32 cur_pos tensor"): row
+    (the write slot comes from a device-side int32 position tensor): row
     b*hkv + g of the new token goes to slot cur_pos[b] of its cache row,
     compressed as compress_kv does; nothing else changes;
   * partial results over disjoint key sets and their merge: kernbench2

@@ -24,10 +24,11 @@
  *    causal); W <= 0 means no window;
  *  - a row whose band is empty gets uniform weights over all s_k keys of its
  *    sequence, i.e. the mean of V (SKaiNET-transformers PR #419, Summary:
- *    "empty sliding-window bands reproduce the engine's uniform softmax");
+ *    a sliding-window row whose band holds no key falls back to the
+ *    engine's uniform softmax);
  *    with s_k = 0 the row is zero;
  *  - the epilogue ops are applied to the normalised output in list order
- *    (fkl_python PR #6, Summary, "epilogue=[ops]").
+ *    (fkl_python PR #6, Summary: the epilogue op list).
  *
  * The quantiser is written in IEEE fp32 because its codes and scales are
  * compared bit for bit: amax = max|x|, s = amax / 127 (fp32 division),

@@ -9,7 +9,7 @@ randomized Hadamard transform (random +-1 signs applied BEFORE the Hadamard
 transform), normalised by its L2 norm, each coordinate quantised to 2-4 bits
 by Lloyd-Max scalar quantisation against a precomputed codebook of the
 Beta(d/2, d/2) distribution, and the codes bit-packed; K4/V2 by default,
-"9.14x smaller than FP32".
+which the page puts at 9.14 times less memory than an fp32 cache.
 
 Readings (the page fixes no more than the above):
   * rotation: y = H (s * x) / sqrt(d), H the Sylvester-ordered Hadamard

@@ -1,6 +1,6 @@
 """GPU parity of fa_attention_decode (int8 KV cache) against the fp64 oracle
-on the dequantised cache (fkl_python PR #6, Verification: "FA decode step
-s_q=1 vs s_k=256 int8"; bf16 output gate: max abs <= 2e-2
+on the dequantised cache (fkl_python PR #6, Verification: a one-query
+decode step over 256 int8-cached keys; bf16 output gate: max abs <= 2e-2
 and relative L2 <= 5e-3)."""
 import numpy as np
 import pytest

@@ -1,6 +1,7 @@
 """GPU parity of fa_attention_decode over a bf16 KV cache against the fp64
-oracle on the same bf16 values (the decode step of fkl_python PR #6,
-Verification, "FA decode step s_q=1 vs s_k=256", with an uncompressed cache;
+oracle on the same bf16 values (the one-query decode step that fkl_python
+PR #6, Verification, checks against 256 cached keys, here with an
+uncompressed cache;
 bf16 output gate: max abs <= 2e-2 and relative L2 <= 5e-3).
 Cache rows outside the attended band may hold any bytes, NaN and Inf
 included; they must not reach the result."""
@@ -70,7 +71,7 @@ def test_decode_bf16_window_epilogue_and_poisoned_rows(d):
     ref = oracle_decode_bf16(w, window=window, epilogue=epi)
     g = got.float().numpy().reshape(ref.shape)
     assert np.isfinite(g).all()
-    assert_close_bf16(g, ref, atol=2 * 2e-2)  # |Mul(2)| doubles the absolute error
+    assert_close_bf16(g, ref)
 
 
 def test_decode_bf16_empty_cache_and_split_invariance():

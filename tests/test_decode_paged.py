@@ -1,9 +1,9 @@
 """GPU parity of fa_attention_decode_paged: decode over a page pool through a
-block table (SKaiNET-transformers PR #419, Summary: positional KV caches hand
-the kernel "copy-free views instead of copying the whole prefix").  The pages
+block table (SKaiNET-transformers PR #419, Summary: the kernel reads the
+cached prefix where it lies rather than a per-token copy of it).  The pages
 of a dense cache scattered over a pool in random order must give the dense
-decode's output bit for bit (the page's "in-place == copied views"), and the
-oracle's within the bf16 gate."""
+decode's output bit for bit (the page's tests compare the in-place view with
+the copied one), and the oracle's within the bf16 gate."""
 import numpy as np
 import pytest
 import torch

@@ -1,6 +1,7 @@
 """GPU parity of the fp32 CUDA-core path of fa_attention_fwd against the fp64
-oracle: max abs error <= 1e-5 (fkl_python PR #6, Verification: "FA dense d64
-causal", "FA dense d32 ragged 33/127", "FA fused epilogue == host-applied").
+oracle: max abs error <= 1e-5 (fkl_python PR #6, Verification: the dense
+causal check at head size 64, the ragged 33/127 check at head size 32, and
+the fused epilogue checked against the same ops applied on the host).
 """
 import numpy as np
 import pytest
@@ -81,8 +82,8 @@ def test_varlen_ragged_33_127():
 
 
 def test_epilogue_fused_equals_host_applied():
-    """fkl_python PR #6, Verification: 'FA fused epilogue == host-applied
-    (err=0.0)'.  In fp32 the fused Mul(2.0), Add(0.5) must equal the same ops
+    """fkl_python PR #6, Verification: the fused epilogue equals the host-
+    applied one with zero error.  In fp32 the fused Mul(2.0), Add(0.5) must equal the same ops
     applied on the host in fp32, bit for bit; changing the values or the
     list's length instantiates no new kernel."""
     from flashattention_attention_b200 import fa
@@ -123,8 +124,8 @@ I8_CASES = [
 
 @pytest.mark.parametrize("case", I8_CASES, ids=lambda c: "-".join(map(str, c)))
 def test_int8_kv_exact_vs_dequantised_oracle(case):
-    """fkl_python PR #6, Verification, 'FA int8-KV exact vs dequantized
-    oracle': fp32 queries over an int8 cache made by fa_compress_kv from fp32
+    """fkl_python PR #6, Verification: attention over the int8 cache agrees
+    with an oracle run on the dequantised cache.  fp32 queries over an int8 cache made by fa_compress_kv from fp32
     K/V (codes and scales bit-exact with the oracle's quantiser) match the fp64
     oracle run on the dequantised cache within the fp32 gate."""
     from flashattention_attention_b200 import fa

@@ -1,14 +1,14 @@
 """GPU parity of the tensor-core prefill over an int8 KV cache (codes +
 per-token fp32 scales made by fa_compress_kv) against the fp64 oracle on the
-dequantised cache (fkl_python PR #6, Verification: "FA int8-KV exact vs
-dequantized oracle"; bf16 output gate: max abs <= 2e-2, relative L2 <= 5e-3;
+dequantised cache (fkl_python PR #6, Verification: int8-cache attention
+against an oracle on the dequantised cache; bf16 output gate: max abs <= 2e-2, relative L2 <= 5e-3;
 codes and scales bit-exact)."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from conftest import assert_close_bf16
+from conftest import assert_close_bf16, assert_close_bf16_planes
 from flashattention_attention_b200 import inputs
 
 pytestmark = pytest.mark.gpu
@@ -63,9 +63,8 @@ def test_dense_int8(case):
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("epilogue", [(), (("mul", 2.0), ("add", 0.5))], ids=["plain", "mul2add"])
 def test_varlen_int8_window(d, epilogue):
-    """Sequence starts at arbitrary rows, so scale addresses are unaligned.
-    With an epilogue Mul(a) the output's absolute error scales by |a|, so the
-    absolute bound is |a| times the gate (relative L2 is unchanged)."""
+    """Sequence starts at arbitrary rows, so scale addresses are unaligned;
+    the gate is the same with and without the epilogue."""
     lengths = [33, 127, 1, 300, 129, 255]
     w = inputs.varlen_prefill("t", lengths=lengths, hq=8, hkv=2, d=d, dtype=torch.bfloat16,
                               causal=True, window=90, seed=d)
@@ -75,14 +74,13 @@ def test_varlen_int8_window(d, epilogue):
                      cu_seqlens_q=cu.cuda(), max_seqlen_q=max(lengths))
     ref = oracle.attention(w.q, kd, vd, hq=8, hkv=2, causal=True, window=90, epilogue=list(epilogue),
                            cu_seqlens_q=cu.numpy())
-    gain = max([1.0] + [abs(v) for op, v in epilogue if op == "mul"])
-    assert_close_bf16(got.float().numpy(), ref, atol=2e-2 * gain)
+    assert_close_bf16(got.float().numpy(), ref, what=f"varlen int8 d={d} {epilogue}")
 
 
 def test_int8_matches_bf16_path_on_dequantised_values_within_quantisation_error():
-    """fkl_python PR #6, Verification: 'int8-KV end-to-end quant error bounded
-    (3.9e-03)': the int8 path stays within ~1e-2 of the bf16 path on the
-    unquantised inputs."""
+    """fkl_python PR #6, Verification: the page bounds the end-to-end error
+    the int8 cache adds (it measured 3.9e-3); here the int8 path stays within
+    ~1e-2 of the bf16 path on the unquantised inputs."""
     w = inputs.dense_prefill("t", batch=1, hq=4, hkv=2, s_q=256, s_k=256, d=64,
                              dtype=torch.bfloat16, causal=True, seed=9)
     from flashattention_attention_b200 import fa
@@ -95,7 +93,8 @@ def test_int8_matches_bf16_path_on_dequantised_values_within_quantisation_error(
 
 def test_full_size_int8_long_prefill():
     """B=1, Hq=64, Hkv=8, S=16384, d=128, causal, int8 KV, epilogue [Mul(0.5)]:
-    sampled rows of two KV groups (16 query heads) computed by the oracle."""
+    the bench's launch; every row of two whole KV groups (the first and the
+    last, 16 query heads) checked against the oracle on the dequantised cache."""
     w = inputs.int8kv_long_prefill()
     gpu_kv, _ = compress_both(w.k, w.v)
     got = gpu_fwd_i8(w.q, gpu_kv, hq=64, hkv=8, causal=True, epilogue=w.epilogue)
@@ -104,12 +103,6 @@ def test_full_size_int8_long_prefill():
     heads = [g * 8 + j for g in groups for j in range(8)]
     rk, rks = oracle.compress_kv(w.k[groups])
     rv, rvs = oracle.compress_kv(w.v[groups])
-    q_sub = w.q[heads]
-    rng = np.random.default_rng(2)
-    rows = sorted({(0, int(h), int(i)) for h, i in zip(rng.integers(0, 16, 96), rng.integers(0, 16384, 96))}
-                  | {(0, 0, 0), (0, 15, 16383), (0, 3, 127), (0, 9, 128)})
-    ref = oracle.attention(q_sub, oracle.dequantize(rk, rks), oracle.dequantize(rv, rvs), hq=16, hkv=2,
-                           causal=True, epilogue=w.epilogue, rows=rows)
-    g = np.stack([got[heads[h], i].float().numpy() for _, h, i in rows])
-    r = np.stack([ref[h, i] for _, h, i in rows])
-    assert_close_bf16(g, r, what="full-size int8 prefill sample")
+    ref = oracle.attention(w.q[heads], oracle.dequantize(rk, rks), oracle.dequantize(rv, rvs), hq=16, hkv=2,
+                           causal=True, epilogue=w.epilogue)
+    assert_close_bf16_planes(got[heads], ref, what="full-size int8 prefill, two KV groups")

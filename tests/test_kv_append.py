@@ -1,6 +1,6 @@
 """GPU parity of fa_kv_append: a one-token cache write at a device-side slot
-(FlashRT QKV Cache RoPE, Kernels: "selects the cache slot from a CUDA int32
-cur_pos tensor for graph-friendly decode"), quantised on the way in with the
+(FlashRT QKV Cache RoPE, Kernels: the slot is read from a device-side int32
+position, so a captured decode graph can reuse it), quantised on the way in with the
 int8 scheme of fkl_python PR #6, Summary.  The caches after the call must
 equal the oracle's plain definition bit for bit, and a captured CUDA graph
 of append + decode steps must match the oracle step by step."""

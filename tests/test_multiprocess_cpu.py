@@ -57,7 +57,8 @@ def test_reference_arm_under_torchrun_world2():
     times the oracle and prints one JSON line, rank 1 exits 0 without work."""
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
            "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
-           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"]
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3",
+           "--ref-step-seconds", "0.5"]
     r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT,
                        env=dict(os.environ, OMP_NUM_THREADS="2"))
     assert r.returncode == 0, r.stderr[-2000:]

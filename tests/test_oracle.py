@@ -158,8 +158,8 @@ def pin_single_key_and_row0():
 
 
 def pin_empty_band():
-    """SKaiNET-transformers PR #419, Summary: an empty sliding-window band
-    reproduces the uniform softmax, i.e. the mean of all V rows.  Here s_q > s_k
+    """SKaiNET-transformers PR #419, Summary: a row whose sliding-window band
+    holds no key falls back to the uniform softmax, i.e. the mean of all V rows.  Here s_q > s_k
     under causal masking leaves the first s_q - s_k rows with no visible key."""
     rng = np.random.default_rng(5)
     s_q, s_k, d = 10, 4, 8
@@ -288,7 +288,8 @@ def pin_quantiser_invariants():
 
 
 def pin_compression_ratio():
-    """fkl_python PR #6, Verification: 'KV compression ratio 3.76x (>3.5x)'.
+    """fkl_python PR #6, Verification: the compressed cache is 3.76 times
+    smaller than fp32, against a gate of 3.5.
     Measured from the oracle's output buffers at head_dim 64 against fp32."""
     with open(os.path.join(GOLDEN, "compression_ratio.txt")) as f:
         fields = dict(line.split("=", 1) for line in f.read().split("\n")

@@ -108,8 +108,8 @@ def test_bit_packing_is_lsb_first():
 
 
 def test_k4_v2_is_9_14_times_smaller_than_fp32():
-    """The page: default K4/V2 "9.14x smaller than FP32" (d = 64: 512 bytes
-    of fp32 K and V per token and head against 56)."""
+    """The page puts the default K4/V2 at 9.14 times less memory than fp32
+    (d = 64: 512 bytes of fp32 K and V per token and head against 56)."""
     d = 64
     ratio = (2 * 4 * d) / (tq.bytes_per_row(d, 4) + tq.bytes_per_row(d, 2))
     assert round(ratio, 2) == 9.14

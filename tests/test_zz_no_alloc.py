@@ -5,10 +5,13 @@ not trigger the implicit synchronisation of a cudaMalloc).  Its partials live
 in a scratch array built into the library instead of a caller workspace.
 
 Called through the C ABI and compared with fa_attention_decode on the same
-inputs, within the bf16 tolerance the decode tests use, on two calls in a row
-with different problems (the shared scratch keeps the previous call's
-contents, which must not leak into the next result).  This file is collected
-last so that a failure here never hides another test.
+inputs and with the fp64 oracle on the dequantised cache, within the bf16
+tolerance the decode tests use, on two calls in a row with different
+problems (the shared scratch keeps the previous call's contents, which must
+not leak into the next result).  A cache length past the capacity is clamped
+and reported through fa_check_device_error, which reads this entry point's
+own status word.  This file is collected last so that a failure here never
+hides another test.
 """
 import ctypes
 
@@ -16,6 +19,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from conftest import assert_close_bf16
 from flashattention_attention_b200 import inputs
 
@@ -54,7 +58,15 @@ def _existing(q, kc, ks, vc, vs, lens, hq, hkv, split_keys=0, epilogue=()):
     return out
 
 
+def _oracle(w, hq, hkv, epilogue=()):
+    rk, rks = oracle.compress_kv(w.k)
+    rv, rvs = oracle.compress_kv(w.v)
+    return oracle.decode(w.q, oracle.dequantize(rk, rks), oracle.dequantize(rv, rvs), w.lengths, hq=hq, hkv=hkv,
+                         epilogue=epilogue)
+
+
 def test_noalloc_matches_decode_on_two_calls_in_a_row():
+    from flashattention_attention_b200 import fa
     # first call: a larger problem that fills more of the scratch
     w1, *a1 = _prepare(21, [4000, 1500, 3000, 64], 32, 8, 4096)
     first = _noalloc(*a1, 32, 8)
@@ -63,6 +75,7 @@ def test_noalloc_matches_decode_on_two_calls_in_a_row():
     w2, *a2 = _prepare(22, [700, 2049], 16, 2, 4096)
     epi = [("mul", 2.0), ("add", 0.5)]
     second = _noalloc(*a2, 16, 2, split_keys=256, epilogue=epi)
+    assert fa.check_device_error() == fa.FA_OK
 
     ref1 = _existing(*a1, 32, 8)
     ref2 = _existing(*a2, 16, 2, split_keys=256, epilogue=epi)
@@ -70,6 +83,28 @@ def test_noalloc_matches_decode_on_two_calls_in_a_row():
     assert_close_bf16(second.float().cpu().numpy(), ref2.float().cpu().numpy(), what="second call")
     # the same split choice runs the same kernels: identical bits
     assert torch.equal(second, ref2)
+    # and both agree with the oracle on the dequantised cache
+    o1 = _oracle(w1, 32, 8)
+    o2 = _oracle(w2, 16, 2, epilogue=epi)
+    assert_close_bf16(first.float().cpu().numpy().reshape(o1.shape), o1, what="first call vs oracle")
+    assert_close_bf16(second.float().cpu().numpy().reshape(o2.shape), o2, what="second call vs oracle")
+
+
+def test_noalloc_reports_a_cache_length_past_the_capacity():
+    """L_b > capacity is clamped to the capacity and reported: the result is
+    attention over the whole cache, and fa_check_device_error (which reads
+    this entry point's own status word) returns FA_ERR_INVALID once, then
+    FA_OK again."""
+    from flashattention_attention_b200 import fa
+    cap = 1024
+    w, q, kc, ks, vc, vs, lens = _prepare(23, [cap, 300], 8, 2, cap)
+    assert fa.check_device_error() == fa.FA_OK
+    over = torch.tensor([cap + 77, 300], dtype=torch.int32, device="cuda")
+    got = _noalloc(q, kc, ks, vc, vs, over, 8, 2)
+    assert fa.check_device_error() == fa.FA_ERR_INVALID
+    assert fa.check_device_error() == fa.FA_OK  # read and cleared
+    ref = _oracle(w, 8, 2)  # w.lengths = [cap, 300]: the clamped problem
+    assert_close_bf16(got.float().cpu().numpy().reshape(ref.shape), ref, what="clamped length vs oracle")
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch():
