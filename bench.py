@@ -366,6 +366,8 @@ def gpu_arm(args, rank, world, dist):
         ring_rank_steps(args, dev, peaks, world, dist, result)
         decode_and_quant(args, dev, peaks, world, dist, result)
         turboquant_decode(args, dev, peaks, world, dist, result)
+        if world > 1:
+            ring_across_ranks(args, dev, peaks, world, dist, result)
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, flops_tiles, flops_exact, args.cpu_seconds)
     summarise(result)
@@ -559,6 +561,51 @@ def ring_rank_steps(args, dev, peaks, world, dist, result):
                          "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                                       "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4)}}}
     del q, kb, vb, blocks, o, lse, acc_o, acc_l, out
+    torch.cuda.empty_cache()
+
+
+def ring_job_flops(world, block=4096, batch=4, hq=32, d=128):
+    """FLOPs of the causal prefill over world * block positions that the
+    ring computes (128x128 tiles intersecting the band), all ranks together."""
+    S = world * block
+    return batch * hq * 4 * d * TILE * TILE * band_tiles(S, S, True, 0)[0]
+
+
+def ring_across_ranks(args, dev, peaks, world, dist, result):
+    """The context-parallel ring itself on N GPUs: each rank holds one
+    4096-position block of every sequence (B=4, Hq=32, Hkv=8, d=128, causal)
+    and ring.ring_attention_fwd passes the K/V blocks around the ranks with
+    NCCL point-to-point sends between the ranks' own memory (no peer loads,
+    no multicast) while each step's kernel merges its block in the
+    epilogue.  Each rank draws its own block (seed = rank).  The step time
+    is the max over ranks; value is the whole causal attention over N * 4096
+    positions divided by it."""
+    import torch
+    from flashattention_attention_b200 import fa, inputs, ring
+    rank = dist.get_rank()
+    w = inputs.dense_prefill(f"ring_block{rank}", batch=4, hq=32, hkv=8, s_q=4096, s_k=4096, d=128,
+                             dtype=torch.bfloat16, causal=True, seed=100 + rank)
+    q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
+    steps = max(10, args.steps // 4)
+
+    def step():
+        ring.ring_attention_fwd(q, k, v, hq=w.hq, hkv=w.hkv, causal=True, group=dist.group.WORLD)
+
+    try:
+        ms = time_launches(step, steps, args.warmup, torch, dist)
+        assert fa.check_device_error() == fa.FA_OK
+        flops = ring_job_flops(world)
+        tf = flops / (ms * 1e-3) / 1e12
+        result["ring_cp_across_ranks"] = {
+            "workload": f"ring_cp{world}_causal_b4_hq32_hkv8_block4096_d128_bf16", "value": round(tf, 2),
+            "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "nccl_ranks": world, "flops_per_step": flops,
+            "flops_counting": "128x128 tiles of the whole causal band over all ranks' positions",
+            "transfers": "NCCL point-to-point K/V blocks between ranks, timed",
+            "roofline": {"bound": "tensor", "achieved": round(tf / world, 2), "per": "GPU", "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(tf / world / peaks["bf16_tflops"], 4)}}
+    except Exception as e:  # reported in the line, never fatal to it
+        result["ring_cp_across_ranks"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    del q, k, v
     torch.cuda.empty_cache()
 
 

@@ -49,7 +49,8 @@
 namespace fa {
 namespace {
 
-constexpr int kWarps = 4;
+constexpr int kWarps = 4;    // compute warps (workers) per CTA
+constexpr int kThreads = (kWarps + 1) * 32;  // plus one producer warp
 constexpr int kTile = 32;    // keys per tile
 constexpr int kMaxCtasPerSm = 2;  // int8 and bf16 at d = 64; bf16 at d = 128 fits one
 constexpr int kMaxWorkers = 4096;
@@ -67,7 +68,12 @@ struct SkArgs {
   int32_t* counters;        // [B*hkv]: workers done with each segment (zeroed by the plan)
   __nv_bfloat16* out;       // [B*hq, D]
   Epilogue epi;
+  // Groups of more than 8 query heads (the MMA's N) run as kv_split passes
+  // over their KV head, each serving group = (hq / hkv_real) / kv_split heads:
+  // hkv counts these virtual KV heads (hkv_real * kv_split), and only cache
+  // addressing uses the real head g / kv_split.
   int batch, hq, hkv, group, cap, window;
+  int hkv_real, kv_split;
   // paged cache (null table: dense [B*hkv, cap, d]): pool [num_pages, hkv,
   // page_size, d]; key j of sequence b lives in page block_table[b*max_pages + j/page_size]
   const int32_t* block_table;
@@ -295,7 +301,7 @@ __device__ __forceinline__ int seq_tiles(const SkArgs& A, const int32_t* pre, in
 __device__ __forceinline__ void set_segment(const SkArgs& A, Cursor& c) {
   int k_lo;
   key_range(clamp_len(A.seqlens[c.b], A.cap), A.window, k_lo, c.t_begin);
-  c.kv_row0 = (static_cast<int64_t>(c.b) * A.hkv + c.g) * A.cap;
+  c.kv_row0 = (static_cast<int64_t>(c.b) * A.hkv_real + c.g / A.kv_split) * A.cap;
 }
 __device__ __forceinline__ Cursor locate(const SkArgs& A, const int32_t* pre, long long x) {
   int lo = 0, hi = A.batch - 1;  // largest b with prefix[b] <= x
@@ -353,11 +359,11 @@ __device__ __forceinline__ int64_t tile_row(const SkArgs& A, const Cursor& c, in
     pc.pg = pg;
     pc.next = page_id(A, c.b, lp + 1);  // consumed page_size / 32 tiles later
   }
-  return (static_cast<int64_t>(pc.pg) * A.hkv + c.g) * A.page_size + key0 % A.page_size;
+  return (static_cast<int64_t>(pc.pg) * A.hkv_real + c.g / A.kv_split) * A.page_size + key0 % A.page_size;
 }
 
 template <int D, bool kBF>
-__global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
+__global__ void __launch_bounds__(kThreads, Geom<D, kBF>::kCtas)
     decode_sk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const SkArgs A) {
   using G = Geom<D, kBF>;
@@ -370,14 +376,20 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kStages * G::kStageBytes);
   __shared__ int abort_flag;
 
+  // full[w][s]: the producer's TMA landed stage s of worker w's ring;
+  // empty[w][s]: worker w is done reading it
+  uint64_t* empty_bars = bars + kWarps * kStages;
   int32_t* s_pre = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + 256);
-  __shared__ int32_t warp_sums[kWarps];
+  __shared__ int32_t warp_sums[kWarps + 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, qq = lane & 3;
   if (threadIdx.x == 0) abort_flag = 0;
-  if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&bars[warp * kStages + s], 1);
+  if (warp < kWarps && lane == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars[warp * kStages + s], 1);
+      mbar_init(&empty_bars[warp * kStages + s], 1);
+    }
     fence_barrier_init();
   }
   // the tile prefix over sequences: computed here for small batches (no
@@ -385,7 +397,7 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
   const int32_t* pre = A.prefix;
   if (A.smem_prefix) {
     int32_t carry = 0;
-    for (int b0 = 0; b0 < A.batch; b0 += kWarps * 32) {
+    for (int b0 = 0; b0 < A.batch; b0 += kThreads) {
       const int b = b0 + static_cast<int>(threadIdx.x);
       const int32_t own = b < A.batch ? tiles_of(clamp_len(A.seqlens[b], A.cap), A.window) * A.hkv : 0;
       int32_t incl = own;
@@ -399,7 +411,7 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
       int32_t before = carry;
       for (int v = 0; v < warp; ++v) before += warp_sums[v];
       if (b < A.batch) s_pre[b] = before + incl - own;
-      for (int v = warp; v < kWarps; ++v) before += warp_sums[v];
+      for (int v = warp; v < kWarps + 1; ++v) before += warp_sums[v];
       carry = before;  // the same in every thread: the running total
       __syncthreads();
     }
@@ -412,6 +424,62 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
 
   const long long T = pre[A.batch];
   const long long P = effective_workers(A, T);
+  if (warp == kWarps) {
+    // ---------------------------------------------------------------- producer
+    // Lanes 0 .. kWarps-1 keep the workers' rings full, lane l for worker l
+    // with that worker's own cursor.  The lanes run together: each round,
+    // every lane whose next stage its worker has released (a non-blocking
+    // probe) refills it, so up to four refills share one pass of the issue
+    // code and no load issue sits in a compute warp.  Gives up (status word)
+    // when no ring frees a stage for a whole watchdog budget.
+    if (T == 0) return;
+    const long long wl = static_cast<long long>(blockIdx.x) * kWarps + lane;
+    int n = 0;
+    Cursor ic;
+    PageCursor ipc;
+    if (lane < kWarps && wl < P) {
+      const long long tf = worker_begin(wl, T, P);
+      n = static_cast<int>(worker_begin(wl + 1, T, P) - tf);
+      ic = locate(A, pre, tf);
+    }
+    int i = 0;
+    long long t0 = clock64();
+    while (__any_sync(0xffffffffu, i < n)) {
+      const int s = i % kStages;
+      const bool ready = i < n && (i < kStages ||
+                                   mbar_test_wait(smem_u32(&empty_bars[lane * kStages + s]), ((i / kStages) - 1) & 1));
+      if (ready) {
+        const int key0 = ic.t_begin + ic.t * kTile;
+        const int64_t row = tile_row(A, ic, key0, ipc);
+        uint8_t* st = smem + (lane * kStages + s) * G::kStageBytes;
+        uint64_t* bar = &bars[lane * kStages + s];
+        mbar_expect_tx(bar, 2 * G::kTileBytes + G::kScaleBytes);
+        if constexpr (kBF) {
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(st + c * G::kChunkBytes, &tm_k, bar, 64 * c, static_cast<int>(row));
+            tma_load_2d(st + G::kTileBytes + c * G::kChunkBytes, &tm_v, bar, 64 * c, static_cast<int>(row));
+          }
+        } else {
+          tma_load_2d(st, &tm_k, bar, 0, static_cast<int>(row));
+          tma_load_2d(st + G::kTileBytes, &tm_v, bar, 0, static_cast<int>(row));
+          bulk_load(st + G::kScaleOff, A.k_scales + row, kTile * 4, bar);
+          bulk_load(st + G::kScaleOff + kTile * 4, A.v_scales + row, kTile * 4, bar);
+        }
+        advance(A, pre, ic);
+        ++i;
+      }
+      if (__any_sync(0xffffffffu, ready)) {
+        t0 = clock64();
+      } else if (clock64() - t0 > A.wd.budget) {
+        if (lane == 0) record_status(A.wd, kStatusTimeout);
+        return;
+      } else {
+        __nanosleep(32);  // leave the issue slots of this sub-partition to its worker
+      }
+    }
+    return;
+  }
   const long long w = static_cast<long long>(blockIdx.x) * kWarps + warp;
   if (T == 0 || w >= P) return;
   const long long t_first = worker_begin(w, T, P);
@@ -419,34 +487,6 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
   if (my_tiles <= 0) return;
 
   auto stage_ptr = [&](int s) { return smem + (warp * kStages + s) * G::kStageBytes; };
-  // issue cursor (lane 0 runs it kStages tiles ahead of the compute cursor)
-  Cursor ic = locate(A, pre, t_first);
-  PageCursor ipc;
-  auto issue = [&](int i) {
-    const int s = i % kStages;
-    const int key0 = ic.t_begin + ic.t * kTile;
-    const int64_t row = tile_row(A, ic, key0, ipc);
-    uint8_t* st = stage_ptr(s);
-    uint64_t* bar = &bars[warp * kStages + s];
-    mbar_expect_tx(bar, 2 * G::kTileBytes + G::kScaleBytes);
-    if constexpr (kBF) {
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_2d(st + c * G::kChunkBytes, &tm_k, bar, 64 * c, static_cast<int>(row));
-        tma_load_2d(st + G::kTileBytes + c * G::kChunkBytes, &tm_v, bar, 64 * c, static_cast<int>(row));
-      }
-    } else {
-      tma_load_2d(st, &tm_k, bar, 0, static_cast<int>(row));
-      tma_load_2d(st + G::kTileBytes, &tm_v, bar, 0, static_cast<int>(row));
-      bulk_load(st + G::kScaleOff, A.k_scales + row, kTile * 4, bar);
-      bulk_load(st + G::kScaleOff + kTile * 4, A.v_scales + row, kTile * 4, bar);
-    }
-    advance(A, pre, ic);
-  };
-  if (lane == 0) {
-    for (int i = 0; i < min(kStages, my_tiles); ++i) issue(i);
-  }
-
   // ---- per-segment state
   uint32_t qb0[kSteps], qb1[kSteps];
   float qs0 = 0.f, qs1 = 0.f;
@@ -825,10 +865,11 @@ __global__ void __launch_bounds__(kWarps * 32, Geom<D, kBF>::kCtas)
       }
     }
 
+    // this warp is done with the stage: hand it back to the producer
     __syncwarp();
-    if (lane == 0 && i + kStages < my_tiles) {
+    if (lane == 0) {
       fence_proxy_async_smem();
-      issue(i + kStages);
+      mbar_arrive(&empty_bars[warp * kStages + s]);
     }
     advance(A, pre, cc);
   }
@@ -864,7 +905,12 @@ fa_status launch_sk(const fa_decode_params& p, const fa_kv_pages* pages, int n_w
   st = encode_tensor_map(&tmv, dt, 2, p.v_cache, dims, strides, box, sw);
   if (st != FA_OK) return st;
 
-  const int group = p.hq / p.hkv;
+  // a group of G > 8 query heads runs as `split` passes of G / split <= 8
+  const int full_group = p.hq / p.hkv;
+  int split = (full_group + 7) / 8;
+  while (full_group % split != 0) ++split;
+  const int group = full_group / split;
+  const int hkv = p.hkv * split;
   uint8_t* base = static_cast<uint8_t*>(ws);
   SkArgs A;
   A.q = static_cast<const __nv_bfloat16*>(p.q);
@@ -875,13 +921,15 @@ fa_status launch_sk(const fa_decode_params& p, const fa_kv_pages* pages, int n_w
   A.counters = reinterpret_cast<int32_t*>(base) + (p.batch + 1);
   A.out = static_cast<__nv_bfloat16*>(p.out);
   A.epi = make_epilogue(p.epilogue, p.n_epilogue);
-  const size_t o_recs = static_cast<size_t>(p.batch * p.hkv + n_workers) * group;
+  const size_t o_recs = static_cast<size_t>(p.batch * hkv + n_workers) * group;
   A.rec_o = reinterpret_cast<float*>(base + plan_bytes(p.batch, p.hq));
   A.rec_ml = A.rec_o + o_recs * D;
   A.batch = p.batch;
   A.hq = p.hq;
-  A.hkv = p.hkv;
+  A.hkv = hkv;
   A.group = group;
+  A.hkv_real = p.hkv;
+  A.kv_split = split;
   A.cap = p.capacity;
   A.block_table = pages != nullptr ? pages->block_table : nullptr;
   A.max_pages = pages != nullptr ? pages->max_pages : 1;
@@ -899,7 +947,7 @@ fa_status launch_sk(const fa_decode_params& p, const fa_kv_pages* pages, int n_w
     note_variant(reinterpret_cast<const void*>(plan));
     note_variant(reinterpret_cast<const void*>(kern));
   }
-  plan<<<1, 1024, 0, ctx.stream>>>(p.cache_seqlens, p.batch, p.hq, p.hkv, p.capacity, p.window,
+  plan<<<1, 1024, 0, ctx.stream>>>(p.cache_seqlens, p.batch, p.hq, hkv, p.capacity, p.window,
                                    reinterpret_cast<int32_t*>(base), A.counters, A.out, A.epi, ctx.wd.word);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   A.smem_prefix = p.batch <= G::kPrefixCap ? 1 : 0;
@@ -911,7 +959,7 @@ fa_status launch_sk(const fa_decode_params& p, const fa_kv_pages* pages, int n_w
   // kernel runs and waits for it only before touching the counters
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(n_workers / kWarps));
-  cfg.blockDim = dim3(kWarps * 32);
+  cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = ctx.stream;
   cudaLaunchAttribute attr[1];

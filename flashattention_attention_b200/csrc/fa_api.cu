@@ -345,7 +345,6 @@ fa_status decode_args(const fa_decode_params* p) {
   if (p->kv_dtype != FA_I8 && p->kv_dtype != FA_BF16) return FA_ERR_INVALID;
   if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
   if (p->head_dim != 64 && p->head_dim != 128) return FA_ERR_UNSUPPORTED;
-  if (p->hq / p->hkv > 8) return FA_ERR_UNSUPPORTED;
   if (p->batch == 0) return FA_OK;
   if (p->q == nullptr || p->k_cache == nullptr || p->v_cache == nullptr || p->out == nullptr ||
       p->cache_seqlens == nullptr)

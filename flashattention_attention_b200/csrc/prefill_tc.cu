@@ -54,6 +54,9 @@
 // layout and fence it to the async proxy.  The softmax is then the bf16 one.
 // That variant runs 16 warps and rebalances registers with setmaxnreg
 // (softmax 192, the rest 64).
+#include <cstdlib>
+#include <mutex>
+
 #include "internal.h"
 #include "layout.cuh"
 #include "umma.cuh"
@@ -62,43 +65,74 @@ namespace fa {
 namespace {
 
 constexpr int kBM = 128;  // query rows per Q tile
-constexpr int kBN = 128;  // keys per K/V tile
-constexpr int kLoadWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kConvWarp0 = 12;  // int8 variant: warps 12-15 convert K/V tiles
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
+// Exponentials of the softmax: every kPolyEvery-th pair of scores is
+// computed by exp2_poly2 (FMA and integer pipes) instead of the MUFU; 0: all
+// on the MUFU.
+#ifndef FA_EXP2_POLY_EVERY
+#define FA_EXP2_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = FA_EXP2_POLY_EVERY;
 constexpr uint32_t kChunkBytes = kSwizzleChunkRows * 128;  // [128 rows x 64 bf16]
 
-template <int D, bool kI8>
+// BN keys per K/V tile, NT Q tiles (query heads) per CTA.  Warps 0 .. 4 NT - 1
+// run the softmax (four per Q tile), then the producer, the MMA issuer and,
+// for int8 K/V, two idle warps and four converters.
+template <int D, bool kI8, bool kPair = false, int BN_ = 128, int NT_ = 2>
 struct TcGeom {
+  static constexpr int BN = BN_;
+  static constexpr int NT = NT_;
+  static constexpr int kLoadWarp = 4 * NT;
+  static constexpr int kMmaWarp = 4 * NT + 1;
+  static constexpr int kConvWarp0 = 4 * NT + 4;
   // K is consumed one step before V (S(j) precedes PV(j)), so K gets the
-  // deeper ring: a slot refills with the TMA latency hidden behind ~2 steps
-  static constexpr int kKStages = 3;
-  static constexpr int kVStages = (D == 128) ? 2 : 3;
+  // deeper ring: a slot refills with the TMA latency hidden behind ~2 steps.
+  // A CTA of a pair holds half of every K and V tile (64 keys of K, 64 dims
+  // of V), so its rings can be deeper.
+  static constexpr int kKStages = kPair ? (kI8 ? 3 : 4) : (NT == 4 ? 6 : 3);
+  static constexpr int kVStages = kPair ? (kI8 ? 3 : 4) : (NT == 4 ? 6 : ((D == 128) ? 2 : 3));
   static constexpr uint32_t kQBytes = kBM * D * 2;
-  static constexpr uint32_t kKVBytes = kBN * D * 2;   // one bf16 K or V tile
-  static constexpr uint32_t kI8Bytes = kBN * D;       // one int8 tile
-  static constexpr uint32_t kKOff = 2 * kQBytes;
-  static constexpr uint32_t kVOff = kKOff + kKStages * kKVBytes;
-  // int8 staging: at d = 128 in the upper half of each bf16 slot (a row's
-  // bf16 output overwrites only that row's int8 bytes); at d = 64 separate
-  static constexpr bool kInPlace = (D == 128);
-  static constexpr uint32_t kStageOff = kVOff + kVStages * kKVBytes;
-  static constexpr uint32_t kStageBytes = (kI8 && !kInPlace) ? (kKStages + kVStages) * kI8Bytes : 0;
+  static constexpr int kKRows = kPair ? BN / 2 : BN;               // K rows in this CTA's slot
+  static constexpr uint32_t kKChunk = kKRows * 128;                 // one 64-dim chunk of them
+  static constexpr uint32_t kKBytes = kKRows * D * 2;               // this CTA's bf16 K slot
+  static constexpr uint32_t kVChunk = BN * 128;                     // 64 dims of every key of a tile
+  static constexpr uint32_t kVBytes = BN * (kPair ? D / 2 : D) * 2;  // this CTA's bf16 V slot
+  static constexpr uint32_t kKI8Bytes = kKBytes / 2;                // the same slots as int8
+  static constexpr uint32_t kVI8Bytes = kVBytes / 2;
+  static constexpr uint32_t kKOff = NT * kQBytes;
+  static constexpr uint32_t kVOff = kKOff + kKStages * kKBytes;
+  // int8 staging: at d = 128 (one CTA) in the upper half of each bf16 slot
+  // (a row's bf16 output overwrites only that row's int8 bytes); otherwise
+  // separate
+  static constexpr bool kInPlace = (D == 128) && !kPair;
+  static constexpr uint32_t kStageOff = kVOff + kVStages * kVBytes;
+  static constexpr uint32_t kStageBytes = (kI8 && !kInPlace) ? kKStages * kKI8Bytes + kVStages * kVI8Bytes : 0;
   static constexpr uint32_t kBarOff = kStageOff + kStageBytes;
-  static constexpr uint32_t kSmem = kBarOff + 256 + 1024;
-  static constexpr int kThreads = kI8 ? 512 : 320;
+  static constexpr uint32_t kSmem = kBarOff + 512 + 1024;
+  // int8: 2 idle warps and 4 converters; four Q tiles: a fifth warpgroup
+  // (producer, MMA, 2 idle) so registers can move between warpgroups
+  static constexpr int kThreads = (4 * NT + ((kI8 || NT == 4) ? (kI8 ? 8 : 4) : 2)) * 32;
+  // setmaxnreg split (0: none): the softmax warpgroups take kRegsHi, the
+  // others give back down to 64 (the totals match the launch's pool)
+  static constexpr int kRegsHi = kI8 ? 192 : (NT == 4 ? 104 : 0);
+  // TMEM columns: S_t (P_t over its first BN / 2 columns) and O_t
+  static constexpr uint32_t s_col(int t) { return t * BN; }
+  static constexpr uint32_t o_col(int t) { return NT * BN + t * D; }
+  static_assert(NT * (BN + D) <= 512, "TMEM columns");
   __host__ __device__ static constexpr uint32_t k_stage(int s) {
-    return kInPlace ? kKOff + s * kKVBytes + kKVBytes / 2 : kStageOff + s * kI8Bytes;
+    return kInPlace ? kKOff + s * kKBytes + kKBytes / 2 : kStageOff + s * kKI8Bytes;
   }
   __host__ __device__ static constexpr uint32_t v_stage(int s) {
-    return kInPlace ? kVOff + s * kKVBytes + kKVBytes / 2 : kStageOff + (kKStages + s) * kI8Bytes;
+    return kInPlace ? kVOff + s * kVBytes + kVBytes / 2 : kStageOff + kKStages * kKI8Bytes + s * kVI8Bytes;
   }
 };
 static_assert(TcGeom<128, false>::kSmem <= 232448, "shared memory budget");
 static_assert(TcGeom<128, true>::kSmem <= 232448, "shared memory budget");
 static_assert(TcGeom<64, true>::kSmem <= 232448, "shared memory budget");
+static_assert(TcGeom<128, false, true>::kSmem <= 232448, "shared memory budget");
+static_assert(TcGeom<128, true, true>::kSmem <= 232448, "shared memory budget");
+static_assert(TcGeom<64, false, false, 64, 4>::kSmem <= 232448, "shared memory budget");
 
 struct PrefillArgs {
   SeqLayout L;
@@ -112,6 +146,7 @@ struct PrefillArgs {
   const float* v_scales;
   int64_t k_plane_rows;   // rows per K plane (the scales share K's row numbering)
   int batch, hq, hkv, group, n_qblocks, two_tiles;
+  int heads_per_item;    // 1, 2 (head pair), or 4 (CTA pair: two heads per CTA)
   float scale_log2;      // |softmax scale| * log2(e), > 0
   uint32_t negate_s;     // 1: the MMA negates Q (a negative softmax scale)
   Epilogue epi;
@@ -142,6 +177,29 @@ __device__ __forceinline__ uint2 dequant4_bf16(uint32_t w, float2 s2) {
   return make_uint2(pack_bf16x2(y01.x, y01.y), pack_bf16x2(y23.x, y23.y));
 }
 
+// NC 16-byte chunks of int8 codes, from chunk c0 of row `row` of a staged
+// tile with RL-byte rows (128- or 64-byte swizzle as TMA wrote it), times the
+// row's scale, rounded to bf16 and written as pieces of output chunk c / 4
+// (128-byte rows with the 128-byte swizzle, chunks dst_chunk bytes apart).
+// Each thread reads its own row's bytes before writing that row.
+template <int NC, int RL>
+__device__ __forceinline__ void convert_int8_row(const uint8_t* src_tile, uint8_t* dst_tile, uint32_t dst_chunk,
+                                                 int row, int c0, float sc) {
+  const float2 s2 = make_float2(sc, sc);
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    const int c = c0 + i;
+    const int pc = (RL == 128) ? (c ^ (row & 7)) : (c ^ ((row >> 1) & 3));
+    const uint4 w = *reinterpret_cast<const uint4*>(src_tile + row * RL + pc * 16);
+    const int h = c / 4, j0 = 2 * (c % 4);
+    uint8_t* out = dst_tile + h * dst_chunk + row * 128;
+    const uint2 y0 = dequant4_bf16(w.x, s2), y1 = dequant4_bf16(w.y, s2);
+    const uint2 y2 = dequant4_bf16(w.z, s2), y3 = dequant4_bf16(w.w, s2);
+    *reinterpret_cast<uint4*>(out + ((j0 ^ (row & 7)) * 16)) = make_uint4(y0.x, y0.y, y1.x, y1.y);
+    *reinterpret_cast<uint4*>(out + (((j0 + 1) ^ (row & 7)) * 16)) = make_uint4(y2.x, y2.y, y3.x, y3.y);
+  }
+}
+
 // One work item: 128 query rows of one head pair (or one head), in the
 // longest-first order (highest q-block first, then sequence, then head pair).
 struct Item {
@@ -151,14 +209,17 @@ struct Item {
 };
 // False for an item with no row or no visible key (the empty-band kernel
 // writes such rows).
-__device__ __forceinline__ bool item_of(const PrefillArgs& A, int item, Item& w) {
-  const int n_pairs = A.two_tiles ? A.hq / 2 : A.hq;
-  const int per_qb = A.batch * n_pairs;
+// In a CTA pair, CTA `rank` takes heads 2 rank and 2 rank + 1 of the item's
+// four (all of one GQA group: the group size is a multiple of 4).
+template <int BN>
+__device__ __forceinline__ bool item_of(const PrefillArgs& A, int item, Item& w, int rank = 0) {
+  const int n_sets = A.hq / A.heads_per_item;
+  const int per_qb = A.batch * n_sets;
   const int qb = A.n_qblocks - 1 - item / per_qb;
   const int rem = item % per_qb;
-  w.b = rem / n_pairs;
-  const int pair = rem % n_pairs;
-  w.h0 = A.two_tiles ? 2 * pair : pair;
+  w.b = rem / n_sets;
+  const int set = rem % n_sets;
+  w.h0 = A.heads_per_item * set + 2 * rank;
   w.g = w.h0 / A.group;
   w.sq = seq_of(A.L, w.b, w.h0, w.g);
   w.i0 = qb * kBM;
@@ -169,8 +230,8 @@ __device__ __forceinline__ bool item_of(const PrefillArgs& A, int item, Item& w)
   band_of(A.L, i_last, w.sq.s_q, w.sq.s_k, lo_last, hi_last);
   const int k_lo = max(0, lo_first);
   const int k_hi = min(w.sq.s_k, hi_last);
-  w.j_lo = k_lo / kBN;
-  w.n_iter = k_hi > k_lo ? (k_hi + kBN - 1) / kBN - w.j_lo : 0;
+  w.j_lo = k_lo / BN;
+  w.n_iter = k_hi > k_lo ? (k_hi + BN - 1) / BN - w.j_lo : 0;
   if (w.n_iter == 0) return false;
   // dense planes are (b*h + h), varlen planes are h with the sequence
   // starting at cu[b] inside the plane
@@ -182,7 +243,7 @@ __device__ __forceinline__ bool item_of(const PrefillArgs& A, int item, Item& w)
   return true;
 }
 
-// TMA plane and row of the 128-key tile starting at key0 of item w (paged:
+// TMA plane and row of the key tile starting at key0 of item w (paged:
 // through the block table; a page id outside the pool reads page 0 and is
 // reported).
 __device__ __forceinline__ void kv_tile(const PrefillArgs& A, const Item& w, int key0, int& plane, int& row) {
@@ -205,12 +266,13 @@ __device__ __forceinline__ int item_at(int c, int G, int k) {
   return (round & 1) ? base + (G - 1 - c) : base + c;
 }
 
-template <int D, bool kI8>
-__global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
+template <int D, bool kI8, bool kPair, int BN, int NT>
+__global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const PrefillArgs A) {
-  using G = TcGeom<D, kI8>;
+  using G = TcGeom<D, kI8, kPair, BN, NT>;
   constexpr int KS = G::kKStages, VS = G::kVStages;
+  constexpr int kLoadWarp = G::kLoadWarp, kMmaWarp = G::kMmaWarp, kConvWarp0 = G::kConvWarp0;
   extern __shared__ uint8_t tc_smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -220,64 +282,99 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
   uint64_t* k_empty = k_full + KS;
   uint64_t* v_full = k_empty + KS;
   uint64_t* v_empty = v_full + VS;
-  uint64_t* s_full = v_empty + VS;  // [2]
-  uint64_t* p_full = s_full + 2;   // [2 tiles][2 halves of the keys]
-  uint64_t* o_done = p_full + 4;   // [2]
-  uint64_t* drain = o_done + 2;
+  uint64_t* s_full = v_empty + VS;  // [NT]
+  uint64_t* p_full = s_full + NT;  // [NT tiles][2 halves of the keys]
+  uint64_t* o_done = p_full + 2 * NT;  // [NT]
+  uint64_t* drain = o_done + NT;
   uint64_t* kraw_full = drain + 1;   // [KS] int8 variant: TMA landed the int8 K tile
   uint64_t* vraw_full = kraw_full + KS;
   uint64_t* q_empty = vraw_full + VS;  // every S MMA of an item has read Q
-  uint64_t* o_free = q_empty + 1;       // [2] the softmax warps have read O_t out
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 2);
+  uint64_t* o_free = q_empty + 1;       // [NT] the softmax warps have read O_t out
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + NT);
   __shared__ int abort_flag;
 
-  // Persistent CTAs: CTA c takes one item per round of gridDim.x items of the
-  // longest-first order (item_at); every role walks the same sequence, with
-  // the K/V ring and every barrier phase counted across items.
-  const int n_items = A.n_qblocks * A.batch * (A.two_tiles ? A.hq / 2 : A.hq);
-  const int ntile = A.two_tiles ? 2 : 1;
+  // A CTA pair (cluster of two) runs M = 256 MMAs: CTA 0 issues them and owns
+  // the barriers they wait on; CTA 1's producer, converters and softmax warps
+  // signal those barriers remotely, and every MMA completion is signalled to
+  // the same barrier in both CTAs.
+  const int rank = kPair ? static_cast<int>(cluster_ctarank()) : 0;
+  const bool leader = rank == 0;
+  auto lead = [&](uint64_t* b) -> uint32_t { return kPair ? mapa_shared(smem_u32(b), 0) : smem_u32(b); };
+  // a barrier of the issuing CTA that some arrivals reach from the peer CTA
+  auto wait_x = [&](uint64_t* b, uint32_t ph) -> bool {
+    return kPair ? wait_parity<true>(b, ph, A.wd, &abort_flag) : wait_parity(b, ph, A.wd, &abort_flag);
+  };
+  // warp-level arrival on a barrier counted per thread (one CTA) or per warp
+  // of both CTAs (pair); the caller has made its TMEM / smem writes visible
+  auto arrive_x = [&](uint64_t* b) {
+    if constexpr (kPair) {
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(lead(b));
+    } else {
+      mbar_arrive(b);
+    }
+  };
+  auto commit = [&](uint64_t* b) {
+    if constexpr (kPair) mma_commit_pair_both(b);
+    else mma_commit(b);
+  };
+  // Persistent CTAs (pairs): unit u takes one item per round of n_units items
+  // of the longest-first order (item_at); every role of both CTAs of a pair
+  // walks the same sequence, with the K/V ring and every barrier phase
+  // counted across items.
+  const int unit = kPair ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int n_units = kPair ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
+  const int n_items = A.n_qblocks * A.batch * (A.hq / A.heads_per_item);
+  const int ntile = kPair ? 2 : A.heads_per_item;
+  constexpr uint32_t kArrivals = kPair ? 8 : kBM;  // warps of both CTAs, or threads of one
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(q_full, 1);
-    // bf16: TMA completes k_full / v_full; int8: the 128 converter threads do
+    // bf16: TMA completes k_full / v_full; int8: the converter threads do
     for (int s = 0; s < KS; ++s) {
-      mbar_init(k_full + s, kI8 ? 128 : 1);
+      mbar_init(k_full + s, kI8 ? kArrivals : 1);
       mbar_init(k_empty + s, 1);
       mbar_init(kraw_full + s, 1);
     }
     for (int s = 0; s < VS; ++s) {
-      mbar_init(v_full + s, kI8 ? 128 : 1);
+      mbar_init(v_full + s, kI8 ? kArrivals : 1);
       mbar_init(v_empty + s, 1);
       mbar_init(vraw_full + s, 1);
     }
-    for (int t = 0; t < 2; ++t) {
+    for (int t = 0; t < NT; ++t) {
       mbar_init(s_full + t, 1);
-      mbar_init(p_full + 2 * t, kBM);
-      mbar_init(p_full + 2 * t + 1, kBM);
+      mbar_init(p_full + 2 * t, kArrivals);
+      mbar_init(p_full + 2 * t + 1, kArrivals);
       mbar_init(o_done + t, 1);
+      mbar_init(o_free + t, kArrivals);
     }
     mbar_init(drain, 1);
     mbar_init(q_empty, 1);
-    mbar_init(o_free, kBM);
-    mbar_init(o_free + 1, kBM);
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(tmem_slot, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Roles split by warpgroup first: warpgroups 0-1 softmax, 2-3 the rest.
-  // int8 variant registers: 512 threads launched at 128; warpgroups 0-1 take
-  // 192, warpgroups 2-3 give back down to 64: 256*192 + 256*64 = 512*128.
-  if (warp >= 8) {
-  if constexpr (kI8) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
+  // Roles split by warpgroup first: the first NT warpgroups softmax, the rest
+  // the other roles.  int8 variant registers: 512 threads launched at 128;
+  // warpgroups 0-1 take 192, warpgroups 2-3 give back down to 64:
+  // 256*192 + 256*64 = 512*128.
+  if (warp >= 4 * NT) {
+  if constexpr (G::kRegsHi > 0) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -286,40 +383,54 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       prefetch_tensormap(&tm_v);
       int base = 0, done = 0;  // K/V tiles and items before this one
       bool ok = true;
-      for (int k = 0, item; ok && (item = item_at(blockIdx.x, gridDim.x, k)) < n_items; ++k) {
+      for (int k = 0, item; ok && (item = item_at(unit, n_units, k)) < n_items; ++k) {
         Item w;
-        if (!item_of(A, item, w)) continue;
+        if (!item_of<BN>(A, item, w, rank)) continue;
         // Q of this item once every S MMA of the previous one has read its Q
-        if (done > 0 && !wait_parity(q_empty, (done - 1) & 1, A.wd, &abort_flag)) break;
-        mbar_expect_tx(q_full, ntile * G::kQBytes);
+        if (done > 0 && !wait_parity<kPair>(q_empty, (done - 1) & 1, A.wd, &abort_flag)) break;
+        if (leader) mbar_expect_tx(q_full, (kPair ? 2 : 1) * ntile * G::kQBytes);
         for (int t = 0; t < ntile; ++t)
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem + t * G::kQBytes + c * kChunkBytes, &tm_q, q_full, 64 * c, w.q_prow, w.q_plane + t);
+          for (int c = 0; c < D / 64; ++c) {
+            uint8_t* dst = smem + t * G::kQBytes + c * kChunkBytes;
+            if constexpr (kPair) tma_load_3d_pair(dst, &tm_q, lead(q_full), 64 * c, w.q_prow, w.q_plane + t);
+            else tma_load_3d(dst, &tm_q, q_full, 64 * c, w.q_prow, w.q_plane + t);
+          }
         for (int it = 0; it < w.n_iter; ++it) {
           const int gi = base + it;
           int s = gi % KS, u = gi / KS;
           int kplane, krow;
-          kv_tile(A, w, (w.j_lo + it) * kBN, kplane, krow);
-          if (u > 0 && !(ok = wait_parity(k_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
+          kv_tile(A, w, (w.j_lo + it) * BN, kplane, krow);
+          if (u > 0 && !(ok = wait_parity<kPair>(k_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
+          // a pair's CTA r brings keys [64 r, 64 r + 64) of K and dims
+          // [D/2 r, D/2 r + D/2) of V
+          const int k_row = krow + (kPair ? 64 * rank : 0);
           if constexpr (kI8) {
-            mbar_expect_tx(kraw_full + s, G::kI8Bytes);
-            tma_load_3d(smem + G::k_stage(s), &tm_k, kraw_full + s, 0, krow, kplane);
-          } else {
-            mbar_expect_tx(k_full + s, G::kKVBytes);
+            mbar_expect_tx(kraw_full + s, G::kKI8Bytes);
+            tma_load_3d(smem + G::k_stage(s), &tm_k, kraw_full + s, 0, k_row, kplane);
+          } else if constexpr (kPair) {
+            if (leader) mbar_expect_tx(k_full + s, 2 * G::kKBytes);
             for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(smem + G::kKOff + s * G::kKVBytes + c * kChunkBytes, &tm_k, k_full + s, 64 * c, krow,
+              tma_load_3d_pair(smem + G::kKOff + s * G::kKBytes + c * G::kKChunk, &tm_k, lead(k_full + s), 64 * c,
+                               k_row, kplane);
+          } else {
+            mbar_expect_tx(k_full + s, G::kKBytes);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(smem + G::kKOff + s * G::kKBytes + c * G::kKChunk, &tm_k, k_full + s, 64 * c, krow,
                           kplane);
           }
           s = gi % VS;
           u = gi / VS;
-          if (u > 0 && !(ok = wait_parity(v_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
+          if (u > 0 && !(ok = wait_parity<kPair>(v_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
           if constexpr (kI8) {
-            mbar_expect_tx(vraw_full + s, G::kI8Bytes);
-            tma_load_3d(smem + G::v_stage(s), &tm_v, vraw_full + s, 0, krow, kplane);
+            mbar_expect_tx(vraw_full + s, G::kVI8Bytes);
+            tma_load_3d(smem + G::v_stage(s), &tm_v, vraw_full + s, kPair ? (D / 2) * rank : 0, krow, kplane);
+          } else if constexpr (kPair) {
+            if (leader) mbar_expect_tx(v_full + s, 2 * G::kVBytes);
+            tma_load_3d_pair(smem + G::kVOff + s * G::kVBytes, &tm_v, lead(v_full + s), (D / 2) * rank, krow, kplane);
           } else {
-            mbar_expect_tx(v_full + s, G::kKVBytes);
+            mbar_expect_tx(v_full + s, G::kVBytes);
             for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(smem + G::kVOff + s * G::kKVBytes + c * kChunkBytes, &tm_v, v_full + s, 64 * c, krow,
+              tma_load_3d(smem + G::kVOff + s * G::kVBytes + c * G::kVChunk, &tm_v, v_full + s, 64 * c, krow,
                           kplane);
           }
         }
@@ -329,33 +440,40 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // a negative softmax scale is folded into the S MMA (negated A operand),
       // so the softmax only ever sees a positive scale
-      const uint32_t idesc_s = umma_idesc_f16(kBM, kBN, 1, 1, false) | (A.negate_s << 13);
-      constexpr uint32_t idesc_o = umma_idesc_f16(kBM, D, 1, 1, true);
+      constexpr int kM = kPair ? 2 * kBM : kBM;
+      const uint32_t idesc_s = umma_idesc_f16(kM, BN, 1, 1, false) | (A.negate_s << 13);
+      constexpr uint32_t idesc_o = umma_idesc_f16(kM, D, 1, 1, true);
       const uint32_t q_base = smem_u32(smem);
       // operand descriptors are built once; a k-step only moves the start
       // address (its 14-bit field never carries: every address is < 2^18)
       const uint64_t dq0 = umma_desc_sw128(q_base, 16, 1024);
       const uint64_t dk0 = umma_desc_sw128(q_base + G::kKOff, 16, 1024);
-      const uint64_t dv0 = umma_desc_sw128(q_base + G::kVOff, kChunkBytes, 1024);
+      const uint64_t dv0 = umma_desc_sw128(q_base + G::kVOff, G::kVChunk, 1024);
       auto issue_s = [&](int t, int st) {
         const uint64_t dq = dq0 + ((t * G::kQBytes) >> 4);
-        const uint64_t dk = dk0 + ((st * G::kKVBytes) >> 4);
+        const uint64_t dk = dk0 + ((st * G::kKBytes) >> 4);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = ((k / 4) * kChunkBytes + (k % 4) * 32) >> 4;
-          mma_ss(tmem + t * kBN, dq + off, dk + off, idesc_s, k > 0 ? 1u : 0u);
+          const uint32_t off_q = ((k / 4) * kChunkBytes + (k % 4) * 32) >> 4;
+          const uint32_t off_k = ((k / 4) * G::kKChunk + (k % 4) * 32) >> 4;
+          if constexpr (kPair) mma_ss_pair(tmem + G::s_col(t), dq + off_q, dk + off_k, idesc_s, k > 0 ? 1u : 0u);
+          else mma_ss(tmem + G::s_col(t), dq + off_q, dk + off_k, idesc_s, k > 0 ? 1u : 0u);
         }
       };
-      // O_t += P_t V over keys [64 h, 64 h + 64)
+      // O_t += P_t V over keys [BN/2 h, BN/2 h + BN/2) (16-key MMA steps)
       auto issue_pv_half = [&](int t, int st, int h, bool accumulate) {
-        const uint64_t dv = dv0 + ((st * G::kKVBytes) >> 4);
+        const uint64_t dv = dv0 + ((st * G::kVBytes) >> 4);
+        constexpr int kHalf = BN / 32;
 #pragma unroll
-        for (int k = 4 * h; k < 4 * h + 4; ++k) {
-          mma_ts(tmem + 256 + t * D, tmem + t * kBN + k * 8, dv + ((k * 2048) >> 4), idesc_o,
-                 (accumulate || k > 0) ? 1u : 0u);
+        for (int k = kHalf * h; k < kHalf * h + kHalf; ++k) {
+          const uint32_t acc = (accumulate || k > 0) ? 1u : 0u;
+          if constexpr (kPair)
+            mma_ts_pair(tmem + G::o_col(t), tmem + G::s_col(t) + k * 8, dv + ((k * 2048) >> 4), idesc_o, acc);
+          else
+            mma_ts(tmem + G::o_col(t), tmem + G::s_col(t) + k * 8, dv + ((k * 2048) >> 4), idesc_o, acc);
         }
       };
       int base = 0, done = 0;  // K/V tiles and items before the current one
@@ -365,116 +483,113 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       auto issue_pv = [&](int t, int j) -> bool {
         const int gj = base + j;
         const int vs = gj % VS;
-        if (j == 0 && done > 0 && !wait_parity(o_free + t, (done - 1) & 1, A.wd, &abort_flag)) return false;
-        if (!wait_parity(p_full + 2 * t, gj & 1, A.wd, &abort_flag)) return false;
-        if (t == 0 && !wait_parity(v_full + vs, (gj / VS) & 1, A.wd, &abort_flag)) return false;
+        if (j == 0 && done > 0 && !wait_x(o_free + t, (done - 1) & 1)) return false;
+        if (!wait_x(p_full + 2 * t, gj & 1)) return false;
+        if (t == 0 && !wait_x(v_full + vs, (gj / VS) & 1)) return false;
         tc_fence_after();
         issue_pv_half(t, vs, 0, j > 0);
-        if (!wait_parity(p_full + 2 * t + 1, gj & 1, A.wd, &abort_flag)) return false;
+        if (!wait_x(p_full + 2 * t + 1, gj & 1)) return false;
         tc_fence_after();
         issue_pv_half(t, vs, 1, true);
         return true;
       };
       bool ok = true;
-      for (int k = 0, item; ok && (item = item_at(blockIdx.x, gridDim.x, k)) < n_items; ++k) {
+      for (int k = 0, item; ok && (item = item_at(unit, n_units, k)) < n_items; ++k) {
         Item w;
-        if (!item_of(A, item, w)) continue;
-        if (!(ok = wait_parity(q_full, done & 1, A.wd, &abort_flag))) break;
+        if (!item_of<BN>(A, item, w, rank)) continue;
+        if (!(ok = wait_x(q_full, done & 1))) break;
         for (int it = 0; ok && it < w.n_iter; ++it) {
           const int gi = base + it;
           const int s = gi % KS;
-          if (!(ok = wait_parity(k_full + s, (gi / KS) & 1, A.wd, &abort_flag))) break;
+          if (!(ok = wait_x(k_full + s, (gi / KS) & 1))) break;
           tc_fence_after();
           for (int t = 0; t < ntile; ++t) {
             if (it > 0) {
               if (!(ok = issue_pv(t, it - 1))) break;
-              if (t == ntile - 1) mma_commit(v_empty + (gi - 1) % VS);
+              if (t == ntile - 1) commit(v_empty + (gi - 1) % VS);
             }
             issue_s(t, s);
-            mma_commit(s_full + t);
+            commit(s_full + t);
           }
-          if (ok) mma_commit(k_empty + s);
+          if (ok) commit(k_empty + s);
         }
         if (!ok) break;
-        mma_commit(q_empty);  // Q is free once this item's S MMAs complete
+        commit(q_empty);  // Q is free once this item's S MMAs complete
         for (int t = 0; t < ntile; ++t) {
           if (!(ok = issue_pv(t, w.n_iter - 1))) break;
-          mma_commit(o_done + t);
+          commit(o_done + t);
         }
         if (!ok) break;
-        mma_commit(v_empty + (base + w.n_iter - 1) % VS);
+        commit(v_empty + (base + w.n_iter - 1) % VS);
         base += w.n_iter;
         ++done;
       }
       // every MMA this thread issued has completed before TMEM is released
-      mma_commit(drain);
+      commit(drain);
       wait_parity(drain, 0, A.wd);
     }
   } else if (kI8 && warp >= kConvWarp0) {
     // ------------------------------------------------------------ int8 -> bf16 converters
-    // thread r rewrites row r of each int8 K and V tile as bf16 in the
-    // 128-byte-swizzled K-major (K) / MN-major (V) operand layout
+    // One CTA: thread r rewrites key row r of each int8 K and V tile as bf16
+    // in the 128-byte-swizzled K-major (K) / MN-major (V) operand layout.
+    // Pair: this CTA's K slot holds 64 key rows (thread r converts half row
+    // r / 2, dims [64 (r % 2), +64)) and its V slot 64 dims of 128 key rows
+    // (thread r converts row r).
     const int r = static_cast<int>(threadIdx.x) - kConvWarp0 * 32;
-    auto convert_row = [&](const uint8_t* src_tile, uint8_t* dst_tile, float sc) {
-      const float2 s2 = make_float2(sc, sc);
-#pragma unroll
-      for (int c = 0; c < D / 16; ++c) {  // 16-byte int8 chunks of the row
-        const int pc = (D == 128) ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
-        const uint4 w = *reinterpret_cast<const uint4*>(src_tile + r * D + pc * 16);
-        const int h = c / 4, j0 = 2 * (c % 4);
-        uint8_t* row = dst_tile + h * kChunkBytes + r * 128;
-        const uint2 y0 = dequant4_bf16(w.x, s2), y1 = dequant4_bf16(w.y, s2);
-        const uint2 y2 = dequant4_bf16(w.z, s2), y3 = dequant4_bf16(w.w, s2);
-        *reinterpret_cast<uint4*>(row + ((j0 ^ (r & 7)) * 16)) = make_uint4(y0.x, y0.y, y1.x, y1.y);
-        *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ (r & 7)) * 16)) = make_uint4(y2.x, y2.y, y3.x, y3.y);
-      }
-    };
+    const int k_r = kPair ? r / 2 : r;                  // K row this thread converts
+    const int k_c0 = kPair ? (r % 2) * 4 : 0;           // its first 16-byte chunk
+    constexpr int k_nc = kPair ? 4 : D / 16;
+    constexpr int v_rl = kPair ? D / 2 : D;             // staged V row bytes
     int base = 0;
     bool ok = true;
-    for (int k = 0, item; ok && (item = item_at(blockIdx.x, gridDim.x, k)) < n_items; ++k) {
+    for (int k = 0, item; ok && (item = item_at(unit, n_units, k)) < n_items; ++k) {
       Item w;
-      if (!item_of(A, item, w)) continue;
+      if (!item_of<BN>(A, item, w, rank)) continue;
       for (int it = 0; it < w.n_iter; ++it) {
         const int gi = base + it;
         const int s = gi % KS, sv = gi % VS;
         const uint32_t ph = (gi / KS) & 1, phv = (gi / VS) & 1;
-        // this thread's key row: its two scales, loaded ahead of the waits (0
+        // this thread's key rows: their scales, loaded ahead of the waits (0
         // past the sequence end, so those rows become zeros; the softmax masks them)
-        const int key0 = (w.j_lo + it) * kBN;
+        const int key0 = (w.j_lo + it) * BN;
+        const int kkey = key0 + (kPair ? 64 * rank : 0) + k_r, vkey = key0 + r;
         float ksc = 0.f, vsc = 0.f;
-        if (key0 + r < w.sq.s_k) {
+        {
           int kplane, krow;
           kv_tile(A, w, key0, kplane, krow);
-          const int64_t at = static_cast<int64_t>(kplane) * A.k_plane_rows + krow + r;
-          ksc = __ldg(A.k_scales + at);
-          vsc = __ldg(A.v_scales + at);
+          const int64_t at = static_cast<int64_t>(kplane) * A.k_plane_rows + krow;
+          if (kkey < w.sq.s_k) ksc = __ldg(A.k_scales + at + (kkey - key0));
+          if (vkey < w.sq.s_k) vsc = __ldg(A.v_scales + at + r);
         }
         if (!(ok = __all_sync(0xffffffffu, wait_parity(kraw_full + s, ph, A.wd, &abort_flag)))) break;
-        convert_row(smem + G::k_stage(s), smem + G::kKOff + s * G::kKVBytes, ksc);
+        convert_int8_row<k_nc, D>(smem + G::k_stage(s), smem + G::kKOff + s * G::kKBytes, G::kKChunk, k_r, k_c0,
+                                  ksc);
         fence_proxy_async_smem();
-        mbar_arrive(k_full + s);
+        arrive_x(k_full + s);
         if (!(ok = __all_sync(0xffffffffu, wait_parity(vraw_full + sv, phv, A.wd, &abort_flag)))) break;
-        convert_row(smem + G::v_stage(sv), smem + G::kVOff + sv * G::kKVBytes, vsc);
+        convert_int8_row<v_rl / 16, v_rl>(smem + G::v_stage(sv), smem + G::kVOff + sv * G::kVBytes, G::kVChunk, r,
+                                          0, vsc);
         fence_proxy_async_smem();
-        mbar_arrive(v_full + sv);
+        arrive_x(v_full + sv);
       }
       base += w.n_iter;
     }
   }
   } else {
-  if constexpr (kI8) asm volatile("setmaxnreg.inc.sync.aligned.u32 192;" ::: "memory");
+  if constexpr (G::kRegsHi == 192) asm volatile("setmaxnreg.inc.sync.aligned.u32 192;" ::: "memory");
+  if constexpr (G::kRegsHi == 104) asm volatile("setmaxnreg.inc.sync.aligned.u32 104;" ::: "memory");
   if (warp / 4 < ntile) {
     // ------------------------------------------------------------ softmax
     const int t = warp / 4, quarter = warp % 4;
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_tm = tmem + lane_base + t * kBN;
-    const uint32_t o_tm = tmem + lane_base + 256 + t * D;
+    const uint32_t s_tm = tmem + lane_base + G::s_col(t);
+    const uint32_t o_tm = tmem + lane_base + G::o_col(t);
     int base = 0, done = 0;  // K/V tiles and items before the current one
     bool ok = true;
-    for (int k = 0, item; ok && (item = item_at(blockIdx.x, gridDim.x, k)) < n_items; ++k) {
+    for (int k = 0, item; ok && (item = item_at(unit, n_units, k)) < n_items; ++k) {
     Item w;
-    if (!item_of(A, item, w)) continue;
+    if (!item_of<BN>(A, item, w, rank)) continue;
     const int i = w.i0 + r;
     int lo, hi;
     band_of(A.L, i, w.sq.s_q, w.sq.s_k, lo, hi);
@@ -488,35 +603,39 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
     }
     float m_used = -INFINITY, l = 0.f;
     for (int it = 0; it < w.n_iter; ++it) {
-      ok = __all_sync(0xffffffffu, wait_parity(s_full + t, (base + it) & 1, A.wd, &abort_flag));
+      ok = __all_sync(0xffffffffu, wait_parity<kPair>(s_full + t, (base + it) & 1, A.wd, &abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t raw[4][32];
-      tmem_ld32(s_tm + 0, raw[0]);
-      tmem_ld32(s_tm + 32, raw[1]);
-      tmem_ld32(s_tm + 64, raw[2]);
-      tmem_ld32(s_tm + 96, raw[3]);
+      constexpr int kCh = BN / 32;  // 32-column chunks of the S row
+      uint32_t raw[kCh][32];
+#pragma unroll
+      for (int c = 0; c < kCh; ++c) tmem_ld32(s_tm + 32 * c, raw[c]);
       tmem_wait_ld();
-      const int kb = (w.j_lo + it) * kBN;
-      if (!(kb >= lo && kb + kBN <= hi)) {
+      const int kb = (w.j_lo + it) * BN;
+      if (!(kb >= lo && kb + BN <= hi)) {
         // boundary tile: keys outside this row's band become -inf (the
         // softmax scale is positive, so masking before it is the same)
         const int va = lo - kb, vb = hi - kb;
 #pragma unroll
-        for (int c = 0; c < kBN; ++c)
+        for (int c = 0; c < BN; ++c)
           if (c < va || c >= vb) raw[c / 32][c % 32] = 0xff800000u;
       }
-      // row max of the raw scores: eight independent chains of 3-input max
-      float g8[8];
+      // row max of the raw scores: BN / 16 independent chains of 3-input max
+      float g8[2 * kCh];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < 2 * kCh; ++k) {
         const uint32_t* v = &raw[k / 2][(k % 2) * 16];
         float g = max3f(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
 #pragma unroll
         for (int e = 3; e < 15; e += 2) g = max3f(g, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
         g8[k] = fmaxf(g, __uint_as_float(v[15]));
       }
-      const float m_raw = fmaxf(max3f(g8[0], g8[1], g8[2]), max3f(max3f(g8[3], g8[4], g8[5]), g8[6], g8[7]));
+      float m_raw;
+      if constexpr (kCh == 4) {
+        m_raw = fmaxf(max3f(g8[0], g8[1], g8[2]), max3f(max3f(g8[3], g8[4], g8[5]), g8[6], g8[7]));
+      } else {
+        m_raw = fmaxf(max3f(g8[0], g8[1], g8[2]), g8[3]);
+      }
       const float m_tile = m_raw * A.scale_log2;
       const float m_new = fmaxf(m_used, m_tile);
       const bool need = m_new > m_used + kRescaleThreshold;
@@ -528,23 +647,27 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       const float2 sc2 = make_float2(A.scale_log2, A.scale_log2);
       const float2 nm2 = make_float2(neg_m, neg_m);
-      float2 lacc[8];
+      constexpr int kL = kCh == 4 ? 8 : 4;  // independent row-sum chains
+      float2 lacc[kL];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) lacc[k] = make_float2(0.f, 0.f);
+      for (int k = 0; k < kL; ++k) lacc[k] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < kCh; ++cc) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           // p = 2^(s * scale * log2(e) - m): one packed FMA for two scores
           const float2 x = fma2(make_float2(__uint_as_float(raw[cc][2 * e]), __uint_as_float(raw[cc][2 * e + 1])),
                                 sc2, nm2);
-          const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          lacc[e % 8] = add2(lacc[e % 8], pp);
+          // every kPolyEvery-th pair of a 32-column chunk on the FMA pipe
+          const float2 pp = (kPolyEvery > 0 && e % kPolyEvery == kPolyEvery - 1)
+                                ? exp2_poly2(x)
+                                : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          lacc[e % kL] = add2(lacc[e % kL], pp);
           pk[e] = pack_bf16x2(pp.x, pp.y);
         }
         tmem_st16(s_tm + cc * 16, pk);
-        if (cc == 1 && it > 0 && __any_sync(0xffffffffu, need)) {
+        if (cc == kCh / 2 - 1 && it > 0 && __any_sync(0xffffffffu, need)) {
           // O_t is idle here (PV_t of the previous step has completed, this
           // step's starts only after the signal below): rescale it if some
           // row's max moved (rare; the first half's scores are dead by now)
@@ -558,21 +681,23 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
             tmem_st32(o_tm + oc * 32, o);
           }
         }
-        if (cc % 2 == 1) {
-          // keys [64 h, 64 h + 64) of P are in TMEM: let the PV MMA start on them
+        if (cc % (kCh / 2) == kCh / 2 - 1) {
+          // keys [BN/2 h, BN/2 h + BN/2) of P are in TMEM: let the PV MMA start on them
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(p_full + 2 * t + cc / 2);
+          arrive_x(p_full + 2 * t + cc / (kCh / 2));
         }
       }
+      if constexpr (kL == 8) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) lacc[k] = add2(lacc[k], lacc[k + 4]);
+        for (int k = 0; k < 4; ++k) lacc[k] = add2(lacc[k], lacc[k + 4]);
+      }
       lacc[0] = add2(lacc[0], lacc[2]);
       lacc[1] = add2(lacc[1], lacc[3]);
       lacc[0] = add2(lacc[0], lacc[1]);
       l = l * alpha + (lacc[0].x + lacc[0].y);
     }
-    if (ok) ok = __all_sync(0xffffffffu, wait_parity(o_done + t, done & 1, A.wd, &abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, wait_parity<kPair>(o_done + t, done & 1, A.wd, &abort_flag));
     if (!ok) break;
     tc_fence_after();
     const bool has_keys = lo < hi;
@@ -607,7 +732,7 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
       if (oc == D / 32 - 1) {
         // O_t is in registers: the next item's first PV may overwrite it
         tc_fence_before();
-        mbar_arrive(o_free + t);
+        arrive_x(o_free + t);
       }
       float y[32];
 #pragma unroll
@@ -649,15 +774,50 @@ __global__ void __launch_bounds__(TcGeom<D, kI8>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // pair: CTA 0's MMAs (all complete: its issuer drained them) wrote this
+  // CTA's TMEM and read its shared memory, and this CTA's arrivals reached
+  // CTA 0's barriers; neither CTA releases TMEM or exits before both are here
+  if constexpr (kPair) cluster_sync_all();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    if constexpr (kPair) tmem_dealloc_pair(tmem, 512);
+    else tmem_dealloc(tmem, 512);
   }
 }
 
-template <int D, bool kI8>
+
+
+// Clusters of two of this kernel that fit on the device at once (cached per
+// device and variant); 0 when the query fails.
+template <typename K>
+int max_pair_clusters(K kern, uint32_t smem, int threads) {
+  static std::mutex mu;
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cached[dev] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * static_cast<unsigned>(device_sm_count()));
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <int D, bool kI8, bool kPair, int BN = 128, int NT = 2>
 fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowSink& sink, const LaunchCtx& ctx) {
-  using G = TcGeom<D, kI8>;
+  using G = TcGeom<D, kI8, kPair, BN, NT>;
   const bool varlen = p.cu_seqlens_q != nullptr;
   const uint64_t q_rows = varlen ? p.total_q : p.seqlen_q;
   // paged keys: planes of page_size rows, one per (page, KV head)
@@ -675,24 +835,33 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowS
                                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != FA_OK) return st;
   }
+  // K boxes: G::kKRows key rows (a pair's CTA takes 64 of each 128-key
+  // tile); V boxes: BN keys of 64 dims (one CTA: every dim chunk in turn;
+  // pair: this CTA's half)
+  const uint32_t krows = static_cast<uint32_t>(G::kKRows);
   if constexpr (kI8) {
-    // int8 rows of D bytes, one box per tile (128 B or 64 B swizzle)
-    const uint32_t box[3] = {static_cast<uint32_t>(D), static_cast<uint32_t>(kSwizzleChunkRows), 1};
+    // int8 rows: K boxes of whole rows (D bytes), V boxes of this CTA's
+    // dims (D bytes, or D / 2 in a pair): 128- or 64-byte swizzle
     const uint64_t dims[3] = {static_cast<uint64_t>(D), k_rows, k_planes};
     const uint64_t strides[2] = {static_cast<uint64_t>(D), k_rows * D};
-    const CUtensorMapSwizzle sw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    fa_status st = encode_tensor_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, p.k, dims, strides, box, sw);
+    const uint32_t kbox[3] = {static_cast<uint32_t>(D), krows, 1};
+    const uint32_t vw = kPair ? D / 2 : D;
+    const uint32_t vbox[3] = {vw, static_cast<uint32_t>(BN), 1};
+    const CUtensorMapSwizzle ksw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUtensorMapSwizzle vsw = vw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    fa_status st = encode_tensor_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, p.k, dims, strides, kbox, ksw);
     if (st != FA_OK) return st;
-    st = encode_tensor_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, p.v, dims, strides, box, sw);
+    st = encode_tensor_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, p.v, dims, strides, vbox, vsw);
     if (st != FA_OK) return st;
   } else {
-    const uint32_t box[3] = {64, static_cast<uint32_t>(kSwizzleChunkRows), 1};
     const uint64_t dims[3] = {static_cast<uint64_t>(D), k_rows, k_planes};
     const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, k_rows * D * 2};
-    fa_status st = encode_tensor_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.k, dims, strides, box,
+    const uint32_t kbox[3] = {64, krows, 1};
+    const uint32_t vbox[3] = {64, static_cast<uint32_t>(BN), 1};
+    fa_status st = encode_tensor_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.k, dims, strides, kbox,
                                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != FA_OK) return st;
-    st = encode_tensor_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.v, dims, strides, box,
+    st = encode_tensor_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.v, dims, strides, vbox,
                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != FA_OK) return st;
   }
@@ -712,6 +881,7 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowS
   A.hkv = p.hkv;
   A.group = p.hq / p.hkv;
   A.two_tiles = (A.group % 2 == 0) ? 1 : 0;
+  A.heads_per_item = (kPair || NT == 4) ? 4 : (A.two_tiles ? 2 : 1);
   const int max_sq = varlen ? p.max_seqlen_q : p.seqlen_q;
   A.n_qblocks = (max_sq + kBM - 1) / kBM;
   // the softmax works with a positive scale: a negative one negates Q inside
@@ -721,32 +891,83 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowS
   A.negate_s = p.softmax_scale < 0.f ? 1u : 0u;
   A.epi = make_epilogue(p.epilogue, p.n_epilogue);
   A.wd = ctx.wd;
-  const long long n_pairs = A.two_tiles ? p.hq / 2 : p.hq;
-  const long long items = static_cast<long long>(A.n_qblocks) * p.batch * n_pairs;
+  const long long items = static_cast<long long>(A.n_qblocks) * p.batch * (p.hq / A.heads_per_item);
   if (items == 0) return FA_OK;
   if (items > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-  // persistent: one CTA per SM (the shared memory allows no second), each
-  // walking its share of the items
-  const long long grid = items < device_sm_count() ? items : device_sm_count();
-  auto kern = prefill_tc_kernel<D, kI8>;
+  auto kern = prefill_tc_kernel<D, kI8, kPair, BN, NT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem) != cudaSuccess)
     return FA_ERR_CUDA;
   note_variant(reinterpret_cast<const void*>(kern));
-  kern<<<static_cast<unsigned>(grid), G::kThreads, G::kSmem, ctx.stream>>>(tq, tk, tv, A);
-  return cuda_status(cudaGetLastError());
+  if constexpr (kPair) {
+    // persistent clusters of two CTAs (one per SM), as many as fit at once
+    const int fit = max_pair_clusters(kern, G::kSmem, G::kThreads);
+    if (fit <= 0) return FA_ERR_CUDA;
+    const long long clusters = items < fit ? items : fit;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
+    cfg.blockDim = dim3(G::kThreads);
+    cfg.dynamicSmemBytes = G::kSmem;
+    cfg.stream = ctx.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, A));
+  } else {
+    // persistent: one CTA per SM (the shared memory allows no second), each
+    // walking its share of the items
+    const long long grid = items < device_sm_count() ? items : device_sm_count();
+    kern<<<static_cast<unsigned>(grid), G::kThreads, G::kSmem, ctx.stream>>>(tq, tk, tv, A);
+    return cuda_status(cudaGetLastError());
+  }
+}
+
+// The CTA-pair kernel (one K/V fetch for four heads of a group) serves d =
+// 128 when every item's four heads share one KV head (group size a multiple
+// of 4) and FA_PREFILL_PAIR=1 (read once).  It is not the default: its
+// cross-SM hand-offs (the peer's P to the issuing CTA, completions back)
+// lengthen the softmax -> PV -> S chain that bounds this kernel, and it
+// measured slower than one CTA per head pair on every workload.
+bool use_pair(const fa_fwd_params& p) {
+  static const bool enabled = [] {
+    const char* e = std::getenv("FA_PREFILL_PAIR");
+    return e != nullptr && e[0] == '1';
+  }();
+  return enabled && p.head_dim == 128 && (p.hq / p.hkv) % 4 == 0;
 }
 
 }  // namespace
 
+// d = 64 bf16 with every four consecutive heads in one GQA group: one CTA
+// takes four heads (a whole group of four) with 64-key tiles, so four
+// softmax tiles share the SM's exponential units and every K/V tile serves
+// the four heads.  Selected by FA_PREFILL_QUAD=1 (read once): it measured
+// slower than the two-head kernel on the varlen window workload (each
+// 64-key step pays the same waits and hand-offs as a 128-key one).
+bool use_quad(const fa_fwd_params& p) {
+  static const bool enabled = [] {
+    const char* e = std::getenv("FA_PREFILL_QUAD");
+    return e != nullptr && e[0] == '1';
+  }();
+  return enabled && p.head_dim == 64 && p.kv_dtype != FA_I8 && (p.hq / p.hkv) % 4 == 0;
+}
+
 fa_status launch_prefill_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowSink& sink,
                             const LaunchCtx& ctx) {
+  const bool pair = use_pair(p);
   if (p.kv_dtype == FA_I8) {
-    if (p.head_dim == 128) return launch_tc<128, true>(p, pages, sink, ctx);
-    if (p.head_dim == 64) return launch_tc<64, true>(p, pages, sink, ctx);
+    if (p.head_dim == 128) return pair ? launch_tc<128, true, true>(p, pages, sink, ctx)
+                                       : launch_tc<128, true, false>(p, pages, sink, ctx);
+    if (p.head_dim == 64) return launch_tc<64, true, false>(p, pages, sink, ctx);
     return FA_ERR_UNSUPPORTED;
   }
-  if (p.head_dim == 128) return launch_tc<128, false>(p, pages, sink, ctx);
-  if (p.head_dim == 64) return launch_tc<64, false>(p, pages, sink, ctx);
+  if (p.head_dim == 128) return pair ? launch_tc<128, false, true>(p, pages, sink, ctx)
+                                     : launch_tc<128, false, false>(p, pages, sink, ctx);
+  if (p.head_dim == 64) return use_quad(p) ? launch_tc<64, false, false, 64, 4>(p, pages, sink, ctx)
+                                           : launch_tc<64, false, false>(p, pages, sink, ctx);
   return FA_ERR_UNSUPPORTED;
 }
 

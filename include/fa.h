@@ -170,7 +170,9 @@ FA_API fa_status fa_attention_fwd(const fa_fwd_params *p, fa_stream_t stream);
  * keys each warp is given (fewer, longer ranges).  capacity must be a
  * multiple of 32; cache entries at or past L_b may hold any bytes (they never
  * reach the result).
- * Supported: head_dim 128 (FA_I8 and FA_BF16) or 64; hq / hkv <= 8.
+ * Supported: head_dim 128 (FA_I8 and FA_BF16) or 64; any hq / hkv (a group
+ * of more than 8 query heads is served in passes of at most 8 heads, each
+ * reading the KV head's cache once).
  */
 typedef struct {
     const void *q;
@@ -192,8 +194,8 @@ typedef struct {
     size_t workspace_bytes;
 } fa_decode_params;
 
-/* Bytes of decode workspace at these sizes (any hkv dividing hq with
- * hq / hkv <= 8; the count of SMs of the current device enters it). */
+/* Bytes of decode workspace at these sizes (any hkv dividing hq; the count
+ * of SMs of the current device enters it). */
 FA_API size_t fa_decode_workspace_size(int32_t batch, int32_t hq, int32_t capacity, int32_t head_dim);
 
 FA_API fa_status fa_attention_decode(const fa_decode_params *p, fa_stream_t stream);

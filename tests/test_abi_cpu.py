@@ -148,7 +148,7 @@ def test_decode_rejects_bad_arguments(fa):
     assert call(decode_p(fa, max_seqlen=2048)) == fa.FA_ERR_INVALID     # above capacity
     assert call(decode_p(fa, split_keys=100)) == fa.FA_ERR_INVALID
     assert call(decode_p(fa, head_dim=96)) == fa.FA_ERR_UNSUPPORTED
-    assert call(decode_p(fa, hq=32, hkv=2)) == fa.FA_ERR_UNSUPPORTED    # group of 16
+    assert call(decode_p(fa, hq=32, hkv=2)) != fa.FA_ERR_UNSUPPORTED    # a group of 16 runs in two passes
     assert call(decode_p(fa, k_scales=None)) == fa.FA_ERR_INVALID
     assert call(decode_p(fa, workspace_bytes=16)) == fa.FA_ERR_WORKSPACE
     assert call(decode_p(fa, workspace=None)) == fa.FA_ERR_WORKSPACE

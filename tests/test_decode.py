@@ -48,6 +48,9 @@ CASES = [
     (2, 16, 2, 128, 768, [700, 100]),         # G = 8
     (2, 4, 2, 64, 1024, [999, 64]),           # d = 64
     (1, 2, 1, 128, 256, [256]),               # the page's s_k = 256 decode step
+    (2, 32, 2, 128, 1024, [1000, 77]),        # G = 16: two passes of 8 heads
+    (2, 24, 2, 64, 512, [300, 512]),          # G = 12: two passes of 6
+    (1, 9, 1, 128, 512, [400]),               # G = 9: three passes of 3
 ]
 
 

@@ -46,11 +46,12 @@ def paginate(dense, scales, lengths, hkv, page_size, extra, rng):
 
 
 @pytest.mark.parametrize("int8", [True, False])
-@pytest.mark.parametrize("d,page_size,window", [(128, 64, 0), (128, 256, 0), (64, 32, 0), (128, 64, 300)])
-def test_paged_equals_dense(int8, d, page_size, window):
+@pytest.mark.parametrize("d,page_size,window,hq,hkv", [(128, 64, 0, 16, 4), (128, 256, 0, 16, 4), (64, 32, 0, 16, 4),
+                                                       (128, 64, 300, 16, 4), (128, 64, 0, 32, 2)])
+def test_paged_equals_dense(int8, d, page_size, window, hq, hkv):
     fa = _fa()
-    rng = np.random.default_rng(d + page_size + window + int8)
-    B, hq, hkv, cap = 6, 16, 4, 1024
+    rng = np.random.default_rng(d + page_size + window + int8 + hq)
+    B, cap = 6, 1024
     lengths = [1000, 1, 0, 512, 1024, 333]
     k = torch.from_numpy(rng.standard_normal((B * hkv, cap, d)).astype(np.float32)).bfloat16()
     v = torch.from_numpy(rng.standard_normal((B * hkv, cap, d)).astype(np.float32)).bfloat16()

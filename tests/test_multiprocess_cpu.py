@@ -155,3 +155,18 @@ def test_ring_schedule_gloo(tmp_path, world, causal):
                        start_method="spawn")
     errs = [float(open(tmp_path / f"ring{r}.txt").read()) for r in range(world)]
     assert max(errs) < 1e-12, errs
+
+
+def test_ring_job_flops_counts_the_whole_band():
+    """The N-GPU ring line counts the causal band over all ranks' positions:
+    one rank is the single-GPU headline step; N ranks is the same tile rule
+    over N * 4096 positions (a triangle of 32 N (32 N + 1) / 2 tiles per
+    head plane)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from flashattention_attention_b200 import inputs
+    w = inputs.gqa_causal_prefill()
+    assert bench.ring_job_flops(1) == bench.prefill_flops(w)[0]
+    for n in (2, 4, 8):
+        t = 32 * n
+        assert bench.ring_job_flops(n) == 4 * 32 * 4 * 128 * 128 * 128 * (t * (t + 1) // 2)
