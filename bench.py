@@ -662,7 +662,7 @@ def decode_and_quant(args, dev, peaks, world, dist, result):
     """int8-KV decode and the quantiser on the decode workload."""
     import torch
     from flashattention_attention_b200 import fa, inputs
-    dw = inputs.int8kv_decode()
+    dw = inputs.int8kv_decode(batch=4) if args.profile_small else inputs.int8kv_decode()
     if args.only in ("all", "quant"):
         # the quantiser over every valid (token, kv-head) row of K and V, packed
         rows = torch.cat([t[b * dw.hkv:(b + 1) * dw.hkv, :dw.lengths[b]].reshape(-1, dw.d)
@@ -936,8 +936,8 @@ def main():
                     help="oracle seconds per sampled step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-small", action="store_true",
-                    help="profiler captures: the int8-KV long prefill at S=8192 (same kernel, inputs still "
-                         "larger than L2)")
+                    help="profiler captures: the int8-KV long prefill at S=8192 and the decodes over 4 of the "
+                         "16 sequences (same kernels, inputs still larger than L2)")
     ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "quant", "prefill_int8", "varlen", "ring", "tq"],
                     help="time one part only (used for profiler captures)")
     args = ap.parse_args()

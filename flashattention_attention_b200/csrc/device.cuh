@@ -368,29 +368,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return d;
 }
 
-// 2^x for a pair of fp32 values on the FMA and integer pipes, leaving the
-// MUFU to the other exponentials of a row.  Range reduction: adding 1.5 * 2^23
-// rounds x to the nearest integer n in the low mantissa bits of the sum (exact
-// for |x| < 2^22), so x = n + f with f in [-1/2, 1/2] computed exactly.  2^f
-// is a degree-3 polynomial whose coefficients were fitted for this file to
-// the least maximum relative error on [-1/2, 1/2] (Remez exchange on a dense
-// grid; 7.5e-5 in fp32 Horner evaluation, far below the bf16 rounding of P),
-// and n is added to the exponent field.  x is clamped to >= -125 so the result
-// stays a normal number: below that it returns about 2^-125 instead of 0 (an
-// exponential that small changes no fp32 sum it enters).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = add2(x, make_float2(12582912.f, 12582912.f));
-  const float2 n = add2(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = fma2(n, make_float2(-1.f, -1.f), x);
-  float2 p = fma2(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.2426111251f, 0.2426111251f));
-  p = fma2(p, f, make_float2(0.6932609677f, 0.6932609677f));
-  p = fma2(p, f, make_float2(0.9999280572f, 0.9999280572f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
 // Epilogue op list as kernel argument data (values never compiled in).
 struct Epilogue {
   int n;

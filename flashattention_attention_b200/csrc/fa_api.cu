@@ -77,6 +77,12 @@ fa_status make_ctx(fa_stream_t s, LaunchCtx* ctx) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Head sizes of the tensor-core prefill: bf16 K/V 32, 64, 96 or 128; int8 K/V 64 or 128.
+bool tc_head_dim_ok(int d, int kv_dtype) {
+  if (kv_dtype == FA_I8) return d == 64 || d == 128;
+  return d == 32 || d == 64 || d == 96 || d == 128;
+}
+
 bool epilogue_ok(const fa_epi_op* ops, int n) {
   if (n < 0 || n > FA_MAX_EPILOGUE) return false;
   for (int i = 0; i < n; ++i) {
@@ -206,7 +212,7 @@ fa_status fwd_args(const fa_fwd_params* p, bool* launch, bool need_out = true) {
     if (p->kv_dtype == FA_I8 && !no_keys && (p->k_scales == nullptr || p->v_scales == nullptr))
       return FA_ERR_INVALID;
     if (p->kv_dtype == FA_I8 && (!aligned16(p->k_scales) || !aligned16(p->v_scales))) return FA_ERR_INVALID;
-    if (p->head_dim != 64 && p->head_dim != 128) return FA_ERR_UNSUPPORTED;
+    if (!tc_head_dim_ok(p->head_dim, p->kv_dtype)) return FA_ERR_UNSUPPORTED;
   } else {
     return FA_ERR_INVALID;
   }
@@ -301,7 +307,7 @@ fa_status fa_attention_fwd_paged(const fa_fwd_params* p, const fa_kv_pages* page
   if (!std::isfinite(p->softmax_scale)) return FA_ERR_INVALID;
   if (p->q_dtype != FA_BF16 || (p->kv_dtype != FA_BF16 && p->kv_dtype != FA_I8)) return FA_ERR_INVALID;
   if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
-  if (p->head_dim != 64 && p->head_dim != 128) return FA_ERR_UNSUPPORTED;
+  if (!tc_head_dim_ok(p->head_dim, p->kv_dtype)) return FA_ERR_UNSUPPORTED;
   if (p->kv_dtype == FA_I8 && (p->k_scales == nullptr || p->v_scales == nullptr || !aligned16(p->k_scales) ||
                                !aligned16(p->v_scales)))
     return FA_ERR_INVALID;

@@ -67,13 +67,6 @@ namespace {
 constexpr int kBM = 128;  // query rows per Q tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
-// Exponentials of the softmax: every kPolyEvery-th pair of scores is
-// computed by exp2_poly2 (FMA and integer pipes) instead of the MUFU; 0: all
-// on the MUFU.
-#ifndef FA_EXP2_POLY_EVERY
-#define FA_EXP2_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = FA_EXP2_POLY_EVERY;
 constexpr uint32_t kChunkBytes = kSwizzleChunkRows * 128;  // [128 rows x 64 bf16]
 
 // BN keys per K/V tile, NT Q tiles (query heads) per CTA.  Warps 0 .. 4 NT - 1
@@ -92,6 +85,12 @@ struct TcGeom {
   // of V), so its rings can be deeper.
   static constexpr int kKStages = kPair ? (kI8 ? 3 : 4) : (NT == 4 ? 6 : 3);
   static constexpr int kVStages = kPair ? (kI8 ? 3 : 4) : (NT == 4 ? 6 : ((D == 128) ? 2 : 3));
+  // D = 64 kNFull + 32 kTail: kNFull chunks of 64 dims (128-byte rows,
+  // 128-byte swizzle), then, for an odd multiple of 32, one chunk of 32 dims
+  // (64-byte rows, 64-byte swizzle) after them
+  static constexpr int kNFull = D / 64;
+  static constexpr bool kTail = (D % 64) == 32;
+  static_assert(D % 32 == 0, "head size");
   static constexpr uint32_t kQBytes = kBM * D * 2;
   static constexpr int kKRows = kPair ? BN / 2 : BN;               // K rows in this CTA's slot
   static constexpr uint32_t kKChunk = kKRows * 128;                 // one 64-dim chunk of them
@@ -269,7 +268,9 @@ __device__ __forceinline__ int item_at(int c, int G, int k) {
 template <int D, bool kI8, bool kPair, int BN, int NT>
 __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const PrefillArgs A) {
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q32,
+                      const __grid_constant__ CUtensorMap tm_k32, const __grid_constant__ CUtensorMap tm_v32,
+                      const PrefillArgs A) {
   using G = TcGeom<D, kI8, kPair, BN, NT>;
   constexpr int KS = G::kKStages, VS = G::kVStages;
   constexpr int kLoadWarp = G::kLoadWarp, kMmaWarp = G::kMmaWarp, kConvWarp0 = G::kConvWarp0;
@@ -389,12 +390,16 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
         // Q of this item once every S MMA of the previous one has read its Q
         if (done > 0 && !wait_parity<kPair>(q_empty, (done - 1) & 1, A.wd, &abort_flag)) break;
         if (leader) mbar_expect_tx(q_full, (kPair ? 2 : 1) * ntile * G::kQBytes);
-        for (int t = 0; t < ntile; ++t)
-          for (int c = 0; c < D / 64; ++c) {
+        for (int t = 0; t < ntile; ++t) {
+          for (int c = 0; c < G::kNFull; ++c) {
             uint8_t* dst = smem + t * G::kQBytes + c * kChunkBytes;
             if constexpr (kPair) tma_load_3d_pair(dst, &tm_q, lead(q_full), 64 * c, w.q_prow, w.q_plane + t);
             else tma_load_3d(dst, &tm_q, q_full, 64 * c, w.q_prow, w.q_plane + t);
           }
+          if constexpr (G::kTail)
+            tma_load_3d(smem + t * G::kQBytes + G::kNFull * kChunkBytes, &tm_q32, q_full, 64 * G::kNFull, w.q_prow,
+                        w.q_plane + t);
+        }
         for (int it = 0; it < w.n_iter; ++it) {
           const int gi = base + it;
           int s = gi % KS, u = gi / KS;
@@ -414,9 +419,12 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
                                k_row, kplane);
           } else {
             mbar_expect_tx(k_full + s, G::kKBytes);
-            for (int c = 0; c < D / 64; ++c)
+            for (int c = 0; c < G::kNFull; ++c)
               tma_load_3d(smem + G::kKOff + s * G::kKBytes + c * G::kKChunk, &tm_k, k_full + s, 64 * c, krow,
                           kplane);
+            if constexpr (G::kTail)
+              tma_load_3d(smem + G::kKOff + s * G::kKBytes + G::kNFull * G::kKChunk, &tm_k32, k_full + s,
+                          64 * G::kNFull, krow, kplane);
           }
           s = gi % VS;
           u = gi / VS;
@@ -429,9 +437,12 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
             tma_load_3d_pair(smem + G::kVOff + s * G::kVBytes, &tm_v, lead(v_full + s), (D / 2) * rank, krow, kplane);
           } else {
             mbar_expect_tx(v_full + s, G::kVBytes);
-            for (int c = 0; c < D / 64; ++c)
+            for (int c = 0; c < G::kNFull; ++c)
               tma_load_3d(smem + G::kVOff + s * G::kVBytes + c * G::kVChunk, &tm_v, v_full + s, 64 * c, krow,
                           kplane);
+            if constexpr (G::kTail)
+              tma_load_3d(smem + G::kVOff + s * G::kVBytes + G::kNFull * G::kVChunk, &tm_v32, v_full + s,
+                          64 * G::kNFull, krow, kplane);
           }
         }
         base += w.n_iter;
@@ -445,22 +456,35 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
       // so the softmax only ever sees a positive scale
       constexpr int kM = kPair ? 2 * kBM : kBM;
       const uint32_t idesc_s = umma_idesc_f16(kM, BN, 1, 1, false) | (A.negate_s << 13);
-      constexpr uint32_t idesc_o = umma_idesc_f16(kM, D, 1, 1, true);
+      // PV in up to two MMAs: the 64-dim chunks (N = 64 kNFull) and the 32-dim tail
+      constexpr uint32_t idesc_o = umma_idesc_f16(kM, G::kNFull > 0 ? 64 * G::kNFull : 32, 1, 1, true);
+      constexpr uint32_t idesc_o32 = umma_idesc_f16(kM, 32, 1, 1, true);
       const uint32_t q_base = smem_u32(smem);
       // operand descriptors are built once; a k-step only moves the start
       // address (its 14-bit field never carries: every address is < 2^18)
       const uint64_t dq0 = umma_desc_sw128(q_base, 16, 1024);
       const uint64_t dk0 = umma_desc_sw128(q_base + G::kKOff, 16, 1024);
       const uint64_t dv0 = umma_desc_sw128(q_base + G::kVOff, G::kVChunk, 1024);
+      // 32-dim tails (64-byte swizzle): Q of tile 0, K and V of stage 0
+      const uint64_t dq32 = umma_desc_sw64(q_base + G::kNFull * kChunkBytes, 16, 512);
+      const uint64_t dk32 = umma_desc_sw64(q_base + G::kKOff + G::kNFull * G::kKChunk, 16, 512);
+      const uint64_t dv32 = umma_desc_sw64(q_base + G::kVOff + G::kNFull * G::kVChunk, 16, 512);
       auto issue_s = [&](int t, int st) {
         const uint64_t dq = dq0 + ((t * G::kQBytes) >> 4);
         const uint64_t dk = dk0 + ((st * G::kKBytes) >> 4);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 0; k < 4 * G::kNFull; ++k) {
           const uint32_t off_q = ((k / 4) * kChunkBytes + (k % 4) * 32) >> 4;
           const uint32_t off_k = ((k / 4) * G::kKChunk + (k % 4) * 32) >> 4;
           if constexpr (kPair) mma_ss_pair(tmem + G::s_col(t), dq + off_q, dk + off_k, idesc_s, k > 0 ? 1u : 0u);
           else mma_ss(tmem + G::s_col(t), dq + off_q, dk + off_k, idesc_s, k > 0 ? 1u : 0u);
+        }
+        if constexpr (G::kTail) {
+          const uint64_t tq = dq32 + ((t * G::kQBytes) >> 4), tk = dk32 + ((st * G::kKBytes) >> 4);
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+            mma_ss(tmem + G::s_col(t), tq + ((k * 32) >> 4), tk + ((k * 32) >> 4), idesc_s,
+                   (G::kNFull > 0 || k > 0) ? 1u : 0u);
         }
       };
       // O_t += P_t V over keys [BN/2 h, BN/2 h + BN/2) (16-key MMA steps)
@@ -470,10 +494,15 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
 #pragma unroll
         for (int k = kHalf * h; k < kHalf * h + kHalf; ++k) {
           const uint32_t acc = (accumulate || k > 0) ? 1u : 0u;
-          if constexpr (kPair)
+          if constexpr (kPair) {
             mma_ts_pair(tmem + G::o_col(t), tmem + G::s_col(t) + k * 8, dv + ((k * 2048) >> 4), idesc_o, acc);
-          else
-            mma_ts(tmem + G::o_col(t), tmem + G::s_col(t) + k * 8, dv + ((k * 2048) >> 4), idesc_o, acc);
+          } else {
+            if constexpr (G::kNFull > 0)
+              mma_ts(tmem + G::o_col(t), tmem + G::s_col(t) + k * 8, dv + ((k * 2048) >> 4), idesc_o, acc);
+            if constexpr (G::kTail)
+              mma_ts(tmem + G::o_col(t) + 64 * G::kNFull, tmem + G::s_col(t) + k * 8,
+                     dv32 + ((st * G::kVBytes + k * 1024) >> 4), idesc_o32, acc);
+          }
         }
       };
       int base = 0, done = 0;  // K/V tiles and items before the current one
@@ -659,10 +688,7 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
           // p = 2^(s * scale * log2(e) - m): one packed FMA for two scores
           const float2 x = fma2(make_float2(__uint_as_float(raw[cc][2 * e]), __uint_as_float(raw[cc][2 * e + 1])),
                                 sc2, nm2);
-          // every kPolyEvery-th pair of a 32-column chunk on the FMA pipe
-          const float2 pp = (kPolyEvery > 0 && e % kPolyEvery == kPolyEvery - 1)
-                                ? exp2_poly2(x)
-                                : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           lacc[e % kL] = add2(lacc[e % kL], pp);
           pk[e] = pack_bf16x2(pp.x, pp.y);
         }
@@ -865,6 +891,26 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowS
                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != FA_OK) return st;
   }
+  // 32-dim tails (64-byte swizzle): boxes of 32 dims, the same rows
+  CUtensorMap tq32 = tq, tk32 = tk, tv32 = tv;
+  if constexpr (G::kTail) {
+    const uint64_t qdims[3] = {static_cast<uint64_t>(D), q_rows, q_planes};
+    const uint64_t qstr[2] = {static_cast<uint64_t>(D) * 2, q_rows * D * 2};
+    const uint32_t qbox[3] = {32, static_cast<uint32_t>(kSwizzleChunkRows), 1};
+    fa_status st = encode_tensor_map(&tq32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.q, qdims, qstr, qbox,
+                                     CU_TENSOR_MAP_SWIZZLE_64B);
+    if (st != FA_OK) return st;
+    const uint64_t kdims[3] = {static_cast<uint64_t>(D), k_rows, k_planes};
+    const uint64_t kstr[2] = {static_cast<uint64_t>(D) * 2, k_rows * D * 2};
+    const uint32_t kbox[3] = {32, krows, 1};
+    const uint32_t vbox[3] = {32, static_cast<uint32_t>(BN), 1};
+    st = encode_tensor_map(&tk32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.k, kdims, kstr, kbox,
+                           CU_TENSOR_MAP_SWIZZLE_64B);
+    if (st != FA_OK) return st;
+    st = encode_tensor_map(&tv32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.v, kdims, kstr, vbox,
+                           CU_TENSOR_MAP_SWIZZLE_64B);
+    if (st != FA_OK) return st;
+  }
   PrefillArgs A;
   A.L = pages != nullptr ? SeqLayout::paged(p, *pages) : SeqLayout::from(p);
   A.out = static_cast<__nv_bfloat16*>(p.out);
@@ -915,12 +961,12 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowS
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cuda_status(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, A));
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, tq32, tk32, tv32, A));
   } else {
     // persistent: one CTA per SM (the shared memory allows no second), each
     // walking its share of the items
     const long long grid = items < device_sm_count() ? items : device_sm_count();
-    kern<<<static_cast<unsigned>(grid), G::kThreads, G::kSmem, ctx.stream>>>(tq, tk, tv, A);
+    kern<<<static_cast<unsigned>(grid), G::kThreads, G::kSmem, ctx.stream>>>(tq, tk, tv, tq32, tk32, tv32, A);
     return cuda_status(cudaGetLastError());
   }
 }
@@ -968,6 +1014,8 @@ fa_status launch_prefill_tc(const fa_fwd_params& p, const fa_kv_pages* pages, co
                                      : launch_tc<128, false, false>(p, pages, sink, ctx);
   if (p.head_dim == 64) return use_quad(p) ? launch_tc<64, false, false, 64, 4>(p, pages, sink, ctx)
                                            : launch_tc<64, false, false>(p, pages, sink, ctx);
+  if (p.head_dim == 32) return launch_tc<32, false, false>(p, pages, sink, ctx);
+  if (p.head_dim == 96) return launch_tc<96, false, false>(p, pages, sink, ctx);
   return FA_ERR_UNSUPPORTED;
 }
 

@@ -7,9 +7,11 @@
 //   [46,48) descriptor version, 1 on sm_100
 //   [49,52) base offset (0: every operand tile here is 1024-byte aligned)
 //   [52]    LBO mode (0)
-//   [61,64) layout: 2 = 128-byte swizzle
+//   [61,64) layout: 2 = 128-byte swizzle, 4 = 64-byte swizzle
 // Operands are staged by TMA with the 128-byte swizzle, in chunks of
-// [rows x 64 bf16] (128 bytes per row, 8-row / 1024-byte swizzle atoms):
+// [rows x 64 bf16] (128 bytes per row, 8-row / 1024-byte swizzle atoms), and
+// a head size that is an odd multiple of 32 keeps its last 32 dims in a
+// chunk of 64-byte rows with the 64-byte swizzle:
 //   K-major (Q, K: the reduction dim contiguous): SBO = 1024 (next 8 rows),
 //     LBO unused; the k-th 16-element step starts 32*k bytes further inside
 //     a chunk, the next 64 elements one chunk further.
@@ -29,14 +31,25 @@ namespace fa {
 
 constexpr uint32_t kSwizzleChunkRows = 128;  // rows per TMA box in the tensor-core kernels
 
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+// layout: 2 = 128-byte swizzle, 4 = 64-byte swizzle
+__device__ __forceinline__ uint64_t umma_desc(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t layout) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1u) << 46;
-  d |= static_cast<uint64_t>(2u) << 61;
+  d |= static_cast<uint64_t>(layout) << 61;
   return d;
+}
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return umma_desc(smem_addr, lbo_bytes, sbo_bytes, 2u);
+}
+// 64-byte swizzle (rows of 32 bf16): 8-row / 512-byte atoms.  K-major: SBO =
+// 512 (next 8 rows), a 16-element k-step starts 32 bytes further.  MN-major:
+// SBO = 512 (next 8 K rows), a 16-row k-step starts 16 * 64 bytes further.
+__device__ __forceinline__ uint64_t umma_desc_sw64(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return umma_desc(smem_addr, lbo_bytes, sbo_bytes, 4u);
 }
 
 // a_fmt/b_fmt: 0 = f16, 1 = bf16.

@@ -190,12 +190,15 @@ def paginate_varlen(x, scales, lens, hkv, page_size, rng, extra=3):
 
 
 @pytest.mark.parametrize("int8", [False, True])
-@pytest.mark.parametrize("d,page_size,window", [(128, 128, 0), (128, 256, 0), (64, 128, 200)])
+@pytest.mark.parametrize("d,page_size,window", [(128, 128, 0), (128, 256, 0), (64, 128, 200), (96, 128, 0),
+                                                (32, 256, 100)])
 def test_paged_prefill_equals_varlen(int8, d, page_size, window):
     """Chunked prefill over a paged cache: each sequence's new queries (fewer
     than its keys, bottom-right causal) attend to its whole prefix read from
     shuffled pages; bit-identical to the contiguous varlen prefill, and the
     oracle's within the bf16 gate."""
+    if int8 and d not in (64, 128):
+        pytest.skip("int8 K/V on the tensor cores: head sizes 64 and 128")
     fa = _fa()
     rng = np.random.default_rng(50 + d + page_size + window + int8)
     hq, hkv = 8, 2
@@ -229,10 +232,7 @@ def test_paged_prefill_equals_varlen(int8, d, page_size, window):
                 if vs is not None:
                     vsp[pg, :, :e - a] = vs[:, a:e]
     cuda = lambda t: None if t is None else t.cuda()
-    # the gate bounds the attention output; an epilogue with gain 2 would
-    # double the int8 path's operand rounding (c * s to bf16) before it, so
-    # the int8 cases take the long-context int8 workload's own Mul(0.5)
-    epi = [("mul", 0.5)] if int8 else [("mul", 2.0), ("add", 0.5)]
+    epi = [("mul", 2.0), ("add", 0.5)]
     ref_gpu = fa.attention_fwd(q, cuda(kc), cuda(vc), hq=hq, hkv=hkv, causal=True, window=window, epilogue=epi,
                                k_scales=cuda(ks), v_scales=cuda(vs), cu_seqlens_q=cu_q.cuda(),
                                cu_seqlens_k=cu_k.cuda(), max_seqlen_q=max(q_lens), max_seqlen_k=max(k_lens))

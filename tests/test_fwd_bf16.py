@@ -34,6 +34,12 @@ DENSE = [
     (1, 8, 1, 64, 700, 128, False, 200),   # window without causal
     (1, 2, 2, 1, 1, 64, True, 0),
     (1, 6, 3, 384, 384, 64, True, 0),      # G = 2
+    (2, 4, 2, 33, 127, 32, True, 0),       # ragged 33/127 at d = 32 (fkl_python PR #6, Verification)
+    (2, 4, 2, 33, 127, 32, False, 0),
+    (1, 6, 2, 130, 50, 32, True, 0),       # d = 32 with empty-band rows
+    (1, 8, 2, 300, 300, 96, True, 0),      # d = 96: a 64-dim chunk and a 32-dim tail
+    (1, 4, 1, 257, 700, 96, False, 200),
+    (1, 4, 4, 200, 333, 96, True, 0),
 ]
 
 
@@ -47,7 +53,7 @@ def test_dense(case):
     assert_close_bf16(got.float().numpy(), ref, what=str(case))
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [32, 64, 96, 128])
 @pytest.mark.parametrize("causal,window", [(True, 0), (True, 100), (False, 0)])
 def test_varlen(d, causal, window):
     lengths = [33, 127, 1, 300, 129, 256]
