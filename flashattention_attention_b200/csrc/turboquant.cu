@@ -213,6 +213,19 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
+// Four 8x8 b16 matrices loaded transposed; lane l gives the row address of
+// matrix l / 8, row l % 8.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+// The 8x8 b16 matrix whose row g / 4, columns 2 (g % 4) .. +1 lane g holds,
+// transposed (one movmatrix).
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
 // D (fp32) += A (16x16 fp16, row) . B (16x8 fp16, col)
 __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                         uint32_t b0, uint32_t b1) {
@@ -262,28 +275,33 @@ __device__ __forceinline__ uint32_t to_nibbles(uint32_t f) {
 //     [t d/4, t d/4 + d/4) of its rows, four per k-step, and the rotated
 //     queries' B fragments (fp16, registers) use the same order.  A
 //     fragments come from the packed codes by byte permutes (dequant4).
-//   online softmax per head on the S fragments; p ||v|| goes to shared memory
-//   O_rot [channels x heads] += sum_j p_j ||v_j|| level[code_j] with the lanes
-//     over the channels (one broadcast read of a key's p for all heads).
+//   online softmax per head on the S fragments; P'[key, head] = p ||v_key||
+//     in fp16, turned from S fragments into B fragments by 8x8 transposes.
+//   V: lane j dequantises key j's codes into an fp16 tile [32 keys x D] in
+//     shared memory (a pair table of fp16 levels; 16-byte chunks of each row
+//     swizzled by the key's low bits, so ldmatrix reads are conflict-free),
+//     then O_rot^T [D x 8 heads] += Vlev^T . P' on mma.sync (channels on M,
+//     heads on N, keys on K), the A fragments read by ldmatrix.trans.
 template <int D, int KB, int VB, int G>
 __global__ void __launch_bounds__(kDecodeWarps * 32)
     tq_decode_kernel(TqArgs A) {
   constexpr int E = D / 32;
   constexpr int KROW = D * KB / 8;  // bytes of a packed K row
   constexpr int VROW = D * VB / 8;
-  constexpr int LVB = E * VB;       // V code bits per lane (its E channels)
   constexpr int VU2 = VROW / 8;     // 8-byte words of a 32-key V block per lane
-  constexpr int GP = (G + 1) / 2;   // head pairs
   constexpr int KS = D / 16;        // k-steps of the score MMA
   constexpr int SB = D * KB / 32;   // bytes of a thread's quarter of a K row
   constexpr int SW = (SB + 3) / 4;
-  constexpr int PG = G < 4 ? G : 4 * ((G + 3) / 4);  // p row stride (16-byte rows from 4 heads up)
+  constexpr int MT = D / 16;        // channel tiles of the V MMA
+  constexpr uint32_t kVdqBytes = kDecodeWarps * 32 * D * 2;      // fp16 V tiles of the warps
+  constexpr uint32_t kSoBytes = kDecodeWarps * G * D * 4;         // the warps' O rows at the end
   __shared__ __align__(16) float qr[D][G];
-  __shared__ __align__(8) float2 vtab[1 << (2 * VB)];  // V pair table: (level[c & m], level[c >> b])
+  __shared__ uint32_t vtab[1 << (2 * VB)];  // V pair table: fp16 (level[c & m], level[c >> b])
   __shared__ __align__(16) uint2 vblk[kDecodeWarps][32 * VU2];  // a warp's staged V codes
-  __shared__ __align__(16) float ps[kDecodeWarps][32][PG];      // p ||v|| per key and head
   __shared__ float s_m[kDecodeWarps][G], s_l[kDecodeWarps][G];
-  __shared__ __align__(16) float s_o[kDecodeWarps][G][D];
+  // the V tiles during the key loop, the per-warp O rows after it
+  __shared__ __align__(128) unsigned char vbuf[kVdqBytes > kSoBytes ? kVdqBytes : kSoBytes];
+  float(*s_o)[G][D] = reinterpret_cast<float(*)[G][D]>(vbuf);
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gq = lane >> 2, tq = lane & 3;  // fragment row group and column pair
@@ -297,7 +315,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   const int k0 = split * A.split_keys;
   const int k1 = min(len, k0 + A.split_keys);
   for (int c = threadIdx.x; c < (1 << (2 * VB)); c += blockDim.x)
-    vtab[c] = make_float2(A.v_levels[c & ((1 << VB) - 1)], A.v_levels[c >> VB]);
+    vtab[c] = pack_h2(A.v_levels[c & ((1 << VB) - 1)], A.v_levels[c >> VB]);
   // the upper half of the K levels as fp16 byte planes (8 entries, zero-padded)
   uint32_t pl[2] = {0u, 0u}, ph[2] = {0u, 0u};
 #pragma unroll
@@ -332,11 +350,11 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   }
 
   float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};  // heads 2 tq, 2 tq + 1
-  float2 o[GP][E];  // heads (2p, 2p + 1) of channel e of this lane
+  // O_rot^T fragments: channels 16 mi + gq (+ 8), heads 2 tq, 2 tq + 1
+  float o[MT][4];
 #pragma unroll
-  for (int pi = 0; pi < GP; ++pi)
-#pragma unroll
-    for (int e = 0; e < E; ++e) o[pi][e] = make_float2(0.f, 0.f);
+  for (int mi = 0; mi < MT; ++mi) o[mi][0] = o[mi][1] = o[mi][2] = o[mi][3] = 0.f;
+  const uint32_t vdq = smem_u32(vbuf) + warp * (32 * D * 2);
   const int64_t plane = static_cast<int64_t>(b) * A.hkv + g;
   const uint8_t* kc = A.kc + plane * A.cap * KROW;
   const uint8_t* vc = A.vc + plane * A.cap * VROW;
@@ -449,63 +467,65 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
       m2[hh] = m_new;
       l2[hh] *= alpha2[hh];
     }
+    // P' = p ||v|| (0 for heads past the group) as B fragments of the V MMA:
+    // the S fragment rows are keys and its columns heads; one transpose per
+    // 8x8 gives thread (g, t) keys 2t, 2t + 1 of head g
+    uint32_t pb[2][2];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int mt = 0; mt < 2; ++mt) {
+      float pv[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const int hh = t & 1;
         const int r4 = 2 * mt + (t >> 1);
-        const int kk = 16 * mt + gq + 8 * (t >> 1);
         const float pe = sv[mt][t] == -INFINITY ? 0.f : exp2f(sv[mt][t] - m2[hh]);
         l2[hh] += pe;
-        const int h = 2 * tq + hh;
-        if (h < G) ps[warp][kk][h] = pe * nv4[r4];
+        pv[t] = 2 * tq + hh < G ? pe * nv4[r4] : 0.f;
       }
-    // the O rows of every head take their alpha (held by lane h / 2)
+      pb[mt][0] = transpose8x8(pack_h2(pv[0], pv[1]));
+      pb[mt][1] = transpose8x8(pack_h2(pv[2], pv[3]));
+    }
+    // O columns (heads 2 tq, 2 tq + 1) take their alpha
 #pragma unroll
-    for (int pi = 0; pi < GP; ++pi) {
-      const float a0 = __shfl_sync(0xffffffffu, alpha2[0], pi);
-      const float a1 = __shfl_sync(0xffffffffu, alpha2[1], pi);
-#pragma unroll
-      for (int e = 0; e < E; ++e) o[pi][e] = make_float2(o[pi][e].x * a0, o[pi][e].y * a1);
+    for (int mi = 0; mi < MT; ++mi) {
+      o[mi][0] *= alpha2[0];
+      o[mi][1] *= alpha2[1];
+      o[mi][2] *= alpha2[0];
+      o[mi][3] *= alpha2[1];
     }
     __syncwarp();
-    // V: the lanes over the channels, one key at a time
-    const int n = min(32, k1 - c0);
-    const int bitpos = lane * LVB;
-    const uint32_t* vw = reinterpret_cast<const uint32_t*>(vblk[warp]) + (bitpos >> 5);
-    const int sh = bitpos & 31;
-    const bool two = sh + LVB > 32;  // this lane's bits cross into the next word
-    for (int j = 0; j < n; ++j) {
-      const uint32_t w0 = vw[j * (VROW / 4)];
-      const uint32_t w1 = two ? vw[j * (VROW / 4) + 1] : 0u;
-      const uint32_t bits = __funnelshift_r(w0, w1, sh);
-      float lev[E];
+    // V: lane j dequantises key j (codes of keys past the chunk's end are
+    // zero, and their P' is 0), then the MMAs over the two 16-key halves
+    {
+      constexpr int NW = VROW / 4;
+      uint32_t vw[NW];
+      const uint32_t* row = reinterpret_cast<const uint32_t*>(vblk[warp]) + lane * NW;
 #pragma unroll
-      for (int e = 0; e < E; e += 2) {
-        const float2 t = vtab[(bits >> (e * VB)) & ((1u << (2 * VB)) - 1u)];
-        lev[e] = t.x;
-        lev[e + 1] = t.y;
+      for (int t = 0; t < NW; ++t) vw[t] = row[t];
+#pragma unroll
+      for (int c16 = 0; c16 < D / 8; ++c16) {  // 8 channels = four level pairs per 16-byte chunk
+        uint32_t h[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) h[q] = vtab[code_at<2 * VB, NW>(vw, (8 * c16 + 2 * q) * VB)];
+        const uint32_t at = vdq + lane * (D * 2) + ((c16 ^ (lane & 7)) * 16);
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(at), "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3])
+                     : "memory");
       }
-      float pj[2 * GP];
-      if constexpr (G >= 4) {
+      __syncwarp();
+      // ldmatrix.trans of 8x8 block i = lane / 8: keys 8 (i / 2) + lane % 8 of
+      // the 16-key half, channels 16 mi + 8 (i % 2) ..
+      const int blk = lane >> 3, rr = lane & 7;
 #pragma unroll
-        for (int g4 = 0; g4 < G; g4 += 4) {
-          const float4 p4 = *reinterpret_cast<const float4*>(&ps[warp][j][g4]);
-          pj[g4] = p4.x; pj[g4 + 1] = p4.y; pj[g4 + 2] = p4.z; pj[g4 + 3] = p4.w;
+      for (int mt = 0; mt < 2; ++mt) {
+        const int key = 16 * mt + 8 * (blk >> 1) + rr;
+#pragma unroll
+        for (int mi = 0; mi < MT; ++mi) {
+          const int c16 = 2 * mi + (blk & 1);
+          uint32_t a[4];
+          ldsm_x4_trans(vdq + key * (D * 2) + ((c16 ^ (key & 7)) * 16), a);
+          mma_f16(o[mi], a[0], a[1], a[2], a[3], pb[mt][0], pb[mt][1]);
         }
-      } else if constexpr (G == 2) {
-        const float2 p2 = *reinterpret_cast<const float2*>(&ps[warp][j][0]);
-        pj[0] = p2.x; pj[1] = p2.y;
-      } else {
-        pj[0] = ps[warp][j][0];
-        pj[1] = 0.f;
       }
-#pragma unroll
-      for (int pi = 0; pi < GP; ++pi)
-#pragma unroll
-        for (int e = 0; e < E; ++e)
-          o[pi][e] = fma2(make_float2(pj[2 * pi], pj[2 * pi + 1]), make_float2(lev[e], lev[e]), o[pi][e]);
     }
   }
 
@@ -523,10 +543,19 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
       s_l[warp][h] = l;
     }
   }
+  __syncthreads();  // every warp's V tile reads are done: vbuf becomes the O rows
 #pragma unroll
-  for (int gi = 0; gi < G; ++gi)
+  for (int mi = 0; mi < MT; ++mi) {
+    const int c = 16 * mi + gq;
 #pragma unroll
-    for (int e = 0; e < E; ++e) s_o[warp][gi][lane * E + e] = gi % 2 == 0 ? o[gi / 2][e].x : o[gi / 2][e].y;
+    for (int hh = 0; hh < 2; ++hh) {
+      const int h = 2 * tq + hh;
+      if (h < G) {
+        s_o[warp][h][c] = o[mi][hh];
+        s_o[warp][h][c + 8] = o[mi][2 + hh];
+      }
+    }
+  }
   __syncthreads();
   for (int idx = threadIdx.x; idx < G * (D + 2); idx += blockDim.x) {
     const int gi = idx / (D + 2), c = idx % (D + 2);
