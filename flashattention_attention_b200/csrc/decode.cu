@@ -90,12 +90,19 @@ struct Geom {
   static constexpr int kScaleBytes = kBF ? 0 : 2 * kTile * 4;    // K and V scales (int8)
   static constexpr int kScaleOff = 2 * kTileBytes;
   static constexpr int kStageBytes = ((2 * kTileBytes + kScaleBytes) + 1023) / 1024 * 1024;
-  // int8: 128B (d = 128) or 64B (d = 64) swizzle of whole rows; bf16: 128B
-  // swizzle of 64-dim chunks [32 rows x 128 B]
-  static constexpr int kSwzMask = (kBF || D == 128) ? 0x70 : 0x30;
+  // bf16: 128-byte swizzle of 64-dim chunks [32 rows x 128 B], then for D =
+  // 32 or 96 a 32-dim tail chunk [32 rows x 64 B] with the 64-byte swizzle.
+  // int8 rows: D = 64 and 128 fill one TMA box with the 64- / 128-byte
+  // swizzle; D = 256 is two 128-byte halves (two boxes, 4 KB apart in the
+  // tile); D = 32 and 96 are plain rows
+  static constexpr int kSwzMask = (kBF || D == 128 || D == 256) ? 0x70 : (D == 64 ? 0x30 : 0);
+  static constexpr int kRowBytes = kBF ? 128 : (D > 128 ? 128 : D);  // bytes per row of one box
+  static constexpr int kHalves = (!kBF && D > 128) ? D / 128 : 1;   // int8 boxes per tile row
   static constexpr int kChunkBytes = kTile * 128;
+  static constexpr int kNFull = D / 64;                 // bf16: full 64-dim chunks
+  static constexpr bool kTail = kBF && (D % 64) == 32;  // bf16: a 32-dim tail chunk
   static constexpr int kStages = 3;
-  static constexpr int kCtas = (kBF && D == 128) ? 1 : 2;
+  static constexpr int kCtas = ((kBF && (D == 128 || D == 96)) || D == 256) ? 1 : 2;
   static constexpr int kSmem = kWarps * kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
   // sequences whose tile prefix fits in the shared memory the CTAs per SM
   // leave over (228 KB per SM, 1 KB reserved per CTA, 256 B margin)
@@ -106,6 +113,10 @@ static_assert(2 * Geom<128, false>::kSmem <= 232448 && 2 * Geom<64, false>::kSme
                   2 * Geom<64, true>::kSmem <= 232448,
               "CTAs per SM");
 static_assert(Geom<128, false>::kCtas <= kMaxCtasPerSm && Geom<64, true>::kCtas <= kMaxCtasPerSm, "workers");
+static_assert(2 * Geom<32, false>::kSmem <= 232448 && 2 * Geom<96, false>::kSmem <= 232448 &&
+                  Geom<256, false>::kSmem <= 232448 && 2 * Geom<32, true>::kSmem <= 232448 &&
+                  Geom<96, true>::kSmem <= 232448,
+              "CTAs per SM");
 
 // TMA swizzle of a byte offset inside a tile whose base is aligned to the
 // swizzle period: bits [4,7) (128B) or [4,6) (64B) ^= bits [7,10) / [7,9).
@@ -113,15 +124,31 @@ template <int D, bool kBF>
 __device__ __forceinline__ uint32_t swz(uint32_t lin) {
   return lin ^ ((lin >> 3) & Geom<D, kBF>::kSwzMask);
 }
+// Offset of byte b of int8 row r inside a tile (the box halves of D = 256).
+template <int D>
+__device__ __forceinline__ uint32_t i8_off(int r, int b) {
+  using G = Geom<D, false>;
+  return (b / G::kRowBytes) * (kTile * G::kRowBytes) + swz<D, false>(r * G::kRowBytes + b % G::kRowBytes);
+}
 // Shared address of element (key r, dim c) of a bf16 tile at `tile`.
 template <int D>
 __device__ __forceinline__ uint32_t bf_addr(uint32_t tile, int r, int c) {
-  return tile + (c / 64) * Geom<D, true>::kChunkBytes + swz<D, true>(r * 128 + (c % 64) * 2);
+  using G = Geom<D, true>;
+  if (G::kTail && c / 64 == G::kNFull) {  // the 32-dim tail: 64-byte rows, 64-byte swizzle
+    const uint32_t lin = r * 64 + (c % 64) * 2;
+    return tile + G::kNFull * G::kChunkBytes + (lin ^ ((lin >> 3) & 0x30));
+  }
+  return tile + (c / 64) * G::kChunkBytes + swz<D, true>(r * 128 + (c % 64) * 2);
 }
 
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -365,11 +392,17 @@ __device__ __forceinline__ int64_t tile_row(const SkArgs& A, const Cursor& c, in
 template <int D, bool kBF>
 __global__ void __launch_bounds__(kThreads, Geom<D, kBF>::kCtas)
     decode_sk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_k32, const __grid_constant__ CUtensorMap tm_v32,
                      const SkArgs A) {
   using G = Geom<D, kBF>;
   constexpr int kStages = G::kStages;
   constexpr int kSteps = D / 16;      // k-steps of the S MMA
-  constexpr int kChunks = D / 64;     // 16-byte chunks per thread per K row
+  constexpr int kChunks = D / 64;     // 16-byte chunks per thread per K row (d = 64, 128)
+  // d = 64 and 128: thread qq owns dims [qq D/4, (qq+1) D/4) of every K row
+  // (16-byte loads); other head sizes: dims [32 c + 8 qq, +8) of every 32-dim
+  // block c (8-byte loads).  Either way k-step ks reads one 4-byte word of
+  // the thread's dims, and Q's fragments take the same dims in that order.
+  constexpr bool kQuarter = (D == 64 || D == 128);
   constexpr int kMT = D / 16;         // O^T m-tiles (dims)
   extern __shared__ uint8_t dec_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dec_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -456,13 +489,22 @@ __global__ void __launch_bounds__(kThreads, Geom<D, kBF>::kCtas)
         mbar_expect_tx(bar, 2 * G::kTileBytes + G::kScaleBytes);
         if constexpr (kBF) {
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
+          for (int c = 0; c < G::kNFull; ++c) {
             tma_load_2d(st + c * G::kChunkBytes, &tm_k, bar, 64 * c, static_cast<int>(row));
             tma_load_2d(st + G::kTileBytes + c * G::kChunkBytes, &tm_v, bar, 64 * c, static_cast<int>(row));
           }
+          if constexpr (G::kTail) {
+            tma_load_2d(st + G::kNFull * G::kChunkBytes, &tm_k32, bar, 64 * G::kNFull, static_cast<int>(row));
+            tma_load_2d(st + G::kTileBytes + G::kNFull * G::kChunkBytes, &tm_v32, bar, 64 * G::kNFull,
+                        static_cast<int>(row));
+          }
         } else {
-          tma_load_2d(st, &tm_k, bar, 0, static_cast<int>(row));
-          tma_load_2d(st + G::kTileBytes, &tm_v, bar, 0, static_cast<int>(row));
+#pragma unroll
+          for (int h = 0; h < G::kHalves; ++h) {
+            tma_load_2d(st + h * kTile * G::kRowBytes, &tm_k, bar, G::kRowBytes * h, static_cast<int>(row));
+            tma_load_2d(st + G::kTileBytes + h * kTile * G::kRowBytes, &tm_v, bar, G::kRowBytes * h,
+                        static_cast<int>(row));
+          }
           bulk_load(st + G::kScaleOff, A.k_scales + row, kTile * 4, bar);
           bulk_load(st + G::kScaleOff + kTile * 4, A.v_scales + row, kTile * 4, bar);
         }
@@ -519,7 +561,8 @@ __global__ void __launch_bounds__(kThreads, Geom<D, kBF>::kCtas)
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       uint4 raw = make_uint4(0, 0, 0, 0);
-      if (head_ok) raw = *reinterpret_cast<const uint4*>(A.q + static_cast<int64_t>(hq_idx) * D + qq * (D / 4) + 8 * c);
+      const int dim0 = kQuarter ? qq * (D / 4) + 8 * c : 32 * c + 8 * qq;
+      if (head_ok) raw = *reinterpret_cast<const uint4*>(A.q + static_cast<int64_t>(hq_idx) * D + dim0);
       const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -718,19 +761,30 @@ __global__ void __launch_bounds__(kThreads, Geom<D, kBF>::kCtas)
     for (int mt = 0; mt < 2; ++mt) {
       sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
       const int r0 = 16 * mt + gq, r1 = r0 + 8;
-      uint4 ka[kChunks], kb[kChunks];
+      // this thread's K words of rows r0, r1: word ks feeds k-step ks
+      uint32_t kwa[kSteps], kwb[kSteps];
+      if constexpr (kQuarter) {
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) {
-        const uint32_t off = (qq * kChunks + c) * 16;
-        ka[c] = lds128(kt + swz<D, false>(r0 * D + off));
-        kb[c] = lds128(kt + swz<D, false>(r1 * D + off));
+        for (int c = 0; c < kChunks; ++c) {
+          const uint32_t off = (qq * kChunks + c) * 16;
+          const uint4 a4 = lds128(kt + swz<D, false>(r0 * D + off));
+          const uint4 b4 = lds128(kt + swz<D, false>(r1 * D + off));
+          kwa[4 * c] = a4.x; kwa[4 * c + 1] = a4.y; kwa[4 * c + 2] = a4.z; kwa[4 * c + 3] = a4.w;
+          kwb[4 * c] = b4.x; kwb[4 * c + 1] = b4.y; kwb[4 * c + 2] = b4.z; kwb[4 * c + 3] = b4.w;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          const uint2 a2 = lds64(kt + i8_off<D>(r0, 32 * c + 8 * qq));
+          const uint2 b2 = lds64(kt + i8_off<D>(r1, 32 * c + 8 * qq));
+          kwa[2 * c] = a2.x; kwa[2 * c + 1] = a2.y;
+          kwb[2 * c] = b2.x; kwb[2 * c + 1] = b2.y;
+        }
       }
 #pragma unroll
       for (int ks = 0; ks < kSteps; ++ks) {
-        const uint4& A4 = ka[ks / 4];
-        const uint4& B4 = kb[ks / 4];
-        const uint32_t wa = (ks % 4 == 0) ? A4.x : (ks % 4 == 1) ? A4.y : (ks % 4 == 2) ? A4.z : A4.w;
-        const uint32_t wb = (ks % 4 == 0) ? B4.x : (ks % 4 == 1) ? B4.y : (ks % 4 == 2) ? B4.z : B4.w;
+        const uint32_t wa = kwa[ks];
+        const uint32_t wb = kwb[ks];
         uint32_t ae, ao, be, bo;
         i8x4_to_f16x2_biased(wa, ae, ao);
         i8x4_to_f16x2_biased(wb, be, bo);
@@ -852,10 +906,10 @@ __global__ void __launch_bounds__(kThreads, Geom<D, kBF>::kCtas)
 #pragma unroll
       for (int pr = 0; pr < D / 32; ++pr) {
         const uint32_t xw = (8 * pr + gq) * 4;  // byte offset of this thread's word
-        const uint32_t w0 = lds32(vt + swz<D, false>((kk0 + 0) * D + xw));
-        const uint32_t w1 = lds32(vt + swz<D, false>((kk0 + 1) * D + xw));
-        const uint32_t w2 = lds32(vt + swz<D, false>((kk0 + 8) * D + xw));
-        const uint32_t w3 = lds32(vt + swz<D, false>((kk0 + 9) * D + xw));
+        const uint32_t w0 = lds32(vt + i8_off<D>(kk0 + 0, xw));
+        const uint32_t w1 = lds32(vt + i8_off<D>(kk0 + 1, xw));
+        const uint32_t w2 = lds32(vt + i8_off<D>(kk0 + 8, xw));
+        const uint32_t w3 = lds32(vt + i8_off<D>(kk0 + 9, xw));
         const uint32_t t01l = prmt(w0, w1, 0x5410), t01h = prmt(w0, w1, 0x7632);
         const uint32_t t23l = prmt(w2, w3, 0x5410), t23h = prmt(w2, w3, 0x7632);
         mma16816(o[2 * pr], i8x2_to_f16x2_even(t01l), i8x2_to_f16x2_odd(t01l), i8x2_to_f16x2_even(t23l),
@@ -897,13 +951,24 @@ fa_status launch_sk(const fa_decode_params& p, const fa_kv_pages* pages, int n_w
   const uint64_t dims[2] = {static_cast<uint64_t>(D), rows};
   const uint64_t strides[1] = {static_cast<uint64_t>(D) * (kBF ? 2 : 1)};
   // int8: one box of whole rows; bf16: boxes of 64 dims (128 bytes) per row
-  const uint32_t box[2] = {static_cast<uint32_t>(kBF ? 64 : D), static_cast<uint32_t>(kTile)};
-  const CUtensorMapSwizzle sw = (kBF || D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  // bf16: boxes of 64 dims (128 bytes) per row; int8: boxes of G::kRowBytes
+  const uint32_t box[2] = {static_cast<uint32_t>(kBF ? 64 : G::kRowBytes), static_cast<uint32_t>(kTile)};
+  const CUtensorMapSwizzle sw = G::kSwzMask == 0x70   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : G::kSwzMask == 0x30 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
   const CUtensorMapDataType dt = kBF ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   fa_status st = encode_tensor_map(&tmk, dt, 2, p.k_cache, dims, strides, box, sw);
   if (st != FA_OK) return st;
   st = encode_tensor_map(&tmv, dt, 2, p.v_cache, dims, strides, box, sw);
   if (st != FA_OK) return st;
+  CUtensorMap tmk32 = tmk, tmv32 = tmv;  // bf16 32-dim tails: boxes of 32 dims, 64-byte swizzle
+  if constexpr (G::kTail) {
+    const uint32_t box32[2] = {32, static_cast<uint32_t>(kTile)};
+    st = encode_tensor_map(&tmk32, dt, 2, p.k_cache, dims, strides, box32, CU_TENSOR_MAP_SWIZZLE_64B);
+    if (st != FA_OK) return st;
+    st = encode_tensor_map(&tmv32, dt, 2, p.v_cache, dims, strides, box32, CU_TENSOR_MAP_SWIZZLE_64B);
+    if (st != FA_OK) return st;
+  }
 
   // a group of G > 8 query heads runs as `split` passes of G / split <= 8
   const int full_group = p.hq / p.hkv;
@@ -967,7 +1032,7 @@ fa_status launch_sk(const fa_decode_params& p, const fa_kv_pages* pages, int n_w
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, kern, tmk, tmv, A));
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, tmk, tmv, tmk32, tmv32, A));
 }
 
 // the most workers any variant runs (int8 and bf16 at d = 64: two CTAs per
@@ -994,9 +1059,14 @@ fa_status launch_decode(const fa_decode_params& p, const fa_kv_pages* pages, int
   if (p.kv_dtype == FA_I8) {
     if (p.head_dim == 128) return launch_sk<128, false>(p, pages, variant_workers<128, false>(), mt, p.workspace, true, ctx);
     if (p.head_dim == 64) return launch_sk<64, false>(p, pages, variant_workers<64, false>(), mt, p.workspace, true, ctx);
+    if (p.head_dim == 32) return launch_sk<32, false>(p, pages, variant_workers<32, false>(), mt, p.workspace, true, ctx);
+    if (p.head_dim == 96) return launch_sk<96, false>(p, pages, variant_workers<96, false>(), mt, p.workspace, true, ctx);
+    if (p.head_dim == 256) return launch_sk<256, false>(p, pages, variant_workers<256, false>(), mt, p.workspace, true, ctx);
   } else if (p.kv_dtype == FA_BF16) {
     if (p.head_dim == 128) return launch_sk<128, true>(p, pages, variant_workers<128, true>(), mt, p.workspace, true, ctx);
     if (p.head_dim == 64) return launch_sk<64, true>(p, pages, variant_workers<64, true>(), mt, p.workspace, true, ctx);
+    if (p.head_dim == 32) return launch_sk<32, true>(p, pages, variant_workers<32, true>(), mt, p.workspace, true, ctx);
+    if (p.head_dim == 96) return launch_sk<96, true>(p, pages, variant_workers<96, true>(), mt, p.workspace, true, ctx);
   }
   return FA_ERR_UNSUPPORTED;
 }
@@ -1109,6 +1179,9 @@ fa_status launch_decode_noalloc(const fa_decode_params& p, int split_keys, long 
   // (no note_variant here: its bookkeeping set may allocate host memory)
   if (p.head_dim == 128) return launch_sk<128, false>(p, nullptr, workers, min_tiles_of(split_keys), scratch, false, ctx);
   if (p.head_dim == 64) return launch_sk<64, false>(p, nullptr, workers, min_tiles_of(split_keys), scratch, false, ctx);
+  if (p.head_dim == 32) return launch_sk<32, false>(p, nullptr, workers, min_tiles_of(split_keys), scratch, false, ctx);
+  if (p.head_dim == 96) return launch_sk<96, false>(p, nullptr, workers, min_tiles_of(split_keys), scratch, false, ctx);
+  if (p.head_dim == 256) return launch_sk<256, false>(p, nullptr, workers, min_tiles_of(split_keys), scratch, false, ctx);
   return FA_ERR_UNSUPPORTED;
 }
 

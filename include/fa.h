@@ -118,7 +118,7 @@ FA_API fa_status fa_compress_kv(const void *x, fa_dtype x_dtype, int64_t rows, i
  * path c * s is formed exactly in fp32 and rounded once to bf16, the
  * tensor-core operand type.  out has q's dtype.
  * head_dim: F32 path any multiple of 32 up to 256; BF16 path 32, 64, 96 or 128
- * with FA_BF16 K/V, 64 or 128 with FA_I8 K/V.
+ * (FA_BF16 or FA_I8 K/V).
  * A problem without keys (seqlen_k = 0, or varlen total_k = 0 with
  * cu_seqlens_k given) reads no K or V: k, v and the scales may be NULL.
  */
@@ -171,7 +171,7 @@ FA_API fa_status fa_attention_fwd(const fa_fwd_params *p, fa_stream_t stream);
  * keys each warp is given (fewer, longer ranges).  capacity must be a
  * multiple of 32; cache entries at or past L_b may hold any bytes (they never
  * reach the result).
- * Supported: head_dim 128 (FA_I8 and FA_BF16) or 64; any hq / hkv (a group
+ * Supported: head_dim 32, 64, 96 or 128 (FA_I8 and FA_BF16), 256 (FA_I8); any hq / hkv (a group
  * of more than 8 query heads is served in passes of at most 8 heads, each
  * reading the KV head's cache once).
  */

@@ -51,6 +51,10 @@ CASES = [
     (2, 32, 2, 128, 1024, [1000, 77]),        # G = 16: two passes of 8 heads
     (2, 24, 2, 64, 512, [300, 512]),          # G = 12: two passes of 6
     (1, 9, 1, 128, 512, [400]),               # G = 9: three passes of 3
+    (3, 8, 2, 32, 1024, [1000, 33, 512]),     # d = 32
+    (2, 8, 2, 96, 1024, [999, 100]),          # d = 96
+    (2, 8, 2, 256, 1024, [700, 1024]),        # d = 256
+    (1, 32, 2, 256, 512, [300]),              # d = 256 with a group of 16
 ]
 
 

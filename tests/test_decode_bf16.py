@@ -43,6 +43,8 @@ CASES = [
     (1, 2, 1, 128, 256, [256]),               # the page's s_k = 256 decode step
     (2, 32, 2, 128, 1024, [1000, 77]),        # G = 16: two passes of 8 heads
     (1, 12, 1, 64, 512, [333]),               # G = 12: two passes of 6
+    (3, 8, 2, 32, 1024, [1000, 33, 512]),     # d = 32: one 32-dim chunk (64-byte swizzle)
+    (2, 8, 2, 96, 1024, [999, 100]),          # d = 96: a 64-dim chunk and a 32-dim tail
 ]
 
 
