@@ -616,7 +616,7 @@ def turboquant_decode(args, dev, peaks, world, dist, result):
     the whole cache."""
     import torch
     from flashattention_attention_b200 import fa, inputs
-    w = inputs.int8kv_decode()
+    w = inputs.int8kv_decode(batch=4) if args.profile_small else inputs.int8kv_decode()
     s = inputs.rotation_signs(w.d, 0).to(dev)
     lk, lv = fa.tq_codebook(w.d, 4).to(dev), fa.tq_codebook(w.d, 2).to(dev)
     k, v = w.k.to(dev), w.v.to(dev)
@@ -936,8 +936,8 @@ def main():
                     help="oracle seconds per sampled step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-small", action="store_true",
-                    help="profiler captures: the int8-KV long prefill at S=8192 and the decodes over 4 of the "
-                         "16 sequences (same kernels, inputs still larger than L2)")
+                    help="profiler captures: the int8-KV long prefill at S=8192 and the decodes (int8, bf16, "
+                         "TurboQuant) over 4 of the 16 sequences (same kernels, inputs still larger than L2)")
     ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "quant", "prefill_int8", "varlen", "ring", "tq"],
                     help="time one part only (used for profiler captures)")
     args = ap.parse_args()

@@ -77,9 +77,9 @@ fa_status make_ctx(fa_stream_t s, LaunchCtx* ctx) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Head sizes of the tensor-core prefill: bf16 K/V 32, 64, 96 or 128; int8 K/V 64 or 128.
+// Head sizes of the tensor-core prefill (bf16 or int8 K/V): 32, 64, 96 or 128.
 bool tc_head_dim_ok(int d, int kv_dtype) {
-  if (kv_dtype == FA_I8) return d == 64 || d == 128;
+  (void)kv_dtype;
   return d == 32 || d == 64 || d == 96 || d == 128;
 }
 
@@ -350,7 +350,10 @@ fa_status decode_args(const fa_decode_params* p) {
   if (!std::isfinite(p->softmax_scale)) return FA_ERR_INVALID;
   if (p->kv_dtype != FA_I8 && p->kv_dtype != FA_BF16) return FA_ERR_INVALID;
   if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
-  if (p->head_dim != 64 && p->head_dim != 128) return FA_ERR_UNSUPPORTED;
+  // int8 cache: 32, 64, 96, 128, 256; bf16 cache: 32, 64, 96, 128
+  if (!(p->head_dim == 32 || p->head_dim == 64 || p->head_dim == 96 || p->head_dim == 128 ||
+        (p->head_dim == 256 && p->kv_dtype == FA_I8)))
+    return FA_ERR_UNSUPPORTED;
   if (p->batch == 0) return FA_OK;
   if (p->q == nullptr || p->k_cache == nullptr || p->v_cache == nullptr || p->out == nullptr ||
       p->cache_seqlens == nullptr)

@@ -83,8 +83,8 @@ struct TcGeom {
   // deeper ring: a slot refills with the TMA latency hidden behind ~2 steps.
   // A CTA of a pair holds half of every K and V tile (64 keys of K, 64 dims
   // of V), so its rings can be deeper.
-  static constexpr int kKStages = kPair ? (kI8 ? 3 : 4) : (NT == 4 ? 6 : 3);
-  static constexpr int kVStages = kPair ? (kI8 ? 3 : 4) : (NT == 4 ? 6 : ((D == 128) ? 2 : 3));
+  static constexpr int kKStages = kPair ? (kI8 ? 3 : 4) : (NT == 4 ? 6 : ((kI8 && D == 96) ? 2 : 3));
+  static constexpr int kVStages = kPair ? (kI8 ? 3 : 4) : (NT == 4 ? 6 : ((D == 128 || (kI8 && D == 96)) ? 2 : 3));
   // D = 64 kNFull + 32 kTail: kNFull chunks of 64 dims (128-byte rows,
   // 128-byte swizzle), then, for an odd multiple of 32, one chunk of 32 dims
   // (64-byte rows, 64-byte swizzle) after them
@@ -132,6 +132,8 @@ static_assert(TcGeom<64, true>::kSmem <= 232448, "shared memory budget");
 static_assert(TcGeom<128, false, true>::kSmem <= 232448, "shared memory budget");
 static_assert(TcGeom<128, true, true>::kSmem <= 232448, "shared memory budget");
 static_assert(TcGeom<64, false, false, 64, 4>::kSmem <= 232448, "shared memory budget");
+static_assert(TcGeom<96, false>::kSmem <= 232448 && TcGeom<96, true>::kSmem <= 232448, "shared memory budget");
+static_assert(TcGeom<32, true>::kSmem <= 232448, "shared memory budget");
 
 struct PrefillArgs {
   SeqLayout L;
@@ -181,21 +183,32 @@ __device__ __forceinline__ uint2 dequant4_bf16(uint32_t w, float2 s2) {
 // row's scale, rounded to bf16 and written as pieces of output chunk c / 4
 // (128-byte rows with the 128-byte swizzle, chunks dst_chunk bytes apart).
 // Each thread reads its own row's bytes before writing that row.
-template <int NC, int RL>
+template <int NC, int RL, int kNFull = 8>
 __device__ __forceinline__ void convert_int8_row(const uint8_t* src_tile, uint8_t* dst_tile, uint32_t dst_chunk,
                                                  int row, int c0, float sc) {
   const float2 s2 = make_float2(sc, sc);
 #pragma unroll
   for (int i = 0; i < NC; ++i) {
     const int c = c0 + i;
-    const int pc = (RL == 128) ? (c ^ (row & 7)) : (c ^ ((row >> 1) & 3));
+    // staged row: 128-, 64- or 32-byte swizzle (RL = 128, 64, 32), plain rows otherwise
+    const int pc = (RL == 128) ? (c ^ (row & 7))
+                 : (RL == 64) ? (c ^ ((row >> 1) & 3))
+                 : (RL == 32) ? (c ^ ((row >> 2) & 1))
+                              : c;
     const uint4 w = *reinterpret_cast<const uint4*>(src_tile + row * RL + pc * 16);
     const int h = c / 4, j0 = 2 * (c % 4);
-    uint8_t* out = dst_tile + h * dst_chunk + row * 128;
     const uint2 y0 = dequant4_bf16(w.x, s2), y1 = dequant4_bf16(w.y, s2);
     const uint2 y2 = dequant4_bf16(w.z, s2), y3 = dequant4_bf16(w.w, s2);
-    *reinterpret_cast<uint4*>(out + ((j0 ^ (row & 7)) * 16)) = make_uint4(y0.x, y0.y, y1.x, y1.y);
-    *reinterpret_cast<uint4*>(out + (((j0 + 1) ^ (row & 7)) * 16)) = make_uint4(y2.x, y2.y, y3.x, y3.y);
+    if (h < kNFull) {  // a 64-dim chunk: 128-byte rows, 128-byte swizzle
+      uint8_t* out = dst_tile + h * dst_chunk + row * 128;
+      *reinterpret_cast<uint4*>(out + ((j0 ^ (row & 7)) * 16)) = make_uint4(y0.x, y0.y, y1.x, y1.y);
+      *reinterpret_cast<uint4*>(out + (((j0 + 1) ^ (row & 7)) * 16)) = make_uint4(y2.x, y2.y, y3.x, y3.y);
+    } else {  // the 32-dim tail: 64-byte rows, 64-byte swizzle
+      uint8_t* out = dst_tile + h * dst_chunk + row * 64;
+      const int sw = (row >> 1) & 3;
+      *reinterpret_cast<uint4*>(out + ((j0 ^ sw) * 16)) = make_uint4(y0.x, y0.y, y1.x, y1.y);
+      *reinterpret_cast<uint4*>(out + (((j0 + 1) ^ sw) * 16)) = make_uint4(y2.x, y2.y, y3.x, y3.y);
+    }
   }
 }
 
@@ -591,13 +604,14 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
           if (vkey < w.sq.s_k) vsc = __ldg(A.v_scales + at + r);
         }
         if (!(ok = __all_sync(0xffffffffu, wait_parity(kraw_full + s, ph, A.wd, &abort_flag)))) break;
-        convert_int8_row<k_nc, D>(smem + G::k_stage(s), smem + G::kKOff + s * G::kKBytes, G::kKChunk, k_r, k_c0,
-                                  ksc);
+        convert_int8_row<k_nc, D, G::kNFull>(smem + G::k_stage(s), smem + G::kKOff + s * G::kKBytes, G::kKChunk,
+                                             k_r, k_c0, ksc);
         fence_proxy_async_smem();
         arrive_x(k_full + s);
         if (!(ok = __all_sync(0xffffffffu, wait_parity(vraw_full + sv, phv, A.wd, &abort_flag)))) break;
-        convert_int8_row<v_rl / 16, v_rl>(smem + G::v_stage(sv), smem + G::kVOff + sv * G::kVBytes, G::kVChunk, r,
-                                          0, vsc);
+        convert_int8_row<v_rl / 16, v_rl, kPair ? 8 : G::kNFull>(smem + G::v_stage(sv),
+                                                                 smem + G::kVOff + sv * G::kVBytes, G::kVChunk, r, 0,
+                                                                 vsc);
         fence_proxy_async_smem();
         arrive_x(v_full + sv);
       }
@@ -873,8 +887,13 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowS
     const uint32_t kbox[3] = {static_cast<uint32_t>(D), krows, 1};
     const uint32_t vw = kPair ? D / 2 : D;
     const uint32_t vbox[3] = {vw, static_cast<uint32_t>(BN), 1};
-    const CUtensorMapSwizzle ksw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    const CUtensorMapSwizzle vsw = vw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    auto sw_of = [](uint32_t bytes) {
+      return bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+           : bytes == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+           : bytes == 32  ? CU_TENSOR_MAP_SWIZZLE_32B
+                          : CU_TENSOR_MAP_SWIZZLE_NONE;
+    };
+    const CUtensorMapSwizzle ksw = sw_of(D), vsw = sw_of(vw);
     fa_status st = encode_tensor_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, p.k, dims, strides, kbox, ksw);
     if (st != FA_OK) return st;
     st = encode_tensor_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, p.v, dims, strides, vbox, vsw);
@@ -1008,6 +1027,8 @@ fa_status launch_prefill_tc(const fa_fwd_params& p, const fa_kv_pages* pages, co
     if (p.head_dim == 128) return pair ? launch_tc<128, true, true>(p, pages, sink, ctx)
                                        : launch_tc<128, true, false>(p, pages, sink, ctx);
     if (p.head_dim == 64) return launch_tc<64, true, false>(p, pages, sink, ctx);
+    if (p.head_dim == 32) return launch_tc<32, true, false>(p, pages, sink, ctx);
+    if (p.head_dim == 96) return launch_tc<96, true, false>(p, pages, sink, ctx);
     return FA_ERR_UNSUPPORTED;
   }
   if (p.head_dim == 128) return pair ? launch_tc<128, false, true>(p, pages, sink, ctx)

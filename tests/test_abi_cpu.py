@@ -84,7 +84,7 @@ def test_fwd_rejects_bad_arguments(fa):
     p.head_dim = 160  # multiple of 32 but no bf16 tensor-core kernel (32, 64, 96, 128)
     assert call_fwd(fa, p) == fa.FA_ERR_UNSUPPORTED
     p = fwd(fa)
-    p.head_dim, p.kv_dtype = 96, fa.FA_I8  # int8 K/V: 64 and 128 only
+    p.head_dim, p.kv_dtype = 160, fa.FA_I8  # int8 K/V: 32, 64, 96, 128
     p.k_scales, p.v_scales = 0x50000, 0x58000
     assert call_fwd(fa, p) == fa.FA_ERR_UNSUPPORTED
     p = fwd(fa)
@@ -151,7 +151,7 @@ def test_decode_rejects_bad_arguments(fa):
     assert call(decode_p(fa, capacity=1000)) == fa.FA_ERR_INVALID       # not a multiple of 32
     assert call(decode_p(fa, max_seqlen=2048)) == fa.FA_ERR_INVALID     # above capacity
     assert call(decode_p(fa, split_keys=100)) == fa.FA_ERR_INVALID
-    assert call(decode_p(fa, head_dim=96)) == fa.FA_ERR_UNSUPPORTED
+    assert call(decode_p(fa, head_dim=160)) == fa.FA_ERR_UNSUPPORTED   # int8 cache: 32, 64, 96, 128, 256
     assert call(decode_p(fa, hq=32, hkv=2)) != fa.FA_ERR_UNSUPPORTED    # a group of 16 runs in two passes
     assert call(decode_p(fa, k_scales=None)) == fa.FA_ERR_INVALID
     assert call(decode_p(fa, workspace_bytes=16)) == fa.FA_ERR_WORKSPACE

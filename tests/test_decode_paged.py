@@ -47,8 +47,11 @@ def paginate(dense, scales, lengths, hkv, page_size, extra, rng):
 
 @pytest.mark.parametrize("int8", [True, False])
 @pytest.mark.parametrize("d,page_size,window,hq,hkv", [(128, 64, 0, 16, 4), (128, 256, 0, 16, 4), (64, 32, 0, 16, 4),
-                                                       (128, 64, 300, 16, 4), (128, 64, 0, 32, 2)])
+                                                       (128, 64, 300, 16, 4), (128, 64, 0, 32, 2), (96, 64, 0, 16, 4),
+                                                       (256, 128, 0, 8, 2)])
 def test_paged_equals_dense(int8, d, page_size, window, hq, hkv):
+    if not int8 and d == 256:
+        pytest.skip("bf16 cache decode: head sizes up to 128")
     fa = _fa()
     rng = np.random.default_rng(d + page_size + window + int8 + hq)
     B, cap = 6, 1024
@@ -197,8 +200,6 @@ def test_paged_prefill_equals_varlen(int8, d, page_size, window):
     than its keys, bottom-right causal) attend to its whole prefix read from
     shuffled pages; bit-identical to the contiguous varlen prefill, and the
     oracle's within the bf16 gate."""
-    if int8 and d not in (64, 128):
-        pytest.skip("int8 K/V on the tensor cores: head sizes 64 and 128")
     fa = _fa()
     rng = np.random.default_rng(50 + d + page_size + window + int8)
     hq, hkv = 8, 2

@@ -46,6 +46,9 @@ DENSE = [
     (1, 6, 2, 130, 50, 128, True, 0),      # empty-band rows (mean of dequantised V)
     (2, 4, 2, 33, 127, 64, True, 0),       # ragged 33/127
     (1, 16, 2, 256, 256, 128, True, 0),    # G = 8
+    (2, 4, 2, 33, 127, 32, True, 0),       # d = 32: the 32-dim tail chunk only
+    (1, 8, 2, 300, 300, 96, True, 0),      # d = 96: a 64-dim chunk and a 32-dim tail
+    (1, 4, 1, 257, 700, 96, False, 200),
 ]
 
 
@@ -60,7 +63,7 @@ def test_dense_int8(case):
     assert_close_bf16(got.float().numpy(), ref, what=str(case))
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [32, 64, 96, 128])
 @pytest.mark.parametrize("epilogue", [(), (("mul", 2.0), ("add", 0.5))], ids=["plain", "mul2add"])
 def test_varlen_int8_window(d, epilogue):
     """Sequence starts at arbitrary rows, so scale addresses are unaligned;
