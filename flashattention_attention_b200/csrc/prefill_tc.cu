@@ -83,8 +83,10 @@ struct TcGeom {
   // deeper ring: a slot refills with the TMA latency hidden behind ~2 steps.
   // A CTA of a pair holds half of every K and V tile (64 keys of K, 64 dims
   // of V), so its rings can be deeper.
-  static constexpr int kKStages = kPair ? (kI8 ? 3 : 4) : (NT == 4 ? 6 : ((kI8 && D == 96) ? 2 : 3));
-  static constexpr int kVStages = kPair ? (kI8 ? 3 : 4) : (NT == 4 ? 6 : ((D == 128 || (kI8 && D == 96)) ? 2 : 3));
+  static constexpr int kKStages = kPair ? (kI8 ? 3 : 4)
+                                 : (NT == 4 ? 6 : ((kI8 && D == 96) || D > 128 ? 2 : 3));
+  static constexpr int kVStages = kPair ? (kI8 ? 3 : 4)
+                                 : (NT == 4 ? 6 : ((D == 128 || (kI8 && D == 96) || D > 128) ? 2 : 3));
   // D = 64 kNFull + 32 kTail: kNFull chunks of 64 dims (128-byte rows,
   // 128-byte swizzle), then, for an odd multiple of 32, one chunk of 32 dims
   // (64-byte rows, 64-byte swizzle) after them
@@ -134,6 +136,8 @@ static_assert(TcGeom<128, true, true>::kSmem <= 232448, "shared memory budget");
 static_assert(TcGeom<64, false, false, 64, 4>::kSmem <= 232448, "shared memory budget");
 static_assert(TcGeom<96, false>::kSmem <= 232448 && TcGeom<96, true>::kSmem <= 232448, "shared memory budget");
 static_assert(TcGeom<32, true>::kSmem <= 232448, "shared memory budget");
+static_assert(TcGeom<256, false, false, 64, 1>::kSmem <= 232448 && TcGeom<224, false, false, 64, 1>::kSmem <= 232448,
+              "shared memory budget");
 
 struct PrefillArgs {
   SeqLayout L;
@@ -395,6 +399,10 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
+      // every K/V tile is read again by the later q-blocks of its sequence
+      // (and the other head pairs of its group), each Q tile once: K/V stay
+      // in L2 ahead of the Q stream
+      const uint64_t pol_q = l2_policy_evict_first(), pol_kv = l2_policy_evict_last();
       int base = 0, done = 0;  // K/V tiles and items before this one
       bool ok = true;
       for (int k = 0, item; ok && (item = item_at(unit, n_units, k)) < n_items; ++k) {
@@ -407,11 +415,11 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
           for (int c = 0; c < G::kNFull; ++c) {
             uint8_t* dst = smem + t * G::kQBytes + c * kChunkBytes;
             if constexpr (kPair) tma_load_3d_pair(dst, &tm_q, lead(q_full), 64 * c, w.q_prow, w.q_plane + t);
-            else tma_load_3d(dst, &tm_q, q_full, 64 * c, w.q_prow, w.q_plane + t);
+            else tma_load_3d_hint(dst, &tm_q, q_full, 64 * c, w.q_prow, w.q_plane + t, pol_q);
           }
           if constexpr (G::kTail)
-            tma_load_3d(smem + t * G::kQBytes + G::kNFull * kChunkBytes, &tm_q32, q_full, 64 * G::kNFull, w.q_prow,
-                        w.q_plane + t);
+            tma_load_3d_hint(smem + t * G::kQBytes + G::kNFull * kChunkBytes, &tm_q32, q_full, 64 * G::kNFull,
+                             w.q_prow, w.q_plane + t, pol_q);
         }
         for (int it = 0; it < w.n_iter; ++it) {
           const int gi = base + it;
@@ -424,7 +432,7 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
           const int k_row = krow + (kPair ? 64 * rank : 0);
           if constexpr (kI8) {
             mbar_expect_tx(kraw_full + s, G::kKI8Bytes);
-            tma_load_3d(smem + G::k_stage(s), &tm_k, kraw_full + s, 0, k_row, kplane);
+            tma_load_3d_hint(smem + G::k_stage(s), &tm_k, kraw_full + s, 0, k_row, kplane, pol_kv);
           } else if constexpr (kPair) {
             if (leader) mbar_expect_tx(k_full + s, 2 * G::kKBytes);
             for (int c = 0; c < D / 64; ++c)
@@ -433,29 +441,30 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
           } else {
             mbar_expect_tx(k_full + s, G::kKBytes);
             for (int c = 0; c < G::kNFull; ++c)
-              tma_load_3d(smem + G::kKOff + s * G::kKBytes + c * G::kKChunk, &tm_k, k_full + s, 64 * c, krow,
-                          kplane);
+              tma_load_3d_hint(smem + G::kKOff + s * G::kKBytes + c * G::kKChunk, &tm_k, k_full + s, 64 * c, krow,
+                               kplane, pol_kv);
             if constexpr (G::kTail)
-              tma_load_3d(smem + G::kKOff + s * G::kKBytes + G::kNFull * G::kKChunk, &tm_k32, k_full + s,
-                          64 * G::kNFull, krow, kplane);
+              tma_load_3d_hint(smem + G::kKOff + s * G::kKBytes + G::kNFull * G::kKChunk, &tm_k32, k_full + s,
+                               64 * G::kNFull, krow, kplane, pol_kv);
           }
           s = gi % VS;
           u = gi / VS;
           if (u > 0 && !(ok = wait_parity<kPair>(v_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
           if constexpr (kI8) {
             mbar_expect_tx(vraw_full + s, G::kVI8Bytes);
-            tma_load_3d(smem + G::v_stage(s), &tm_v, vraw_full + s, kPair ? (D / 2) * rank : 0, krow, kplane);
+            tma_load_3d_hint(smem + G::v_stage(s), &tm_v, vraw_full + s, kPair ? (D / 2) * rank : 0, krow, kplane,
+                             pol_kv);
           } else if constexpr (kPair) {
             if (leader) mbar_expect_tx(v_full + s, 2 * G::kVBytes);
             tma_load_3d_pair(smem + G::kVOff + s * G::kVBytes, &tm_v, lead(v_full + s), (D / 2) * rank, krow, kplane);
           } else {
             mbar_expect_tx(v_full + s, G::kVBytes);
             for (int c = 0; c < G::kNFull; ++c)
-              tma_load_3d(smem + G::kVOff + s * G::kVBytes + c * G::kVChunk, &tm_v, v_full + s, 64 * c, krow,
-                          kplane);
+              tma_load_3d_hint(smem + G::kVOff + s * G::kVBytes + c * G::kVChunk, &tm_v, v_full + s, 64 * c, krow,
+                               kplane, pol_kv);
             if constexpr (G::kTail)
-              tma_load_3d(smem + G::kVOff + s * G::kVBytes + G::kNFull * G::kVChunk, &tm_v32, v_full + s,
-                          64 * G::kNFull, krow, kplane);
+              tma_load_3d_hint(smem + G::kVOff + s * G::kVBytes + G::kNFull * G::kVChunk, &tm_v32, v_full + s,
+                               64 * G::kNFull, krow, kplane, pol_kv);
           }
         }
         base += w.n_iter;
@@ -946,7 +955,7 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowS
   A.hkv = p.hkv;
   A.group = p.hq / p.hkv;
   A.two_tiles = (A.group % 2 == 0) ? 1 : 0;
-  A.heads_per_item = (kPair || NT == 4) ? 4 : (A.two_tiles ? 2 : 1);
+  A.heads_per_item = (kPair || NT == 4) ? 4 : (NT == 1 || !A.two_tiles ? 1 : 2);
   const int max_sq = varlen ? p.max_seqlen_q : p.seqlen_q;
   A.n_qblocks = (max_sq + kBM - 1) / kBM;
   // the softmax works with a positive scale: a negative one negates Q inside
@@ -1037,6 +1046,11 @@ fa_status launch_prefill_tc(const fa_fwd_params& p, const fa_kv_pages* pages, co
                                            : launch_tc<64, false, false>(p, pages, sink, ctx);
   if (p.head_dim == 32) return launch_tc<32, false, false>(p, pages, sink, ctx);
   if (p.head_dim == 96) return launch_tc<96, false, false>(p, pages, sink, ctx);
+  // above 128: one Q tile per CTA (S of a 64-key tile + O of D columns in TMEM)
+  if (p.head_dim == 160) return launch_tc<160, false, false, 64, 1>(p, pages, sink, ctx);
+  if (p.head_dim == 192) return launch_tc<192, false, false, 64, 1>(p, pages, sink, ctx);
+  if (p.head_dim == 224) return launch_tc<224, false, false, 64, 1>(p, pages, sink, ctx);
+  if (p.head_dim == 256) return launch_tc<256, false, false, 64, 1>(p, pages, sink, ctx);
   return FA_ERR_UNSUPPORTED;
 }
 

@@ -81,7 +81,7 @@ def test_fwd_rejects_bad_arguments(fa):
     p.head_dim = 48  # not a multiple of 32
     assert call_fwd(fa, p) == fa.FA_ERR_INVALID
     p = fwd(fa)
-    p.head_dim = 160  # multiple of 32 but no bf16 tensor-core kernel (32, 64, 96, 128)
+    p.head_dim = 288  # multiple of 32 but no bf16 tensor-core kernel (32 .. 256)
     assert call_fwd(fa, p) == fa.FA_ERR_UNSUPPORTED
     p = fwd(fa)
     p.head_dim, p.kv_dtype = 160, fa.FA_I8  # int8 K/V: 32, 64, 96, 128
@@ -278,7 +278,7 @@ def test_fwd_paged_rejects_bad_arguments(fa):
     assert call(cu_seqlens_k=None) == fa.FA_ERR_INVALID      # per-sequence key counts required
     assert call(block_table=None) == fa.FA_ERR_INVALID
     assert call(q_dtype=fa.FA_F32, kv_dtype=fa.FA_F32) == fa.FA_ERR_INVALID   # tensor-core path only
-    assert call(head_dim=160) == fa.FA_ERR_UNSUPPORTED
+    assert call(head_dim=288) == fa.FA_ERR_UNSUPPORTED
     assert call(kv_dtype=fa.FA_I8) == fa.FA_ERR_INVALID       # int8 needs scales
     assert call(seqlen_q=0) == fa.FA_OK                       # nothing to do
 
@@ -341,7 +341,7 @@ def test_fwd_acc_rejects_bad_arguments(fa):
             v=FakeTensor(0x30000, (2, 64, 128), torch.float32), out=FakeTensor(0x40000, (4, 64, 128), torch.float32))
     assert call(p) == fa.FA_ERR_UNSUPPORTED                   # fp32 path
     p = fwd(fa)
-    p.head_dim = 160
+    p.head_dim = 288
     assert call(p) == fa.FA_ERR_UNSUPPORTED
     p = fwd(fa)
     p.seqlen_q = 0

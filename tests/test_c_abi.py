@@ -36,7 +36,7 @@ int main(void) {
   p.batch = 1; p.hq = 3; p.hkv = 2; p.head_dim = 128; p.seqlen_q = p.seqlen_k = 64;
   p.q_dtype = FA_BF16; p.kv_dtype = FA_BF16; p.softmax_scale = 0.125f;
   CHECK(fa_attention_fwd(&p, NULL) == FA_ERR_INVALID);  /* hq % hkv != 0 */
-  p.hq = 4; p.head_dim = 160;  /* a multiple of 32 without a tensor-core kernel */
+  p.hq = 4; p.head_dim = 288;  /* a multiple of 32 without a tensor-core kernel */
   CHECK(fa_attention_fwd(&p, NULL) == FA_ERR_UNSUPPORTED);
   p.head_dim = 128; p.seqlen_q = 0;
   CHECK(fa_attention_fwd(&p, NULL) == FA_OK);  /* nothing to do */

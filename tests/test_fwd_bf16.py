@@ -40,6 +40,11 @@ DENSE = [
     (1, 8, 2, 300, 300, 96, True, 0),      # d = 96: a 64-dim chunk and a 32-dim tail
     (1, 4, 1, 257, 700, 96, False, 200),
     (1, 4, 4, 200, 333, 96, True, 0),
+    (1, 4, 2, 300, 300, 256, True, 0),     # d = 256: one Q tile per CTA, 64-key tiles
+    (2, 2, 1, 33, 127, 256, False, 0),
+    (1, 4, 2, 257, 700, 192, True, 150),   # d = 192 with a window
+    (1, 2, 2, 130, 50, 160, True, 0),      # d = 160 (a 32-dim tail) with empty-band rows
+    (1, 8, 2, 200, 200, 224, False, 0),    # d = 224
 ]
 
 
@@ -53,7 +58,7 @@ def test_dense(case):
     assert_close_bf16(got.float().numpy(), ref, what=str(case))
 
 
-@pytest.mark.parametrize("d", [32, 64, 96, 128])
+@pytest.mark.parametrize("d", [32, 64, 96, 128, 256])
 @pytest.mark.parametrize("causal,window", [(True, 0), (True, 100), (False, 0)])
 def test_varlen(d, causal, window):
     lengths = [33, 127, 1, 300, 129, 256]
