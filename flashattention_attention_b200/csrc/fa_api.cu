@@ -79,9 +79,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Head sizes of the tensor-core prefill: 32, 64, 96 or 128 (bf16 or int8 K/V);
 // 160, 192, 224 or 256 (bf16 K/V).
-bool tc_head_dim_ok(int d, int kv_dtype) {
-  if (d == 32 || d == 64 || d == 96 || d == 128) return true;
-  return kv_dtype != FA_I8 && (d == 160 || d == 192 || d == 224 || d == 256);
+bool tc_head_dim_ok(int d, int /*kv_dtype*/) {
+  return d == 32 || d == 64 || d == 96 || d == 128 || d == 160 || d == 192 || d == 224 || d == 256;
 }
 
 bool epilogue_ok(const fa_epi_op* ops, int n) {

@@ -53,7 +53,9 @@
 // round once to bf16, the tensor-core operand type, write it in the operand
 // layout and fence it to the async proxy.  The softmax is then the bf16 one.
 // That variant runs 16 warps and rebalances registers with setmaxnreg
-// (softmax 192, the rest 64).
+// (softmax 192, the rest 64).  Above d = 128 (one Q tile, 64-key tiles, 12
+// warps) two converter threads share a key row, and the int8 tiles land in
+// rings of their own so the bf16 operand slots fit beside the Q tile.
 #include <cstdlib>
 #include <mutex>
 
@@ -86,7 +88,14 @@ struct TcGeom {
   static constexpr int kKStages = kPair ? (kI8 ? 3 : 4)
                                  : (NT == 4 ? 6 : ((kI8 && D == 96) || D > 128 ? 2 : 3));
   static constexpr int kVStages = kPair ? (kI8 ? 3 : 4)
-                                 : (NT == 4 ? 6 : ((D == 128 || (kI8 && D == 96) || D > 128) ? 2 : 3));
+                                 : (NT == 4 ? 6 : (kI8 && D > 128 ? 1 : ((D == 128 || (kI8 && D == 96) || D > 128) ? 2 : 3)));
+  // int8 above d = 128: the int8 tiles land in rings of their own (a slot
+  // is refilled once the converters have read it), so the bf16 operand slots
+  // (one V slot, two K slots) fit beside a 64 KB Q tile; otherwise an int8
+  // tile and its bf16 slot share the ring position
+  static constexpr bool kSplitRaw = kI8 && D > 128;
+  static constexpr int kRawKStages = !kI8 ? 0 : (kSplitRaw ? 2 : kKStages);
+  static constexpr int kRawVStages = !kI8 ? 0 : (kSplitRaw ? 2 : kVStages);
   // D = 64 kNFull + 32 kTail: kNFull chunks of 64 dims (128-byte rows,
   // 128-byte swizzle), then, for an odd multiple of 32, one chunk of 32 dims
   // (64-byte rows, 64-byte swizzle) after them
@@ -108,15 +117,29 @@ struct TcGeom {
   // separate
   static constexpr bool kInPlace = (D == 128) && !kPair;
   static constexpr uint32_t kStageOff = kVOff + kVStages * kVBytes;
-  static constexpr uint32_t kStageBytes = (kI8 && !kInPlace) ? kKStages * kKI8Bytes + kVStages * kVI8Bytes : 0;
+  static constexpr uint32_t kStageBytes =
+      (kI8 && !kInPlace) ? kRawKStages * kKI8Bytes + kRawVStages * kVI8Bytes : 0;
   static constexpr uint32_t kBarOff = kStageOff + kStageBytes;
+  // mbarriers (8 bytes each, the order of the kernel's pointers) + the TMEM address
+  static constexpr uint32_t kBarBytes =
+      8 * (1 + 2 * kKStages + 2 * kVStages + 5 * NT + 1 + 2 * kRawKStages + 2 * kRawVStages + 1) + 4;
+  static_assert(kBarBytes <= 512, "barrier area");
   static constexpr uint32_t kSmem = kBarOff + 512 + 1024;
   // int8: 2 idle warps and 4 converters; four Q tiles: a fifth warpgroup
   // (producer, MMA, 2 idle) so registers can move between warpgroups
-  static constexpr int kThreads = (4 * NT + ((kI8 || NT == 4) ? (kI8 ? 8 : 4) : 2)) * 32;
+  // (int8 above 128: 2 idle warps, 4 K converters and 4 V converters)
+  static constexpr int kThreads = (4 * NT + ((kI8 || NT == 4) ? (kI8 ? (kSplitRaw ? 12 : 8) : 4) : 2)) * 32;
   // setmaxnreg split (0: none): the softmax warpgroups take kRegsHi, the
   // others give back down to 64 (the totals match the launch's pool)
+  // (int8 with one Q tile, 512 threads: one softmax warpgroup at 192, three
+  // at 96: 128*192 + 384*96 <= 512*128)
   static constexpr int kRegsHi = kI8 ? 192 : (NT == 4 ? 104 : 0);
+  static constexpr int kRegsLo = kSplitRaw ? 96 : 64;
+  // the registers a launch of kThreads threads gets per thread, which the
+  // split redistributes (setmaxnreg.inc waits for registers the pool lacks)
+  static constexpr int kLaunchRegs = (65536 / kThreads) / 8 * 8;
+  static_assert(kRegsHi == 0 || 128 * NT * kRegsHi + (kThreads - 128 * NT) * kRegsLo <= kThreads * kLaunchRegs,
+                "setmaxnreg budget");
   // TMEM columns: S_t (P_t over its first BN / 2 columns) and O_t
   static constexpr uint32_t s_col(int t) { return t * BN; }
   static constexpr uint32_t o_col(int t) { return NT * BN + t * D; }
@@ -125,7 +148,7 @@ struct TcGeom {
     return kInPlace ? kKOff + s * kKBytes + kKBytes / 2 : kStageOff + s * kKI8Bytes;
   }
   __host__ __device__ static constexpr uint32_t v_stage(int s) {
-    return kInPlace ? kVOff + s * kVBytes + kVBytes / 2 : kStageOff + kKStages * kKI8Bytes + s * kVI8Bytes;
+    return kInPlace ? kVOff + s * kVBytes + kVBytes / 2 : kStageOff + kRawKStages * kKI8Bytes + s * kVI8Bytes;
   }
 };
 static_assert(TcGeom<128, false>::kSmem <= 232448, "shared memory budget");
@@ -137,6 +160,8 @@ static_assert(TcGeom<64, false, false, 64, 4>::kSmem <= 232448, "shared memory b
 static_assert(TcGeom<96, false>::kSmem <= 232448 && TcGeom<96, true>::kSmem <= 232448, "shared memory budget");
 static_assert(TcGeom<32, true>::kSmem <= 232448, "shared memory budget");
 static_assert(TcGeom<256, false, false, 64, 1>::kSmem <= 232448 && TcGeom<224, false, false, 64, 1>::kSmem <= 232448,
+              "shared memory budget");
+static_assert(TcGeom<256, true, false, 64, 1>::kSmem <= 232448 && TcGeom<224, true, false, 64, 1>::kSmem <= 232448,
               "shared memory budget");
 
 struct PrefillArgs {
@@ -216,6 +241,39 @@ __device__ __forceinline__ void convert_int8_row(const uint8_t* src_tile, uint8_
   }
 }
 
+// Above d = 128 (64-key tiles, int8 rows staged without swizzle, D bytes
+// each): thread (row, h) converts D / 32 of the row's D / 16 chunks of 16
+// codes, chunk c0 + 2i (mod D / 16) at step i, with c0 = h + a row + b h +
+// f (row / 2).  The two threads of a row cover it once; a, b, f were found
+// by an exhaustive search so that the 8 lanes of each shared-memory phase
+// (4 rows x 2 halves) read 8 different bank groups, and write at most 2 to
+// one (only where the 32-dim tail's 64-byte rows are involved).
+template <int D, int kNFull>
+__device__ __forceinline__ void convert_int8_half_row(const uint8_t* src_tile, uint8_t* dst_tile, uint32_t dst_chunk,
+                                                      int row, int h, float sc) {
+  constexpr int U = D / 16;
+  constexpr int a = D == 256 ? 2 : 0, b = D == 256 ? 2 : 0, f = D == 192 ? 2 : 0;
+  const float2 s2 = make_float2(sc, sc);
+  const uint8_t* src = src_tile + row * D;
+  int c = (h + a * row + b * h + f * (row >> 1)) % U;
+#pragma unroll
+  for (int i = 0; i < U / 2; ++i) {
+    const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
+    const uint2 y0 = dequant4_bf16(w.x, s2), y1 = dequant4_bf16(w.y, s2);
+    const uint2 y2 = dequant4_bf16(w.z, s2), y3 = dequant4_bf16(w.w, s2);
+    const int hc = c >> 2, j0 = 2 * (c & 3);
+    // a 64-dim chunk: 128-byte rows, 128-byte swizzle; the 32-dim tail:
+    // 64-byte rows, 64-byte swizzle
+    const bool tail = hc >= kNFull;
+    const int sw = tail ? ((row >> 1) & 3) : (row & 7);
+    uint8_t* out = dst_tile + hc * dst_chunk + row * (tail ? 64 : 128);
+    *reinterpret_cast<uint4*>(out + ((j0 ^ sw) * 16)) = make_uint4(y0.x, y0.y, y1.x, y1.y);
+    *reinterpret_cast<uint4*>(out + (((j0 + 1) ^ sw) * 16)) = make_uint4(y2.x, y2.y, y3.x, y3.y);
+    c += 2;
+    if (c >= U) c -= U;
+  }
+}
+
 // One work item: 128 query rows of one head pair (or one head), in the
 // longest-first order (highest q-block first, then sequence, then head pair).
 struct Item {
@@ -289,7 +347,7 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_k32, const __grid_constant__ CUtensorMap tm_v32,
                       const PrefillArgs A) {
   using G = TcGeom<D, kI8, kPair, BN, NT>;
-  constexpr int KS = G::kKStages, VS = G::kVStages;
+  constexpr int KS = G::kKStages, VS = G::kVStages, RKS = G::kRawKStages, RVS = G::kRawVStages;
   constexpr int kLoadWarp = G::kLoadWarp, kMmaWarp = G::kMmaWarp, kConvWarp0 = G::kConvWarp0;
   extern __shared__ uint8_t tc_smem_raw[];
   uint8_t* smem =
@@ -304,9 +362,11 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
   uint64_t* p_full = s_full + NT;  // [NT tiles][2 halves of the keys]
   uint64_t* o_done = p_full + 2 * NT;  // [NT]
   uint64_t* drain = o_done + NT;
-  uint64_t* kraw_full = drain + 1;   // [KS] int8 variant: TMA landed the int8 K tile
-  uint64_t* vraw_full = kraw_full + KS;
-  uint64_t* q_empty = vraw_full + VS;  // every S MMA of an item has read Q
+  uint64_t* kraw_full = drain + 1;   // [RKS] int8 variant: TMA landed the int8 K tile
+  uint64_t* vraw_full = kraw_full + RKS;
+  uint64_t* kraw_empty = vraw_full + RVS;  // [RKS] separate int8 rings: the converters have read it
+  uint64_t* vraw_empty = kraw_empty + RKS;
+  uint64_t* q_empty = vraw_empty + RVS;  // every S MMA of an item has read Q
   uint64_t* o_free = q_empty + 1;       // [NT] the softmax warps have read O_t out
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + NT);
   __shared__ int abort_flag;
@@ -354,12 +414,18 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
     for (int s = 0; s < KS; ++s) {
       mbar_init(k_full + s, kI8 ? kArrivals : 1);
       mbar_init(k_empty + s, 1);
-      mbar_init(kraw_full + s, 1);
     }
     for (int s = 0; s < VS; ++s) {
       mbar_init(v_full + s, kI8 ? kArrivals : 1);
       mbar_init(v_empty + s, 1);
+    }
+    for (int s = 0; s < RKS; ++s) {
+      mbar_init(kraw_full + s, 1);
+      mbar_init(kraw_empty + s, kArrivals);
+    }
+    for (int s = 0; s < RVS; ++s) {
       mbar_init(vraw_full + s, 1);
+      mbar_init(vraw_empty + s, kArrivals);
     }
     for (int t = 0; t < NT; ++t) {
       mbar_init(s_full + t, 1);
@@ -392,7 +458,8 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
   // warpgroups 0-1 take 192, warpgroups 2-3 give back down to 64:
   // 256*192 + 256*64 = 512*128.
   if (warp >= 4 * NT) {
-  if constexpr (G::kRegsHi > 0) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
+  if constexpr (G::kRegsHi > 0 && G::kRegsLo == 64) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
+  if constexpr (G::kRegsHi > 0 && G::kRegsLo == 96) asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -426,7 +493,14 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
           int s = gi % KS, u = gi / KS;
           int kplane, krow;
           kv_tile(A, w, (w.j_lo + it) * BN, kplane, krow);
-          if (u > 0 && !(ok = wait_parity<kPair>(k_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
+          if constexpr (G::kSplitRaw) {
+            // separate int8 ring: its slot is free once the converters read it
+            s = gi % RKS;
+            u = gi / RKS;
+            if (u > 0 && !(ok = wait_parity(kraw_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
+          } else if (u > 0 && !(ok = wait_parity<kPair>(k_empty + s, (u - 1) & 1, A.wd, &abort_flag))) {
+            break;
+          }
           // a pair's CTA r brings keys [64 r, 64 r + 64) of K and dims
           // [D/2 r, D/2 r + D/2) of V
           const int k_row = krow + (kPair ? 64 * rank : 0);
@@ -447,9 +521,15 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
               tma_load_3d_hint(smem + G::kKOff + s * G::kKBytes + G::kNFull * G::kKChunk, &tm_k32, k_full + s,
                                64 * G::kNFull, krow, kplane, pol_kv);
           }
-          s = gi % VS;
-          u = gi / VS;
-          if (u > 0 && !(ok = wait_parity<kPair>(v_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
+          if constexpr (G::kSplitRaw) {
+            s = gi % RVS;
+            u = gi / RVS;
+            if (u > 0 && !(ok = wait_parity(vraw_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
+          } else {
+            s = gi % VS;
+            u = gi / VS;
+            if (u > 0 && !(ok = wait_parity<kPair>(v_empty + s, (u - 1) & 1, A.wd, &abort_flag))) break;
+          }
           if constexpr (kI8) {
             mbar_expect_tx(vraw_full + s, G::kVI8Bytes);
             tma_load_3d_hint(smem + G::v_stage(s), &tm_v, vraw_full + s, kPair ? (D / 2) * rank : 0, krow, kplane,
@@ -578,6 +658,52 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
       // every MMA this thread issued has completed before TMEM is released
       commit(drain);
       wait_parity(drain, 0, A.wd);
+    }
+  } else if (G::kSplitRaw && warp >= kConvWarp0) {
+    // ------------------------------------------------------------ int8 -> bf16 converters, d > 128
+    // Warps kConvWarp0 .. +3 convert K, the next four V, two threads per
+    // key row of the 64-key tiles.  A tile's int8 slot is released once
+    // read; its bf16 slot is written once the MMAs that read the slot's
+    // previous tile have completed.
+    const int r = static_cast<int>(threadIdx.x) - kConvWarp0 * 32;
+    const bool is_v = r >= 128;  // warp-uniform
+    const int row = (r & 127) >> 1, h = r & 1;
+    uint64_t* raw_full = is_v ? vraw_full : kraw_full;
+    uint64_t* raw_empty = is_v ? vraw_empty : kraw_empty;
+    uint64_t* op_full = is_v ? v_full : k_full;
+    uint64_t* op_empty = is_v ? v_empty : k_empty;
+    const int n_raw = is_v ? RVS : RKS, n_op = is_v ? VS : KS;
+    const float* scales = is_v ? A.v_scales : A.k_scales;
+    static_assert(!G::kSplitRaw ||
+                      (G::kKChunk == G::kVChunk && G::kKBytes == G::kVBytes && G::kKI8Bytes == G::kVI8Bytes),
+                  "K and V slots alike");
+    const uint32_t op_off = is_v ? G::kVOff : G::kKOff;
+    int base = 0;
+    bool ok = true;
+    for (int k = 0, item; ok && (item = item_at(unit, n_units, k)) < n_items; ++k) {
+      Item w;
+      if (!item_of<BN>(A, item, w, rank)) continue;
+      for (int it = 0; it < w.n_iter; ++it) {
+        const int gi = base + it;
+        const int key0 = (w.j_lo + it) * BN;
+        float sc = 0.f;  // 0 past the sequence end: those rows become zeros
+        if (key0 + row < w.sq.s_k) {
+          int kplane, krow;
+          kv_tile(A, w, key0, kplane, krow);
+          sc = __ldg(scales + static_cast<int64_t>(kplane) * A.k_plane_rows + krow + row);
+        }
+        const int rs = gi % n_raw, s = gi % n_op;
+        if (!(ok = __all_sync(0xffffffffu, wait_parity(raw_full + rs, (gi / n_raw) & 1, A.wd, &abort_flag)))) break;
+        if (gi >= n_op &&
+            !(ok = __all_sync(0xffffffffu, wait_parity(op_empty + s, (gi / n_op - 1) & 1, A.wd, &abort_flag))))
+          break;
+        convert_int8_half_row<D, G::kNFull>(smem + (is_v ? G::v_stage(rs) : G::k_stage(rs)),
+                                            smem + op_off + s * G::kKBytes, G::kKChunk, row, h, sc);
+        fence_proxy_async_smem();
+        mbar_arrive(raw_empty + rs);
+        mbar_arrive(op_full + s);
+      }
+      base += w.n_iter;
     }
   } else if (kI8 && warp >= kConvWarp0) {
     // ------------------------------------------------------------ int8 -> bf16 converters
@@ -890,7 +1016,8 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowS
   const uint32_t krows = static_cast<uint32_t>(G::kKRows);
   if constexpr (kI8) {
     // int8 rows: K boxes of whole rows (D bytes), V boxes of this CTA's
-    // dims (D bytes, or D / 2 in a pair): 128- or 64-byte swizzle
+    // dims (D bytes, or D / 2 in a pair): the 128-, 64- or 32-byte swizzle
+    // of that width, unswizzled rows otherwise (d = 96 and above 128)
     const uint64_t dims[3] = {static_cast<uint64_t>(D), k_rows, k_planes};
     const uint64_t strides[2] = {static_cast<uint64_t>(D), k_rows * D};
     const uint32_t kbox[3] = {static_cast<uint32_t>(D), krows, 1};
@@ -928,16 +1055,18 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowS
     fa_status st = encode_tensor_map(&tq32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.q, qdims, qstr, qbox,
                                      CU_TENSOR_MAP_SWIZZLE_64B);
     if (st != FA_OK) return st;
-    const uint64_t kdims[3] = {static_cast<uint64_t>(D), k_rows, k_planes};
-    const uint64_t kstr[2] = {static_cast<uint64_t>(D) * 2, k_rows * D * 2};
-    const uint32_t kbox[3] = {32, krows, 1};
-    const uint32_t vbox[3] = {32, static_cast<uint32_t>(BN), 1};
-    st = encode_tensor_map(&tk32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.k, kdims, kstr, kbox,
-                           CU_TENSOR_MAP_SWIZZLE_64B);
-    if (st != FA_OK) return st;
-    st = encode_tensor_map(&tv32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.v, kdims, kstr, vbox,
-                           CU_TENSOR_MAP_SWIZZLE_64B);
-    if (st != FA_OK) return st;
+    if constexpr (!kI8) {  // int8 rows come in whole through tk / tv
+      const uint64_t kdims[3] = {static_cast<uint64_t>(D), k_rows, k_planes};
+      const uint64_t kstr[2] = {static_cast<uint64_t>(D) * 2, k_rows * D * 2};
+      const uint32_t kbox[3] = {32, krows, 1};
+      const uint32_t vbox[3] = {32, static_cast<uint32_t>(BN), 1};
+      st = encode_tensor_map(&tk32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.k, kdims, kstr, kbox,
+                             CU_TENSOR_MAP_SWIZZLE_64B);
+      if (st != FA_OK) return st;
+      st = encode_tensor_map(&tv32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.v, kdims, kstr, vbox,
+                             CU_TENSOR_MAP_SWIZZLE_64B);
+      if (st != FA_OK) return st;
+    }
   }
   PrefillArgs A;
   A.L = pages != nullptr ? SeqLayout::paged(p, *pages) : SeqLayout::from(p);
@@ -1038,6 +1167,11 @@ fa_status launch_prefill_tc(const fa_fwd_params& p, const fa_kv_pages* pages, co
     if (p.head_dim == 64) return launch_tc<64, true, false>(p, pages, sink, ctx);
     if (p.head_dim == 32) return launch_tc<32, true, false>(p, pages, sink, ctx);
     if (p.head_dim == 96) return launch_tc<96, true, false>(p, pages, sink, ctx);
+    // above 128: one Q tile per CTA, 64-key tiles, separate int8 rings
+    if (p.head_dim == 160) return launch_tc<160, true, false, 64, 1>(p, pages, sink, ctx);
+    if (p.head_dim == 192) return launch_tc<192, true, false, 64, 1>(p, pages, sink, ctx);
+    if (p.head_dim == 224) return launch_tc<224, true, false, 64, 1>(p, pages, sink, ctx);
+    if (p.head_dim == 256) return launch_tc<256, true, false, 64, 1>(p, pages, sink, ctx);
     return FA_ERR_UNSUPPORTED;
   }
   if (p.head_dim == 128) return pair ? launch_tc<128, false, true>(p, pages, sink, ctx)

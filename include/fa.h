@@ -117,8 +117,8 @@ FA_API fa_status fa_compress_kv(const void *x, fa_dtype x_dtype, int64_t rows, i
  * (fkl_python PR #6, Summary): exactly in fp32 on the F32 path; on the BF16
  * path c * s is formed exactly in fp32 and rounded once to bf16, the
  * tensor-core operand type.  out has q's dtype.
- * head_dim: F32 path any multiple of 32 up to 256; BF16 path 32, 64, 96 or 128
- * (FA_BF16 or FA_I8 K/V), and 160, 192, 224 or 256 (FA_BF16 K/V).
+ * head_dim: F32 path any multiple of 32 up to 256; BF16 path 32, 64, 96, 128,
+ * 160, 192, 224 or 256 (FA_BF16 or FA_I8 K/V).
  * A problem without keys (seqlen_k = 0, or varlen total_k = 0 with
  * cu_seqlens_k given) reads no K or V: k, v and the scales may be NULL.
  */

@@ -81,10 +81,10 @@ def test_fwd_rejects_bad_arguments(fa):
     p.head_dim = 48  # not a multiple of 32
     assert call_fwd(fa, p) == fa.FA_ERR_INVALID
     p = fwd(fa)
-    p.head_dim = 288  # multiple of 32 but no bf16 tensor-core kernel (32 .. 256)
+    p.head_dim = 288  # multiple of 32 but no tensor-core kernel (32 .. 256)
     assert call_fwd(fa, p) == fa.FA_ERR_UNSUPPORTED
     p = fwd(fa)
-    p.head_dim, p.kv_dtype = 160, fa.FA_I8  # int8 K/V: 32, 64, 96, 128
+    p.head_dim, p.kv_dtype = 288, fa.FA_I8  # int8 K/V: the same head sizes
     p.k_scales, p.v_scales = 0x50000, 0x58000
     assert call_fwd(fa, p) == fa.FA_ERR_UNSUPPORTED
     p = fwd(fa)

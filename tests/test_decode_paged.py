@@ -194,7 +194,7 @@ def paginate_varlen(x, scales, lens, hkv, page_size, rng, extra=3):
 
 @pytest.mark.parametrize("int8", [False, True])
 @pytest.mark.parametrize("d,page_size,window", [(128, 128, 0), (128, 256, 0), (64, 128, 200), (96, 128, 0),
-                                                (32, 256, 100)])
+                                                (32, 256, 100), (256, 128, 0), (160, 256, 300)])
 def test_paged_prefill_equals_varlen(int8, d, page_size, window):
     """Chunked prefill over a paged cache: each sequence's new queries (fewer
     than its keys, bottom-right causal) attend to its whole prefix read from

@@ -49,6 +49,11 @@ DENSE = [
     (2, 4, 2, 33, 127, 32, True, 0),       # d = 32: the 32-dim tail chunk only
     (1, 8, 2, 300, 300, 96, True, 0),      # d = 96: a 64-dim chunk and a 32-dim tail
     (1, 4, 1, 257, 700, 96, False, 200),
+    (1, 4, 2, 300, 300, 256, True, 0),     # d = 256: one Q tile per CTA, 64-key tiles, own int8 rings
+    (2, 2, 1, 33, 127, 256, False, 0),
+    (1, 4, 2, 257, 700, 192, True, 150),   # d = 192 with a window
+    (1, 2, 2, 130, 50, 160, True, 0),      # d = 160 (a 32-dim tail) with empty-band rows
+    (1, 8, 2, 200, 200, 224, False, 0),    # d = 224: three 64-dim chunks and a 32-dim tail
 ]
 
 
@@ -63,7 +68,7 @@ def test_dense_int8(case):
     assert_close_bf16(got.float().numpy(), ref, what=str(case))
 
 
-@pytest.mark.parametrize("d", [32, 64, 96, 128])
+@pytest.mark.parametrize("d", [32, 64, 96, 128, 160, 256])
 @pytest.mark.parametrize("epilogue", [(), (("mul", 2.0), ("add", 0.5))], ids=["plain", "mul2add"])
 def test_varlen_int8_window(d, epilogue):
     """Sequence starts at arbitrary rows, so scale addresses are unaligned;
