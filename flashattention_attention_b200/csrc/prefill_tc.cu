@@ -88,7 +88,7 @@ struct TcGeom {
   static constexpr int kKStages = kPair ? (kI8 ? 3 : 4)
                                  : (NT == 4 ? 6 : ((kI8 && D == 96) || D > 128 ? 2 : 3));
   static constexpr int kVStages = kPair ? (kI8 ? 3 : 4)
-                                 : (NT == 4 ? 6 : (kI8 && D > 128 ? 1 : ((D == 128 || (kI8 && D == 96) || D > 128) ? 2 : 3)));
+                                 : (NT == 4 ? 6 : (kI8 && D > 128 ? 1 : ((D == 128 || D == 96 || D > 128) ? 2 : 3)));
   // int8 above d = 128: the int8 tiles land in rings of their own (a slot
   // is refilled once the converters have read it), so the bf16 operand slots
   // (one V slot, two K slots) fit beside a 64 KB Q tile; otherwise an int8
@@ -97,19 +97,25 @@ struct TcGeom {
   static constexpr int kRawKStages = !kI8 ? 0 : (kSplitRaw ? 2 : kKStages);
   static constexpr int kRawVStages = !kI8 ? 0 : (kSplitRaw ? 2 : kVStages);
   // D = 64 kNFull + 32 kTail: kNFull chunks of 64 dims (128-byte rows,
-  // 128-byte swizzle), then, for an odd multiple of 32, one chunk of 32 dims
-  // (64-byte rows, 64-byte swizzle) after them
+  // 128-byte swizzle), then, for an odd multiple of 32, a 32-dim tail: as a
+  // further 64-dim chunk whose upper half TMA fills with zeros (one PV MMA
+  // with N = D), except with int8 K/V at d = 96, whose separate int8
+  // staging leaves no room for padded slots: there the tail is a chunk of
+  // 32 dims (64-byte rows, 64-byte swizzle) with MMAs of its own
   static constexpr int kNFull = D / 64;
   static constexpr bool kTail = (D % 64) == 32;
+  static constexpr bool kTailSw64 = kTail && kI8 && D == 96;
+  static constexpr int kNChunks = kNFull + ((kTail && !kTailSw64) ? 1 : 0);  // 128-byte-swizzled chunks
+  static constexpr int kDP = kTailSw64 ? D : 64 * kNChunks;                  // dims per staged bf16 row
   static_assert(D % 32 == 0, "head size");
-  static constexpr uint32_t kQBytes = kBM * D * 2;
+  static constexpr uint32_t kQBytes = kBM * kDP * 2;
   static constexpr int kKRows = kPair ? BN / 2 : BN;               // K rows in this CTA's slot
   static constexpr uint32_t kKChunk = kKRows * 128;                 // one 64-dim chunk of them
-  static constexpr uint32_t kKBytes = kKRows * D * 2;               // this CTA's bf16 K slot
+  static constexpr uint32_t kKBytes = kKRows * kDP * 2;             // this CTA's bf16 K slot
   static constexpr uint32_t kVChunk = BN * 128;                     // 64 dims of every key of a tile
-  static constexpr uint32_t kVBytes = BN * (kPair ? D / 2 : D) * 2;  // this CTA's bf16 V slot
-  static constexpr uint32_t kKI8Bytes = kKBytes / 2;                // the same slots as int8
-  static constexpr uint32_t kVI8Bytes = kVBytes / 2;
+  static constexpr uint32_t kVBytes = BN * (kPair ? D / 2 : kDP) * 2;  // this CTA's bf16 V slot
+  static constexpr uint32_t kKI8Bytes = kKRows * D;                 // the int8 tiles (unpadded rows)
+  static constexpr uint32_t kVI8Bytes = BN * (kPair ? D / 2 : D);
   static constexpr uint32_t kKOff = NT * kQBytes;
   static constexpr uint32_t kVOff = kKOff + kKStages * kKBytes;
   // int8 staging: at d = 128 (one CTA) in the upper half of each bf16 slot
@@ -162,6 +168,9 @@ static_assert(TcGeom<32, true>::kSmem <= 232448, "shared memory budget");
 static_assert(TcGeom<256, false, false, 64, 1>::kSmem <= 232448 && TcGeom<224, false, false, 64, 1>::kSmem <= 232448,
               "shared memory budget");
 static_assert(TcGeom<256, true, false, 64, 1>::kSmem <= 232448 && TcGeom<224, true, false, 64, 1>::kSmem <= 232448,
+              "shared memory budget");
+static_assert(TcGeom<160, false, false, 64, 1>::kSmem <= 232448 && TcGeom<160, true, false, 64, 1>::kSmem <= 232448 &&
+                  TcGeom<192, true, false, 64, 1>::kSmem <= 232448 && TcGeom<32, false>::kSmem <= 232448,
               "shared memory budget");
 
 struct PrefillArgs {
@@ -344,7 +353,6 @@ template <int D, bool kI8, bool kPair, int BN, int NT>
 __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q32,
-                      const __grid_constant__ CUtensorMap tm_k32, const __grid_constant__ CUtensorMap tm_v32,
                       const PrefillArgs A) {
   using G = TcGeom<D, kI8, kPair, BN, NT>;
   constexpr int KS = G::kKStages, VS = G::kVStages, RKS = G::kRawKStages, RVS = G::kRawVStages;
@@ -479,12 +487,12 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
         if (done > 0 && !wait_parity<kPair>(q_empty, (done - 1) & 1, A.wd, &abort_flag)) break;
         if (leader) mbar_expect_tx(q_full, (kPair ? 2 : 1) * ntile * G::kQBytes);
         for (int t = 0; t < ntile; ++t) {
-          for (int c = 0; c < G::kNFull; ++c) {
+          for (int c = 0; c < G::kNChunks; ++c) {
             uint8_t* dst = smem + t * G::kQBytes + c * kChunkBytes;
             if constexpr (kPair) tma_load_3d_pair(dst, &tm_q, lead(q_full), 64 * c, w.q_prow, w.q_plane + t);
             else tma_load_3d_hint(dst, &tm_q, q_full, 64 * c, w.q_prow, w.q_plane + t, pol_q);
           }
-          if constexpr (G::kTail)
+          if constexpr (G::kTailSw64)
             tma_load_3d_hint(smem + t * G::kQBytes + G::kNFull * kChunkBytes, &tm_q32, q_full, 64 * G::kNFull,
                              w.q_prow, w.q_plane + t, pol_q);
         }
@@ -514,12 +522,10 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
                                k_row, kplane);
           } else {
             mbar_expect_tx(k_full + s, G::kKBytes);
-            for (int c = 0; c < G::kNFull; ++c)
+            // (a padded tail chunk: the dims past D read as zeros)
+            for (int c = 0; c < G::kNChunks; ++c)
               tma_load_3d_hint(smem + G::kKOff + s * G::kKBytes + c * G::kKChunk, &tm_k, k_full + s, 64 * c, krow,
                                kplane, pol_kv);
-            if constexpr (G::kTail)
-              tma_load_3d_hint(smem + G::kKOff + s * G::kKBytes + G::kNFull * G::kKChunk, &tm_k32, k_full + s,
-                               64 * G::kNFull, krow, kplane, pol_kv);
           }
           if constexpr (G::kSplitRaw) {
             s = gi % RVS;
@@ -539,12 +545,9 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
             tma_load_3d_pair(smem + G::kVOff + s * G::kVBytes, &tm_v, lead(v_full + s), (D / 2) * rank, krow, kplane);
           } else {
             mbar_expect_tx(v_full + s, G::kVBytes);
-            for (int c = 0; c < G::kNFull; ++c)
+            for (int c = 0; c < G::kNChunks; ++c)
               tma_load_3d_hint(smem + G::kVOff + s * G::kVBytes + c * G::kVChunk, &tm_v, v_full + s, 64 * c, krow,
                                kplane, pol_kv);
-            if constexpr (G::kTail)
-              tma_load_3d_hint(smem + G::kVOff + s * G::kVBytes + G::kNFull * G::kVChunk, &tm_v32, v_full + s,
-                               64 * G::kNFull, krow, kplane, pol_kv);
           }
         }
         base += w.n_iter;
@@ -558,8 +561,13 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
       // so the softmax only ever sees a positive scale
       constexpr int kM = kPair ? 2 * kBM : kBM;
       const uint32_t idesc_s = umma_idesc_f16(kM, BN, 1, 1, false) | (A.negate_s << 13);
-      // PV in up to two MMAs: the 64-dim chunks (N = 64 kNFull) and the 32-dim tail
-      constexpr uint32_t idesc_o = umma_idesc_f16(kM, G::kNFull > 0 ? 64 * G::kNFull : 32, 1, 1, true);
+      // PV: one MMA over every dim (N = D; a padded tail chunk's upper half
+      // is never read), or, with a 64-byte-swizzled tail, the 64-dim chunks
+      // (N = 64 kNFull) and the tail (N = 32)
+      constexpr uint32_t idesc_o =
+          umma_idesc_f16(kM, G::kTailSw64 ? (G::kNFull > 0 ? 64 * G::kNFull : 32) : D, 1, 1, true);
+      // S: 16-dim k-steps over the 128-byte-swizzled chunks (2 in a padded tail)
+      constexpr int kSSteps = 4 * G::kNFull + ((G::kTail && !G::kTailSw64) ? 2 : 0);
       constexpr uint32_t idesc_o32 = umma_idesc_f16(kM, 32, 1, 1, true);
       const uint32_t q_base = smem_u32(smem);
       // operand descriptors are built once; a k-step only moves the start
@@ -567,7 +575,7 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
       const uint64_t dq0 = umma_desc_sw128(q_base, 16, 1024);
       const uint64_t dk0 = umma_desc_sw128(q_base + G::kKOff, 16, 1024);
       const uint64_t dv0 = umma_desc_sw128(q_base + G::kVOff, G::kVChunk, 1024);
-      // 32-dim tails (64-byte swizzle): Q of tile 0, K and V of stage 0
+      // 64-byte-swizzled 32-dim tails (int8 K/V at d = 96): Q of tile 0, K and V of stage 0
       const uint64_t dq32 = umma_desc_sw64(q_base + G::kNFull * kChunkBytes, 16, 512);
       const uint64_t dk32 = umma_desc_sw64(q_base + G::kKOff + G::kNFull * G::kKChunk, 16, 512);
       const uint64_t dv32 = umma_desc_sw64(q_base + G::kVOff + G::kNFull * G::kVChunk, 16, 512);
@@ -575,13 +583,13 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
         const uint64_t dq = dq0 + ((t * G::kQBytes) >> 4);
         const uint64_t dk = dk0 + ((st * G::kKBytes) >> 4);
 #pragma unroll
-        for (int k = 0; k < 4 * G::kNFull; ++k) {
+        for (int k = 0; k < kSSteps; ++k) {
           const uint32_t off_q = ((k / 4) * kChunkBytes + (k % 4) * 32) >> 4;
           const uint32_t off_k = ((k / 4) * G::kKChunk + (k % 4) * 32) >> 4;
           if constexpr (kPair) mma_ss_pair(tmem + G::s_col(t), dq + off_q, dk + off_k, idesc_s, k > 0 ? 1u : 0u);
           else mma_ss(tmem + G::s_col(t), dq + off_q, dk + off_k, idesc_s, k > 0 ? 1u : 0u);
         }
-        if constexpr (G::kTail) {
+        if constexpr (G::kTailSw64) {
           const uint64_t tq = dq32 + ((t * G::kQBytes) >> 4), tk = dk32 + ((st * G::kKBytes) >> 4);
 #pragma unroll
           for (int k = 0; k < 2; ++k)
@@ -599,9 +607,9 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
           if constexpr (kPair) {
             mma_ts_pair(tmem + G::o_col(t), tmem + G::s_col(t) + k * 8, dv + ((k * 2048) >> 4), idesc_o, acc);
           } else {
-            if constexpr (G::kNFull > 0)
+            if constexpr (G::kNChunks > 0)
               mma_ts(tmem + G::o_col(t), tmem + G::s_col(t) + k * 8, dv + ((k * 2048) >> 4), idesc_o, acc);
-            if constexpr (G::kTail)
+            if constexpr (G::kTailSw64)
               mma_ts(tmem + G::o_col(t) + 64 * G::kNFull, tmem + G::s_col(t) + k * 8,
                      dv32 + ((st * G::kVBytes + k * 1024) >> 4), idesc_o32, acc);
           }
@@ -697,7 +705,7 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
         if (gi >= n_op &&
             !(ok = __all_sync(0xffffffffu, wait_parity(op_empty + s, (gi / n_op - 1) & 1, A.wd, &abort_flag))))
           break;
-        convert_int8_half_row<D, G::kNFull>(smem + (is_v ? G::v_stage(rs) : G::k_stage(rs)),
+        convert_int8_half_row<D, G::kNChunks>(smem + (is_v ? G::v_stage(rs) : G::k_stage(rs)),
                                             smem + op_off + s * G::kKBytes, G::kKChunk, row, h, sc);
         fence_proxy_async_smem();
         mbar_arrive(raw_empty + rs);
@@ -739,12 +747,12 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
           if (vkey < w.sq.s_k) vsc = __ldg(A.v_scales + at + r);
         }
         if (!(ok = __all_sync(0xffffffffu, wait_parity(kraw_full + s, ph, A.wd, &abort_flag)))) break;
-        convert_int8_row<k_nc, D, G::kNFull>(smem + G::k_stage(s), smem + G::kKOff + s * G::kKBytes, G::kKChunk,
+        convert_int8_row<k_nc, D, G::kNChunks>(smem + G::k_stage(s), smem + G::kKOff + s * G::kKBytes, G::kKChunk,
                                              k_r, k_c0, ksc);
         fence_proxy_async_smem();
         arrive_x(k_full + s);
         if (!(ok = __all_sync(0xffffffffu, wait_parity(vraw_full + sv, phv, A.wd, &abort_flag)))) break;
-        convert_int8_row<v_rl / 16, v_rl, kPair ? 8 : G::kNFull>(smem + G::v_stage(sv),
+        convert_int8_row<v_rl / 16, v_rl, kPair ? 8 : G::kNChunks>(smem + G::v_stage(sv),
                                                                  smem + G::kVOff + sv * G::kVBytes, G::kVChunk, r, 0,
                                                                  vsc);
         fence_proxy_async_smem();
@@ -1046,27 +1054,17 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowS
                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != FA_OK) return st;
   }
-  // 32-dim tails (64-byte swizzle): boxes of 32 dims, the same rows
-  CUtensorMap tq32 = tq, tk32 = tk, tv32 = tv;
-  if constexpr (G::kTail) {
+  // the 64-byte-swizzled Q tail (int8 K/V at d = 96): boxes of 32 dims, the
+  // same rows.  Every other tail is a 64-dim box of tq / tk / tv whose dims
+  // past D read as zeros.
+  CUtensorMap tq32 = tq;
+  if constexpr (G::kTailSw64) {
     const uint64_t qdims[3] = {static_cast<uint64_t>(D), q_rows, q_planes};
     const uint64_t qstr[2] = {static_cast<uint64_t>(D) * 2, q_rows * D * 2};
     const uint32_t qbox[3] = {32, static_cast<uint32_t>(kSwizzleChunkRows), 1};
     fa_status st = encode_tensor_map(&tq32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.q, qdims, qstr, qbox,
                                      CU_TENSOR_MAP_SWIZZLE_64B);
     if (st != FA_OK) return st;
-    if constexpr (!kI8) {  // int8 rows come in whole through tk / tv
-      const uint64_t kdims[3] = {static_cast<uint64_t>(D), k_rows, k_planes};
-      const uint64_t kstr[2] = {static_cast<uint64_t>(D) * 2, k_rows * D * 2};
-      const uint32_t kbox[3] = {32, krows, 1};
-      const uint32_t vbox[3] = {32, static_cast<uint32_t>(BN), 1};
-      st = encode_tensor_map(&tk32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.k, kdims, kstr, kbox,
-                             CU_TENSOR_MAP_SWIZZLE_64B);
-      if (st != FA_OK) return st;
-      st = encode_tensor_map(&tv32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.v, kdims, kstr, vbox,
-                             CU_TENSOR_MAP_SWIZZLE_64B);
-      if (st != FA_OK) return st;
-    }
   }
   PrefillArgs A;
   A.L = pages != nullptr ? SeqLayout::paged(p, *pages) : SeqLayout::from(p);
@@ -1118,12 +1116,12 @@ fa_status launch_tc(const fa_fwd_params& p, const fa_kv_pages* pages, const RowS
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cuda_status(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, tq32, tk32, tv32, A));
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, tq32, A));
   } else {
     // persistent: one CTA per SM (the shared memory allows no second), each
     // walking its share of the items
     const long long grid = items < device_sm_count() ? items : device_sm_count();
-    kern<<<static_cast<unsigned>(grid), G::kThreads, G::kSmem, ctx.stream>>>(tq, tk, tv, tq32, tk32, tv32, A);
+    kern<<<static_cast<unsigned>(grid), G::kThreads, G::kSmem, ctx.stream>>>(tq, tk, tv, tq32, A);
     return cuda_status(cudaGetLastError());
   }
 }
