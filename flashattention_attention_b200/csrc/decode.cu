@@ -101,7 +101,9 @@ struct Geom {
   static constexpr int kChunkBytes = kTile * 128;
   static constexpr int kNFull = D / 64;                 // bf16: full 64-dim chunks
   static constexpr bool kTail = kBF && (D % 64) == 32;  // bf16: a 32-dim tail chunk
-  static constexpr int kStages = 3;
+  // stages per worker ring (a bf16 tile at D = 256 is 32 KB: one stage,
+  // the producer refilling it as soon as its worker releases it)
+  static constexpr int kStages = (kBF && D == 256) ? 1 : 3;
   static constexpr int kCtas = ((kBF && (D == 128 || D == 96)) || D == 256) ? 1 : 2;
   static constexpr int kSmem = kWarps * kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
   // sequences whose tile prefix fits in the shared memory the CTAs per SM
@@ -114,7 +116,8 @@ static_assert(2 * Geom<128, false>::kSmem <= 232448 && 2 * Geom<64, false>::kSme
               "CTAs per SM");
 static_assert(Geom<128, false>::kCtas <= kMaxCtasPerSm && Geom<64, true>::kCtas <= kMaxCtasPerSm, "workers");
 static_assert(2 * Geom<32, false>::kSmem <= 232448 && 2 * Geom<96, false>::kSmem <= 232448 &&
-                  Geom<256, false>::kSmem <= 232448 && 2 * Geom<32, true>::kSmem <= 232448 &&
+                  Geom<256, false>::kSmem <= 232448 && Geom<256, true>::kSmem <= 232448 &&
+                  2 * Geom<32, true>::kSmem <= 232448 &&
                   Geom<96, true>::kSmem <= 232448,
               "CTAs per SM");
 
@@ -1067,6 +1070,7 @@ fa_status launch_decode(const fa_decode_params& p, const fa_kv_pages* pages, int
     if (p.head_dim == 64) return launch_sk<64, true>(p, pages, variant_workers<64, true>(), mt, p.workspace, true, ctx);
     if (p.head_dim == 32) return launch_sk<32, true>(p, pages, variant_workers<32, true>(), mt, p.workspace, true, ctx);
     if (p.head_dim == 96) return launch_sk<96, true>(p, pages, variant_workers<96, true>(), mt, p.workspace, true, ctx);
+    if (p.head_dim == 256) return launch_sk<256, true>(p, pages, variant_workers<256, true>(), mt, p.workspace, true, ctx);
   }
   return FA_ERR_UNSUPPORTED;
 }

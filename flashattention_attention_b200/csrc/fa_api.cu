@@ -350,9 +350,8 @@ fa_status decode_args(const fa_decode_params* p) {
   if (!std::isfinite(p->softmax_scale)) return FA_ERR_INVALID;
   if (p->kv_dtype != FA_I8 && p->kv_dtype != FA_BF16) return FA_ERR_INVALID;
   if (p->head_dim <= 0 || p->head_dim % 32 != 0) return FA_ERR_INVALID;
-  // int8 cache: 32, 64, 96, 128, 256; bf16 cache: 32, 64, 96, 128
-  if (!(p->head_dim == 32 || p->head_dim == 64 || p->head_dim == 96 || p->head_dim == 128 ||
-        (p->head_dim == 256 && p->kv_dtype == FA_I8)))
+  // int8 or bf16 cache: 32, 64, 96, 128, 256
+  if (!(p->head_dim == 32 || p->head_dim == 64 || p->head_dim == 96 || p->head_dim == 128 || p->head_dim == 256))
     return FA_ERR_UNSUPPORTED;
   if (p->batch == 0) return FA_OK;
   if (p->q == nullptr || p->k_cache == nullptr || p->v_cache == nullptr || p->out == nullptr ||

@@ -171,7 +171,7 @@ FA_API fa_status fa_attention_fwd(const fa_fwd_params *p, fa_stream_t stream);
  * keys each warp is given (fewer, longer ranges).  capacity must be a
  * multiple of 32; cache entries at or past L_b may hold any bytes (they never
  * reach the result).
- * Supported: head_dim 32, 64, 96 or 128 (FA_I8 and FA_BF16), 256 (FA_I8); any hq / hkv (a group
+ * Supported: head_dim 32, 64, 96, 128 or 256 (FA_I8 and FA_BF16); any hq / hkv (a group
  * of more than 8 query heads is served in passes of at most 8 heads, each
  * reading the KV head's cache once).
  */

@@ -45,6 +45,8 @@ CASES = [
     (1, 12, 1, 64, 512, [333]),               # G = 12: two passes of 6
     (3, 8, 2, 32, 1024, [1000, 33, 512]),     # d = 32: one 32-dim chunk (64-byte swizzle)
     (2, 8, 2, 96, 1024, [999, 100]),          # d = 96: a 64-dim chunk and a 32-dim tail
+    (2, 8, 2, 256, 1024, [1000, 33]),         # d = 256: four 64-dim chunks, one ring stage per worker
+    (1, 16, 1, 256, 512, [512]),              # d = 256, G = 16
 ]
 
 
@@ -57,7 +59,7 @@ def test_decode_bf16_cases(case):
     assert_close_bf16(got.float().numpy().reshape(ref.shape), ref, what=str(case))
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_decode_bf16_window_epilogue_and_poisoned_rows(d):
     """Rows past L_b and, with a window, rows before L_b - W are NaN / Inf in
     both caches; the result must equal the oracle on the clean cache."""

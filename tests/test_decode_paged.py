@@ -50,8 +50,6 @@ def paginate(dense, scales, lengths, hkv, page_size, extra, rng):
                                                        (128, 64, 300, 16, 4), (128, 64, 0, 32, 2), (96, 64, 0, 16, 4),
                                                        (256, 128, 0, 8, 2)])
 def test_paged_equals_dense(int8, d, page_size, window, hq, hkv):
-    if not int8 and d == 256:
-        pytest.skip("bf16 cache decode: head sizes up to 128")
     fa = _fa()
     rng = np.random.default_rng(d + page_size + window + int8 + hq)
     B, cap = 6, 1024
