@@ -53,7 +53,7 @@
 // round once to bf16, the tensor-core operand type, write it in the operand
 // layout and fence it to the async proxy.  The softmax is then the bf16 one.
 // That variant runs 16 warps and rebalances registers with setmaxnreg
-// (softmax 192, the rest 64).  Above d = 128 (one Q tile, 64-key tiles, 12
+// (softmax 176, the rest 80).  Above d = 128 (one Q tile, 64-key tiles, 12
 // warps) two converter threads share a key row, and the int8 tiles land in
 // rings of their own so the bf16 operand slots fit beside the Q tile.
 #include <cstdlib>
@@ -137,10 +137,10 @@ struct TcGeom {
   static constexpr int kThreads = (4 * NT + ((kI8 || NT == 4) ? (kI8 ? (kSplitRaw ? 12 : 8) : 4) : 2)) * 32;
   // setmaxnreg split (0: none): the softmax warpgroups take kRegsHi, the
   // others give back down to 64 (the totals match the launch's pool)
-  // (int8 with one Q tile, 512 threads: one softmax warpgroup at 192, three
-  // at 96: 128*192 + 384*96 <= 512*128)
-  static constexpr int kRegsHi = kI8 ? 192 : (NT == 4 ? 104 : 0);
-  static constexpr int kRegsLo = kSplitRaw ? 96 : 64;
+  // (int8, two Q tiles: 2 x 128 threads at 176, 2 x 128 at 80 = 512 * 128;
+  // with one Q tile, 512 threads: one softmax warpgroup at 192, three at 96)
+  static constexpr int kRegsHi = kI8 ? (kSplitRaw ? 192 : 176) : (NT == 4 ? 104 : 0);
+  static constexpr int kRegsLo = kSplitRaw ? 96 : (NT == 4 ? 64 : 80);
   // the registers a launch of kThreads threads gets per thread, which the
   // split redistributes (setmaxnreg.inc waits for registers the pool lacks)
   static constexpr int kLaunchRegs = (65536 / kThreads) / 8 * 8;
@@ -462,12 +462,10 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   // Roles split by warpgroup first: the first NT warpgroups softmax, the rest
-  // the other roles.  int8 variant registers: 512 threads launched at 128;
-  // warpgroups 0-1 take 192, warpgroups 2-3 give back down to 64:
-  // 256*192 + 256*64 = 512*128.
+  // the other roles, which give registers back to the softmax warpgroups
+  // where TcGeom sets a split (kRegsHi / kRegsLo).
   if (warp >= 4 * NT) {
-  if constexpr (G::kRegsHi > 0 && G::kRegsLo == 64) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
-  if constexpr (G::kRegsHi > 0 && G::kRegsLo == 96) asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
+  if constexpr (G::kRegsHi > 0) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(G::kRegsLo) : "memory");
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -762,8 +760,7 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
     }
   }
   } else {
-  if constexpr (G::kRegsHi == 192) asm volatile("setmaxnreg.inc.sync.aligned.u32 192;" ::: "memory");
-  if constexpr (G::kRegsHi == 104) asm volatile("setmaxnreg.inc.sync.aligned.u32 104;" ::: "memory");
+  if constexpr (G::kRegsHi > 0) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(G::kRegsHi) : "memory");
   if (warp / 4 < ntile) {
     // ------------------------------------------------------------ softmax
     const int t = warp / 4, quarter = warp % 4;
