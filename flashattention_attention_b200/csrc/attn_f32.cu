@@ -10,8 +10,8 @@
 // max m and sum l in fp32, exp2 with log2(e) folded into the scale).
 // With an int8 KV cache (fkl_python PR #6, Verification: int8-cache
 // attention checked against an oracle on the dequantised cache) each K/V element enters the shared tile as c * s
-// computed in fp32, which is exact (|c| <= 127 times an fp32 scale), so the
-// kernel sees the dequantised cache itself.
+// rounded once to fp32 (a 7-bit |c| times a 24-bit significand can need 31
+// bits: relative error at most 2^-24, far inside the fp32 path's tolerance).
 //
 // empty_rows_kernel: rows whose band is empty (causal with s_q > s_k leaves
 // rows i < s_q - s_k without keys; s_k = 0 leaves every row without keys)

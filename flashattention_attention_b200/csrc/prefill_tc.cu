@@ -49,11 +49,11 @@
 // for both products and never widens the cache in global memory): TMA
 // brings each int8 tile into shared memory (at d = 128 into the upper half of
 // the bf16 slot it becomes); four converter warps, one thread per key row,
-// dequantise it as c * s in fp32 (exact: |c| <= 127 times an fp32 scale),
-// round once to bf16, the tensor-core operand type, write it in the operand
-// layout and fence it to the async proxy.  The softmax is then the bf16 one.
+// dequantise it as c * s in fp32 (dequant4_bf16 below), round it to bf16,
+// the tensor-core operand type, write it in the operand layout and fence it
+// to the async proxy.  The softmax is then the bf16 one.
 // That variant runs 16 warps and rebalances registers with setmaxnreg
-// (softmax 176, the rest 80).  Above d = 128 (one Q tile, 64-key tiles, 12
+// (softmax 176, the rest 80).  Above d = 128 (one Q tile, 64-key tiles, 16
 // warps) two converter threads share a key row, and the int8 tiles land in
 // rings of their own so the bf16 operand slots fit beside the Q tile.
 #include <cstdlib>
@@ -197,11 +197,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Four signed bytes of w times the row scale, each product rounded once to
-// bf16 (two bf16x2 words).  Each byte b, flipped to b ^ 0x80 = c + 128, is
-// placed in the low mantissa byte of 2^23, so the float is 2^23 + 128 + c and
-// one exact subtraction leaves c; c * s is then exact in fp32 (8 x 24 bits
-// fit), and the bf16 cast is the only rounding.
+// Four signed bytes of w times the row scale, as bf16 (two bf16x2 words).
+// Each byte b, flipped to b ^ 0x80 = c + 128, is placed in the low mantissa
+// byte of 2^23, so the float is 2^23 + 128 + c and one exact subtraction
+// leaves c.  c * s is rounded to fp32 (a 7-bit |c| times a 24-bit
+// significand can need 31 bits) and then to bf16; that differs from one
+// rounding of c * s to bf16 only when the fp32 result lands exactly halfway
+// between two bf16 values, by one bf16 unit in the last place.
 __device__ __forceinline__ uint2 dequant4_bf16(uint32_t w, float2 s2) {
   const uint32_t x = w ^ 0x80808080u;
   uint32_t f[4];

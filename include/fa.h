@@ -114,9 +114,9 @@ FA_API fa_status fa_compress_kv(const void *x, fa_dtype x_dtype, int64_t rows, i
  * with k_scales/v_scales [batch*hkv, seqlen_k] dense or [hkv, total_k]
  * varlen, one fp32 scale per (token, kv-head) as fa_compress_kv writes them
  * (16-byte aligned on the BF16 path).  The kernels dequantise c * s on chip
- * (fkl_python PR #6, Summary): exactly in fp32 on the F32 path; on the BF16
- * path c * s is formed exactly in fp32 and rounded once to bf16, the
- * tensor-core operand type.  out has q's dtype.
+ * (fkl_python PR #6, Summary): rounded to fp32 on the F32 path (relative
+ * error at most 2^-24); on the BF16 path rounded to fp32 and then to bf16,
+ * the tensor-core operand type.  out has q's dtype.
  * head_dim: F32 path any multiple of 32 up to 256; BF16 path 32, 64, 96, 128,
  * 160, 192, 224 or 256 (FA_BF16 or FA_I8 K/V).
  * A problem without keys (seqlen_k = 0, or varlen total_k = 0 with
