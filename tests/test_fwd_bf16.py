@@ -104,6 +104,13 @@ def test_epilogue_and_determinism():
     assert_close_bf16(outs[0].float().numpy(), ref)
     ref2 = oracle.attention(w.q, w.k, w.v, hq=4, hkv=2, causal=True, epilogue=[("mul", -1.5), ("add", 3.0)])
     assert_close_bf16(outs[1].float().numpy(), ref2)
+    # the most ops a call takes (FA_MAX_EPILOGUE = 8), still no new kernel
+    longest = [("mul", 2.0), ("add", 0.5), ("mul", 0.25), ("add", -1.0), ("mul", 3.0), ("add", 0.125),
+               ("mul", -0.5), ("add", 2.0)]
+    got = gpu_fwd(w.q, w.k, w.v, hq=4, hkv=2, causal=True, epilogue=longest)
+    assert fa.kernel_variants_used() == variants
+    ref3 = oracle.attention(w.q, w.k, w.v, hq=4, hkv=2, causal=True, epilogue=longest)
+    assert_close_bf16(got.float().numpy(), ref3)
 
 
 def test_gqa_equals_repeated_kv():

@@ -90,8 +90,10 @@ def test_epilogue_fused_equals_host_applied():
     w = inputs.tiny_fp32_causal()
     base = run_dense(w.q, w.k, w.v, w.hq, w.hkv, causal=True, scale=w.scale).numpy()
     variants = fa.kernel_variants_used()
+    longest = [("mul", 2.0), ("add", 0.5), ("mul", 0.25), ("add", -1.0), ("mul", 3.0), ("add", 0.125),
+               ("mul", -0.5), ("add", 2.0)]  # the most ops a call takes (FA_MAX_EPILOGUE)
     for epi in ([("mul", 2.0), ("add", 0.5)], [("mul", -3.0), ("add", 1.25)], [("add", 0.5)],
-                [("mul", 2.0), ("add", 0.5), ("mul", 0.25)]):
+                [("mul", 2.0), ("add", 0.5), ("mul", 0.25)], longest):
         fused = run_dense(w.q, w.k, w.v, w.hq, w.hkv, causal=True, scale=w.scale, epilogue=epi).numpy()
         host = base.copy()
         for op, val in epi:
