@@ -274,7 +274,11 @@ __device__ __forceinline__ uint32_t to_nibbles(uint32_t f) {
 //     so their order inside a k-step is free: thread (g, t) takes channels
 //     [t d/4, t d/4 + d/4) of its rows, four per k-step, and the rotated
 //     queries' B fragments (fp16, registers) use the same order.  A
-//     fragments come from the packed codes by byte permutes (dequant4).
+//     fragments come from the packed codes: with 4-bit codes each code byte
+//     (two channels) indexes a table of fp16 level pairs in dynamic shared
+//     memory, 32 KB with one copy per lane so every lane reads its own bank
+//     (one load per fragment register); other widths by byte permutes
+//     (dequant4).
 //   online softmax per head on the S fragments; P'[key, head] = p ||v_key||
 //     in fp16, turned from S fragments into B fragments by 8x8 transposes.
 //   V: lane j dequantises key j's codes into an fp16 tile [32 keys x D] in
@@ -282,8 +286,9 @@ __device__ __forceinline__ uint32_t to_nibbles(uint32_t f) {
 //     swizzled by the key's low bits, so ldmatrix reads are conflict-free),
 //     then O_rot^T [D x 8 heads] += Vlev^T . P' on mma.sync (channels on M,
 //     heads on N, keys on K), the A fragments read by ldmatrix.trans.
+// Three CTAs per SM: at most 168 registers a thread.
 template <int D, int KB, int VB, int G>
-__global__ void __launch_bounds__(kDecodeWarps * 32)
+__global__ void __launch_bounds__(kDecodeWarps * 32, 3)
     tq_decode_kernel(TqArgs A) {
   constexpr int E = D / 32;
   constexpr int KROW = D * KB / 8;  // bytes of a packed K row
@@ -302,6 +307,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   // the V tiles during the key loop, the per-warp O rows after it
   __shared__ __align__(128) unsigned char vbuf[kVdqBytes > kSoBytes ? kVdqBytes : kSoBytes];
   float(*s_o)[G][D] = reinterpret_cast<float(*)[G][D]>(vbuf);
+  // 4-bit K codes: fp16 level pairs of every code byte, one copy per lane
+  // (entry e of lane l at word 32 e + l), so each lane reads its own bank
+  extern __shared__ __align__(16) uint32_t ktab[];
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gq = lane >> 2, tq = lane & 3;  // fragment row group and column pair
@@ -316,7 +324,16 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   const int k1 = min(len, k0 + A.split_keys);
   for (int c = threadIdx.x; c < (1 << (2 * VB)); c += blockDim.x)
     vtab[c] = pack_h2(A.v_levels[c & ((1 << VB) - 1)], A.v_levels[c >> VB]);
-  // the upper half of the K levels as fp16 byte planes (8 entries, zero-padded)
+  if constexpr (KB == 4) {
+    if (k0 < k1) {
+      for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
+        const int e = i >> 5;
+        ktab[i] = pack_h2(A.k_levels[e & 15], A.k_levels[e >> 4]);
+      }
+    }
+  }
+  // other widths: the upper half of the K levels as fp16 byte planes (8
+  // entries, zero-padded)
   uint32_t pl[2] = {0u, 0u}, ph[2] = {0u, 0u};
 #pragma unroll
   for (int jj = 0; jj < (1 << (KB - 1)); ++jj) {
@@ -437,8 +454,20 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         uint32_t a0, a1, a2, a3;
-        dequant4<KB>(to_nibbles<KB>(code_at<4 * KB, SW>(kc4[2 * mt], 4 * ks * KB)), pl, ph, a0, a2);
-        dequant4<KB>(to_nibbles<KB>(code_at<4 * KB, SW>(kc4[2 * mt + 1], 4 * ks * KB)), pl, ph, a1, a3);
+        if constexpr (KB == 4) {
+          // the code bytes of channels 4 ks .. +3: each byte is the table
+          // index of its fp16 pair (offset 128 bytes per entry)
+          const uint32_t* kt = ktab + lane;
+          const uint32_t w0 = kc4[2 * mt][ks >> 1] >> (16 * (ks & 1));
+          const uint32_t w1 = kc4[2 * mt + 1][ks >> 1] >> (16 * (ks & 1));
+          a0 = kt[(w0 << 5) & 0x1fe0u];
+          a2 = kt[(w0 >> 3) & 0x1fe0u];
+          a1 = kt[(w1 << 5) & 0x1fe0u];
+          a3 = kt[(w1 >> 3) & 0x1fe0u];
+        } else {
+          dequant4<KB>(to_nibbles<KB>(code_at<4 * KB, SW>(kc4[2 * mt], 4 * ks * KB)), pl, ph, a0, a2);
+          dequant4<KB>(to_nibbles<KB>(code_at<4 * KB, SW>(kc4[2 * mt + 1], 4 * ks * KB)), pl, ph, a1, a3);
+        }
         mma_f16(sacc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
       }
     }
@@ -617,9 +646,13 @@ __global__ void __launch_bounds__(256)
 
 template <int D, int KB, int VB>
 fa_status launch_decode_g(const TqArgs& A, int group, dim3 grid, cudaStream_t st) {
+  // 4-bit K: the replicated pair table in dynamic shared memory
+  constexpr int kDyn = KB == 4 ? 256 * 32 * 4 : 0;
   auto go = [&](auto kern) {
     note_variant(reinterpret_cast<const void*>(kern));
-    kern<<<grid, kDecodeWarps * 32, 0, st>>>(A);
+    if (kDyn > 0 && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDyn) != cudaSuccess)
+      return FA_ERR_CUDA;
+    kern<<<grid, kDecodeWarps * 32, kDyn, st>>>(A);
     return cuda_status(cudaGetLastError());
   };
   switch (group) {
