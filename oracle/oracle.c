@@ -17,7 +17,7 @@
  * paper and the online softmax trick), so the plain definition is the
  * oracle.
  *
- * Readings taken where the pages are silent (each also listed in the design doc):
+ * Readings taken where the pages are silent:
  *  - causal alignment is bottom-right: query row i of a sequence with s_q
  *    queries and s_k keys sits at key position p = i + s_k - s_q;
  *  - a window W > 0 keeps keys j with p - W < j (W keys including self when
