@@ -943,9 +943,13 @@ __global__ void __launch_bounds__(TcGeom<D, kI8, kPair, BN, NT>::kThreads, 1)
 #pragma unroll
       for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
       if (store) {
+        // written once and never read here: marked to leave L2 before the
+        // K/V tiles that later q-blocks read again
         uint4* dst = reinterpret_cast<uint4*>(orow + oc * 32);
+        const uint64_t pol_o = l2_policy_evict_first();
 #pragma unroll
-        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        for (int v = 0; v < 4; ++v)
+          stg_v4_hint(dst + v, make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]), pol_o);
       }
     }
     base += w.n_iter;
