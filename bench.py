@@ -53,6 +53,7 @@ KERNEL_SOURCES = {
     "prefill_tc_kernel<128,int8>": ["prefill_tc.cu", "umma.cuh", "device.cuh", "layout.cuh"],
     "prefill_tc_kernel<64,bf16>": ["prefill_tc.cu", "umma.cuh", "device.cuh", "layout.cuh"],
     "decode_sk_kernel<128>": ["decode.cu", "device.cuh"],
+    "decode_sk_kernel<128,bf16>": ["decode.cu", "device.cuh"],
     "compress_rows8_kernel<bf16,16>": ["quant.cu", "device.cuh"],
 }
 
@@ -725,7 +726,8 @@ def decode_and_quant(args, dev, peaks, world, dist, result):
                                  "unit": "GB/s", "us_per_step": round(bf_ms * 1e3, 2), "bytes_per_step": bf_bytes,
                                  "roofline": {"bound": "hbm", "kernel": "decode_sk_kernel<128,bf16> + decode_plan_kernel",
                                               "achieved": round(bf_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                              "frac": round(bf_gbs / peaks["hbm_gbs"], 4), "traffic": None}}
+                                              "frac": round(bf_gbs / peaks["hbm_gbs"], 4),
+                                              "traffic": measured_traffic("decode_sk_kernel<128,bf16>")}}
         del kb, vb
         torch.cuda.empty_cache()
     assert fa.check_device_error() == fa.FA_OK
