@@ -38,7 +38,8 @@
 // chunks of 128-byte rows (128-byte swizzle); K fragments come from ldmatrix,
 // V^T fragments from ldmatrix.trans, Q enters the bf16 MMA as it is and P is
 // rounded to bf16.  A stage is twice as large, so d = 128 runs one CTA per
-// SM.  Cache rows outside [k_lo, L) may hold any bytes (NaN included): their
+// SM, and at d = 256 (32 KB for a K and a V tile) each worker's ring holds
+// one stage.  Cache rows outside [k_lo, L) may hold any bytes (NaN included): their
 // scores are masked, and in a tile that holds such rows the V rows are zeroed
 // in shared memory before P V, so 0 * NaN never reaches O.
 #include <mutex>

@@ -27,6 +27,15 @@
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 after it.
 // P (bf16, two per 32-bit column) overwrites the first 64 columns of its S
 // tile and is the A operand of O += P V straight from TMEM.
+// Above d = 128 two O tiles no longer fit beside their S tiles: one Q tile
+// per CTA and 64-key K/V tiles (S [0,64), O [64,64+D)).
+//
+// Operand tiles are 64-dim chunks in the 128-byte swizzle; a 32-dim remainder
+// of the head size is one more such chunk whose upper half the TMA fills
+// with zeros (int8 K/V at d = 96: a 32-dim chunk in the 64-byte swizzle).
+// L2 policies: Q loads evict_first (read once), K/V loads evict_last (read
+// again by later q-blocks and the group's other head pairs), output stores
+// evict_first.
 //
 // Result modes: the normalised output (epilogue applied, bf16); that output
 // with each row's log-sum-exp (a partial result over the given keys); or,
@@ -258,7 +267,7 @@ __device__ __forceinline__ void convert_int8_row(const uint8_t* src_tile, uint8_
 // f (row / 2).  The two threads of a row cover it once; a, b, f were found
 // by an exhaustive search so that the 8 lanes of each shared-memory phase
 // (4 rows x 2 halves) read 8 different bank groups, and write at most 2 to
-// one (only where the 32-dim tail's 64-byte rows are involved).
+// one (2 only at d = 160 and 224; no order of this family does better).
 template <int D, int kNFull>
 __device__ __forceinline__ void convert_int8_half_row(const uint8_t* src_tile, uint8_t* dst_tile, uint32_t dst_chunk,
                                                       int row, int h, float sc) {

@@ -1,9 +1,11 @@
 // quant.cu -- per-row int8 KV quantiser (fkl_python PR #6, Summary: the
 // cache compressed on the GPU to int8 codes per token, one fp32 scale each).
 //
-// One warp per row.  Each lane holds 4 consecutive elements per 128-element
-// chunk (8-byte bf16 / 16-byte fp32 vector loads, fully coalesced), the warp
-// reduces max|x| with xor-shuffles, and every lane forms c = rint(x / s) with
+// compress_kernel (any d): one warp per row; compress_rows8_kernel (d = 64
+// and 128, further below): eight lanes per row.  In the first, each lane
+// holds 4 consecutive elements per 128-element chunk (8-byte bf16 / 16-byte
+// fp32 vector loads, fully coalesced), the warp reduces max|x| with
+// xor-shuffles, and every lane forms c = rint(x / s) with
 // s = amax / 127 (IEEE division, once per row), rounds half to even, and
 // stores its 4 codes as one packed 32-bit word.  Each warp handles several
 // rows so that enough loads are in flight to stream HBM.
